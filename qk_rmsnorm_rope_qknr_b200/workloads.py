@@ -1,0 +1,194 @@
+"""Seeded synthetic inputs for the fused Q/K RMSNorm + RoPE workloads.
+
+This module only draws inputs (and counts their bytes); it holds none of the
+transform's arithmetic, and both the CUDA path and the oracle consume the very
+tensors it returns. Draw order per workload: qkv (or q then k), q_weight,
+k_weight, then the outlier mask; every draw uses one torch.Generator seeded
+with the workload's seed, on the device the caller names (so inputs drawn on
+"cpu" and on "cuda" differ; a test always feeds one tensor to both sides).
+
+Workloads (shapes from the two API pages' parameter lists, sizes from the
+video-DiT and MiniMax-H3 geometries the pages name):
+  tiny3d      3D form, 32 tokens, 4+4+4 heads of 64, grid 2x4x4, 16/24/24
+  table_hs    table form, half-split, q [4096,32,128], k [4096,8,128], rd 96, fp32 table
+  table_il    table form, adjacent pairs, q,k [2048,24,128] (x3, 1% outliers x20),
+              rd 128, bf16 table
+  video3d     3D form, [1,15360,(32+32+32)*128], grid 16x30x32, 16/56/56, bf16 out
+  fp8neox     3D form, [2,29760,(24+24+24)*128] ~N(0, 2^2), grid 31x24x40,
+              32/48/48, NeoX pairs, E4M3 out (scales 0.5 / 0.25)
+  fp8neox_nonorm  fp8neox with is_qk_norm=False
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Form3D:
+    name: str
+    batch: int
+    seq: int
+    ppf: int
+    pph: int
+    ppw: int
+    cf: int
+    ch: int
+    cw: int
+    hq: int
+    hk: int
+    hv: int
+    head_dim: int
+    eps: float = 1e-6
+    base: float = 10000.0
+    interleave: bool = True
+    is_qk_norm: bool = True
+    output_fp8: bool = False
+    q_scale: float = 1.0
+    v_scale: float = 1.0
+    std: float = 1.0
+    seed: int = 0
+    input_2d: bool = False
+    form: str = "3d"
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seq
+
+    @property
+    def row(self) -> int:
+        return (self.hq + self.hk + self.hv) * self.head_dim
+
+    def params(self) -> dict:
+        """Keyword arguments of the 3D entry point (the page's names)."""
+        return dict(ppf=self.ppf, pph=self.pph, ppw=self.ppw, num_frame_channels=self.cf,
+                    num_height_channels=self.ch, num_width_channels=self.cw,
+                    num_heads_q=self.hq, num_heads_k=self.hk, num_heads_v=self.hv,
+                    head_dim=self.head_dim, eps=self.eps, base=self.base,
+                    interleave=self.interleave, is_qk_norm=self.is_qk_norm,
+                    output_fp8=self.output_fp8, output_quant_scale=self.q_scale,
+                    v_quant_scale=self.v_scale)
+
+
+@dataclasses.dataclass(frozen=True)
+class FormTable:
+    name: str
+    tokens: int
+    hq: int
+    hk: int
+    head_dim: int
+    rotary_dim: int
+    table_f32: bool
+    interleaved: bool
+    eps: float = 1e-6
+    std: float = 1.0
+    outlier_frac: float = 0.0
+    outlier_mult: float = 1.0
+    rope_base: float = 10000.0
+    seed: int = 0
+    form: str = "table"
+
+
+WORKLOADS = {
+    "tiny3d": Form3D("tiny3d", batch=1, seq=32, ppf=2, pph=4, ppw=4, cf=16, ch=24, cw=24, hq=4,
+                     hk=4, hv=4, head_dim=64, input_2d=True),
+    "table_hs": FormTable("table_hs", tokens=4096, hq=32, hk=8, head_dim=128, rotary_dim=96,
+                          table_f32=True, interleaved=False),
+    "table_il": FormTable("table_il", tokens=2048, hq=24, hk=24, head_dim=128, rotary_dim=128,
+                          table_f32=False, interleaved=True, std=3.0, outlier_frac=0.01,
+                          outlier_mult=20.0),
+    "video3d": Form3D("video3d", batch=1, seq=15360, ppf=16, pph=30, ppw=32, cf=16, ch=56,
+                      cw=56, hq=32, hk=32, hv=32, head_dim=128),
+    "fp8neox": Form3D("fp8neox", batch=2, seq=29760, ppf=31, pph=24, ppw=40, cf=32, ch=48,
+                      cw=48, hq=24, hk=24, hv=24, head_dim=128, interleave=False,
+                      output_fp8=True, q_scale=0.5, v_scale=0.25, std=2.0),
+    "fp8neox_nonorm": Form3D("fp8neox_nonorm", batch=2, seq=29760, ppf=31, pph=24, ppw=40,
+                             cf=32, ch=48, cw=48, hq=24, hk=24, hv=24, head_dim=128,
+                             interleave=False, is_qk_norm=False, output_fp8=True, q_scale=0.5,
+                             v_scale=0.25, std=2.0),
+}
+
+
+def _normal(g: torch.Generator, shape, std: float, device) -> torch.Tensor:
+    x = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    return (x * std).to(torch.bfloat16) if std != 1.0 else x.to(torch.bfloat16)
+
+
+def _weight(g: torch.Generator, n: int, device) -> torch.Tensor:
+    w = torch.randn(n, generator=g, dtype=torch.float32, device=device)
+    return (1.0 + 0.1 * w).to(torch.bfloat16)
+
+
+def rope_table_input(tokens: int, rotary_dim: int, base: float, f32: bool,
+                     device="cpu") -> torch.Tensor:
+    """A caller-built [tokens, rotary_dim] table [cos(theta) | sin(theta)] with
+    theta[t, i] = t * base^(-2i/rotary_dim), built in float64 and stored as
+    float32 or bfloat16 (the input the table form consumes)."""
+    half = rotary_dim // 2
+    pos = torch.arange(tokens, dtype=torch.float64).unsqueeze(1)
+    inv = base ** (-2.0 * torch.arange(half, dtype=torch.float64) / rotary_dim)
+    theta = pos * inv.unsqueeze(0)
+    tbl = torch.cat([torch.cos(theta), torch.sin(theta)], dim=1)
+    return tbl.to(torch.float32 if f32 else torch.bfloat16).to(device)
+
+
+def make_inputs(w, device="cpu", tokens: Optional[int] = None, seed: Optional[int] = None):
+    """Inputs of workload `w` (a Form3D / FormTable or its name) on `device`.
+
+    tokens overrides the token count (3D: a 2D [tokens, row] input; it must stay
+    a multiple of ppf*pph*ppw for the 3D form's own rule) for smaller cases.
+    Returns a dict of tensors.
+    """
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed if seed is None else seed)
+    if w.form == "3d":
+        if tokens is None:
+            shape = (w.seq, w.row) if w.input_2d else (w.batch, w.seq, w.row)
+        else:
+            shape = (tokens, w.row)
+        qkv = _normal(g, shape, w.std, device)
+        qw = _weight(g, w.hq * w.head_dim, device)
+        kw = _weight(g, w.hk * w.head_dim, device)
+        return dict(qkv=qkv, q_weight=qw, k_weight=kw)
+    T = w.tokens if tokens is None else tokens
+    q = _normal(g, (T, w.hq, w.head_dim), w.std, device)
+    k = _normal(g, (T, w.hk, w.head_dim), w.std, device)
+    qw = _weight(g, w.head_dim, device)
+    kw = _weight(g, w.head_dim, device)
+    if w.outlier_frac > 0:
+        mq = torch.rand(q.shape, generator=g, device=device) < w.outlier_frac
+        mk = torch.rand(k.shape, generator=g, device=device) < w.outlier_frac
+        q = torch.where(mq, (q.float() * w.outlier_mult).to(torch.bfloat16), q)
+        k = torch.where(mk, (k.float() * w.outlier_mult).to(torch.bfloat16), k)
+    table = rope_table_input(T, w.rotary_dim, w.rope_base, w.table_f32, device)
+    return dict(q=q, k=k, q_weight=qw, k_weight=kw, rope_table=table)
+
+
+def algorithmic_bytes(w, tokens: Optional[int] = None) -> int:
+    """Bytes one launch must move at minimum: every input read once, every
+    output written once, the weights (and table) read once."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    if w.form == "3d":
+        T = w.tokens if tokens is None else tokens
+        out_b = 1 if w.output_fp8 else 2
+        per_tok = w.row * 2 + w.row * out_b
+        weights = 2 * (w.hq + w.hk) * w.head_dim if w.is_qk_norm else 0
+        return T * per_tok + weights
+    T = w.tokens if tokens is None else tokens
+    per_tok = 2 * 2 * (w.hq + w.hk) * w.head_dim + w.rotary_dim * (4 if w.table_f32 else 2)
+    return T * per_tok + 2 * 2 * w.head_dim
+
+
+def bytes_per_token(w) -> float:
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    return algorithmic_bytes(w) / w.tokens
+
+
+_ = math

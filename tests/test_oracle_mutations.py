@@ -1,0 +1,76 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case copies oracle/qknr_oracle.c, plants one mistake by a textual edit,
+compiles the copy on the CPU, and runs the pins of test_oracle_pins.py against
+it: at least one pin must fail. (The direction of the FP8 scale is a reading
+the pages leave open, so no case flips it.)
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle as O
+from tests import test_oracle_pins as P
+
+SRC = os.path.join(os.path.dirname(O.__file__), "qknr_oracle.c")
+
+MUTATIONS = {
+    "rotation_sign_a": ("out[pa[j]] = a * cos_t[j] - b * sin_t[j];",
+                        "out[pa[j]] = a * cos_t[j] + b * sin_t[j];"),
+    "rotation_sign_b": ("out[pb[j]] = b * cos_t[j] + a * sin_t[j];",
+                        "out[pb[j]] = b * cos_t[j] - a * sin_t[j];"),
+    "dropped_eps": ("sqrt(ssq / (double)n + eps)", "sqrt(ssq / (double)n)"),
+    "mean_over_n_plus_1": ("sqrt(ssq / (double)n + eps)", "sqrt(ssq / (double)(n + 1) + eps)"),
+    "per_head_norm_in_3d": (
+        "qknr_oracle_rmsnorm(x, n, pass ? wk : wq, eps, y); /* across all H heads */",
+        "for (int32_t hh = 0; hh < H; ++hh) qknr_oracle_rmsnorm(x + (int64_t)hh * D, D, "
+        "(pass ? wk : wq) + (int64_t)hh * D, eps, y + (int64_t)hh * D);"),
+    "weight_reversed": ("y[c] = x[c] * r * (weight ? weight[c] : 1.0);",
+                        "y[c] = x[c] * r * (weight ? weight[n - 1 - c] : 1.0);"),
+    "frequency_exponent_halved": ("pow(base, -2.0 * i / C[a])", "pow(base, -1.0 * i / C[a])"),
+    "frequency_over_head_dim": ("pow(base, -2.0 * i / C[a])",
+                                "pow(base, -2.0 * i / (C[0] + C[1] + C[2]))"),
+    "axis_order_swapped": ("int64_t pos[3] = {f, h, w};", "int64_t pos[3] = {w, h, f};"),
+    "position_height_index": ("*h = (s / ppw) % pph;", "*h = (s / pph) % ppw;"),
+    "pos_offset_ignored": ("int64_t s = (t + pos_offset) % P;", "int64_t s = t % P;"),
+    "half_split_mirrored": ("pb[j] = interleaved ? 2 * j + 1 : j + rotary_dim / 2;",
+                            "pb[j] = interleaved ? 2 * j + 1 : rotary_dim - 1 - j;"),
+    "table_sin_column": ("s[j] = row[R / 2 + j];\n            } else {",
+                         "s[j] = row[2 * j + 1];\n            } else {"),
+    "bf16_ties_away": ("return fl + fmod(fl, 2.0);", "return fl + 1.0;"),
+    "bf16_no_subnormal_floor": ("if (e < -126) e = -126;", ""),
+    "e4m3_no_saturation": ("if (v > 448.0) v = 448.0;", ""),
+    "e4m3_subnormal_floor": ("if (e < -6) e = -6;", "if (e < -7) e = -7;"),
+    "v_uses_qk_scale": ("qknr_oracle_e4m3_from_double(ev[i] * v_scale)",
+                        "qknr_oracle_e4m3_from_double(ev[i] * q_scale)"),
+    "norm_flag_ignored": ("if (is_qk_norm)\n            qknr_oracle_rmsnorm",
+                          "if (1)\n            qknr_oracle_rmsnorm"),
+}
+
+# cheap pins first, so a planted mistake is usually caught within a second
+ORDER = sorted(P.ALL_PINS, key=lambda f: ("rounding_vs_torch" in f.__name__, f.__name__))
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-o", str(so),
+                    str(path), "-lm"], check=True)
+    O.use_library(str(so))
+    try:
+        caught = []
+        for pin in ORDER:
+            try:
+                pin()
+            except (AssertionError, ValueError):
+                caught.append(pin.__name__)
+                break
+        assert caught, f"no pin caught the planted mistake {name}"
+    finally:
+        O.use_library()
