@@ -1,0 +1,359 @@
+#!/usr/bin/env python
+"""Benchmark of the fused Q/K RMSNorm + RoPE hot path on B200.
+
+One step = one call of the 3D entry point (across-heads RMSNorm + 3D RoPE +
+V copy) over one batch of the video-DiT workload: packed bf16 QKV
+[1, 15360, (32+32+32)*128], patch grid 16x30x32, channels 16/56/56,
+interleaved pairs, bf16 out. Inputs are seeded synthetic tensors resident in
+HBM; the 377 MB input (plus 377 MB output) exceeds the 126 MB L2, so no flush
+is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle, bounded sample
+
+Under torchrun each rank processes its own batch (weak scaling, no
+collective on the data path); rank 0 prints one JSON line.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "tokens/s and achieved HBM GB/s (% of B200 peak) for fused QK-norm+RoPE, 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu
+# capture summarised in profiles/, valid only for the kernel sources whose
+# hash is stored beside it (null otherwise).
+TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "qk_rmsnorm_rope_qknr_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# --------------------------------------------------------------- oracle arm --
+def oracle_sample(w, inp_cpu, budget_s: float, chunk: int = 256):
+    """Time the fp64 oracle on consecutive token chunks of the workload until
+    budget_s of CPU work is spent; returns (tokens, seconds, threads)."""
+    import oracle as O
+    from tests._util import t2u16
+
+    qkv = inp_cpu["qkv"].reshape(-1, inp_cpu["qkv"].shape[-1])
+    qw, kw = t2u16(inp_cpu["q_weight"]), t2u16(inp_cpu["k_weight"])
+    p = w.params()
+    done, spent = 0, 0.0
+    T = qkv.shape[0]
+    while spent < budget_s and done < T:
+        n = min(chunk, T - done)
+        bits = t2u16(qkv[done:done + n])
+        t0 = time.perf_counter()
+        O.rope_3d(bits, qw, kw, pos_offset=done, **p)
+        spent += time.perf_counter() - t0
+        done += n
+    return done, spent, O.threads()
+
+
+def run_reference(args, w):
+    """--impl reference: the oracle as it stands, on the host cores."""
+    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = W.make_inputs(w, device="cpu")
+    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, min(per_step, 2.0))
+    toks, secs = 0, 0.0
+    threads = 1
+    for _ in range(args.steps):
+        n, s, threads = oracle_sample(w, inp, per_step)
+        toks += n
+        secs += s
+    value = toks / secs
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "tokens": w.tokens, "sample": "leading tokens"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{toks // max(1, args.steps)} leading tokens per step of "
+                                   f"{w.name}"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm --
+def run_gpu(args, w):
+    import torch
+
+    import qk_rmsnorm_rope_qknr_b200 as Q
+    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    Q.lib()
+
+    # Each rank: its own batch of the workload (seed offset by rank).
+    inp = W.make_inputs(w, device=dev, seed=w.seed + rank)
+    T = w.tokens
+    odt = torch.float8_e4m3fn if w.output_fp8 else torch.bfloat16
+    outs = [torch.empty(T, h, w.head_dim, dtype=odt, device=dev) for h in (w.hq, w.hk, w.hv)]
+    p = w.params()
+    qkv, qw, kw = inp["qkv"], inp["q_weight"], inp["k_weight"]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        Q.qknr_rope_3d(qkv, qw, kw, *outs, stream=stream, **p)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # Timed region: K steps, per-launch events on the launching stream.
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    if pg:
+        t = torch.tensor([total_ms, statistics.mean(launch_ms)], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms, avg_launch_ms = t.tolist()
+    else:
+        avg_launch_ms = statistics.mean(launch_ms)
+    ms_per_step = total_ms / args.steps
+    tokens_per_s = world * T / (ms_per_step / 1e3)
+
+    alg_bytes = W.algorithmic_bytes(w)
+    peak, peak_kind = measured_peaks()
+    achieved = alg_bytes / (avg_launch_ms / 1e3) / 1e9
+    tr = TRAFFIC.get(w.name)
+    traffic = tr[0] if tr and tr[1] == kernel_source_hash() else None
+
+    # End to end through the C ABI with host buffers: copy the step's input
+    # from pinned host memory, run, copy the outputs back, every step.
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(args, w, qkv, qw, kw, outs, p, stream, dev, world, pg)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = {"qkv": qkv[:, :min(T, 4096)].cpu() if qkv.dim() == 3 else qkv[:4096].cpu(),
+                   "q_weight": qw.cpu(), "k_weight": kw.cpu()}
+        n, s, threads = oracle_sample(w, inp_cpu, args.cpu_seconds)
+        cpu = {"value": n / s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"first {n} tokens of {w.name} ({s:.1f} s of fp64 oracle work)"}
+
+    if rank == 0:
+        clk = clocks.summary()
+        line = {
+            "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "tokens_per_gpu": T,
+                       "qkv_shape": list(qkv.shape), "grid": [w.ppf, w.pph, w.ppw],
+                       "channels": [w.cf, w.ch, w.cw], "heads": [w.hq, w.hk, w.hv],
+                       "head_dim": w.head_dim, "interleave": w.interleave,
+                       "is_qk_norm": w.is_qk_norm, "output_fp8": w.output_fp8,
+                       "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": f"no flush: inputs {qkv.numel() * 2 / 1e6:.0f} MB > 126 MB L2"},
+            "hbm_gbs": achieved, "hbm_pct_of_peak": 100.0 * achieved / peak,
+            "kernel_us": avg_launch_ms * 1e3,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": alg_bytes},
+            "cpu_baseline": cpu, "clocks": clk, "e2e": e2e, "gpu_launches": args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def measure_e2e(args, w, qkv, qw, kw, outs, p, stream, dev, world, pg):
+    import torch
+
+    import qk_rmsnorm_rope_qknr_b200 as Q
+
+    h_in = torch.empty(qkv.shape, dtype=qkv.dtype).pin_memory()
+    h_in.copy_(qkv.cpu())
+    h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    d_in = torch.empty_like(qkv)
+    steps = max(3, min(args.e2e_steps, args.steps))
+
+    def step():
+        d_in.copy_(h_in, non_blocking=True)
+        Q.qknr_rope_3d(d_in, qw, kw, *outs, stream=stream, **p)
+        for h, o in zip(h_out, outs):
+            h.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = t.item()
+    return {"value": world * w.tokens / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": qkv.numel() * qkv.element_size(),
+            "d2h_bytes_per_step": sum(o.numel() * o.element_size() for o in outs),
+            "steps": steps, "mode": "pinned host -> device copy, kernel, device -> pinned host copy"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="qknr", choices=["qknr", "reference"])
+    ap.add_argument("--workload", default="video3d")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+
+    w = W.WORKLOADS[args.workload]
+    if w.form != "3d":
+        ap.error("the bench times the 3D entry point; pick a 3D workload")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

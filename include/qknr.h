@@ -1,0 +1,167 @@
+/*
+ * qknr.h -- C ABI of libqknr.so: fused Q/K RMSNorm + rotary position embedding
+ * (with V copy and optional FP8 E4M3 output) for B200 (sm_100a).
+ *
+ * Two entry points, one per contract that the source pages state:
+ *
+ *   qknr_rope_table  -- "vllm_omni.diffusion.layers.fused_qk_norm_rope"
+ *                       (vLLM-Omni API docs): module description (public
+ *                       contract bullets) and fused_qk_norm_rope(...).
+ *   qknr_rope_3d     -- "flashinfer.norm.fused_qk_rmsnorm_rope" (FlashInfer
+ *                       API docs): summary, Parameters, Returns.
+ *
+ * Common rules
+ *   - Pointers are plain addresses that the current CUDA device can read or
+ *     write: device memory of that device, managed memory, or page-locked host
+ *     memory registered with CUDA (then the kernel reads and writes it across
+ *     the bus). Anything else is rejected with QKNR_ERR_POINTER before any
+ *     launch.
+ *   - The caller owns every buffer (destination-passing); the library never
+ *     allocates, frees or synchronises. Work is queued on `cuda_stream`
+ *     (a cudaStream_t; NULL = the legacy default stream) and the call returns
+ *     at once. A fault inside the kernel surfaces at the caller's next
+ *     synchronisation on that stream.
+ *   - Every entry point returns a qknr_status. Nothing is thrown across the
+ *     ABI and nothing is written when the status is not QKNR_OK.
+ *     qknr_last_error_detail() names the argument that failed, for this thread.
+ *   - num_tokens == 0 is a valid no-op (QKNR_OK, no launch).
+ *   - bf16 is IEEE-style bfloat16, E4M3 is the OCP FP8 E4M3FN format (bias 7,
+ *     largest finite 448, no infinities); conversions to bf16 round to nearest
+ *     even, conversions to E4M3 round to nearest even and saturate to +-448.
+ *   - All arithmetic is fp32; each output element is rounded once.
+ *
+ * Thread safety: calls may come from several host threads and streams at once.
+ */
+#ifndef QKNR_H_
+#define QKNR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QKNR_ABI_VERSION 1
+
+typedef enum {
+    QKNR_OK = 0,
+    QKNR_ERR_NULL = 1,        /* a pointer that the call needs is NULL               */
+    QKNR_ERR_SHAPE = 2,       /* sizes or parameters break the contract              */
+    QKNR_ERR_UNSUPPORTED = 3, /* allowed by the pages but not built (YARN, factor!=1) */
+    QKNR_ERR_ALIGN = 4,       /* a pointer or row stride misses the 16-byte rule     */
+    QKNR_ERR_ALIAS = 5,       /* an output overlaps an input it may not overlap      */
+    QKNR_ERR_POINTER = 6,     /* a pointer the current device cannot access          */
+    QKNR_ERR_CUDA = 7         /* the CUDA runtime refused the launch                 */
+} qknr_status;
+
+typedef enum {
+    QKNR_DT_BF16 = 0,
+    QKNR_DT_F32 = 1,
+    QKNR_DT_E4M3 = 2
+} qknr_dtype;
+
+/*
+ * Table-driven per-head Q/K RMSNorm + RoPE
+ * ("vllm_omni.diffusion.layers.fused_qk_norm_rope": contract bullets and
+ * fused_qk_norm_rope).
+ *
+ * For every token t and every head h of q (and of k, with k's weight):
+ *   y[d]   = x[d] / sqrt(mean_d'(x[d']^2) + eps) * weight[d]      (d < head_dim)
+ *   pair j = (2j, 2j+1) if interleaved, else (j, j + rotary_dim/2)  (j < rotary_dim/2)
+ *   c = rope_table[t][j], s = rope_table[t][rotary_dim/2 + j]
+ *   out[a] = y[a] c - y[b] s,  out[b] = y[b] c + y[a] s;  channels >= rotary_dim: out = y
+ *
+ * q, k          bf16 [num_tokens, heads, head_dim]: heads dense inside a token,
+ *               tokens q_token_stride / k_token_stride ELEMENTS apart
+ *               (0 = dense, heads*head_dim). Read only.
+ * q_out, k_out  bf16, same shape, their own token strides (0 = dense). May
+ *               equal q / k exactly (in place, then with the same stride);
+ *               any other overlap with an input is QKNR_ERR_ALIAS.
+ * q_weight, k_weight  bf16 [head_dim].
+ * rope_table    [num_tokens, rotary_dim], dense, QKNR_DT_F32 or QKNR_DT_BF16:
+ *               columns [0, rotary_dim/2) hold cos(theta_j), the rest sin(theta_j).
+ * head_dim      1..256; rotary_dim 0 means head_dim, else even and <= head_dim.
+ * heads_q, heads_k >= 0 (a tensor with 0 heads is neither read nor written and
+ *               its pointers may be NULL).
+ * eps           >= 0.
+ * Fast path: every pointer and token stride 16-byte aligned, head_dim a
+ * multiple of 16 and rotary_dim a multiple of 16 (half-split) or 8
+ * (interleaved). Other valid inputs run a general kernel (2-byte alignment).
+ */
+int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
+                    const void* q_weight, const void* k_weight, const void* rope_table,
+                    int32_t table_dtype, int64_t num_tokens, int32_t heads_q, int32_t heads_k,
+                    int32_t head_dim, int32_t rotary_dim, int64_t q_token_stride,
+                    int64_t k_token_stride, int64_t q_out_token_stride,
+                    int64_t k_out_token_stride, float eps, int32_t interleaved,
+                    void* cuda_stream);
+
+/*
+ * Packed-QKV across-heads RMSNorm + 3D RoPE + V copy (+ FP8 E4M3 output)
+ * ("flashinfer.norm.fused_qk_rmsnorm_rope": summary, Parameters, Returns).
+ *
+ * Input row of token t: qkv[t] = [Q heads | K heads | V heads], each head
+ * head_dim bf16 channels, (Hq + Hk + Hv) * head_dim per row, rows dense.
+ *   Q: r = 1 / sqrt(sum over all Hq*head_dim channels of x^2 / (Hq*head_dim) + eps)
+ *      y[c] = x[c] * r * q_weight[c]  (c < Hq*head_dim); K likewise over Hk*head_dim.
+ *      With is_qk_norm == 0, y = x (weights and eps unused, may be NULL).
+ *   Patch of token t: s = (t + pos_offset) mod (ppf*pph*ppw), row-major:
+ *      f = s / (pph*ppw), h = (s / ppw) mod pph, w = s mod ppw.
+ *   Pair slot j < head_dim/2 belongs to the frame axis for j < Cf/2, the height
+ *      axis for the next Ch/2 slots, the width axis for the rest; with i the
+ *      slot's index inside its axis group and C that group's channel count,
+ *      theta_j = pos_axis * base^(-2i/C).
+ *   Each Q and K head rotates its pairs: (2j, 2j+1) if interleave, else
+ *      (j, j + head_dim/2) (NeoX), by theta_j as in qknr_rope_table.
+ *   Outputs: q_out [T, Hq, head_dim], k_out [T, Hk, head_dim], v_out
+ *      [T, Hv, head_dim], dense. bf16; or with output_fp8, E4M3 of
+ *      q*output_quant_scale, k*output_quant_scale and v*v_quant_scale.
+ *      Without output_fp8, v_out is a bit copy of V.
+ *
+ * Validation: tokens divisible by ppf*pph*ppw (pos_offset == 0) or any count
+ * (pos_offset > 0, a shard of a longer sequence); channel counts even,
+ * non-negative, summing to head_dim; head_dim in {64, 128, 256}; heads >= 0 and
+ * Hq + Hk + Hv >= 1; factor == 1 and attention_factor == 1 (YARN is not built:
+ * QKNR_ERR_UNSUPPORTED); qkv and all outputs 16-byte aligned; no output
+ * overlapping qkv or another output.
+ */
+typedef struct {
+    size_t struct_size; /* sizeof(qknr_rope_3d_params); guards against ABI drift */
+    const void* qkv;    /* bf16 [num_tokens, (Hq+Hk+Hv)*head_dim]               */
+    const void* q_weight; /* bf16 [Hq*head_dim]                                   */
+    const void* k_weight; /* bf16 [Hk*head_dim]                                   */
+    void* q_out;        /* bf16 or E4M3 [num_tokens, Hq, head_dim]               */
+    void* k_out;        /* bf16 or E4M3 [num_tokens, Hk, head_dim]               */
+    void* v_out;        /* bf16 or E4M3 [num_tokens, Hv, head_dim]               */
+    int64_t num_tokens;
+    int64_t pos_offset; /* position of the first token in the patch sequence     */
+    int32_t ppf, pph, ppw;
+    int32_t num_frame_channels, num_height_channels, num_width_channels;
+    int32_t num_heads_q, num_heads_k, num_heads_v, head_dim;
+    float eps;
+    float base;
+    int32_t interleave;  /* 1 = adjacent pairs (non-NeoX), 0 = NeoX half split   */
+    float factor, low, high, attention_factor; /* YARN: only factor == 1 accepted */
+    int32_t is_qk_norm;
+    int32_t output_fp8;
+    float output_quant_scale;
+    float v_quant_scale;
+} qknr_rope_3d_params;
+
+int qknr_rope_3d(const qknr_rope_3d_params* params, void* cuda_stream);
+
+/* Static text for a status code. */
+const char* qknr_status_string(int status);
+
+/* Text on the last failing call of this host thread ("" if none). */
+const char* qknr_last_error_detail(void);
+
+/* QKNR_ABI_VERSION of the built library. */
+int qknr_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKNR_H_ */

@@ -1,0 +1,268 @@
+"""qk_rmsnorm_rope_qknr_b200 -- fused Q/K RMSNorm + RoPE (+ V copy, FP8 out) for B200.
+
+A thin ctypes binding over libqknr.so (C ABI in include/qknr.h). Every step of
+the transform runs in the library's CUDA kernels; this module only turns torch
+tensors into pointers, sizes and a stream. There is no CPU or eager fallback:
+if libqknr.so is missing or cannot load, every call raises.
+
+Low-level names mirror the C entry points:
+  qknr_rope_table(...)  table-driven per-head form
+  qknr_rope_3d(...)     packed-QKV across-heads 3D form
+Page-shaped wrappers allocate missing outputs and return them:
+  fused_qk_norm_rope(q, k, q_weight, k_weight, rope_table, eps, *, head_dim=None,
+                     rotary_dim=None, interleaved=False) -> (q, k)
+      ("vllm_omni.diffusion.layers.fused_qk_norm_rope", fused_qk_norm_rope)
+  fused_qk_rmsnorm_rope(qkv, q_weight, k_weight, *, ppf, pph, ppw, ...,
+                        q_out=None, k_out=None, v_out=None) -> (q, k, v)
+      ("flashinfer.norm.fused_qk_rmsnorm_rope", Parameters / Returns)
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqknr.so")
+
+QKNR_OK, QKNR_ERR_NULL, QKNR_ERR_SHAPE, QKNR_ERR_UNSUPPORTED = 0, 1, 2, 3
+QKNR_ERR_ALIGN, QKNR_ERR_ALIAS, QKNR_ERR_POINTER, QKNR_ERR_CUDA = 4, 5, 6, 7
+QKNR_DT_BF16, QKNR_DT_F32, QKNR_DT_E4M3 = 0, 1, 2
+
+EXPORTS = ("qknr_rope_table", "qknr_rope_3d", "qknr_status_string", "qknr_last_error_detail",
+           "qknr_abi_version")
+
+
+class QknrError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"qknr status {status}: {detail}")
+        self.status = status
+
+
+class QknrValueError(QknrError, ValueError):
+    """Shape, parameter, alignment or aliasing errors (the pages raise ValueError)."""
+
+
+class Rope3DParams(C.Structure):
+    _fields_ = [("struct_size", C.c_size_t), ("qkv", C.c_void_p), ("q_weight", C.c_void_p),
+                ("k_weight", C.c_void_p), ("q_out", C.c_void_p), ("k_out", C.c_void_p),
+                ("v_out", C.c_void_p), ("num_tokens", C.c_int64), ("pos_offset", C.c_int64),
+                ("ppf", C.c_int32), ("pph", C.c_int32), ("ppw", C.c_int32),
+                ("num_frame_channels", C.c_int32), ("num_height_channels", C.c_int32),
+                ("num_width_channels", C.c_int32), ("num_heads_q", C.c_int32),
+                ("num_heads_k", C.c_int32), ("num_heads_v", C.c_int32), ("head_dim", C.c_int32),
+                ("eps", C.c_float), ("base", C.c_float), ("interleave", C.c_int32),
+                ("factor", C.c_float), ("low", C.c_float), ("high", C.c_float),
+                ("attention_factor", C.c_float), ("is_qk_norm", C.c_int32),
+                ("output_fp8", C.c_int32), ("output_quant_scale", C.c_float),
+                ("v_quant_scale", C.c_float)]
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """The loaded libqknr.so; raises if it is missing (build it with build())."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libqknr.so not built at {LIB_PATH}; run "
+                              "qk_rmsnorm_rope_qknr_b200.build.build()")
+        L = C.CDLL(LIB_PATH)
+        vp, i32, i64 = C.c_void_p, C.c_int32, C.c_int64
+        L.qknr_rope_table.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                      i64, i64, i64, i64, C.c_float, i32, vp]
+        L.qknr_rope_table.restype = C.c_int
+        L.qknr_rope_3d.argtypes = [C.POINTER(Rope3DParams), vp]
+        L.qknr_rope_3d.restype = C.c_int
+        L.qknr_status_string.argtypes = [C.c_int]
+        L.qknr_status_string.restype = C.c_char_p
+        L.qknr_last_error_detail.restype = C.c_char_p
+        L.qknr_abi_version.restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def build(force: bool = False) -> str:
+    """Compile libqknr.so in-tree (nvcc, sm_100a) if it is missing or stale."""
+    import importlib
+
+    return importlib.import_module(__name__ + ".build").build(force=force)
+
+
+def _check(status: int) -> None:
+    if status == QKNR_OK:
+        return
+    L = lib()
+    detail = (L.qknr_last_error_detail() or b"").decode() or L.qknr_status_string(status).decode()
+    if status in (QKNR_ERR_NULL, QKNR_ERR_SHAPE, QKNR_ERR_UNSUPPORTED, QKNR_ERR_ALIGN,
+                  QKNR_ERR_ALIAS, QKNR_ERR_POINTER):
+        raise QknrValueError(status, detail)
+    raise QknrError(status, detail)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream, *tensors) -> Optional[int]:
+    if stream is not None:
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    for t in tensors:
+        if t is not None and t.is_cuda:
+            return torch.cuda.current_stream(t.device).cuda_stream
+    return None
+
+
+def _table_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return QKNR_DT_F32
+    if t.dtype == torch.bfloat16:
+        return QKNR_DT_BF16
+    raise QknrValueError(QKNR_ERR_SHAPE, f"rope_table dtype {t.dtype} is not float32/bfloat16")
+
+
+def _token_stride(t: torch.Tensor, name: str, heads: int, head_dim: int) -> int:
+    if t.dim() != 3 or t.shape[1] != heads or t.shape[2] != head_dim:
+        raise QknrValueError(QKNR_ERR_SHAPE, f"{name} must be [tokens, {heads}, {head_dim}]")
+    if t.dtype != torch.bfloat16:
+        raise QknrValueError(QKNR_ERR_SHAPE, f"{name} must be bfloat16")
+    if t.shape[0] > 0 and heads > 0 and (t.stride(2) != 1 or (heads > 1 and
+                                                             t.stride(1) != head_dim)):
+        raise QknrValueError(QKNR_ERR_SHAPE, f"{name}: heads must be dense inside a token")
+    return t.stride(0)
+
+
+# --------------------------------------------------------------- C-ABI names --
+def qknr_rope_table(q, k, q_out, k_out, q_weight, k_weight, rope_table, *, eps: float,
+                    rotary_dim: int = 0, interleaved: bool = False, stream=None) -> None:
+    """Table form through the C ABI (destination passing; see include/qknr.h).
+    q/k/q_out/k_out are bf16 [tokens, heads, head_dim] with dense heads."""
+    T, Hq, D = q.shape
+    Hk = k.shape[1]
+    qs = _token_stride(q, "q", Hq, D)
+    ks = _token_stride(k, "k", Hk, D)
+    qos = _token_stride(q_out, "q_out", Hq, D)
+    kos = _token_stride(k_out, "k_out", Hk, D)
+    if k.shape[0] != T or q_out.shape[0] != T or k_out.shape[0] != T:
+        raise QknrValueError(QKNR_ERR_SHAPE, "q, k and outputs differ in token count")
+    R = rotary_dim or D
+    if rope_table.dim() != 2 or tuple(rope_table.shape) != (T, R) or not rope_table.is_contiguous():
+        raise QknrValueError(QKNR_ERR_SHAPE, f"rope_table must be a dense [{T}, {R}] tensor")
+    for n, w in (("q_weight", q_weight), ("k_weight", k_weight)):
+        if w.dtype != torch.bfloat16 or w.numel() != D or not w.is_contiguous():
+            raise QknrValueError(QKNR_ERR_SHAPE, f"{n} must be a dense bf16 [{D}] tensor")
+    st = _stream(stream, q, k, q_out, k_out)
+    _check(lib().qknr_rope_table(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _ptr(q_weight),
+                                 _ptr(k_weight), _ptr(rope_table), _table_dtype(rope_table), T, Hq,
+                                 Hk, D, R, qs, ks, qos, kos, float(eps), int(bool(interleaved)),
+                                 st))
+
+
+def make_3d_params(qkv, q_weight, k_weight, q_out, k_out, v_out, *, ppf, pph, ppw,
+                   num_frame_channels, num_height_channels, num_width_channels, num_heads_q,
+                   num_heads_k, num_heads_v, head_dim, eps=1e-6, base=10000.0, interleave=True,
+                   factor=1.0, low=0.0, high=0.0, attention_factor=1.0, is_qk_norm=True,
+                   output_fp8=False, output_quant_scale=1.0, v_quant_scale=1.0, pos_offset=0,
+                   num_tokens=None) -> Rope3DParams:
+    row = (num_heads_q + num_heads_k + num_heads_v) * head_dim
+    if num_tokens is None:
+        if qkv.dtype != torch.bfloat16 or qkv.shape[-1] != row or not qkv.is_contiguous():
+            raise QknrValueError(QKNR_ERR_SHAPE,
+                                 f"qkv must be a contiguous bf16 tensor [..., {row}]")
+        num_tokens = qkv.numel() // row
+    p = Rope3DParams()
+    p.struct_size = C.sizeof(Rope3DParams)
+    p.qkv, p.q_weight, p.k_weight = _ptr(qkv), _ptr(q_weight), _ptr(k_weight)
+    p.q_out, p.k_out, p.v_out = _ptr(q_out), _ptr(k_out), _ptr(v_out)
+    p.num_tokens, p.pos_offset = int(num_tokens), int(pos_offset)
+    p.ppf, p.pph, p.ppw = ppf, pph, ppw
+    p.num_frame_channels, p.num_height_channels = num_frame_channels, num_height_channels
+    p.num_width_channels = num_width_channels
+    p.num_heads_q, p.num_heads_k, p.num_heads_v = num_heads_q, num_heads_k, num_heads_v
+    p.head_dim = head_dim
+    p.eps, p.base, p.interleave = eps, base, int(bool(interleave))
+    p.factor, p.low, p.high, p.attention_factor = factor, low, high, attention_factor
+    p.is_qk_norm, p.output_fp8 = int(bool(is_qk_norm)), int(bool(output_fp8))
+    p.output_quant_scale, p.v_quant_scale = output_quant_scale, v_quant_scale
+    return p
+
+
+def qknr_rope_3d(qkv, q_weight, k_weight, q_out, k_out, v_out, *, stream=None, **params) -> None:
+    """3D form through the C ABI (destination passing; see include/qknr.h).
+    params are the page's keyword arguments plus pos_offset."""
+    p = make_3d_params(qkv, q_weight, k_weight, q_out, k_out, v_out, **params)
+    odt = torch.float8_e4m3fn if params.get("output_fp8") else torch.bfloat16
+    for n, o, h in (("q_out", q_out, p.num_heads_q), ("k_out", k_out, p.num_heads_k),
+                    ("v_out", v_out, p.num_heads_v)):
+        if h and o is not None:
+            if o.dtype not in (odt, torch.uint8) or not o.is_contiguous() or \
+                    o.numel() != p.num_tokens * h * p.head_dim:
+                raise QknrValueError(QKNR_ERR_SHAPE,
+                                     f"{n} must be a dense {odt} tensor of {p.num_tokens}x{h}x"
+                                     f"{p.head_dim} elements")
+    for n, w, h in (("q_weight", q_weight, p.num_heads_q), ("k_weight", k_weight, p.num_heads_k)):
+        if p.is_qk_norm and h and w is not None and (w.dtype != torch.bfloat16 or
+                                                      w.numel() != h * p.head_dim):
+            raise QknrValueError(QKNR_ERR_SHAPE, f"{n} must be bf16 [{h * p.head_dim}]")
+    st = _stream(stream, qkv, q_out)
+    _check(lib().qknr_rope_3d(C.byref(p), st))
+
+
+# ------------------------------------------------------- page-shaped wrappers --
+def fused_qk_norm_rope(q: torch.Tensor, k: torch.Tensor, q_weight: torch.Tensor,
+                       k_weight: torch.Tensor, rope_table: torch.Tensor, eps: float, *,
+                       head_dim: Optional[int] = None, rotary_dim: Optional[int] = None,
+                       interleaved: bool = False, q_out: Optional[torch.Tensor] = None,
+                       k_out: Optional[torch.Tensor] = None, stream=None
+                       ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Q/K RMSNorm + packed RoPE, table form. Returns new (q, k) unless outputs
+    are given (pass q_out=q, k_out=k to work in place)."""
+    D = head_dim or q.shape[-1]
+    if q.shape[-1] != D or k.shape[-1] != D:
+        raise QknrValueError(QKNR_ERR_SHAPE, f"last dim of q/k must be head_dim={D}")
+    if q_out is None:
+        q_out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
+    if k_out is None:
+        k_out = torch.empty(k.shape, dtype=k.dtype, device=k.device)
+    qknr_rope_table(q, k, q_out, k_out, q_weight, k_weight, rope_table, eps=eps,
+                    rotary_dim=rotary_dim or D, interleaved=interleaved, stream=stream)
+    return q_out, k_out
+
+
+def fused_qk_rmsnorm_rope(qkv: torch.Tensor, q_weight: torch.Tensor, k_weight: torch.Tensor, *,
+                          ppf: int, pph: int, ppw: int, num_frame_channels: int,
+                          num_height_channels: int, num_width_channels: int, num_heads_q: int,
+                          num_heads_k: int, num_heads_v: int, head_dim: int, eps: float = 1e-6,
+                          base: float = 10000.0, interleave: bool = True, factor: float = 1.0,
+                          low: float = 0.0, high: float = 0.0, attention_factor: float = 1.0,
+                          is_qk_norm: bool = True, output_fp8: bool = False,
+                          output_quant_scale: float = 1.0, v_quant_scale: float = 1.0,
+                          q_out: Optional[torch.Tensor] = None,
+                          k_out: Optional[torch.Tensor] = None,
+                          v_out: Optional[torch.Tensor] = None, pos_offset: int = 0,
+                          stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Across-heads Q/K RMSNorm + 3D RoPE + V copy (+ FP8). Outputs are
+    [B, S, H, D] for a 3D qkv and [T, H, D] for a 2D one."""
+    lead = tuple(qkv.shape[:-1])
+    odt = torch.float8_e4m3fn if output_fp8 else torch.bfloat16
+    outs = []
+    for o, h in ((q_out, num_heads_q), (k_out, num_heads_k), (v_out, num_heads_v)):
+        outs.append(o if o is not None else torch.empty(lead + (h, head_dim), dtype=odt,
+                                                        device=qkv.device))
+    qknr_rope_3d(qkv, q_weight, k_weight, *outs, stream=stream, ppf=ppf, pph=pph, ppw=ppw,
+                 num_frame_channels=num_frame_channels, num_height_channels=num_height_channels,
+                 num_width_channels=num_width_channels, num_heads_q=num_heads_q,
+                 num_heads_k=num_heads_k, num_heads_v=num_heads_v, head_dim=head_dim, eps=eps,
+                 base=base, interleave=interleave, factor=factor, low=low, high=high,
+                 attention_factor=attention_factor, is_qk_norm=is_qk_norm,
+                 output_fp8=output_fp8, output_quant_scale=output_quant_scale,
+                 v_quant_scale=v_quant_scale, pos_offset=pos_offset)
+    return tuple(outs)
+
+
+__all__ = ["qknr_rope_table", "qknr_rope_3d", "fused_qk_norm_rope", "fused_qk_rmsnorm_rope",
+           "QknrError", "QknrValueError", "lib", "build", "make_3d_params", "Rope3DParams",
+           "EXPORTS", "LIB_PATH"]

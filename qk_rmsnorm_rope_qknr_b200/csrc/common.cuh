@@ -1,0 +1,116 @@
+// Device helpers shared by the qknr kernels: 128-bit streaming loads and
+// stores, bf16 / E4M3 packing, warp reductions, and the fixed-point angle
+// that keeps cos/sin accurate at any integer position.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qknr {
+
+// Read-only streaming load of 16 bytes: the input is read exactly once, so it
+// bypasses L1 (the data must not be written by the same kernel).
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Streaming load that stays correct when the same kernel later overwrites the
+// address (in-place use): a plain global load marked evict-first.
+__device__ __forceinline__ uint4 ld_cs_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_v2(void* p, uint2 v) {
+    asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+
+// bf16 pair packed in a 32-bit word: low half is the lower-addressed element.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+    f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+    f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
+// Round to nearest even, two floats into one bf16x2 word.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(const float (&f)[8]) {
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                      pack_bf16x2(f[6], f[7]));
+}
+
+// E4M3 (OCP E4M3FN), round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+    uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+    uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+    return lo | (hi << 16);
+}
+
+__device__ __forceinline__ uint2 pack8_e4m3(const float (&f)[8], float scale) {
+    return make_uint2(pack_e4m3x4(f[0] * scale, f[1] * scale, f[2] * scale, f[3] * scale),
+                      pack_e4m3x4(f[4] * scale, f[5] * scale, f[6] * scale, f[7] * scale));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Sum over aligned groups of G lanes (G a power of two <= 32).
+template <int G>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Angle of integer position `pos` for a frequency stored as a 64-bit binary
+// fraction of a turn (turns_q64 = round(omega / (2 pi) * 2^64)). The product
+// wraps modulo 2^64, i.e. modulo whole turns, so no precision is lost to the
+// size of the angle; the top 32 bits give the signed fraction of a turn in
+// [-1/2, 1/2), and sincospif turns it into cos/sin of 2 pi times that fraction.
+__device__ __forceinline__ void turn_sincos(uint32_t pos, uint64_t turns_q64, float* s,
+                                            float* c) {
+    const uint64_t u = (uint64_t)pos * turns_q64;
+    const int32_t hi = (int32_t)(u >> 32);
+    const float half_turns = (float)hi * 4.656612873077392578125e-10f;  // 2^-31
+    sincospif(half_turns, s, c);
+}
+
+// omega / (2 pi) as a 64-bit binary fraction of a turn, omega = base^(-2i/C).
+// Positions are integers, so only the fractional part of the frequency in
+// turns matters (this also covers base < 1, where omega exceeds one turn).
+__device__ __forceinline__ uint64_t turns_q64(double base, int i, int C) {
+    const double two_pi = 6.283185307179586476925286766559;
+    const double two_64 = 18446744073709551616.0;
+    double g = pow(base, -2.0 * (double)i / (double)C) / two_pi;
+    g -= floor(g);
+    const double x = g * two_64;
+    return x >= two_64 ? 0ull : (uint64_t)x;
+}
+
+}  // namespace qknr

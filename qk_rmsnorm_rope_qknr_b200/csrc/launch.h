@@ -1,0 +1,61 @@
+// Internal interface between the C-ABI layer (qknr_abi.cu) and the kernel
+// launchers (rope3d.cu, rope_table.cu). Arguments are already validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qknr {
+
+struct Rope3DArgs {
+    const uint8_t* qkv;       // bf16 [T, (hq+hk+hv)*D]
+    const uint8_t* q_weight;  // bf16 [hq*D] (unused without the norm)
+    const uint8_t* k_weight;  // bf16 [hk*D]
+    uint8_t* q_out;           // bf16 or E4M3 [T, hq, D]
+    uint8_t* k_out;
+    uint8_t* v_out;
+    int64_t num_tokens;
+    int64_t pos_offset;  // reduced modulo ppf*pph*ppw by the host
+    int32_t ppf, pph, ppw;
+    int32_t cf, ch, cw;
+    int32_t hq, hk, hv;
+    int32_t is_qk_norm;
+    int32_t use_table;      // cos/sin table in shared memory (set by the launcher)
+    int32_t table_entries;  // ppf*cf/2 + pph*ch/2 + ppw*cw/2
+    float eps;
+    float q_scale;
+    float v_scale;
+    double base;
+};
+
+struct RopeTableArgs {
+    const uint8_t* q;  // bf16 [T, hq, D], token stride q_stride elements
+    const uint8_t* k;
+    uint8_t* q_out;
+    uint8_t* k_out;
+    const uint8_t* q_weight;  // bf16 [D]
+    const uint8_t* k_weight;
+    const uint8_t* table;  // [T, rd] fp32 or bf16
+    int64_t num_tokens;
+    int64_t q_stride, k_stride, q_out_stride, k_out_stride;  // elements
+    int32_t hq, hk, head_dim, rotary_dim;
+    int32_t table_f32;
+    int32_t interleaved;
+    int32_t in_place;  // an output aliases its input
+    float eps;
+};
+
+// Launch description returned for the benchmark and tests.
+struct LaunchInfo {
+    int grid;
+    int block;
+    int smem;
+    int kernel_id;  // which kernel variant ran
+};
+
+cudaError_t launch_rope3d(const Rope3DArgs& a, int head_dim, int neox, int fp8,
+                          cudaStream_t stream, LaunchInfo* info);
+cudaError_t launch_rope_table(const RopeTableArgs& a, int fast_path, cudaStream_t stream,
+                              LaunchInfo* info);
+
+}  // namespace qknr

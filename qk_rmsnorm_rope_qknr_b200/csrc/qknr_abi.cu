@@ -1,0 +1,380 @@
+// C ABI of libqknr.so (declared in include/qknr.h): argument checks, pointer
+// classification, and dispatch to the kernel launchers. Nothing here
+// allocates, synchronises or touches the data.
+#include "qknr.h"
+
+#include "launch.h"
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+
+namespace {
+
+thread_local char g_detail[320] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int ok() {
+    g_detail[0] = '\0';
+    return QKNR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A pointer the current device can dereference: its own device memory,
+// managed memory, or host memory registered with CUDA (page-locked). On
+// success *dev_ptr is the address a kernel must use.
+int classify(const void* p, const char* name, int device, const void** dev_ptr) {
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(QKNR_ERR_POINTER, "%s: cudaPointerGetAttributes failed (%s)", name,
+                    cudaGetErrorString(e));
+    }
+    switch (attr.type) {
+        case cudaMemoryTypeDevice:
+            if (attr.device != device)
+                return fail(QKNR_ERR_POINTER, "%s: memory of device %d, current device is %d",
+                            name, attr.device, device);
+            *dev_ptr = p;
+            return QKNR_OK;
+        case cudaMemoryTypeManaged:
+            *dev_ptr = p;
+            return QKNR_OK;
+        case cudaMemoryTypeHost:
+            if (attr.devicePointer == nullptr)
+                return fail(QKNR_ERR_POINTER, "%s: host memory not mapped for the device", name);
+            *dev_ptr = attr.devicePointer;
+            return QKNR_OK;
+        default:
+            return fail(QKNR_ERR_POINTER,
+                        "%s: not memory the device can access (pageable host memory?)", name);
+    }
+}
+
+// A [rows, row_bytes] byte region whose rows start stride_bytes apart.
+struct Span {
+    const void* p;
+    uint64_t bytes;  // total extent, first byte to last
+    int64_t row_bytes = 0;
+    int64_t stride_bytes = 0;
+};
+
+// Bytes spanned by a [rows, cols] tensor of `elem` bytes with a row stride of
+// `stride` elements.
+uint64_t span_bytes(int64_t rows, int64_t cols, int64_t stride, int elem) {
+    if (rows <= 0 || cols <= 0) return 0;
+    return (uint64_t)((rows - 1) * stride + cols) * (uint64_t)elem;
+}
+
+Span rows_span(const void* p, int64_t rows, int64_t cols, int64_t stride, int elem) {
+    Span s{p, span_bytes(rows, cols, stride, elem)};
+    s.row_bytes = cols * elem;
+    s.stride_bytes = stride * elem;
+    return s;
+}
+
+// Whether two regions share a byte. Two row sets with the same row stride
+// whose rows interleave without touching (q and k heads inside one packed QKV
+// buffer) do not overlap; other cases fall back to comparing extents.
+bool overlap(Span a, Span b) {
+    if (a.p == nullptr || b.p == nullptr || a.bytes == 0 || b.bytes == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+    if (!(a0 < b0 + b.bytes && b0 < a0 + a.bytes)) return false;
+    const int64_t s = a.stride_bytes;
+    if (s > 0 && s == b.stride_bytes && a.row_bytes <= s && b.row_bytes <= s) {
+        const int64_t d = (int64_t)(b0 - a0);
+        const int64_t m = ((d % s) + s) % s;  // where b's rows start inside a's period
+        if (m >= a.row_bytes && m + b.row_bytes <= s) return false;
+    }
+    return true;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    cudaGetLastError();
+    return fail(QKNR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+namespace qknr {
+int rope3d_max_heads(int head_dim);
+}
+
+extern "C" {
+
+int qknr_abi_version(void) { return QKNR_ABI_VERSION; }
+
+const char* qknr_status_string(int status) {
+    switch (status) {
+        case QKNR_OK: return "ok";
+        case QKNR_ERR_NULL: return "a required pointer is NULL";
+        case QKNR_ERR_SHAPE: return "sizes or parameters break the contract";
+        case QKNR_ERR_UNSUPPORTED: return "not supported by this library";
+        case QKNR_ERR_ALIGN: return "a pointer or stride is not 16-byte aligned";
+        case QKNR_ERR_ALIAS: return "an output overlaps an input";
+        case QKNR_ERR_POINTER: return "a pointer the current device cannot access";
+        case QKNR_ERR_CUDA: return "CUDA runtime error";
+        default: return "unknown status";
+    }
+}
+
+const char* qknr_last_error_detail(void) { return g_detail; }
+
+int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
+                    const void* q_weight, const void* k_weight, const void* rope_table,
+                    int32_t table_dtype, int64_t num_tokens, int32_t heads_q, int32_t heads_k,
+                    int32_t head_dim, int32_t rotary_dim, int64_t q_token_stride,
+                    int64_t k_token_stride, int64_t q_out_token_stride,
+                    int64_t k_out_token_stride, float eps, int32_t interleaved,
+                    void* cuda_stream) {
+    // ---- shape checks (host only) ----
+    if (num_tokens < 0) return fail(QKNR_ERR_SHAPE, "num_tokens < 0");
+    if (heads_q < 0 || heads_k < 0) return fail(QKNR_ERR_SHAPE, "negative head count");
+    if (head_dim < 1 || head_dim > 256)
+        return fail(QKNR_ERR_SHAPE, "head_dim %d outside 1..256", head_dim);
+    const int32_t R = rotary_dim == 0 ? head_dim : rotary_dim;
+    if (R < 2 || (R & 1) || R > head_dim)
+        return fail(QKNR_ERR_SHAPE, "rotary_dim %d must be even and <= head_dim %d", R,
+                    head_dim);
+    if (table_dtype != QKNR_DT_F32 && table_dtype != QKNR_DT_BF16)
+        return fail(QKNR_ERR_SHAPE, "rope_table dtype must be float32 or bfloat16");
+    if (!(eps >= 0.0f) || std::isinf(eps)) return fail(QKNR_ERR_SHAPE, "eps must be >= 0");
+    const int64_t qrow = (int64_t)heads_q * head_dim, krow = (int64_t)heads_k * head_dim;
+    const int64_t qs = q_token_stride ? q_token_stride : qrow;
+    const int64_t ks = k_token_stride ? k_token_stride : krow;
+    const int64_t qos = q_out_token_stride ? q_out_token_stride : qrow;
+    const int64_t kos = k_out_token_stride ? k_out_token_stride : krow;
+    if (qs < qrow || ks < krow || qos < qrow || kos < krow)
+        return fail(QKNR_ERR_SHAPE, "a token stride is smaller than heads*head_dim");
+    if (num_tokens == 0 || (heads_q == 0 && heads_k == 0)) return ok();
+
+    // ---- pointers ----
+    const bool has_q = heads_q > 0, has_k = heads_k > 0;
+    if (!rope_table) return fail(QKNR_ERR_NULL, "rope_table is NULL");
+    if (has_q && (!q || !q_out || !q_weight)) return fail(QKNR_ERR_NULL, "q, q_out or q_weight is NULL");
+    if (has_k && (!k || !k_out || !k_weight)) return fail(QKNR_ERR_NULL, "k, k_out or k_weight is NULL");
+    const int tb = table_dtype == QKNR_DT_F32 ? 4 : 2;
+    const Span sq = rows_span(q, num_tokens, qrow, qs, 2);
+    const Span sk = rows_span(k, num_tokens, krow, ks, 2);
+    const Span sqo = rows_span(q_out, num_tokens, qrow, qos, 2);
+    const Span sko = rows_span(k_out, num_tokens, krow, kos, 2);
+    const Span stab{rope_table, (uint64_t)num_tokens * R * tb};
+    const bool q_inplace = has_q && q_out == q;
+    const bool k_inplace = has_k && k_out == k;
+    if (q_inplace && qos != qs) return fail(QKNR_ERR_ALIAS, "in-place q needs the same stride");
+    if (k_inplace && kos != ks) return fail(QKNR_ERR_ALIAS, "in-place k needs the same stride");
+    if (has_q) {
+        if (!q_inplace && overlap(sqo, sq)) return fail(QKNR_ERR_ALIAS, "q_out overlaps q");
+        if (has_k && overlap(sqo, sk)) return fail(QKNR_ERR_ALIAS, "q_out overlaps k");
+        if (overlap(sqo, stab)) return fail(QKNR_ERR_ALIAS, "q_out overlaps rope_table");
+        if (overlap(sqo, Span{q_weight, (uint64_t)head_dim * 2}) ||
+            (has_k && overlap(sqo, Span{k_weight, (uint64_t)head_dim * 2})))
+            return fail(QKNR_ERR_ALIAS, "q_out overlaps a weight");
+    }
+    if (has_k) {
+        if (!k_inplace && overlap(sko, sk)) return fail(QKNR_ERR_ALIAS, "k_out overlaps k");
+        if (has_q && overlap(sko, sq)) return fail(QKNR_ERR_ALIAS, "k_out overlaps q");
+        if (has_q && overlap(sko, sqo)) return fail(QKNR_ERR_ALIAS, "k_out overlaps q_out");
+        if (overlap(sko, stab)) return fail(QKNR_ERR_ALIAS, "k_out overlaps rope_table");
+        if (overlap(sko, Span{k_weight, (uint64_t)head_dim * 2}) ||
+            (has_q && overlap(sko, Span{q_weight, (uint64_t)head_dim * 2})))
+            return fail(QKNR_ERR_ALIAS, "k_out overlaps a weight");
+    }
+    // 2-byte alignment is the minimum for bf16 / fp32 element access.
+    const uintptr_t any = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                          reinterpret_cast<uintptr_t>(q_out) | reinterpret_cast<uintptr_t>(k_out) |
+                          reinterpret_cast<uintptr_t>(q_weight) |
+                          reinterpret_cast<uintptr_t>(k_weight);
+    if (any & 1u) return fail(QKNR_ERR_ALIGN, "a bf16 pointer is not 2-byte aligned");
+    if (reinterpret_cast<uintptr_t>(rope_table) & (uintptr_t)(tb - 1))
+        return fail(QKNR_ERR_ALIGN, "rope_table is not aligned to its element size");
+
+    // ---- device access ----
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    qknr::RopeTableArgs a{};
+    const void* p = nullptr;
+    int rc;
+    if ((rc = classify(rope_table, "rope_table", dev, &p))) return rc;
+    a.table = static_cast<const uint8_t*>(p);
+    if (has_q) {
+        if ((rc = classify(q, "q", dev, &p))) return rc;
+        a.q = static_cast<const uint8_t*>(p);
+        if ((rc = classify(q_out, "q_out", dev, &p))) return rc;
+        a.q_out = static_cast<uint8_t*>(const_cast<void*>(p));
+        if ((rc = classify(q_weight, "q_weight", dev, &p))) return rc;
+        a.q_weight = static_cast<const uint8_t*>(p);
+    }
+    if (has_k) {
+        if ((rc = classify(k, "k", dev, &p))) return rc;
+        a.k = static_cast<const uint8_t*>(p);
+        if ((rc = classify(k_out, "k_out", dev, &p))) return rc;
+        a.k_out = static_cast<uint8_t*>(const_cast<void*>(p));
+        if ((rc = classify(k_weight, "k_weight", dev, &p))) return rc;
+        a.k_weight = static_cast<const uint8_t*>(p);
+    }
+    a.num_tokens = num_tokens;
+    a.q_stride = qs;
+    a.k_stride = ks;
+    a.q_out_stride = qos;
+    a.k_out_stride = kos;
+    a.hq = heads_q;
+    a.hk = heads_k;
+    a.head_dim = head_dim;
+    a.rotary_dim = R;
+    a.table_f32 = table_dtype == QKNR_DT_F32;
+    a.interleaved = interleaved ? 1 : 0;
+    a.in_place = q_inplace || k_inplace;
+    a.eps = eps;
+
+    // Fast kernel: 16-byte vectors everywhere and rotation pairs inside a lane.
+    const bool vec_ok =
+        aligned16(a.table) && (!has_q || (aligned16(a.q) && aligned16(a.q_out) &&
+                                          aligned16(a.q_weight) && qs % 8 == 0 && qos % 8 == 0)) &&
+        (!has_k || (aligned16(a.k) && aligned16(a.k_out) && aligned16(a.k_weight) &&
+                    ks % 8 == 0 && kos % 8 == 0));
+    const bool shape_ok = head_dim % 16 == 0 && (interleaved ? R % 8 == 0 : R % 16 == 0);
+    qknr::LaunchInfo info{};
+    e = qknr::launch_rope_table(a, vec_ok && shape_ok, static_cast<cudaStream_t>(cuda_stream),
+                                &info);
+    if (e != cudaSuccess) return cuda_fail(e, "table kernel launch");
+    return ok();
+}
+
+int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
+    if (!prm) return fail(QKNR_ERR_NULL, "params is NULL");
+    if (prm->struct_size != sizeof(qknr_rope_3d_params))
+        return fail(QKNR_ERR_SHAPE, "params.struct_size %zu != %zu (header mismatch)",
+                    prm->struct_size, sizeof(qknr_rope_3d_params));
+    const qknr_rope_3d_params& p = *prm;
+    const int D = p.head_dim;
+    if (D != 64 && D != 128 && D != 256)
+        return fail(QKNR_ERR_SHAPE, "head_dim %d must be 64, 128 or 256", D);
+    if (p.num_heads_q < 0 || p.num_heads_k < 0 || p.num_heads_v < 0 ||
+        p.num_heads_q + p.num_heads_k + p.num_heads_v < 1)
+        return fail(QKNR_ERR_SHAPE, "head counts must be >= 0 with at least one head");
+    const int maxh = qknr::rope3d_max_heads(D);
+    if (p.num_heads_q > maxh || p.num_heads_k > maxh)
+        return fail(QKNR_ERR_UNSUPPORTED, "more than %d Q or K heads of %d channels", maxh, D);
+    if (p.ppf < 1 || p.pph < 1 || p.ppw < 1)
+        return fail(QKNR_ERR_SHAPE, "ppf, pph and ppw must be >= 1");
+    const int64_t P = (int64_t)p.ppf * p.pph * p.ppw;
+    if (P > INT32_MAX) return fail(QKNR_ERR_SHAPE, "ppf*pph*ppw exceeds 2^31-1");
+    const int cf = p.num_frame_channels, ch = p.num_height_channels, cw = p.num_width_channels;
+    if (cf < 0 || ch < 0 || cw < 0 || (cf & 1) || (ch & 1) || (cw & 1))
+        return fail(QKNR_ERR_SHAPE, "channel counts must be even and >= 0 (%d/%d/%d)", cf, ch, cw);
+    if (cf + ch + cw != D)
+        return fail(QKNR_ERR_SHAPE, "channels %d+%d+%d != head_dim %d", cf, ch, cw, D);
+    if (p.num_tokens < 0) return fail(QKNR_ERR_SHAPE, "num_tokens < 0");
+    if (p.pos_offset < 0) return fail(QKNR_ERR_SHAPE, "pos_offset < 0");
+    if (p.pos_offset == 0 && p.num_tokens % P != 0)
+        return fail(QKNR_ERR_SHAPE, "num_tokens %lld not divisible by ppf*pph*ppw = %lld",
+                    (long long)p.num_tokens, (long long)P);
+    if (!(p.base > 0.0f) || std::isinf(p.base)) return fail(QKNR_ERR_SHAPE, "base must be > 0");
+    if (p.factor != 1.0f)
+        return fail(QKNR_ERR_UNSUPPORTED, "YARN scaling (factor %g != 1) is not supported",
+                    (double)p.factor);
+    if (p.attention_factor != 1.0f)
+        return fail(QKNR_ERR_SHAPE, "attention_factor must be 1.0 when factor is 1.0");
+    if (p.is_qk_norm && (!(p.eps >= 0.0f) || std::isinf(p.eps)))
+        return fail(QKNR_ERR_SHAPE, "eps must be >= 0");
+    if (p.output_fp8 && (!std::isfinite(p.output_quant_scale) || !std::isfinite(p.v_quant_scale)))
+        return fail(QKNR_ERR_SHAPE, "FP8 scales must be finite");
+    if (p.num_tokens == 0) return ok();
+
+    const int64_t T = p.num_tokens;
+    const int64_t row = (int64_t)(p.num_heads_q + p.num_heads_k + p.num_heads_v) * D;
+    const int ob = p.output_fp8 ? 1 : 2;
+    const bool hq = p.num_heads_q > 0, hk = p.num_heads_k > 0, hv = p.num_heads_v > 0;
+    if (!p.qkv) return fail(QKNR_ERR_NULL, "qkv is NULL");
+    if ((hq && !p.q_out) || (hk && !p.k_out) || (hv && !p.v_out))
+        return fail(QKNR_ERR_NULL, "an output pointer is NULL");
+    if (p.is_qk_norm && ((hq && !p.q_weight) || (hk && !p.k_weight)))
+        return fail(QKNR_ERR_NULL, "a weight pointer is NULL with is_qk_norm");
+    const Span sin_{p.qkv, (uint64_t)T * row * 2};
+    const Span so[3] = {{p.q_out, (uint64_t)T * p.num_heads_q * D * ob},
+                        {p.k_out, (uint64_t)T * p.num_heads_k * D * ob},
+                        {p.v_out, (uint64_t)T * p.num_heads_v * D * ob}};
+    const Span sw[2] = {{p.is_qk_norm ? p.q_weight : nullptr, (uint64_t)p.num_heads_q * D * 2},
+                        {p.is_qk_norm ? p.k_weight : nullptr, (uint64_t)p.num_heads_k * D * 2}};
+    for (int i = 0; i < 3; ++i) {
+        if (overlap(so[i], sin_)) return fail(QKNR_ERR_ALIAS, "an output overlaps qkv");
+        for (int j = 0; j < i; ++j)
+            if (overlap(so[i], so[j])) return fail(QKNR_ERR_ALIAS, "two outputs overlap");
+        for (int j = 0; j < 2; ++j)
+            if (overlap(so[i], sw[j])) return fail(QKNR_ERR_ALIAS, "an output overlaps a weight");
+    }
+    if (!aligned16(p.qkv) || (hq && !aligned16(p.q_out)) || (hk && !aligned16(p.k_out)) ||
+        (hv && !aligned16(p.v_out)))
+        return fail(QKNR_ERR_ALIGN, "qkv and the outputs must be 16-byte aligned");
+    if (p.is_qk_norm && ((hq && !aligned16(p.q_weight)) || (hk && !aligned16(p.k_weight))))
+        return fail(QKNR_ERR_ALIGN, "weights must be 16-byte aligned");
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    qknr::Rope3DArgs a{};
+    const void* ptr = nullptr;
+    int rc;
+    if ((rc = classify(p.qkv, "qkv", dev, &ptr))) return rc;
+    a.qkv = static_cast<const uint8_t*>(ptr);
+    if (hq) {
+        if ((rc = classify(p.q_out, "q_out", dev, &ptr))) return rc;
+        a.q_out = static_cast<uint8_t*>(const_cast<void*>(ptr));
+    }
+    if (hk) {
+        if ((rc = classify(p.k_out, "k_out", dev, &ptr))) return rc;
+        a.k_out = static_cast<uint8_t*>(const_cast<void*>(ptr));
+    }
+    if (hv) {
+        if ((rc = classify(p.v_out, "v_out", dev, &ptr))) return rc;
+        a.v_out = static_cast<uint8_t*>(const_cast<void*>(ptr));
+    }
+    if (p.is_qk_norm && hq) {
+        if ((rc = classify(p.q_weight, "q_weight", dev, &ptr))) return rc;
+        a.q_weight = static_cast<const uint8_t*>(ptr);
+    }
+    if (p.is_qk_norm && hk) {
+        if ((rc = classify(p.k_weight, "k_weight", dev, &ptr))) return rc;
+        a.k_weight = static_cast<const uint8_t*>(ptr);
+    }
+    a.num_tokens = T;
+    a.pos_offset = p.pos_offset % P;
+    a.ppf = p.ppf;
+    a.pph = p.pph;
+    a.ppw = p.ppw;
+    a.cf = cf;
+    a.ch = ch;
+    a.cw = cw;
+    a.hq = p.num_heads_q;
+    a.hk = p.num_heads_k;
+    a.hv = p.num_heads_v;
+    a.is_qk_norm = p.is_qk_norm ? 1 : 0;
+    const int64_t entries = (int64_t)p.ppf * (cf / 2) + (int64_t)p.pph * (ch / 2) +
+                            (int64_t)p.ppw * (cw / 2);
+    a.table_entries = entries > (1 << 20) ? (1 << 20) + 1 : (int32_t)entries;
+    a.eps = p.eps;
+    a.q_scale = p.output_quant_scale;
+    a.v_scale = p.v_quant_scale;
+    a.base = (double)p.base;
+    qknr::LaunchInfo info{};
+    e = qknr::launch_rope3d(a, D, p.interleave ? 0 : 1, p.output_fp8 ? 1 : 0,
+                            static_cast<cudaStream_t>(cuda_stream), &info);
+    if (e != cudaSuccess) return cuda_fail(e, "3D kernel launch");
+    return ok();
+}
+
+}  // extern "C"

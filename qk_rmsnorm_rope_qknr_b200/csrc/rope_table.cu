@@ -1,0 +1,315 @@
+// Table-driven per-head Q/K RMSNorm + RoPE.
+//
+// Computes the operation of "vllm_omni.diffusion.layers.fused_qk_norm_rope"
+// (vLLM-Omni API docs; contract bullets and fused_qk_norm_rope): each head of
+// q [T, Hq, D] and k [T, Hk, D] is RMS-normalised over its D channels, scaled
+// by a [D] weight and rotated by the token's row of a [T, rotary_dim] cos/sin
+// table, pairs (2j, 2j+1) (interleaved) or (j, j + rotary_dim/2) (half split);
+// channels >= rotary_dim are normalised only.
+//
+// Fast kernel: a head is a group of GS lanes (GS = next power of two of D/16);
+// lane l of the group owns two 16-byte vectors of the head, chosen so that
+// every rotation pair sits inside the lane: half split -> vectors l and
+// l + rotary_dim/16 for l < rotary_dim/16, the pass-through vectors two by two
+// after that; interleaved -> vectors l and l + D/16. The group's sum of
+// squares is a GS-lane shuffle reduction: no shared memory, no barrier. Every
+// thread works on U heads at once so that 2U loads are in flight. The table
+// row of a token is read by all its heads and stays in L1.
+//
+// General kernel: one warp per head through shared memory, for the shapes and
+// alignments the fast kernel does not take.
+#include "common.cuh"
+#include "launch.h"
+
+#include <algorithm>
+
+namespace qknr {
+
+namespace {
+
+constexpr int kBlock = 256;
+constexpr int kUnroll = 4;
+
+template <bool F32>
+__device__ __forceinline__ void load_cos_sin8(const uint8_t* tbl_row, int col, int half,
+                                              float (&c)[8], float (&s)[8]) {
+    if constexpr (F32) {
+        const float4* pc = reinterpret_cast<const float4*>(tbl_row + (size_t)col * 4);
+        const float4* ps = reinterpret_cast<const float4*>(tbl_row + (size_t)(half + col) * 4);
+        const float4 c0 = __ldg(pc), c1 = __ldg(pc + 1), s0 = __ldg(ps), s1 = __ldg(ps + 1);
+        c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w;
+        c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
+        s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w;
+        s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
+    } else {
+        const uint4 cv = __ldg(reinterpret_cast<const uint4*>(tbl_row + (size_t)col * 2));
+        const uint4 sv = __ldg(reinterpret_cast<const uint4*>(tbl_row + (size_t)(half + col) * 2));
+        unpack8(cv, c);
+        unpack8(sv, s);
+    }
+}
+
+template <bool F32>
+__device__ __forceinline__ void load_cos_sin4(const uint8_t* tbl_row, int col, int half,
+                                              float* c, float* s) {
+    if constexpr (F32) {
+        const float4 cv = __ldg(reinterpret_cast<const float4*>(tbl_row + (size_t)col * 4));
+        const float4 sv = __ldg(reinterpret_cast<const float4*>(tbl_row + (size_t)(half + col) * 4));
+        c[0] = cv.x; c[1] = cv.y; c[2] = cv.z; c[3] = cv.w;
+        s[0] = sv.x; s[1] = sv.y; s[2] = sv.z; s[3] = sv.w;
+    } else {
+        const uint2 cv = __ldg(reinterpret_cast<const uint2*>(tbl_row + (size_t)col * 2));
+        const uint2 sv = __ldg(reinterpret_cast<const uint2*>(tbl_row + (size_t)(half + col) * 2));
+        c[0] = bf16_lo(cv.x); c[1] = bf16_hi(cv.x); c[2] = bf16_lo(cv.y); c[3] = bf16_hi(cv.y);
+        s[0] = bf16_lo(sv.x); s[1] = bf16_hi(sv.x); s[2] = bf16_lo(sv.y); s[3] = bf16_hi(sv.y);
+    }
+}
+
+template <int GS, bool IL, bool F32>
+__global__ void __launch_bounds__(kBlock) rope_table_fast(const RopeTableArgs a) {
+    const int D = a.head_dim, R = a.rotary_dim;
+    const int L = D / 16;
+    const int l = threadIdx.x % GS;
+    const bool active = l < L;
+    const int H = a.hq + a.hk;
+    const int64_t ngroups = a.num_tokens * H;
+    const int gpb = kBlock / GS;  // groups per block per round
+    const int tb = F32 ? 4 : 2;   // table element bytes
+
+    // Vectors of this lane inside a head and how they rotate.
+    int va, vb;
+    bool across = false, rot_a = false, rot_b = false;
+    if (IL) {
+        va = l; vb = l + L;
+        rot_a = va < R / 8; rot_b = vb < R / 8;
+    } else {
+        const int r16 = R / 16;
+        if (l < r16) {
+            va = l; vb = l + r16; across = true;
+        } else {
+            va = R / 8 + 2 * (l - r16); vb = va + 1;
+        }
+    }
+    uint4 wqa = make_uint4(0, 0, 0, 0), wqb = wqa, wka = wqa, wkb = wqa;
+    if (active) {
+        const uint4* qw = reinterpret_cast<const uint4*>(a.q_weight);
+        const uint4* kw = reinterpret_cast<const uint4*>(a.k_weight);
+        if (a.hq > 0) { wqa = qw[va]; wqb = qw[vb]; }
+        if (a.hk > 0) { wka = kw[va]; wkb = kw[vb]; }
+    }
+    const float inv_d = 1.0f / (float)D;
+
+    for (int64_t g0 = (int64_t)blockIdx.x * gpb * kUnroll; g0 < ngroups;
+         g0 += (int64_t)gridDim.x * gpb * kUnroll) {
+        uint4 xa[kUnroll], xb[kUnroll];
+        int64_t tok[kUnroll];
+        int head[kUnroll];
+        bool isk[kUnroll], ok[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = g0 + (int64_t)u * gpb + threadIdx.x / GS;
+            ok[u] = active && g < ngroups;
+            tok[u] = g / H;
+            const int hh = (int)(g - tok[u] * H);
+            isk[u] = hh >= a.hq;
+            head[u] = isk[u] ? hh - a.hq : hh;
+            if (ok[u]) {
+                const uint8_t* src = isk[u]
+                    ? a.k + ((size_t)tok[u] * a.k_stride + (size_t)head[u] * D) * 2
+                    : a.q + ((size_t)tok[u] * a.q_stride + (size_t)head[u] * D) * 2;
+                xa[u] = ld_cs_v4(src + (size_t)va * 16);
+                xb[u] = ld_cs_v4(src + (size_t)vb * 16);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            float fa[8], fb[8];
+            unpack8(xa[u], fa);
+            unpack8(xb[u], fb);
+            float ss = 0.0f;
+            if (ok[u]) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss += fa[e] * fa[e] + fb[e] * fb[e];
+            }
+            ss = group_sum<GS>(ss);
+            if (!ok[u]) continue;
+            const float r = rsqrtf(ss * inv_d + a.eps);
+            float wa[8], wb[8];
+            unpack8(isk[u] ? wka : wqa, wa);
+            unpack8(isk[u] ? wkb : wqb, wb);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                fa[e] = fa[e] * r * wa[e];
+                fb[e] = fb[e] * r * wb[e];
+            }
+            const uint8_t* trow = a.table + (size_t)tok[u] * R * tb;
+            float oa[8], ob[8];
+            if (IL) {
+                float c[8], s[8];
+                if (rot_a) load_cos_sin4<F32>(trow, 4 * va, R / 2, c, s);
+                if (rot_b) load_cos_sin4<F32>(trow, 4 * vb, R / 2, c + 4, s + 4);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    if (rot_a) {
+                        oa[2 * m] = fa[2 * m] * c[m] - fa[2 * m + 1] * s[m];
+                        oa[2 * m + 1] = fa[2 * m + 1] * c[m] + fa[2 * m] * s[m];
+                    } else {
+                        oa[2 * m] = fa[2 * m]; oa[2 * m + 1] = fa[2 * m + 1];
+                    }
+                    if (rot_b) {
+                        ob[2 * m] = fb[2 * m] * c[4 + m] - fb[2 * m + 1] * s[4 + m];
+                        ob[2 * m + 1] = fb[2 * m + 1] * c[4 + m] + fb[2 * m] * s[4 + m];
+                    } else {
+                        ob[2 * m] = fb[2 * m]; ob[2 * m + 1] = fb[2 * m + 1];
+                    }
+                }
+            } else if (across) {
+                float c[8], s[8];
+                load_cos_sin8<F32>(trow, 8 * va, R / 2, c, s);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    oa[e] = fa[e] * c[e] - fb[e] * s[e];
+                    ob[e] = fb[e] * c[e] + fa[e] * s[e];
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) { oa[e] = fa[e]; ob[e] = fb[e]; }
+            }
+            uint8_t* dst = isk[u]
+                ? a.k_out + ((size_t)tok[u] * a.k_out_stride + (size_t)head[u] * D) * 2
+                : a.q_out + ((size_t)tok[u] * a.q_out_stride + (size_t)head[u] * D) * 2;
+            st_v4(dst + (size_t)va * 16, pack8_bf16(oa));
+            st_v4(dst + (size_t)vb * 16, pack8_bf16(ob));
+        }
+    }
+}
+
+// One warp per head; any head_dim <= 256, any even rotary_dim <= head_dim,
+// 2-byte alignment. The normalised head goes through shared memory so that
+// every lane can read its partner channel.
+template <bool F32>
+__global__ void __launch_bounds__(kBlock) rope_table_general(const RopeTableArgs a) {
+    __shared__ float ybuf[kBlock / 32][256];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int D = a.head_dim, R = a.rotary_dim, half = R / 2;
+    const int H = a.hq + a.hk;
+    const int64_t ngroups = a.num_tokens * H;
+    float* y = ybuf[warp];
+    const uint16_t* qw = reinterpret_cast<const uint16_t*>(a.q_weight);
+    const uint16_t* kw = reinterpret_cast<const uint16_t*>(a.k_weight);
+    for (int64_t g = (int64_t)blockIdx.x * (kBlock / 32) + warp; g < ngroups;
+         g += (int64_t)gridDim.x * (kBlock / 32)) {
+        const int64_t t = g / H;
+        const int hh = (int)(g - t * H);
+        const bool isk = hh >= a.hq;
+        const int head = isk ? hh - a.hq : hh;
+        const uint16_t* src = reinterpret_cast<const uint16_t*>(isk ? a.k : a.q) +
+                              (size_t)t * (isk ? a.k_stride : a.q_stride) + (size_t)head * D;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(isk ? a.k_out : a.q_out) +
+                        (size_t)t * (isk ? a.k_out_stride : a.q_out_stride) + (size_t)head * D;
+        const uint16_t* w = isk ? kw : qw;
+        float x[8];
+        float ss = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int d = lane + 32 * k;
+            x[k] = d < D ? __uint_as_float((uint32_t)src[d] << 16) : 0.0f;
+            ss += x[k] * x[k];
+        }
+        ss = warp_sum(ss);
+        const float r = rsqrtf(ss / (float)D + a.eps);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int d = lane + 32 * k;
+            if (d < D) y[d] = x[k] * r * __uint_as_float((uint32_t)__ldg(w + d) << 16);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int d = lane + 32 * k;
+            if (d >= D) continue;
+            float o = y[d];
+            if (d < R) {
+                int j, p;
+                bool first;
+                if (a.interleaved) {
+                    j = d >> 1; first = (d & 1) == 0; p = d ^ 1;
+                } else {
+                    first = d < half; j = first ? d : d - half; p = first ? d + half : d - half;
+                }
+                float c, s;
+                if (F32) {
+                    const float* tr = reinterpret_cast<const float*>(a.table) + (size_t)t * R;
+                    c = __ldg(tr + j); s = __ldg(tr + half + j);
+                } else {
+                    const uint16_t* tr = reinterpret_cast<const uint16_t*>(a.table) + (size_t)t * R;
+                    c = __uint_as_float((uint32_t)__ldg(tr + j) << 16);
+                    s = __uint_as_float((uint32_t)__ldg(tr + half + j) << 16);
+                }
+                o = first ? y[d] * c - y[p] * s : y[d] * c + y[p] * s;
+            }
+            __nv_bfloat16 b = __float2bfloat16_rn(o);
+            dst[d] = *reinterpret_cast<uint16_t*>(&b);
+        }
+        __syncwarp();
+    }
+}
+
+template <typename K>
+cudaError_t launch_persistent(K kern, int64_t work_blocks, const RopeTableArgs& a,
+                              cudaStream_t stream, LaunchInfo* info, int id) {
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBlock,
+                                                                            0);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * per_sm,
+                                                                 work_blocks));
+    kern<<<grid, kBlock, 0, stream>>>(a);
+    if (info) {
+        info->grid = grid;
+        info->block = kBlock;
+        info->smem = 0;
+        info->kernel_id = id;
+    }
+    return cudaGetLastError();
+}
+
+template <int GS>
+cudaError_t run_fast(const RopeTableArgs& a, cudaStream_t stream, LaunchInfo* info) {
+    const int64_t groups = a.num_tokens * (a.hq + a.hk);
+    const int64_t per_block = (int64_t)(kBlock / GS) * kUnroll;
+    const int64_t blocks = (groups + per_block - 1) / per_block;
+    const int id = 1000 + GS * 10 + (a.interleaved ? 1 : 0) * 2 + (a.table_f32 ? 1 : 0);
+    if (a.interleaved) {
+        return a.table_f32
+            ? launch_persistent(rope_table_fast<GS, true, true>, blocks, a, stream, info, id)
+            : launch_persistent(rope_table_fast<GS, true, false>, blocks, a, stream, info, id);
+    }
+    return a.table_f32
+        ? launch_persistent(rope_table_fast<GS, false, true>, blocks, a, stream, info, id)
+        : launch_persistent(rope_table_fast<GS, false, false>, blocks, a, stream, info, id);
+}
+
+}  // namespace
+
+cudaError_t launch_rope_table(const RopeTableArgs& a, int fast_path, cudaStream_t stream,
+                              LaunchInfo* info) {
+    if (fast_path) {
+        const int L = a.head_dim / 16;
+        if (L <= 1) return run_fast<1>(a, stream, info);
+        if (L <= 2) return run_fast<2>(a, stream, info);
+        if (L <= 4) return run_fast<4>(a, stream, info);
+        if (L <= 8) return run_fast<8>(a, stream, info);
+        return run_fast<16>(a, stream, info);
+    }
+    const int64_t groups = a.num_tokens * (a.hq + a.hk);
+    const int64_t blocks = (groups + kBlock / 32 - 1) / (kBlock / 32);
+    return a.table_f32
+        ? launch_persistent(rope_table_general<true>, blocks, a, stream, info, 2001)
+        : launch_persistent(rope_table_general<false>, blocks, a, stream, info, 2000);
+}
+
+}  // namespace qknr

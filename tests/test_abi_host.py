@@ -1,0 +1,190 @@
+"""Host-side checks of libqknr.so that need no GPU: the library loads, exports
+every entry point declared in include/qknr.h, agrees with the Python struct
+layout, and turns bad arguments into status codes before touching CUDA."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import qk_rmsnorm_rope_qknr_b200 as Q
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qknr.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    Q.build()
+    return Q.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qknr_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    assert {"qknr_rope_table", "qknr_rope_3d", "qknr_status_string"} <= set(names)
+    assert set(names) == set(Q.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_abi_version_and_strings(L):
+    assert L.qknr_abi_version() == 1
+    for s in range(8):
+        assert L.qknr_status_string(s)
+    assert L.qknr_status_string(0) == b"ok"
+
+
+# Fake device addresses: every call below fails validation before any CUDA
+# call, so they are never dereferenced.
+A = 0x7f0000000000
+
+
+def _p3(**over):
+    kw = dict(ppf=2, pph=4, ppw=4, num_frame_channels=16, num_height_channels=24,
+              num_width_channels=24, num_heads_q=4, num_heads_k=4, num_heads_v=4, head_dim=64,
+              num_tokens=32)
+    kw.update(over)
+    qkv = over.pop("qkv_ptr", A)
+    p = Q.make_3d_params(None, None, None, None, None, None, **{k: v for k, v in kw.items()
+                                                                  if k != "qkv_ptr"})
+    T = kw["num_tokens"]
+    p.qkv = qkv
+    p.q_weight = A + (1 << 30)
+    p.k_weight = A + (1 << 30) + 4096
+    p.q_out = A + (2 << 30)
+    p.k_out = A + (3 << 30)
+    p.v_out = A + (4 << 30)
+    _ = T
+    return p
+
+
+def _call3d(L, p):
+    rc = L.qknr_rope_3d(C.byref(p), None)
+    return rc, L.qknr_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("over,code,needle", [
+    (dict(head_dim=96, num_frame_channels=32, num_height_channels=32, num_width_channels=32),
+     Q.QKNR_ERR_SHAPE, "head_dim"),
+    (dict(num_frame_channels=18), Q.QKNR_ERR_SHAPE, "!= head_dim"),
+    (dict(num_frame_channels=15, num_height_channels=25), Q.QKNR_ERR_SHAPE, "even"),
+    (dict(num_width_channels=22), Q.QKNR_ERR_SHAPE, "head_dim"),
+    (dict(num_tokens=33), Q.QKNR_ERR_SHAPE, "divisible"),
+    (dict(ppf=0), Q.QKNR_ERR_SHAPE, "ppf"),
+    (dict(factor=2.0), Q.QKNR_ERR_UNSUPPORTED, "YARN"),
+    (dict(attention_factor=0.5), Q.QKNR_ERR_SHAPE, "attention_factor"),
+    (dict(base=0.0), Q.QKNR_ERR_SHAPE, "base"),
+    (dict(num_heads_q=0, num_heads_k=0, num_heads_v=0), Q.QKNR_ERR_SHAPE, "head"),
+    (dict(num_heads_q=-1), Q.QKNR_ERR_SHAPE, "head"),
+    (dict(num_heads_q=4096), Q.QKNR_ERR_UNSUPPORTED, "heads"),
+    (dict(num_tokens=-1, pos_offset=1), Q.QKNR_ERR_SHAPE, "num_tokens"),
+    (dict(pos_offset=-3), Q.QKNR_ERR_SHAPE, "pos_offset"),
+    (dict(eps=-1.0), Q.QKNR_ERR_SHAPE, "eps"),
+    (dict(qkv_ptr=0), Q.QKNR_ERR_NULL, "qkv"),
+    (dict(qkv_ptr=A + 8), Q.QKNR_ERR_ALIGN, "16-byte"),
+])
+def test_3d_validation(L, over, code, needle):
+    p = _p3(**over)
+    rc, detail = _call3d(L, p)
+    assert rc == code, (rc, detail)
+    assert needle in detail
+
+
+def test_3d_struct_size_guard(L):
+    p = _p3()
+    p.struct_size = C.sizeof(Q.Rope3DParams) - 8
+    rc, detail = _call3d(L, p)
+    assert rc == Q.QKNR_ERR_SHAPE and "struct_size" in detail
+    # the real size passes the guard (and then fails on head_dim, proving the layout)
+    p = _p3(head_dim=32, num_frame_channels=8, num_height_channels=8, num_width_channels=16)
+    rc, detail = _call3d(L, p)
+    assert rc == Q.QKNR_ERR_SHAPE and "head_dim 32" in detail
+
+
+def test_3d_null_outputs_and_weights(L):
+    p = _p3()
+    p.v_out = None
+    assert _call3d(L, p)[0] == Q.QKNR_ERR_NULL
+    p = _p3()
+    p.q_weight = None
+    assert _call3d(L, p)[0] == Q.QKNR_ERR_NULL
+    p = _p3(is_qk_norm=False, num_heads_v=0)
+    p.q_weight = p.k_weight = None
+    p.v_out = None
+    p.q_out = A + (2 << 30) + 8
+    assert _call3d(L, p)[0] == Q.QKNR_ERR_ALIGN     # passes the NULL checks, fails alignment
+
+
+def test_3d_aliasing(L):
+    p = _p3()
+    p.q_out = A + 4096      # inside qkv (32 rows of 1536 bytes)
+    assert _call3d(L, p)[0] == Q.QKNR_ERR_ALIAS
+    p = _p3()
+    p.k_out = p.q_out + 1024
+    assert _call3d(L, p)[0] == Q.QKNR_ERR_ALIAS
+    p = _p3()
+    p.v_out = p.q_weight
+    assert _call3d(L, p)[0] == Q.QKNR_ERR_ALIAS
+
+
+def test_3d_zero_tokens_is_noop(L):
+    p = _p3(num_tokens=0)
+    p.qkv = p.q_out = p.k_out = p.v_out = None
+    assert _call3d(L, p)[0] == Q.QKNR_OK
+
+
+def _table(L, **over):
+    kw = dict(q=A, k=A + (1 << 30), q_out=A + (2 << 30), k_out=A + (3 << 30),
+              q_weight=A + (4 << 30), k_weight=A + (4 << 30) + 4096, rope_table=A + (5 << 30),
+              table_dtype=Q.QKNR_DT_F32, T=16, Hq=4, Hk=2, D=128, R=96, qs=0, ks=0, qos=0,
+              kos=0, eps=1e-6, il=0)
+    kw.update(over)
+    rc = L.qknr_rope_table(kw["q"], kw["k"], kw["q_out"], kw["k_out"], kw["q_weight"],
+                           kw["k_weight"], kw["rope_table"], kw["table_dtype"], kw["T"], kw["Hq"],
+                           kw["Hk"], kw["D"], kw["R"], kw["qs"], kw["ks"], kw["qos"], kw["kos"],
+                           kw["eps"], kw["il"], None)
+    return rc, L.qknr_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(D=0), Q.QKNR_ERR_SHAPE), (dict(D=258, R=96), Q.QKNR_ERR_SHAPE),
+    (dict(R=97), Q.QKNR_ERR_SHAPE), (dict(R=130), Q.QKNR_ERR_SHAPE),
+    (dict(table_dtype=Q.QKNR_DT_E4M3), Q.QKNR_ERR_SHAPE), (dict(T=-1), Q.QKNR_ERR_SHAPE),
+    (dict(Hq=-2), Q.QKNR_ERR_SHAPE), (dict(eps=-1.0), Q.QKNR_ERR_SHAPE),
+    (dict(qs=100), Q.QKNR_ERR_SHAPE), (dict(q=0), Q.QKNR_ERR_NULL),
+    (dict(k_weight=0), Q.QKNR_ERR_NULL), (dict(rope_table=0), Q.QKNR_ERR_NULL),
+    (dict(q_out=A + 64), Q.QKNR_ERR_ALIAS), (dict(k_out=A + (2 << 30) + 256), Q.QKNR_ERR_ALIAS),
+    (dict(q_out=A + (5 << 30)), Q.QKNR_ERR_ALIAS),
+    (dict(q_out=A, qos=1024), Q.QKNR_ERR_ALIAS),          # in place needs the same stride
+    (dict(q=A + 1), Q.QKNR_ERR_ALIGN), (dict(rope_table=A + (5 << 30) + 2), Q.QKNR_ERR_ALIGN),
+])
+def test_table_validation(L, over, code):
+    rc, detail = _table(L, **over)
+    assert rc == code, (rc, detail)
+    assert detail
+
+
+def test_table_noops(L):
+    assert _table(L, T=0, q=0, k=0, q_out=0, k_out=0)[0] == Q.QKNR_OK
+    assert _table(L, Hq=0, Hk=0, q=0, k=0)[0] == Q.QKNR_OK
+
+
+def test_python_wrapper_raises_valueerror(L):
+    import torch
+
+    x = torch.zeros(4, 2, 64, dtype=torch.bfloat16)
+    w = torch.zeros(64, dtype=torch.bfloat16)
+    tbl = torch.zeros(4, 64, dtype=torch.float32)
+    with pytest.raises(ValueError):
+        Q.fused_qk_norm_rope(x, x, w, w, tbl[:, :63], 1e-6)
+    with pytest.raises(ValueError):
+        Q.fused_qk_norm_rope(x.float(), x, w, w, tbl, 1e-6)

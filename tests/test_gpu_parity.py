@@ -1,0 +1,337 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Tolerance (tests/_util.py): bf16 outputs within 2 ulp of the oracle's rounded
+result, with the ulp taken at max(|ref|, 2^-8 * RMS of the head row); E4M3
+outputs within one code step. Pure copies (V in bf16, and Q/K at patch
+(0,0,0) without the norm) must be bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import qk_rmsnorm_rope_qknr_b200 as Q
+from qk_rmsnorm_rope_qknr_b200 import workloads as W
+from tests._util import bf16_mismatch, e4m3_mismatch, t2u16, t2u8
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _p3(w: W.Form3D, **over):
+    p = w.params()
+    p.update(over)
+    return p
+
+
+def run_3d(qkv, qw, kw, stream=None, **p):
+    return Q.fused_qk_rmsnorm_rope(qkv, qw, kw, stream=stream, **p)
+
+
+def oracle_3d(qkv_cpu, qw_cpu, kw_cpu, **p):
+    bits = t2u16(qkv_cpu)
+    qwb = t2u16(qw_cpu) if qw_cpu is not None else None
+    kwb = t2u16(kw_cpu) if kw_cpu is not None else None
+    exact = O.rope_3d(bits, qwb, kwb, exact=True, **p)
+    rounded = O.rope_3d(bits, qwb, kwb, **p)
+    return rounded, exact
+
+
+def assert_3d_close(outs, ref, exact, fp8, what=""):
+    names = ("q", "k", "v")
+    for n, o, r, x in zip(names, outs, ref, exact):
+        T = r.shape[0]
+        if fp8:
+            bad, st = e4m3_mismatch(t2u8(o).reshape(r.shape), r)
+            assert len(bad) == 0, f"{what} {n}: {len(bad)} E4M3 codes off by >1 step {st}"
+        else:
+            g = t2u16(o).reshape(r.shape)
+            if n == "v":
+                assert np.array_equal(g, r), f"{what} v is not a bit copy"
+                continue
+            bad, st = bf16_mismatch(g, r, x)
+            assert len(bad) == 0, f"{what} {n}: {len(bad)} of {g.size} beyond 2 ulp {st}, " \
+                                  f"first at {bad[:3].tolist()}"
+        _ = T
+
+
+def check_3d_case(qkv, qw, kw, **p):
+    outs = run_3d(qkv, qw, kw, **p)
+    torch.cuda.synchronize()
+    cpu = lambda t: None if t is None else t.cpu()  # noqa: E731
+    ref, exact = oracle_3d(cpu(qkv).reshape(-1, qkv.shape[-1]), cpu(qw), cpu(kw), **p)
+    assert_3d_close(outs, ref, exact, p.get("output_fp8", False), str(p))
+    return outs
+
+
+# --------------------------------------------------------------- workloads --
+@pytest.mark.parametrize("name", ["tiny3d", "video3d", "fp8neox", "fp8neox_nonorm"])
+def test_3d_workload_ragged_shard(name):
+    """The workload's geometry on a shard of 3001 tokens that starts mid-grid:
+    several CTAs' worth of tokens per CTA, a ragged end, wrapped positions."""
+    w = W.WORKLOADS[name]
+    T = 32 if name == "tiny3d" else 3001
+    off = 0 if name == "tiny3d" else 12345
+    inp = W.make_inputs(w, device="cpu", tokens=T)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    check_3d_case(g["qkv"], g["q_weight"], g["k_weight"], pos_offset=off, **_p3(w))
+
+
+@pytest.mark.parametrize("name", ["video3d", "fp8neox", "fp8neox_nonorm"])
+def test_3d_workload_full_size_sampled(name):
+    """Full-size workload in the benchmark's launch configuration; the oracle
+    checks 48 sampled tokens one by one (grid corners, batch seam, random), and
+    the V output is checked in full against torch's own conversion."""
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w, device=DEV)
+    qkv = inp["qkv"]
+    p = _p3(w)
+    outs = run_3d(qkv, inp["q_weight"], inp["k_weight"], **p)
+    torch.cuda.synchronize()
+    T = w.tokens
+    P = w.ppf * w.pph * w.ppw
+    rng = np.random.default_rng(7)
+    picks = sorted(set([0, 1, w.ppw, w.pph * w.ppw, P - 1, T - 1] + ([P, P + 1] if T > P else [])
+                       + rng.integers(0, T, 40).tolist()))
+    flat = qkv.reshape(T, -1)
+    qw_cpu, kw_cpu = inp["q_weight"].cpu(), inp["k_weight"].cpu()
+    for t in picks:
+        ref, exact = oracle_3d(flat[t:t + 1].cpu(), qw_cpu, kw_cpu, pos_offset=t, **p)
+        got = [o.reshape(T, -1, w.head_dim)[t:t + 1] for o in outs]
+        assert_3d_close(got, ref, exact, w.output_fp8, f"{name} token {t}")
+    v_in = flat[:, (w.hq + w.hk) * w.head_dim:]
+    v_out = outs[2].reshape(T, -1)
+    if w.output_fp8:
+        want = (v_in.float() * w.v_scale).to(torch.float8_e4m3fn)
+        assert torch.equal(v_out.view(torch.uint8), want.view(torch.uint8))
+    else:
+        assert torch.equal(v_out, v_in)
+
+
+@pytest.mark.parametrize("name", ["table_hs", "table_il"])
+def test_table_workload_full(name):
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w, device="cpu")
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    qo, ko = Q.fused_qk_norm_rope(g["q"], g["k"], g["q_weight"], g["k_weight"], g["rope_table"],
+                                  w.eps, rotary_dim=w.rotary_dim, interleaved=w.interleaved)
+    torch.cuda.synchronize()
+    check_table_against_oracle(inp, qo, ko, w.eps, w.rotary_dim, w.interleaved)
+
+
+def _table_bits(t):
+    return t.numpy() if t.dtype == torch.float32 else t2u16(t)
+
+
+def check_table_against_oracle(inp, qo, ko, eps, rd, il, what=""):
+    args = (t2u16(inp["q"]), t2u16(inp["k"]), t2u16(inp["q_weight"]), t2u16(inp["k_weight"]),
+            _table_bits(inp["rope_table"].cpu().contiguous()), eps, rd)
+    ex_q, ex_k = O.rope_table(*args, interleaved=il, exact=True)
+    rq, rk = O.rope_table(*args, interleaved=il)
+    for n, o, r, x in (("q", qo, rq, ex_q), ("k", ko, rk, ex_k)):
+        bad, st = bf16_mismatch(t2u16(o), r, x)
+        assert len(bad) == 0, f"{what} {n}: {len(bad)} beyond tolerance {st} at {bad[:3].tolist()}"
+
+
+# ------------------------------------------------------------- 3D variants --
+def _rand3d(T, Hq, Hk, Hv, D, std=1.0, seed=0):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    qkv = (torch.randn(T, (Hq + Hk + Hv) * D, generator=g) * std).to(torch.bfloat16)
+    qw = (1 + 0.1 * torch.randn(Hq * D, generator=g)).to(torch.bfloat16)
+    kw = (1 + 0.1 * torch.randn(Hk * D, generator=g)).to(torch.bfloat16)
+    return qkv.to(DEV), qw.to(DEV), kw.to(DEV)
+
+
+CASES_3D = [
+    # (T, Hq, Hk, Hv, D, grid, channels, interleave, fp8, norm, pos_offset)
+    (12, 5, 3, 2, 64, (1, 3, 4), (16, 24, 24), True, False, True, 0),
+    (12, 5, 3, 2, 64, (1, 3, 4), (16, 24, 24), False, True, True, 0),
+    (40, 2, 2, 2, 256, (2, 4, 5), (64, 96, 96), True, True, False, 0),
+    (40, 2, 6, 1, 256, (2, 4, 5), (0, 128, 128), False, False, True, 0),
+    (7, 1, 1, 1, 128, (1, 1, 1), (32, 48, 48), True, False, True, 0),       # P = 1
+    (1, 4, 4, 4, 128, (3, 5, 7), (16, 56, 56), False, False, True, 77),     # a single token
+    (99, 80, 8, 8, 128, (3, 3, 11), (32, 48, 48), True, False, True, 5),    # 2 slots per thread
+    (33, 200, 160, 8, 128, (1, 3, 11), (32, 48, 48), False, True, True, 9),  # 4 slots
+    (64, 4, 4, 40, 64, (4, 4, 4), (16, 24, 24), True, False, True, 0),      # V-heavy row
+    (10000, 2, 2, 2, 64, (1, 1, 10000), (0, 0, 64), True, False, True, 0),  # no smem table
+    (257, 0, 4, 2, 128, (1, 1, 257), (32, 48, 48), True, False, True, 0),   # no Q heads
+    (64, 3, 3, 0, 128, (4, 4, 4), (32, 48, 48), False, True, True, 0),      # no V heads
+]
+
+
+@pytest.mark.parametrize("case", CASES_3D, ids=[str(i) for i in range(len(CASES_3D))])
+def test_3d_variants(case):
+    T, Hq, Hk, Hv, D, grid, ch, il, fp8, norm, off = case
+    qkv, qw, kw = _rand3d(T, Hq, Hk, Hv, D, std=2.0, seed=T + D)
+    p = dict(ppf=grid[0], pph=grid[1], ppw=grid[2], num_frame_channels=ch[0],
+             num_height_channels=ch[1], num_width_channels=ch[2], num_heads_q=Hq, num_heads_k=Hk,
+             num_heads_v=Hv, head_dim=D, eps=1e-5, base=10000.0, interleave=il, is_qk_norm=norm,
+             output_fp8=fp8, output_quant_scale=0.75, v_quant_scale=1.5, pos_offset=off)
+    check_3d_case(qkv, qw if norm else None, kw if norm else None, **p)
+
+
+def test_3d_rope_only_origin_is_bit_copy():
+    qkv, _, _ = _rand3d(16, 4, 4, 4, 64, std=3.0)
+    p = dict(ppf=1, pph=4, ppw=4, num_frame_channels=16, num_height_channels=24,
+             num_width_channels=24, num_heads_q=4, num_heads_k=4, num_heads_v=4, head_dim=64,
+             is_qk_norm=False)
+    q, k, v = run_3d(qkv, None, None, **p)
+    assert torch.equal(q[0].reshape(-1), qkv[0, :256]) and torch.equal(k[0].reshape(-1),
+                                                                         qkv[0, 256:512])
+    assert torch.equal(v.reshape(16, -1), qkv[:, 512:])
+
+
+def test_3d_base_below_one_and_large_positions():
+    """base < 1 makes frequencies above one turn; a 60000-wide grid makes large
+    angles: the fixed-point angle keeps both within tolerance."""
+    qkv, qw, kw = _rand3d(600, 2, 2, 1, 64, seed=3)
+    p = dict(ppf=1, pph=1, ppw=60000, num_frame_channels=16, num_height_channels=16,
+             num_width_channels=32, num_heads_q=2, num_heads_k=2, num_heads_v=1, head_dim=64,
+             base=0.37, pos_offset=59500)
+    check_3d_case(qkv, qw, kw, **p)
+
+
+def test_3d_output_guards_and_poison():
+    """Every output element is written and nothing past the end: outputs are
+    pre-filled with 0xFF (a NaN pattern the op cannot produce from finite
+    inputs) and followed by guard bytes."""
+    T, H, D = 48, 3, 128
+    qkv, qw, kw = _rand3d(T, H, H, H, D)
+    for fp8 in (False, True):
+        eb = 1 if fp8 else 2
+        n = T * H * D * eb
+        bufs = [torch.full((n + 4096,), 0xFF, dtype=torch.uint8, device=DEV) for _ in range(3)]
+        outs = [b[:n] for b in bufs]
+        p = dict(ppf=1, pph=6, ppw=8, num_frame_channels=32, num_height_channels=48,
+                 num_width_channels=48, num_heads_q=H, num_heads_k=H, num_heads_v=H, head_dim=D,
+                 output_fp8=fp8, output_quant_scale=0.5, v_quant_scale=0.5)
+        Q.qknr_rope_3d(qkv, qw, kw, *outs, **p)
+        torch.cuda.synchronize()
+        for b in bufs:
+            assert torch.all(b[n:] == 0xFF), "guard bytes overwritten"
+            body = b[:n]
+            if fp8:
+                assert not torch.any(body == 0xFF)
+            else:
+                assert not torch.any(body.view(torch.int16) == -1)
+
+
+def test_3d_pinned_host_buffers():
+    """The C ABI accepts page-locked host memory: the kernel reads and writes it
+    across the bus. Same results as device buffers."""
+    qkv, qw, kw = _rand3d(64, 4, 4, 4, 64, seed=11)
+    p = dict(ppf=4, pph=4, ppw=4, num_frame_channels=16, num_height_channels=24,
+             num_width_channels=24, num_heads_q=4, num_heads_k=4, num_heads_v=4, head_dim=64)
+    dev_out = run_3d(qkv, qw, kw, **p)
+    h_qkv = qkv.cpu().pin_memory()
+    h_out = [torch.empty(64, 4, 64, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    Q.qknr_rope_3d(h_qkv, qw, kw, *h_out, stream=torch.cuda.current_stream(), **p)
+    torch.cuda.synchronize()
+    for a, b in zip(dev_out, h_out):
+        assert torch.equal(a.cpu(), b)
+
+
+def test_3d_pageable_host_memory_is_rejected():
+    qkv, qw, kw = _rand3d(16, 4, 4, 4, 64)
+    p = dict(ppf=1, pph=4, ppw=4, num_frame_channels=16, num_height_channels=24,
+             num_width_channels=24, num_heads_q=4, num_heads_k=4, num_heads_v=4, head_dim=64)
+    with pytest.raises(ValueError, match="device cannot access|pageable"):
+        Q.fused_qk_rmsnorm_rope(qkv.cpu(), qw, kw, q_out=torch.empty(16, 4, 64, dtype=torch.bfloat16,
+                                                                      device=DEV),
+                                k_out=torch.empty(16, 4, 64, dtype=torch.bfloat16, device=DEV),
+                                v_out=torch.empty(16, 4, 64, dtype=torch.bfloat16, device=DEV),
+                                **p)
+
+
+def test_3d_deterministic_and_streams():
+    w = W.WORKLOADS["tiny3d"]
+    inp = {k: v.to(DEV) for k, v in W.make_inputs(w).items()}
+    a = run_3d(inp["qkv"], inp["q_weight"], inp["k_weight"], **w.params())
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = run_3d(inp["qkv"], inp["q_weight"], inp["k_weight"], stream=s, **w.params())
+    s.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_3d_batch_shape():
+    w = W.WORKLOADS["tiny3d"]
+    qkv, qw, kw = _rand3d(64, 4, 4, 4, 64)
+    q, k, v = run_3d(qkv.reshape(2, 32, -1), qw, kw, **w.params())
+    assert q.shape == (2, 32, 4, 64) and v.shape == (2, 32, 4, 64)
+    q2, _, _ = run_3d(qkv, qw, kw, **w.params())
+    assert torch.equal(q.reshape(64, 4, 64), q2)
+
+
+# ----------------------------------------------------------- table variants --
+def _rand_table_inputs(T, Hq, Hk, D, R, f32, seed=0, std=1.0):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    q = (torch.randn(T, Hq, D, generator=g) * std).to(torch.bfloat16)
+    k = (torch.randn(T, Hk, D, generator=g) * std).to(torch.bfloat16)
+    qw = (1 + 0.1 * torch.randn(D, generator=g)).to(torch.bfloat16)
+    kw = (1 + 0.1 * torch.randn(D, generator=g)).to(torch.bfloat16)
+    tbl = W.rope_table_input(T, R, 10000.0, f32)
+    return dict(q=q, k=k, q_weight=qw, k_weight=kw, rope_table=tbl)
+
+
+CASES_TABLE = [
+    # (T, Hq, Hk, D, R, f32, interleaved)
+    (37, 3, 5, 128, 96, True, False),
+    (37, 3, 5, 128, 64, False, True),
+    (20, 2, 1, 256, 256, True, False),
+    (20, 2, 1, 256, 248, False, True),
+    (50, 4, 4, 16, 16, True, True),
+    (50, 4, 4, 48, 32, True, False),     # 3 lanes per head, padded group of 4
+    (30, 2, 3, 72, 40, True, True),      # head_dim % 16 != 0: general kernel
+    (30, 2, 3, 128, 40, False, False),   # half split with rd % 16 != 0: general kernel
+    (30, 2, 3, 2, 2, True, True),        # smallest head
+    (30, 3, 0, 64, 64, True, False),     # no K heads
+]
+
+
+@pytest.mark.parametrize("case", CASES_TABLE, ids=[str(i) for i in range(len(CASES_TABLE))])
+def test_table_variants(case):
+    T, Hq, Hk, D, R, f32, il = case
+    inp = _rand_table_inputs(T, Hq, Hk, D, R, f32, seed=D + R, std=2.0)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    qo, ko = Q.fused_qk_norm_rope(g["q"], g["k"], g["q_weight"], g["k_weight"], g["rope_table"],
+                                  1e-5, rotary_dim=R, interleaved=il)
+    torch.cuda.synchronize()
+    check_table_against_oracle(inp, qo.cpu(), ko.cpu(), 1e-5, R, il, str(case))
+
+
+def test_table_strided_inplace_and_misaligned():
+    """q and k as views into a packed QKV buffer (token stride 3*H*D), updated
+    in place; then the same with every pointer shifted by one element (general
+    kernel); all must match the oracle on dense copies."""
+    T, H, D, R = 64, 4, 128, 96
+    inp = _rand_table_inputs(T, H, H, D, R, True, seed=5)
+    for shift in (0, 1):
+        buf = torch.zeros(T * 3 * H * D + 64, dtype=torch.bfloat16, device=DEV)
+        packed = buf[shift:shift + T * 3 * H * D].view(T, 3 * H, D)
+        packed[:, :H] = inp["q"].to(DEV)
+        packed[:, H:2 * H] = inp["k"].to(DEV)
+        q, k = packed[:, :H], packed[:, H:2 * H]
+        g = {n: inp[n].to(DEV) for n in ("q_weight", "k_weight", "rope_table")}
+        Q.fused_qk_norm_rope(q, k, g["q_weight"], g["k_weight"], g["rope_table"], 1e-6,
+                             rotary_dim=R, interleaved=False, q_out=q, k_out=k)
+        torch.cuda.synchronize()
+        check_table_against_oracle(inp, q.cpu(), k.cpu(), 1e-6, R, False, f"shift {shift}")
+        assert torch.all(packed[:, 2 * H:] == 0)
+
+
+def test_table_outputs_written_exactly():
+    T, Hq, Hk, D, R = 33, 3, 2, 128, 128
+    inp = _rand_table_inputs(T, Hq, Hk, D, R, False, seed=9)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    qb = torch.full((T * Hq * D + 512,), -1, dtype=torch.int16, device=DEV)
+    kb = torch.full((T * Hk * D + 512,), -1, dtype=torch.int16, device=DEV)
+    qo = qb[:T * Hq * D].view(torch.bfloat16).view(T, Hq, D)
+    ko = kb[:T * Hk * D].view(torch.bfloat16).view(T, Hk, D)
+    Q.fused_qk_norm_rope(g["q"], g["k"], g["q_weight"], g["k_weight"], g["rope_table"], 1e-6,
+                         rotary_dim=R, interleaved=True, q_out=qo, k_out=ko)
+    torch.cuda.synchronize()
+    assert torch.all(qb[T * Hq * D:] == -1) and torch.all(kb[T * Hk * D:] == -1)
+    assert not torch.any(qb[:T * Hq * D] == -1) and not torch.any(kb[:T * Hk * D] == -1)
