@@ -140,7 +140,7 @@ typedef struct {
     int32_t num_frame_channels, num_height_channels, num_width_channels;
     int32_t num_heads_q, num_heads_k, num_heads_v, head_dim;
     float eps;
-    float base;
+    double base;         /* double: at large positions a float base shifts angles */
     int32_t interleave;  /* 1 = adjacent pairs (non-NeoX), 0 = NeoX half split   */
     float factor, low, high, attention_factor; /* YARN: only factor == 1 accepted */
     int32_t is_qk_norm;

@@ -53,7 +53,7 @@ class Rope3DParams(C.Structure):
                 ("num_frame_channels", C.c_int32), ("num_height_channels", C.c_int32),
                 ("num_width_channels", C.c_int32), ("num_heads_q", C.c_int32),
                 ("num_heads_k", C.c_int32), ("num_heads_v", C.c_int32), ("head_dim", C.c_int32),
-                ("eps", C.c_float), ("base", C.c_float), ("interleave", C.c_int32),
+                ("eps", C.c_float), ("base", C.c_double), ("interleave", C.c_int32),
                 ("factor", C.c_float), ("low", C.c_float), ("high", C.c_float),
                 ("attention_factor", C.c_float), ("is_qk_norm", C.c_int32),
                 ("output_fp8", C.c_int32), ("output_quant_scale", C.c_float),

@@ -283,7 +283,7 @@ int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
     if (p.pos_offset == 0 && p.num_tokens % P != 0)
         return fail(QKNR_ERR_SHAPE, "num_tokens %lld not divisible by ppf*pph*ppw = %lld",
                     (long long)p.num_tokens, (long long)P);
-    if (!(p.base > 0.0f) || std::isinf(p.base)) return fail(QKNR_ERR_SHAPE, "base must be > 0");
+    if (!(p.base > 0.0) || std::isinf(p.base)) return fail(QKNR_ERR_SHAPE, "base must be > 0");
     if (p.factor != 1.0f)
         return fail(QKNR_ERR_UNSUPPORTED, "YARN scaling (factor %g != 1) is not supported",
                     (double)p.factor);
@@ -369,7 +369,7 @@ int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
     a.eps = p.eps;
     a.q_scale = p.output_quant_scale;
     a.v_scale = p.v_quant_scale;
-    a.base = (double)p.base;
+    a.base = p.base;
     qknr::LaunchInfo info{};
     e = qknr::launch_rope3d(a, D, p.interleave ? 0 : 1, p.output_fp8 ? 1 : 0,
                             static_cast<cudaStream_t>(cuda_stream), &info);

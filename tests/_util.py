@@ -38,6 +38,8 @@ def bf16_mismatch(gpu_bits, ref_bits, ref_exact, ulps=2.0):
     Arrays are [..., D] (last axis = one head row)."""
     g = u16_to_f64(gpu_bits)
     r = u16_to_f64(ref_bits)
+    if g.size == 0:
+        return np.zeros((0, g.ndim), int), dict(exact_frac=1.0, max_err_ulps=0.0, n=0)
     rms = np.sqrt(np.mean(np.square(ref_exact), axis=-1, keepdims=True))
     scale = np.maximum(np.abs(r), 2.0 ** -8 * rms)
     tol = ulps * ulp_bf16(scale)

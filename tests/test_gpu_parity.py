@@ -202,7 +202,8 @@ def test_3d_output_guards_and_poison():
         eb = 1 if fp8 else 2
         n = T * H * D * eb
         bufs = [torch.full((n + 4096,), 0xFF, dtype=torch.uint8, device=DEV) for _ in range(3)]
-        outs = [b[:n] for b in bufs]
+        odt = torch.float8_e4m3fn if fp8 else torch.bfloat16
+        outs = [b[:n].view(odt) for b in bufs]
         p = dict(ppf=1, pph=6, ppw=8, num_frame_channels=32, num_height_channels=48,
                  num_width_channels=48, num_heads_q=H, num_heads_k=H, num_heads_v=H, head_dim=D,
                  output_fp8=fp8, output_quant_scale=0.5, v_quant_scale=0.5)
