@@ -151,6 +151,28 @@ typedef struct {
 
 int qknr_rope_3d(const qknr_rope_3d_params* params, void* cuda_stream);
 
+/*
+ * Device-side status of this library's kernels on the current device, for
+ * failures that can only be seen on the GPU. Bit 0: a kernel's wait on one of
+ * its own bulk copies ran past its time limit (2 s), so that launch abandoned
+ * its remaining tokens and its outputs are incomplete; the kernel still ended
+ * normally and the CUDA context stays usable. The word accumulates over
+ * launches until cleared. Unlike every other entry point this one
+ * synchronises: it reads the word after the work already queued on
+ * `cuda_stream`, then clears it if `clear` is non-zero.
+ */
+int qknr_device_status(void* cuda_stream, uint32_t* status_out, int32_t clear);
+
+/*
+ * Test hook for the timeout path above (not for production use). While
+ * extra_bytes is non-zero, every later 3D launch on any thread makes each
+ * ring buffer wait for extra_bytes more than its copy delivers, so its waits
+ * run out after limit_ns and the launch takes the abandon path; the copies
+ * themselves complete, so nothing is left in flight. extra_bytes == 0 turns
+ * the hook off (limit_ns is then ignored and the 2 s limit returns).
+ */
+int qknr_test_set_wait_fault(uint32_t extra_bytes, uint64_t limit_ns);
+
 /* Static text for a status code. */
 const char* qknr_status_string(int status);
 

@@ -31,8 +31,8 @@ QKNR_OK, QKNR_ERR_NULL, QKNR_ERR_SHAPE, QKNR_ERR_UNSUPPORTED = 0, 1, 2, 3
 QKNR_ERR_ALIGN, QKNR_ERR_ALIAS, QKNR_ERR_POINTER, QKNR_ERR_CUDA = 4, 5, 6, 7
 QKNR_DT_BF16, QKNR_DT_F32, QKNR_DT_E4M3 = 0, 1, 2
 
-EXPORTS = ("qknr_rope_table", "qknr_rope_3d", "qknr_status_string", "qknr_last_error_detail",
-           "qknr_abi_version")
+EXPORTS = ("qknr_rope_table", "qknr_rope_3d", "qknr_device_status", "qknr_test_set_wait_fault",
+           "qknr_status_string", "qknr_last_error_detail", "qknr_abi_version")
 
 
 class QknrError(RuntimeError):
@@ -81,6 +81,10 @@ def lib() -> C.CDLL:
         L.qknr_status_string.restype = C.c_char_p
         L.qknr_last_error_detail.restype = C.c_char_p
         L.qknr_abi_version.restype = C.c_int
+        L.qknr_device_status.argtypes = [vp, C.POINTER(C.c_uint32), i32]
+        L.qknr_device_status.restype = C.c_int
+        L.qknr_test_set_wait_fault.argtypes = [C.c_uint32, C.c_uint64]
+        L.qknr_test_set_wait_fault.restype = C.c_int
         _lib = L
     return _lib
 
@@ -211,6 +215,16 @@ def qknr_rope_3d(qkv, q_weight, k_weight, q_out, k_out, v_out, *, stream=None, *
     _check(lib().qknr_rope_3d(C.byref(p), st))
 
 
+def qknr_device_status(clear: bool = False, stream=None, device=None) -> int:
+    """Device status word (bit 0: a kernel gave up waiting on its own bulk
+    copy and left its outputs incomplete). Synchronises the stream."""
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    out = C.c_uint32(0)
+    _check(lib().qknr_device_status(_stream(stream), C.byref(out), int(bool(clear))))
+    return out.value
+
+
 # ------------------------------------------------------- page-shaped wrappers --
 def fused_qk_norm_rope(q: torch.Tensor, k: torch.Tensor, q_weight: torch.Tensor,
                        k_weight: torch.Tensor, rope_table: torch.Tensor, eps: float, *,
@@ -263,6 +277,6 @@ def fused_qk_rmsnorm_rope(qkv: torch.Tensor, q_weight: torch.Tensor, k_weight: t
     return tuple(outs)
 
 
-__all__ = ["qknr_rope_table", "qknr_rope_3d", "fused_qk_norm_rope", "fused_qk_rmsnorm_rope",
+__all__ = ["qknr_rope_table", "qknr_rope_3d", "qknr_device_status", "fused_qk_norm_rope", "fused_qk_rmsnorm_rope",
            "QknrError", "QknrValueError", "lib", "build", "make_3d_params", "Rope3DParams",
            "EXPORTS", "LIB_PATH"]

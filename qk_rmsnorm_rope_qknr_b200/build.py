@@ -18,7 +18,7 @@ LIB = os.path.join(PKG, "libqknr.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2,-Wall", "-I", INC,
-         "-I", CSRC, "--expt-relaxed-constexpr"]
+         "-I", CSRC]
 
 
 def _sources():

@@ -26,6 +26,12 @@ struct Rope3DArgs {
     float q_scale;
     float v_scale;
     double base;
+    // Pipelined (bulk-copy) kernel only:
+    int32_t stages;          // ring buffers per token pipeline
+    int32_t groups;          // token pipelines per CTA
+    int32_t v_bulk;          // bf16 V leaves through a bulk store
+    uint32_t stall_tx_bytes; // test hook: extra bytes a stage waits for (0 in use)
+    uint64_t wait_limit_ns;  // a wait on a bulk copy gives up after this long
 };
 
 struct RopeTableArgs {
@@ -55,6 +61,11 @@ struct LaunchInfo {
 
 cudaError_t launch_rope3d(const Rope3DArgs& a, int head_dim, int neox, int fp8,
                           cudaStream_t stream, LaunchInfo* info);
+
+// Status word the pipelined 3D kernel raises (bit 0: a bulk-copy wait timed
+// out and the kernel abandoned its remaining tokens). Read on `stream`, after
+// the work queued before it; optionally cleared.
+cudaError_t read_device_status(uint32_t* out, int clear, cudaStream_t stream);
 cudaError_t launch_rope_table(const RopeTableArgs& a, int fast_path, cudaStream_t stream,
                               LaunchInfo* info);
 

@@ -7,6 +7,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
@@ -15,6 +16,10 @@
 namespace {
 
 thread_local char g_detail[320] = "";
+
+// Timeout-path test hook (qknr_test_set_wait_fault).
+std::atomic<uint32_t> g_fault_extra_bytes{0};
+std::atomic<uint64_t> g_fault_limit_ns{0};
 
 int fail(int code, const char* fmt, ...) {
     va_list ap;
@@ -131,6 +136,23 @@ const char* qknr_status_string(int status) {
 }
 
 const char* qknr_last_error_detail(void) { return g_detail; }
+
+int qknr_test_set_wait_fault(uint32_t extra_bytes, uint64_t limit_ns) {
+    if (extra_bytes != 0 && (extra_bytes % 16 != 0 || limit_ns == 0))
+        return fail(QKNR_ERR_SHAPE, "extra_bytes must be a multiple of 16 and limit_ns > 0");
+    g_fault_limit_ns.store(limit_ns);
+    g_fault_extra_bytes.store(extra_bytes);
+    return ok();
+}
+
+int qknr_device_status(void* cuda_stream, uint32_t* status_out, int32_t clear) {
+    if (!status_out) return fail(QKNR_ERR_NULL, "status_out is NULL");
+    uint32_t v = 0;
+    cudaError_t e = qknr::read_device_status(&v, clear, static_cast<cudaStream_t>(cuda_stream));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    *status_out = v;
+    return ok();
+}
 
 int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
                     const void* q_weight, const void* k_weight, const void* rope_table,
@@ -370,6 +392,8 @@ int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
     a.q_scale = p.output_quant_scale;
     a.v_scale = p.v_quant_scale;
     a.base = p.base;
+    a.stall_tx_bytes = g_fault_extra_bytes.load(std::memory_order_relaxed);
+    a.wait_limit_ns = a.stall_tx_bytes ? g_fault_limit_ns.load() : 0;
     qknr::LaunchInfo info{};
     e = qknr::launch_rope3d(a, D, p.interleave ? 0 : 1, p.output_fp8 ? 1 : 0,
                             static_cast<cudaStream_t>(cuda_stream), &info);

@@ -2,25 +2,43 @@
 //
 // Computes the operation of "flashinfer.norm.fused_qk_rmsnorm_rope" (FlashInfer
 // API docs; summary, Parameters, Returns) in one pass over HBM: every input
-// byte is read once with 128-bit loads, every output byte written once with
-// 128-bit (bf16) or 64-bit (E4M3) stores, and nothing else touches memory.
+// byte is read once, every output byte written once, nothing else touches
+// memory.
 //
-// Layout of the work. A CTA is persistent and walks tokens t = blockIdx.x,
-// blockIdx.x + gridDim.x, ... For one token the CTA holds the whole Q and K
-// part of the row in registers: thread tid owns, for S "slots" (head, l),
-// the two 16-byte vectors l and l + D/16 of that head (l = tid mod D/16, the
-// same for every slot of the thread). Vector l's channel e pairs with vector
-// l + D/16's channel e in NeoX mode; in interleaved mode each vector's
-// adjacent channels pair up. Either way a thread's 8 rotation pairs sit at
-// fixed pair slots, so their frequencies, weights and table columns are set up
-// once per CTA. V vectors are streamed straight to v_out.
+// Thread layout. One token is worked on by a group of threads. A thread owns,
+// for S "slots" (head, l), the two 16-byte vectors l and l + D/16 of that
+// head of Q and of K (l = thread mod D/16, the same for all its slots).
+// Vector l's channel e pairs with vector l + D/16's channel e in NeoX mode; in
+// interleaved mode adjacent channels of one vector pair up. Either way the 8
+// rotation pairs of a thread stay inside the thread, at fixed pair slots.
 //
-// Per token: issue every load, store V, reduce sum(x^2) of Q and of K over the
-// CTA (warp shuffles, one shared-memory exchange, one barrier), then scale,
-// rotate, convert and store. cos/sin come from a per-CTA shared-memory table
-// of every (axis, position, frequency) triple -- at most ppf*Cf/2 + pph*Ch/2 +
-// ppw*Cw/2 entries -- built once per CTA with an exact fixed-point angle, or,
-// when the table would not fit, from the same angle computed per token.
+// Per token: sum x^2 of Q and of K over the group (warp shuffles, one shared
+// exchange, one barrier), then scale, rotate, convert and store.
+//
+// cos/sin: the frequency of pair slot j, base^(-2i/C) / 2pi, is kept as a
+// 64-bit binary fraction of a turn; pos * fraction modulo 2^64 is the exact
+// angle in turns, so no precision is lost at large positions. A shared table
+// holds cos/sin of every (axis, position, frequency) -- at most
+// ppf*Cf/2 + pph*Ch/2 + ppw*Cw/2 entries -- built once per CTA; when it would
+// not fit, the angles are evaluated per token instead.
+//
+// rope3d_mg_kernel (the fast path): one persistent CTA per SM runs G
+// independent token pipelines ("groups"), each with its own named barrier and
+// its own ring of shared-memory row buffers that bulk asynchronous copies (the
+// TMA engine, one instruction per row, tracked by mbarriers) fill ahead of
+// use. The angle table and the norm weights (converted once to fp32, laid out
+// for conflict-free reads) are shared by all groups. Threads keep no row data
+// in registers across the per-token barrier: they read their vectors from the
+// ring before it (for sum x^2) and again after it (to scale and rotate), which
+// keeps registers low enough for ~24 warps per SM. The group's first thread
+// refills a buffer one token later, once every thread has passed the next
+// barrier, and in bf16 mode copies V straight from the ring to v_out with a
+// bulk store. Every wait on a copy is bounded in time; on expiry the group
+// votes through its barrier, raises bit 0 of a device status word, drains its
+// own copies and leaves.
+//
+// rope3d_reg_kernel (fallback for rows too large for the ring): 128-bit
+// loads straight into registers.
 #include "common.cuh"
 #include "launch.h"
 
@@ -28,32 +46,20 @@
 
 namespace qknr {
 
+__device__ unsigned int g_rope3d_status;
+
 namespace {
 
 constexpr int kMaxBlock = 512;
 constexpr int kMaxTableBytes = 64 * 1024;
+constexpr int kSmemPerSm = 227 * 1024;
 
-template <int D, bool NEOX, bool FP8, int S>
-__global__ void __launch_bounds__(kMaxBlock) rope3d_kernel(const Rope3DArgs a) {
-    constexpr int L = D / 16;   // threads per head
-    constexpr int VPH = D / 8;  // 16-byte vectors per head
+// Frequencies of the D/2 pair slots and, if enabled, the cos/sin table.
+template <int D>
+__device__ __forceinline__ void setup_angles(const Rope3DArgs& a, uint64_t* gq, float2* tab) {
     constexpr int HALF = D / 2;
-    constexpr int SV = 2 * S;  // V vectors per thread issued with the Q/K loads
-    constexpr int OUTB = FP8 ? 1 : 2;
-
-    extern __shared__ __align__(16) unsigned char smem[];
-    uint64_t* gq = reinterpret_cast<uint64_t*>(smem);                  // [HALF]
-    float2* red = reinterpret_cast<float2*>(smem + HALF * 8);         // [2][32]
-    float2* tab = reinterpret_cast<float2*>(smem + HALF * 8 + 512);  // [table_entries]
-
-    const int tid = threadIdx.x;
-    const int B = blockDim.x;
-    const int lane = tid & 31, warp = tid >> 5, nwarps = B >> 5;
-    const int l = tid % L;
+    const int tid = threadIdx.x, B = blockDim.x;
     const int hcf = a.cf >> 1, hch = a.ch >> 1, hcw = a.cw >> 1;
-    const bool norm = a.is_qk_norm != 0;
-
-    // Frequencies of the HALF pair slots, as 64-bit fractions of a turn.
     for (int j = tid; j < HALF; j += B) {
         int i, C;
         if (j < hcf) {
@@ -66,8 +72,8 @@ __global__ void __launch_bounds__(kMaxBlock) rope3d_kernel(const Rope3DArgs a) {
         gq[j] = turns_q64(a.base, i, C);
     }
     __syncthreads();
-    const int nf = a.ppf * hcf, nh = a.pph * hch;
     if (a.use_table) {
+        const int nf = a.ppf * hcf, nh = a.pph * hch;
         for (int e = tid; e < a.table_entries; e += B) {
             int pos, j;
             if (e < nf) {
@@ -83,97 +89,504 @@ __global__ void __launch_bounds__(kMaxBlock) rope3d_kernel(const Rope3DArgs a) {
             turn_sincos((uint32_t)pos, gq[j], &s, &c);
             tab[e] = make_float2(c, s);
         }
-        __syncthreads();
     }
+}
 
-    // This thread's 8 pair slots: axis and index inside the axis group.
-    int pax[8], pcol[8];
+// cos/sin of pair slot j for patch (pf, ph, pw).
+__device__ __forceinline__ float2 pair_cos_sin(const Rope3DArgs& a, const uint64_t* gq,
+                                               const float2* tab, int j, int pf, int ph, int pw) {
+    const int hcf = a.cf >> 1, hch = a.ch >> 1, hcw = a.cw >> 1;
+    int pos, col, base;
+    if (j < hcf) {
+        pos = pf; col = j; base = pf * hcf;
+    } else if (j < hcf + hch) {
+        pos = ph; col = j - hcf; base = a.ppf * hcf + ph * hch;
+    } else {
+        pos = pw; col = j - hcf - hch; base = a.ppf * hcf + a.pph * hch + pw * hcw;
+    }
+    if (a.use_table) return tab[base + col];
+    float s, c;
+    turn_sincos((uint32_t)pos, gq[j], &s, &c);
+    return make_float2(c, s);
+}
+
+// Scale by r * weight, rotate the thread's 8 pairs, convert, store one slot.
+// Channel pairs travel as float2 so that the scaling (and the NeoX rotation,
+// whose partners sit in the two vectors) use the packed fp32x2 instructions.
+template <int D, bool NEOX, bool FP8>
+__device__ __forceinline__ void apply_slot(const uint4& va, const uint4& vb, const uint4& wva,
+                                           const uint4& wvb, bool norm, float r,
+                                           const float (&cs)[8], const float (&sn)[8],
+                                           uint8_t* out_head, int l, float scale) {
+    constexpr int L = D / 16;
+    float2 xa[4] = {bf16x2_to_f2(va.x), bf16x2_to_f2(va.y), bf16x2_to_f2(va.z),
+                    bf16x2_to_f2(va.w)};
+    float2 xb[4] = {bf16x2_to_f2(vb.x), bf16x2_to_f2(vb.y), bf16x2_to_f2(vb.z),
+                    bf16x2_to_f2(vb.w)};
+    if (norm) {
+        const float2 r2 = make_float2(r, r);
+        const float2 wa[4] = {bf16x2_to_f2(wva.x), bf16x2_to_f2(wva.y), bf16x2_to_f2(wva.z),
+                              bf16x2_to_f2(wva.w)};
+        const float2 wb[4] = {bf16x2_to_f2(wvb.x), bf16x2_to_f2(wvb.y), bf16x2_to_f2(wvb.z),
+                              bf16x2_to_f2(wvb.w)};
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const int j = NEOX ? 8 * l + k : (k < 4 ? 4 * l + k : 4 * (l + L) + (k - 4));
-        if (j < hcf) {
-            pax[k] = 0; pcol[k] = j;
-        } else if (j < hcf + hch) {
-            pax[k] = 1; pcol[k] = j - hcf;
-        } else {
-            pax[k] = 2; pcol[k] = j - hcf - hch;
+        for (int m = 0; m < 4; ++m) {
+            xa[m] = __fmul2_rn(__fmul2_rn(xa[m], r2), wa[m]);
+            xb[m] = __fmul2_rn(__fmul2_rn(xb[m], r2), wb[m]);
         }
     }
+    float2 oa[4], ob[4];
+    if constexpr (NEOX) {
+        // channel e of vector a pairs with channel e of vector b, slot e
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float2 c = make_float2(cs[2 * m], cs[2 * m + 1]);
+            const float2 sv = make_float2(sn[2 * m], sn[2 * m + 1]);
+            const float2 nsv = make_float2(-sn[2 * m], -sn[2 * m + 1]);
+            oa[m] = __ffma2_rn(xa[m], c, __fmul2_rn(xb[m], nsv));
+            ob[m] = __ffma2_rn(xb[m], c, __fmul2_rn(xa[m], sv));
+        }
+    } else {
+        // channels (2m, 2m+1) of a vector pair up, slot m (vector a) or 4+m (b)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            oa[m].x = xa[m].x * cs[m] - xa[m].y * sn[m];
+            oa[m].y = xa[m].y * cs[m] + xa[m].x * sn[m];
+            ob[m].x = xb[m].x * cs[4 + m] - xb[m].y * sn[4 + m];
+            ob[m].y = xb[m].y * cs[4 + m] + xb[m].x * sn[4 + m];
+        }
+    }
+    if constexpr (FP8) {
+        const float fa[8] = {oa[0].x, oa[0].y, oa[1].x, oa[1].y, oa[2].x, oa[2].y, oa[3].x, oa[3].y};
+        const float fb[8] = {ob[0].x, ob[0].y, ob[1].x, ob[1].y, ob[2].x, ob[2].y, ob[3].x, ob[3].y};
+        uint8_t* p = out_head + 8 * l;
+        st_v2(p, pack8_e4m3(fa, scale));
+        st_v2(p + 8 * L, pack8_e4m3(fb, scale));
+    } else {
+        uint8_t* p = out_head + 16 * l;
+        st_v4(p, make_uint4(f2_to_bf16x2(oa[0]), f2_to_bf16x2(oa[1]), f2_to_bf16x2(oa[2]),
+                            f2_to_bf16x2(oa[3])));
+        st_v4(p + 16 * L, make_uint4(f2_to_bf16x2(ob[0]), f2_to_bf16x2(ob[1]),
+                                     f2_to_bf16x2(ob[2]), f2_to_bf16x2(ob[3])));
+    }
+}
 
-    const int nq = a.hq * L, nk = a.hk * L, nv = a.hv * VPH;
-    // Weights of this thread's slots stay in registers for the whole kernel.
-    uint4 wqa[S], wqb[S], wka[S], wkb[S];
+// As apply_slot, with the weights of the slot given as fp32 from shared
+// memory: w points at float4 index (h*2 + m)*VPH + v for vector v, half m.
+template <int D, bool NEOX, bool FP8>
+__device__ __forceinline__ void apply_slot_wf(const uint4& va, const uint4& vb,
+                                              const float4* wsm_head, bool norm, float r,
+                                              const float (&cs)[8], const float (&sn)[8],
+                                              uint8_t* out_head, int l, float scale) {
+    constexpr int L = D / 16;
+    constexpr int VPH = D / 8;
+    float2 xa[4] = {bf16x2_to_f2(va.x), bf16x2_to_f2(va.y), bf16x2_to_f2(va.z),
+                    bf16x2_to_f2(va.w)};
+    float2 xb[4] = {bf16x2_to_f2(vb.x), bf16x2_to_f2(vb.y), bf16x2_to_f2(vb.z),
+                    bf16x2_to_f2(vb.w)};
+    if (norm) {
+        const float2 r2 = make_float2(r, r);
+        const float4 a0 = wsm_head[l], a1 = wsm_head[VPH + l];
+        const float4 b0 = wsm_head[l + L], b1 = wsm_head[VPH + l + L];
+        const float2 wa[4] = {make_float2(a0.x, a0.y), make_float2(a0.z, a0.w),
+                              make_float2(a1.x, a1.y), make_float2(a1.z, a1.w)};
+        const float2 wb[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w),
+                              make_float2(b1.x, b1.y), make_float2(b1.z, b1.w)};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            xa[m] = __fmul2_rn(__fmul2_rn(xa[m], r2), wa[m]);
+            xb[m] = __fmul2_rn(__fmul2_rn(xb[m], r2), wb[m]);
+        }
+    }
+    float2 oa[4], ob[4];
+    if constexpr (NEOX) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float2 c = make_float2(cs[2 * m], cs[2 * m + 1]);
+            const float2 sv = make_float2(sn[2 * m], sn[2 * m + 1]);
+            const float2 nsv = make_float2(-sn[2 * m], -sn[2 * m + 1]);
+            oa[m] = __ffma2_rn(xa[m], c, __fmul2_rn(xb[m], nsv));
+            ob[m] = __ffma2_rn(xb[m], c, __fmul2_rn(xa[m], sv));
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            oa[m].x = xa[m].x * cs[m] - xa[m].y * sn[m];
+            oa[m].y = xa[m].y * cs[m] + xa[m].x * sn[m];
+            ob[m].x = xb[m].x * cs[4 + m] - xb[m].y * sn[4 + m];
+            ob[m].y = xb[m].y * cs[4 + m] + xb[m].x * sn[4 + m];
+        }
+    }
+    if constexpr (FP8) {
+        const float fa[8] = {oa[0].x, oa[0].y, oa[1].x, oa[1].y, oa[2].x, oa[2].y, oa[3].x, oa[3].y};
+        const float fb[8] = {ob[0].x, ob[0].y, ob[1].x, ob[1].y, ob[2].x, ob[2].y, ob[3].x, ob[3].y};
+        uint8_t* p = out_head + 8 * l;
+        st_v2(p, pack8_e4m3(fa, scale));
+        st_v2(p + 8 * L, pack8_e4m3(fb, scale));
+    } else {
+        uint8_t* p = out_head + 16 * l;
+        st_v4(p, make_uint4(f2_to_bf16x2(oa[0]), f2_to_bf16x2(oa[1]), f2_to_bf16x2(oa[2]),
+                            f2_to_bf16x2(oa[3])));
+        st_v4(p + 16 * L, make_uint4(f2_to_bf16x2(ob[0]), f2_to_bf16x2(ob[1]),
+                                     f2_to_bf16x2(ob[2]), f2_to_bf16x2(ob[3])));
+    }
+}
+
+// Sum of squares of the 16 channels of a vector pair, packed.
+__device__ __forceinline__ float2 ssq_pair(const uint4& va, const uint4& vb, float2 acc) {
+    const uint32_t w[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const float2 x = bf16x2_to_f2(w[m]);
+        acc = __ffma2_rn(x, x, acc);
+    }
+    return acc;
+}
+
+// Pair slots of vector pair (l, l + D/16): NeoX -> 8l..8l+7; interleaved ->
+// 4l..4l+3 and 4(l + D/16)..+3.
+template <int D, bool NEOX>
+__device__ __forceinline__ int slot_of(int l, int k) {
+    constexpr int L = D / 16;
+    return NEOX ? 8 * l + k : (k < 4 ? 4 * l + k : 4 * (l + L) + (k - 4));
+}
+
+template <int S>
+__device__ __forceinline__ void load_weights(const Rope3DArgs& a, int VPH, int L, int l, int tid,
+                                             int B, uint4 (&wqa)[S], uint4 (&wqb)[S],
+                                             uint4 (&wka)[S], uint4 (&wkb)[S]) {
+    const int nq = a.hq * L, nk = a.hk * L;
+    const bool norm = a.is_qk_norm != 0;
 #pragma unroll
     for (int i = 0; i < S; ++i) {
         const int slot = tid + i * B;
         const uint4 one = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
         wqa[i] = wqb[i] = wka[i] = wkb[i] = one;
         if (norm && slot < nq) {
-            const int h = slot / L;
-            const uint4* w = reinterpret_cast<const uint4*>(a.q_weight) + h * VPH + l;
+            const uint4* w = reinterpret_cast<const uint4*>(a.q_weight) + (slot / L) * VPH + l;
             wqa[i] = w[0]; wqb[i] = w[L];
         }
         if (norm && slot < nk) {
-            const int h = slot / L;
-            const uint4* w = reinterpret_cast<const uint4*>(a.k_weight) + h * VPH + l;
+            const uint4* w = reinterpret_cast<const uint4*>(a.k_weight) + (slot / L) * VPH + l;
             wka[i] = w[0]; wkb[i] = w[L];
         }
     }
+}
+
+// ---------------------------------------------------------------------------
+// Pipelined kernel: G token pipelines per CTA, sharing the angle table and
+// the fp32 weights.
+// ---------------------------------------------------------------------------
+constexpr int kCsPitch = 20;  // floats per l-row of the staged cos/sin (16 + pad)
+constexpr int kMaxGroups = 15;
+
+// Shared-memory layout of the pipelined kernel, in bytes from the base.
+struct MgLayout {
+    int ring, full, cst, red, abort, wts, gq, tab, total;
+};
+
+__host__ __device__ inline MgLayout mg_layout(int D, int groups, int stages, int row_bytes,
+                                              int weight_floats, int table_bytes) {
+    MgLayout o;
+    const int L = D / 16, HALF = D / 2;
+    o.ring = 0;
+    o.full = groups * stages * row_bytes;
+    o.cst = (o.full + 8 * groups * stages + 15) & ~15;
+    o.red = o.cst + groups * 2 * L * kCsPitch * 4;
+    o.abort = o.red + groups * 64 * 8;
+    o.wts = o.abort + 16;
+    o.gq = o.wts + weight_floats * 4;
+    o.tab = o.gq + HALF * 8;
+    o.total = o.tab + table_bytes;
+    return o;
+}
+
+template <int D, bool NEOX, bool FP8, int S>
+__global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
+    constexpr int L = D / 16;
+    constexpr int VPH = D / 8;
+    constexpr int HALF = D / 2;
+    constexpr int OUTB = FP8 ? 1 : 2;
+
+    const int G = a.groups;
+    const int Bg = blockDim.x / G;  // threads per group, a multiple of 32
+    const int row_bytes = (a.hq + a.hk + a.hv) * D * 2;
+    const int stages = a.stages;
+    const bool norm = a.is_qk_norm != 0;
+    const MgLayout lay = mg_layout(D, G, stages, row_bytes, norm ? (a.hq + a.hk) * D : 0,
+                                   a.use_table ? a.table_entries * 8 : 0);
+    extern __shared__ __align__(128) unsigned char smem[];
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + lay.abort);
+    float4* wsm = reinterpret_cast<float4*>(smem + lay.wts);
+    uint64_t* gq = reinterpret_cast<uint64_t*>(smem + lay.gq);
+    float2* tab = reinterpret_cast<float2*>(smem + lay.tab);
+
+    const int tid = threadIdx.x;
+    const int g = tid / Bg;
+    const int ctid = tid - g * Bg;
+    unsigned char* ring = smem + lay.ring + (size_t)g * stages * row_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.full) + g * stages;
+    float* cst = reinterpret_cast<float*>(smem + lay.cst) + g * 2 * L * kCsPitch;
+    float2* red = reinterpret_cast<float2*>(smem + lay.red) + g * 64;
+
+    const int64_t NP = (int64_t)gridDim.x * G;  // pipelines in the grid
+    const uint32_t tx = (uint32_t)row_bytes + a.stall_tx_bytes;
+    const int vbytes = a.hv * D * 2;
+    const bool v_bulk = a.v_bulk && vbytes > 0;
+    const size_t v_off = (size_t)(a.hq + a.hk) * D * 2;  // V inside a row
+
+    if (tid == 0) {
+        for (int q = 0; q < G * stages; ++q)
+            mbar_init(reinterpret_cast<uint64_t*>(smem + lay.full) + q, 1);
+        *abort_flag = 0u;
+        fence_mbar_init();
+        // First `stages` rows of every pipeline.
+        for (int q = 0; q < G; ++q) {
+            const int64_t p = (int64_t)blockIdx.x * G + q;
+            unsigned char* rq = smem + lay.ring + (size_t)q * stages * row_bytes;
+            uint64_t* fq = reinterpret_cast<uint64_t*>(smem + lay.full) + q * stages;
+            for (int i = 0; i < stages && p + i * NP < a.num_tokens; ++i) {
+                mbar_arrive_expect_tx(&fq[i], tx);
+                bulk_load(rq + (size_t)i * row_bytes, a.qkv + (p + i * NP) * row_bytes,
+                          row_bytes, &fq[i]);
+            }
+        }
+    }
+    if (norm) {
+        // fp32 weights, float4 index (h*2 + m)*VPH + v for channels 8v+4m..+3 of head h.
+        const int nq4 = a.hq * VPH * 2, n4 = (a.hq + a.hk) * VPH * 2;
+        for (int q = tid; q < n4; q += blockDim.x) {
+            const bool isk = q >= nq4;
+            const int r = isk ? q - nq4 : q;
+            const int h = r / (2 * VPH), m = (r / VPH) & 1, v = r % VPH;
+            const uint2 w = reinterpret_cast<const uint2*>(isk ? a.k_weight : a.q_weight)
+                [((size_t)h * VPH + v) * 2 + m];
+            wsm[q] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+        }
+    }
+    setup_angles<D>(a, gq, tab);
+    __syncthreads();
+
+    // ------------------------------ one pipeline ------------------------------
+    const int64_t p = (int64_t)blockIdx.x * G + g;
+    const int64_t n_local = p < a.num_tokens ? (a.num_tokens - 1 - p) / NP + 1 : 0;
+    const int lane = tid & 31, cwarp = ctid >> 5, nwarps = Bg >> 5;
+    const int l = ctid % L;
+    const int nq = a.hq * L, nk = a.hk * L, nv = a.hv * VPH;
+
+    // Patch of the current token, stepped by the pipeline stride without division.
+    const int hw = a.pph * a.ppw;
+    const int P = a.ppf * hw;
+    int pf, ph, pw, df, dh, dw;
+    {
+        const int s0 = (int)((p + a.pos_offset) % P);
+        pf = s0 / hw; ph = (s0 - pf * hw) / a.ppw; pw = s0 - pf * hw - ph * a.ppw;
+        const int st = (int)(NP % P);
+        df = st / hw; dh = (st - df * hw) / a.ppw; dw = st - df * hw - dh * a.ppw;
+    }
+    // Pair slot this thread stages each token (spread evenly over the warps).
+    const int stage_every = (Bg % HALF == 0) ? Bg / HALF : 0;
+    const int my_j = stage_every ? (ctid % stage_every == 0 ? ctid / stage_every : -1) : -1;
+    const float inv_nq = 1.0f / (float)(a.hq * D > 0 ? a.hq * D : 1);
+    const float inv_nk = 1.0f / (float)(a.hk * D > 0 ? a.hk * D : 1);
+    const int vout_bytes = a.hv * D * OUTB;
+
+    int64_t i = 0;
+    bool aborted = false;
+    for (; i < n_local; ++i) {
+        const int stage = (int)(i % stages);
+        const int parity = (int)(i & 1);
+        const int64_t t = p + i * NP;
+        const bool ok = mbar_wait_abortable(&full[stage], (uint32_t)((i / stages) & 1),
+                                            a.wait_limit_ns, abort_flag);
+        const unsigned char* row = ring + (size_t)stage * row_bytes;
+        if (ctid == 0 && ok && v_bulk) {
+            bulk_store(a.v_out + t * vbytes, row + v_off, (uint32_t)vbytes);
+            bulk_commit();
+        }
+        float2 sq2 = make_float2(0.0f, 0.0f), sk2 = make_float2(0.0f, 0.0f);
+        if (ok) {
+            if (norm) {
+#pragma unroll
+                for (int k = 0; k < S; ++k) {
+                    const int slot = ctid + k * Bg;
+                    const int h = slot / L;
+                    if (slot < nq) {
+                        const uint4* q4 = reinterpret_cast<const uint4*>(row) + h * VPH + l;
+                        sq2 = ssq_pair(q4[0], q4[L], sq2);
+                    }
+                    if (slot < nk) {
+                        const uint4* k4 = reinterpret_cast<const uint4*>(row) + (a.hq + h) * VPH + l;
+                        sk2 = ssq_pair(k4[0], k4[L], sk2);
+                    }
+                }
+            }
+            if (!v_bulk) {
+                const unsigned char* vrow = row + v_off;
+                uint8_t* vout = a.v_out + t * vout_bytes;
+                for (int vi = ctid; vi < nv; vi += Bg) {
+                    const uint4 v = reinterpret_cast<const uint4*>(vrow)[vi];
+                    if constexpr (FP8) {
+                        float f[8];
+                        unpack8(v, f);
+                        st_v2(vout + (size_t)vi * 8, pack8_e4m3(f, a.v_scale));
+                    } else {
+                        st_v4(vout + (size_t)vi * 16, v);
+                    }
+                }
+            }
+        }
+        // This token's cos/sin, staged per l-row: [c_0..c_7][s_0..s_7][pad].
+        {
+            float* cp = cst + parity * L * kCsPitch;
+            for (int j = stage_every ? my_j : ctid; j >= 0 && j < HALF;
+                 j += stage_every ? HALF : Bg) {
+                int rl, k;
+                if (NEOX) {
+                    rl = j >> 3; k = j & 7;
+                } else if (j < 4 * L) {
+                    rl = j >> 2; k = j & 3;
+                } else {
+                    rl = (j - 4 * L) >> 2; k = 4 + ((j - 4 * L) & 3);
+                }
+                const float2 v = pair_cos_sin(a, gq, tab, j, pf, ph, pw);
+                cp[rl * kCsPitch + k] = v.x;
+                cp[rl * kCsPitch + 8 + k] = v.y;
+            }
+        }
+        if (norm) {
+            const float sq = warp_sum(sq2.x + sq2.y);
+            const float sk = warp_sum(sk2.x + sk2.y);
+            if (lane == 0) red[parity * 32 + cwarp] = make_float2(sq, sk);
+        }
+        if (named_barrier_or(1 + g, Bg, !ok)) {
+            aborted = true;
+            if (ctid == 0) *abort_flag = 1u;
+            break;
+        }
+        // Every thread of the group is past token i-1: refill its buffer.
+        if (ctid == 0 && i >= 1 && i - 1 + stages < n_local) {
+            const int ps = (int)((i - 1) % stages);
+            if (v_bulk) bulk_wait_read_all();
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&full[ps], tx);
+            bulk_load(ring + (size_t)ps * row_bytes, a.qkv + (t - NP + stages * NP) * row_bytes,
+                      row_bytes, &full[ps]);
+        }
+        pw += dw;
+        ph += dh + (pw >= a.ppw ? 1 : 0);
+        pw -= pw >= a.ppw ? a.ppw : 0;
+        pf += df + (ph >= a.pph ? 1 : 0);
+        ph -= ph >= a.pph ? a.pph : 0;
+        pf -= pf >= a.ppf ? a.ppf : 0;
+
+        float rq = 1.0f, rk = 1.0f;
+        if (norm) {
+            float tq = 0.0f, tk = 0.0f;
+            for (int w = 0; w < nwarps; ++w) {
+                const float2 v = red[parity * 32 + w];
+                tq += v.x; tk += v.y;
+            }
+            rq = rsqrtf(tq * inv_nq + a.eps);
+            rk = rsqrtf(tk * inv_nk + a.eps);
+        }
+        float cs[8], sn[8];
+        {
+            const float4* cp = reinterpret_cast<const float4*>(cst + (parity * L + l) * kCsPitch);
+            const float4 c0 = cp[0], c1 = cp[1], s0 = cp[2], s1 = cp[3];
+            cs[0] = c0.x; cs[1] = c0.y; cs[2] = c0.z; cs[3] = c0.w;
+            cs[4] = c1.x; cs[5] = c1.y; cs[6] = c1.z; cs[7] = c1.w;
+            sn[0] = s0.x; sn[1] = s0.y; sn[2] = s0.z; sn[3] = s0.w;
+            sn[4] = s1.x; sn[5] = s1.y; sn[6] = s1.z; sn[7] = s1.w;
+        }
+#pragma unroll
+        for (int k = 0; k < S; ++k) {
+            const int slot = ctid + k * Bg;
+            const int h = slot / L;
+            if (slot < nq) {
+                const uint4* q4 = reinterpret_cast<const uint4*>(row) + h * VPH + l;
+                apply_slot_wf<D, NEOX, FP8>(q4[0], q4[L], wsm + h * 2 * VPH, norm, rq, cs, sn,
+                                            a.q_out + (t * a.hq + h) * D * OUTB, l, a.q_scale);
+            }
+            if (slot < nk) {
+                const uint4* k4 = reinterpret_cast<const uint4*>(row) + (a.hq + h) * VPH + l;
+                apply_slot_wf<D, NEOX, FP8>(k4[0], k4[L], wsm + (a.hq + h) * 2 * VPH, norm, rk,
+                                            cs, sn, a.k_out + (t * a.hk + h) * D * OUTB, l,
+                                            a.q_scale);
+            }
+        }
+    }
+    if (ctid == 0) {
+        if (aborted || *abort_flag) {
+            atomicOr(&g_rope3d_status, 1u);
+            // Drain this pipeline's loads that may still be in flight (bounded):
+            // tokens i .. i+stages-2 (refills run one token behind), or the
+            // whole first ring if nothing was consumed yet.
+            const int64_t hi = i == 0 ? stages : i + stages - 1;
+            for (int64_t j = i; j < n_local && j < hi; ++j)
+                mbar_wait_bounded(&full[j % stages], (uint32_t)((j / stages) & 1),
+                                  a.wait_limit_ns);
+        }
+        if (v_bulk) bulk_wait_all();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Fallback kernel: 128-bit loads into registers, no ring.
+// ---------------------------------------------------------------------------
+template <int D, bool NEOX, bool FP8, int S>
+__global__ void __launch_bounds__(kMaxBlock) rope3d_reg_kernel(const Rope3DArgs a) {
+    constexpr int L = D / 16;
+    constexpr int VPH = D / 8;
+    constexpr int HALF = D / 2;
+    constexpr int OUTB = FP8 ? 1 : 2;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    float2* cst = reinterpret_cast<float2*>(smem);     // [2][HALF]
+    float2* red = cst + 2 * HALF;                      // [2][32]
+    uint64_t* gq = reinterpret_cast<uint64_t*>(red + 64);
+    float2* tab = reinterpret_cast<float2*>(gq + HALF);
+
+    const int tid = threadIdx.x;
+    const int B = blockDim.x;
+    const int lane = tid & 31, warp = tid >> 5, nwarps = B >> 5;
+    const int l = tid % L;
+    const bool norm = a.is_qk_norm != 0;
+    const int nq = a.hq * L, nk = a.hk * L, nv = a.hv * VPH;
+
+    setup_angles<D>(a, gq, tab);
+    uint4 wqa[S], wqb[S], wka[S], wkb[S];
+    load_weights<S>(a, VPH, L, l, tid, B, wqa, wqb, wka, wkb);
+    __syncthreads();
 
     const int64_t row_bytes = (int64_t)(a.hq + a.hk + a.hv) * D * 2;
     const int hw = a.pph * a.ppw;
-    const int64_t P = (int64_t)a.ppf * hw;
+    const int P = a.ppf * hw;
+    const int pstep = (int)((int64_t)gridDim.x % P);
+    int s_pos = (int)(((int64_t)blockIdx.x + a.pos_offset) % P);
     const float inv_nq = 1.0f / (float)(a.hq * D > 0 ? a.hq * D : 1);
     const float inv_nk = 1.0f / (float)(a.hk * D > 0 ? a.hk * D : 1);
 
     int parity = 0;
     for (int64_t t = blockIdx.x; t < a.num_tokens; t += gridDim.x, parity ^= 1) {
         const uint8_t* row = a.qkv + t * row_bytes;
-        uint4 qa[S], qb[S], ka[S], kb[S], vv[SV];
+        uint4 qa[S], qb[S], ka[S], kb[S];
 #pragma unroll
-        for (int i = 0; i < S; ++i) {
-            const int slot = tid + i * B;
+        for (int k = 0; k < S; ++k) {
+            const int slot = tid + k * B;
             const int h = slot / L;
             if (slot < nq) {
                 const uint8_t* p = row + (size_t)(h * VPH + l) * 16;
-                qa[i] = ld_nc_v4(p); qb[i] = ld_nc_v4(p + L * 16);
+                qa[k] = ld_nc_v4(p); qb[k] = ld_nc_v4(p + L * 16);
             }
             if (slot < nk) {
                 const uint8_t* p = row + (size_t)((a.hq + h) * VPH + l) * 16;
-                ka[i] = ld_nc_v4(p); kb[i] = ld_nc_v4(p + L * 16);
+                ka[k] = ld_nc_v4(p); kb[k] = ld_nc_v4(p + L * 16);
             }
         }
         const uint8_t* vrow = row + (size_t)(a.hq + a.hk) * VPH * 16;
-#pragma unroll
-        for (int i = 0; i < SV; ++i) {
-            const int vi = tid + i * B;
-            if (vi < nv) vv[i] = ld_nc_v4(vrow + (size_t)vi * 16);
-        }
-
-        // Patch coordinates of this token.
-        const int64_t s64 = (t + a.pos_offset) % P;
-        const int s = (int)s64;
-        const int pf = s / hw;
-        const int rem = s - pf * hw;
-        const int ph = rem / a.ppw;
-        const int pw = rem - ph * a.ppw;
-
-        // V: bit copy (bf16) or E4M3(v * v_scale).
         uint8_t* vout = a.v_out + t * (int64_t)nv * 8 * OUTB;
-#pragma unroll
-        for (int i = 0; i < SV; ++i) {
-            const int vi = tid + i * B;
-            if (vi < nv) {
-                if constexpr (FP8) {
-                    float f[8];
-                    unpack8(vv[i], f);
-                    st_v2(vout + (size_t)vi * 8, pack8_e4m3(f, a.v_scale));
-                } else {
-                    st_v4(vout + (size_t)vi * 16, vv[i]);
-                }
-            }
-        }
-        for (int vi = tid + SV * B; vi < nv; vi += B) {  // heads beyond the up-front batch
+        for (int vi = tid; vi < nv; vi += B) {
             const uint4 v = ld_nc_v4(vrow + (size_t)vi * 16);
             if constexpr (FP8) {
                 float f[8];
@@ -183,159 +596,156 @@ __global__ void __launch_bounds__(kMaxBlock) rope3d_kernel(const Rope3DArgs a) {
                 st_v4(vout + (size_t)vi * 16, v);
             }
         }
-
-        // Across-heads RMS of Q and of K.
+        {
+            const int pf = s_pos / hw;
+            const int rem = s_pos - pf * hw;
+            const int ph = rem / a.ppw;
+            const int pw = rem - ph * a.ppw;
+            for (int j = tid; j < HALF; j += B)
+                cst[parity * HALF + j] = pair_cos_sin(a, gq, tab, j, pf, ph, pw);
+        }
+        s_pos += pstep;
+        if (s_pos >= P) s_pos -= P;
+        if (norm) {
+            float2 sq2 = make_float2(0.0f, 0.0f), sk2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int k = 0; k < S; ++k) {
+                const int slot = tid + k * B;
+                if (slot < nq) sq2 = ssq_pair(qa[k], qb[k], sq2);
+                if (slot < nk) sk2 = ssq_pair(ka[k], kb[k], sk2);
+            }
+            const float sq = warp_sum(sq2.x + sq2.y);
+            const float sk = warp_sum(sk2.x + sk2.y);
+            if (lane == 0) red[parity * 32 + warp] = make_float2(sq, sk);
+        }
+        __syncthreads();
         float rq = 1.0f, rk = 1.0f;
         if (norm) {
-            float sq = 0.0f, sk = 0.0f;
-#pragma unroll
-            for (int i = 0; i < S; ++i) {
-                const int slot = tid + i * B;
-                if (slot < nq) {
-                    float fa[8], fb[8];
-                    unpack8(qa[i], fa); unpack8(qb[i], fb);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) sq += fa[e] * fa[e] + fb[e] * fb[e];
-                }
-                if (slot < nk) {
-                    float fa[8], fb[8];
-                    unpack8(ka[i], fa); unpack8(kb[i], fb);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) sk += fa[e] * fa[e] + fb[e] * fb[e];
-                }
-            }
-            sq = warp_sum(sq);
-            sk = warp_sum(sk);
-            float2* rb = red + parity * 32;
-            if (lane == 0) rb[warp] = make_float2(sq, sk);
-            __syncthreads();
             float tq = 0.0f, tk = 0.0f;
             for (int w = 0; w < nwarps; ++w) {
-                const float2 v = rb[w];
+                const float2 v = red[parity * 32 + w];
                 tq += v.x; tk += v.y;
             }
             rq = rsqrtf(tq * inv_nq + a.eps);
             rk = rsqrtf(tk * inv_nk + a.eps);
         }
-
-        // cos/sin of this thread's 8 pairs.
         float cs[8], sn[8];
-        if (a.use_table) {
-            const int r0 = pf * hcf, r1 = nf + ph * hch, r2 = nf + nh + pw * hcw;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int base = pax[k] == 0 ? r0 : (pax[k] == 1 ? r1 : r2);
-                const float2 v = tab[base + pcol[k]];
-                cs[k] = v.x; sn[k] = v.y;
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int j = NEOX ? 8 * l + k : (k < 4 ? 4 * l + k : 4 * (l + L) + (k - 4));
-                const int pos = pax[k] == 0 ? pf : (pax[k] == 1 ? ph : pw);
-                turn_sincos((uint32_t)pos, gq[j], &sn[k], &cs[k]);
-            }
+        for (int k = 0; k < 8; ++k) {
+            const float2 v = cst[parity * HALF + slot_of<D, NEOX>(l, k)];
+            cs[k] = v.x; sn[k] = v.y;
         }
-
-        // Scale, rotate, convert, store: Q then K.
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int nslot = part ? nk : nq;
-            const float r = part ? rk : rq;
-            const int H = part ? a.hk : a.hq;
-            uint8_t* out = (part ? a.k_out : a.q_out) + t * (int64_t)H * D * OUTB;
-            const float scale = a.q_scale;
-#pragma unroll
-            for (int i = 0; i < S; ++i) {
-                const int slot = tid + i * B;
-                if (slot >= nslot) continue;
-                const int h = slot / L;
-                float xa[8], xb[8];
-                unpack8(part ? ka[i] : qa[i], xa);
-                unpack8(part ? kb[i] : qb[i], xb);
-                if (norm) {
-                    float wa[8], wb[8];
-                    unpack8(part ? wka[i] : wqa[i], wa);
-                    unpack8(part ? wkb[i] : wqb[i], wb);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        xa[e] = xa[e] * r * wa[e];
-                        xb[e] = xb[e] * r * wb[e];
-                    }
-                }
-                float oa[8], ob[8];
-                if constexpr (NEOX) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        oa[e] = xa[e] * cs[e] - xb[e] * sn[e];
-                        ob[e] = xb[e] * cs[e] + xa[e] * sn[e];
-                    }
-                } else {
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        oa[2 * m] = xa[2 * m] * cs[m] - xa[2 * m + 1] * sn[m];
-                        oa[2 * m + 1] = xa[2 * m + 1] * cs[m] + xa[2 * m] * sn[m];
-                        ob[2 * m] = xb[2 * m] * cs[4 + m] - xb[2 * m + 1] * sn[4 + m];
-                        ob[2 * m + 1] = xb[2 * m + 1] * cs[4 + m] + xb[2 * m] * sn[4 + m];
-                    }
-                }
-                if constexpr (FP8) {
-                    uint8_t* p = out + (size_t)h * D + 8 * l;
-                    st_v2(p, pack8_e4m3(oa, scale));
-                    st_v2(p + 8 * L, pack8_e4m3(ob, scale));
-                } else {
-                    uint8_t* p = out + (size_t)(h * VPH + l) * 16;
-                    st_v4(p, pack8_bf16(oa));
-                    st_v4(p + 16 * L, pack8_bf16(ob));
-                }
-            }
+        for (int k = 0; k < S; ++k) {
+            const int slot = tid + k * B;
+            const int h = slot / L;
+            if (slot < nq)
+                apply_slot<D, NEOX, FP8>(qa[k], qb[k], wqa[k], wqb[k], norm, rq, cs, sn,
+                                         a.q_out + (t * a.hq + h) * D * OUTB, l, a.q_scale);
+            if (slot < nk)
+                apply_slot<D, NEOX, FP8>(ka[k], kb[k], wka[k], wkb[k], norm, rk, cs, sn,
+                                         a.k_out + (t * a.hk + h) * D * OUTB, l, a.q_scale);
         }
     }
 }
 
-template <int D, bool NEOX, bool FP8, int S>
-cudaError_t run(const Rope3DArgs& a, int block, cudaStream_t stream, LaunchInfo* info) {
-    auto kern = rope3d_kernel<D, NEOX, FP8, S>;
-    Rope3DArgs args = a;
-    const int fixed = (D / 2) * 8 + 512;
-    const int table_bytes = a.table_entries * 8;
-    args.use_table = table_bytes <= kMaxTableBytes ? 1 : 0;
-    const int smem = fixed + (args.use_table ? table_bytes : 0);
+int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return sms;
+}
+
+template <typename K>
+cudaError_t launch_grid(K kern, int block, int smem, int64_t tokens, const Rope3DArgs& args,
+                        cudaStream_t stream, int* grid_out) {
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              smem);
         if (e != cudaSuccess) return e;
     }
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block,
-                                                                            smem);
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, smem);
     if (e != cudaSuccess) return e;
-    if (per_sm < 1) per_sm = 1;
-    const int64_t want = (int64_t)sms * per_sm;
-    const int grid = (int)std::min<int64_t>(want, a.num_tokens);
+    const int sms = device_sms();
+    if (sms <= 0) return cudaErrorNoDevice;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int grid = (int)std::min<int64_t>((int64_t)sms * per_sm, tokens);
     kern<<<grid, block, smem, stream>>>(args);
+    *grid_out = grid;
+    return cudaGetLastError();
+}
+
+template <int D, bool NEOX, bool FP8, int S>
+cudaError_t run(const Rope3DArgs& a, int block, cudaStream_t stream, LaunchInfo* info) {
+    constexpr int HALF = D / 2;
+    Rope3DArgs args = a;
+    const int table_bytes = a.table_entries * 8;
+    args.use_table = table_bytes <= kMaxTableBytes ? 1 : 0;
+    const int used_table = args.use_table ? table_bytes : 0;
+    const int row_bytes = (a.hq + a.hk + a.hv) * D * 2;
+    const int weight_floats = a.is_qk_norm ? (a.hq + a.hk) * D : 0;
+    // Pipelines per CTA: as many groups as fit in 24 warps and in shared memory,
+    // each with a ring of 3 row buffers (2 if 3 do not fit even for one group).
+    const int warps = block / 32;
+    int groups = std::max(1, std::min(kMaxGroups, 24 / warps));
+    int stages = 0;
+    for (; groups >= 1; --groups) {
+        for (stages = 3; stages >= 2; --stages) {
+            if (mg_layout(D, groups, stages, row_bytes, weight_floats, used_table).total <=
+                kSmemPerSm - 1024)
+                break;
+        }
+        if (stages >= 2) break;
+    }
+    // Do not start more pipelines than there are tokens.
+    const int sms = device_sms();
+    if (sms <= 0) return cudaErrorNoDevice;
+    while (groups > 1 && (int64_t)sms * (groups - 1) >= a.num_tokens) --groups;
+    int grid = 0, smem = 0, id = 0;
+    cudaError_t e;
+    if (groups >= 1 && stages >= 2) {
+        args.stages = stages;
+        args.groups = groups;
+        args.v_bulk = FP8 ? 0 : 1;
+        if (args.wait_limit_ns == 0) args.wait_limit_ns = 2000000000ull;  // 2 s
+        smem = mg_layout(D, groups, stages, row_bytes, weight_floats, used_table).total;
+        auto kern = rope3d_mg_kernel<D, NEOX, FP8, S>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess) {
+            grid = (int)std::min<int64_t>(sms, (a.num_tokens + groups - 1) / groups);
+            kern<<<grid, block * groups, smem, stream>>>(args);
+            e = cudaGetLastError();
+        }
+        id = 3100;
+        block *= groups;
+    } else {
+        smem = 2 * HALF * 8 + 64 * 8 + HALF * 8 + used_table;
+        e = launch_grid(rope3d_reg_kernel<D, NEOX, FP8, S>, block, smem, a.num_tokens, args,
+                        stream, &grid);
+        id = 3000;
+    }
     if (info) {
         info->grid = grid;
         info->block = block;
         info->smem = smem;
-        info->kernel_id = 3000 + D * 10 + (NEOX ? 1 : 0) * 4 + (FP8 ? 2 : 0) + (S > 1);
+        info->kernel_id = id + D / 64 * 10 + (NEOX ? 4 : 0) + (FP8 ? 2 : 0) + (S > 1);
     }
-    return cudaGetLastError();
+    return e;
 }
 
 template <int D, bool NEOX, bool FP8>
 cudaError_t run_s(const Rope3DArgs& a, cudaStream_t stream, LaunchInfo* info) {
     constexpr int L = D / 16;
-    int slots = std::max(std::max(a.hq, a.hk), 1) * L;
-    const int v_vectors = a.hv * (D / 8);
+    const int slots = std::max(std::max(a.hq, a.hk), 1) * L;
     int S = (slots + kMaxBlock - 1) / kMaxBlock;
     if (S > 4) return cudaErrorInvalidValue;  // rejected earlier by the host checks
     S = S <= 1 ? 1 : (S <= 2 ? 2 : 4);
     int block = ((slots + S - 1) / S + 31) / 32 * 32;
-    // With few Q/K heads, widen the block to cover V in the up-front batch.
-    while (block < kMaxBlock && 2 * S * block < v_vectors && block < 256) block += 32;
+    // With few Q/K heads, widen the block so that V and the per-token cos/sin
+    // have enough threads.
+    const int v_vectors = a.hv * (D / 8);
+    while (block < 256 && (block < v_vectors / 2 || block < D / 2)) block += 32;
     switch (S) {
         case 1: return run<D, NEOX, FP8, 1>(a, block, stream, info);
         case 2: return run<D, NEOX, FP8, 2>(a, block, stream, info);
@@ -364,7 +774,20 @@ cudaError_t launch_rope3d(const Rope3DArgs& a, int head_dim, int neox, int fp8,
     }
 }
 
-// Largest number of Q or K heads the 3D kernel takes for a head size
+cudaError_t read_device_status(uint32_t* out, int clear, cudaStream_t stream) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_rope3d_status, sizeof(uint32_t), 0,
+                                              cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && clear) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_rope3d_status, &zero, sizeof(uint32_t), 0,
+                                    cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    }
+    return e;
+}
+
+// Largest number of Q or K heads the 3D kernels take for a head size
 // (S <= 4 slots per thread at 512 threads).
 int rope3d_max_heads(int head_dim) { return 4 * kMaxBlock / (head_dim / 16); }
 

@@ -188,3 +188,9 @@ def test_python_wrapper_raises_valueerror(L):
         Q.fused_qk_norm_rope(x, x, w, w, tbl[:, :63], 1e-6)
     with pytest.raises(ValueError):
         Q.fused_qk_norm_rope(x.float(), x, w, w, tbl, 1e-6)
+
+
+def test_wait_fault_hook_argument_checks(L):
+    assert L.qknr_test_set_wait_fault(8, 1000) == Q.QKNR_ERR_SHAPE
+    assert L.qknr_test_set_wait_fault(16, 0) == Q.QKNR_ERR_SHAPE
+    assert L.qknr_test_set_wait_fault(0, 0) == Q.QKNR_OK

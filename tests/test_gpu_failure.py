@@ -1,0 +1,52 @@
+"""Failure detection on the GPU without faulting it.
+
+The pipelined 3D kernel bounds every wait on its own bulk copies. The test
+hook makes each ring buffer expect 16 bytes more than its copy delivers (a
+count that nothing completes), with a 20 ms limit: the waits run out, the
+launch abandons its tokens, raises bit 0 of the device status word, drains its
+copies and ends. The context must stay usable: a normal call right after
+gives correct results.
+"""
+import pytest
+import torch
+
+import qk_rmsnorm_rope_qknr_b200 as Q
+from qk_rmsnorm_rope_qknr_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _tiny():
+    w = W.WORKLOADS["tiny3d"]
+    inp = {k: v.cuda() for k, v in W.make_inputs(w).items()}
+    return w, inp
+
+
+def test_device_status_clean_after_normal_runs():
+    w, inp = _tiny()
+    Q.qknr_device_status(clear=True)
+    for _ in range(3):
+        Q.fused_qk_rmsnorm_rope(inp["qkv"], inp["q_weight"], inp["k_weight"], **w.params())
+    assert Q.qknr_device_status() == 0
+
+
+def test_wait_timeout_raises_status_and_context_survives():
+    w, inp = _tiny()
+    good = Q.fused_qk_rmsnorm_rope(inp["qkv"], inp["q_weight"], inp["k_weight"], **w.params())
+    torch.cuda.synchronize()
+    Q.qknr_device_status(clear=True)
+    L = Q.lib()
+    assert L.qknr_test_set_wait_fault(16, 20_000_000) == 0
+    try:
+        outs = [torch.zeros_like(o) for o in good]
+        Q.qknr_rope_3d(inp["qkv"], inp["q_weight"], inp["k_weight"], *outs, **w.params())
+        torch.cuda.synchronize()
+    finally:
+        assert L.qknr_test_set_wait_fault(0, 0) == 0
+    assert Q.qknr_device_status(clear=True) & 1
+    assert Q.qknr_device_status() == 0
+    again = Q.fused_qk_rmsnorm_rope(inp["qkv"], inp["q_weight"], inp["k_weight"], **w.params())
+    torch.cuda.synchronize()
+    for a, b in zip(good, again):
+        assert torch.equal(a, b)
+    assert Q.qknr_device_status() == 0
