@@ -251,7 +251,10 @@ __device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred
     return r != 0;
 }
 
-// Packed fp32 pairs (one instruction for two lanes of math on sm_100).
+// Two-lane fp32 math. On sm_100 these map to the packed fp32x2 instructions.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
 __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
     return make_float2(bf16_lo(w), bf16_hi(w));
 }

@@ -92,6 +92,14 @@ __device__ __forceinline__ void setup_angles(const Rope3DArgs& a, uint64_t* gq, 
     }
 }
 
+// cos/sin of an integer position for a stored frequency, out of line so that
+// the table path carries none of its code.
+__device__ __noinline__ float2 direct_cos_sin(uint32_t pos, uint64_t turns) {
+    float s, c;
+    turn_sincos(pos, turns, &s, &c);
+    return make_float2(c, s);
+}
+
 // cos/sin of pair slot j for patch (pf, ph, pw).
 __device__ __forceinline__ float2 pair_cos_sin(const Rope3DArgs& a, const uint64_t* gq,
                                                const float2* tab, int j, int pf, int ph, int pw) {
@@ -105,9 +113,7 @@ __device__ __forceinline__ float2 pair_cos_sin(const Rope3DArgs& a, const uint64
         pos = pw; col = j - hcf - hch; base = a.ppf * hcf + a.pph * hch + pw * hcw;
     }
     if (a.use_table) return tab[base + col];
-    float s, c;
-    turn_sincos((uint32_t)pos, gq[j], &s, &c);
-    return make_float2(c, s);
+    return direct_cos_sin((uint32_t)pos, gq[j]);
 }
 
 // Scale by r * weight, rotate the thread's 8 pairs, convert, store one slot.
@@ -131,8 +137,8 @@ __device__ __forceinline__ void apply_slot(const uint4& va, const uint4& vb, con
                               bf16x2_to_f2(wvb.w)};
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            xa[m] = __fmul2_rn(__fmul2_rn(xa[m], r2), wa[m]);
-            xb[m] = __fmul2_rn(__fmul2_rn(xb[m], r2), wb[m]);
+            xa[m] = mul2(mul2(xa[m], r2), wa[m]);
+            xb[m] = mul2(mul2(xb[m], r2), wb[m]);
         }
     }
     float2 oa[4], ob[4];
@@ -143,8 +149,8 @@ __device__ __forceinline__ void apply_slot(const uint4& va, const uint4& vb, con
             const float2 c = make_float2(cs[2 * m], cs[2 * m + 1]);
             const float2 sv = make_float2(sn[2 * m], sn[2 * m + 1]);
             const float2 nsv = make_float2(-sn[2 * m], -sn[2 * m + 1]);
-            oa[m] = __ffma2_rn(xa[m], c, __fmul2_rn(xb[m], nsv));
-            ob[m] = __ffma2_rn(xb[m], c, __fmul2_rn(xa[m], sv));
+            oa[m] = fma2(xa[m], c, mul2(xb[m], nsv));
+            ob[m] = fma2(xb[m], c, mul2(xa[m], sv));
         }
     } else {
         // channels (2m, 2m+1) of a vector pair up, slot m (vector a) or 4+m (b)
@@ -194,8 +200,8 @@ __device__ __forceinline__ void apply_slot_wf(const uint4& va, const uint4& vb,
                               make_float2(b1.x, b1.y), make_float2(b1.z, b1.w)};
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            xa[m] = __fmul2_rn(__fmul2_rn(xa[m], r2), wa[m]);
-            xb[m] = __fmul2_rn(__fmul2_rn(xb[m], r2), wb[m]);
+            xa[m] = mul2(mul2(xa[m], r2), wa[m]);
+            xb[m] = mul2(mul2(xb[m], r2), wb[m]);
         }
     }
     float2 oa[4], ob[4];
@@ -205,8 +211,8 @@ __device__ __forceinline__ void apply_slot_wf(const uint4& va, const uint4& vb,
             const float2 c = make_float2(cs[2 * m], cs[2 * m + 1]);
             const float2 sv = make_float2(sn[2 * m], sn[2 * m + 1]);
             const float2 nsv = make_float2(-sn[2 * m], -sn[2 * m + 1]);
-            oa[m] = __ffma2_rn(xa[m], c, __fmul2_rn(xb[m], nsv));
-            ob[m] = __ffma2_rn(xb[m], c, __fmul2_rn(xa[m], sv));
+            oa[m] = fma2(xa[m], c, mul2(xb[m], nsv));
+            ob[m] = fma2(xb[m], c, mul2(xa[m], sv));
         }
     } else {
 #pragma unroll
@@ -238,7 +244,7 @@ __device__ __forceinline__ float2 ssq_pair(const uint4& va, const uint4& vb, flo
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
         const float2 x = bf16x2_to_f2(w[m]);
-        acc = __ffma2_rn(x, x, acc);
+        acc = fma2(x, x, acc);
     }
     return acc;
 }
@@ -364,6 +370,9 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
             wsm[q] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
         }
     }
+    // Partial sums of warps a group does not have stay zero.
+    for (int q = tid; q < G * 64; q += blockDim.x)
+        reinterpret_cast<float2*>(smem + lay.red)[q] = make_float2(0.0f, 0.0f);
     setup_angles<D>(a, gq, tab);
     __syncthreads();
 
@@ -384,21 +393,40 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
         const int st = (int)(NP % P);
         df = st / hw; dh = (st - df * hw) / a.ppw; dw = st - df * hw - dh * a.ppw;
     }
-    // Pair slot this thread stages each token (spread evenly over the warps).
-    const int stage_every = (Bg % HALF == 0) ? Bg / HALF : 0;
-    const int my_j = stage_every ? (ctid % stage_every == 0 ? ctid / stage_every : -1) : -1;
+    // Staging: thread ctid < HALF owns pair slot j = ctid each token. Its
+    // destination in the staged cos/sin rows, its axis and its column in the
+    // table are fixed: packed into one word (dst 11 bits, axis 2, column 8).
+    const int hcf = a.cf >> 1, hch = a.ch >> 1, hcw = a.cw >> 1;
+    const int nf = a.ppf * hcf, nh = a.pph * hch;
+    uint32_t stage_code = 0;
+    if (HALF <= Bg && ctid < HALF) {
+        const int j = ctid;
+        int rl, k;
+        if (NEOX) {
+            rl = j >> 3; k = j & 7;
+        } else if (j < 4 * L) {
+            rl = j >> 2; k = j & 3;
+        } else {
+            rl = (j - 4 * L) >> 2; k = 4 + ((j - 4 * L) & 3);
+        }
+        const int axis = j < hcf ? 0 : (j < hcf + hch ? 1 : 2);
+        const int col = axis == 0 ? j : (axis == 1 ? j - hcf : j - hcf - hch);
+        stage_code = (uint32_t)(rl * kCsPitch + k) | ((uint32_t)axis << 11) | ((uint32_t)col << 13);
+    }
     const float inv_nq = 1.0f / (float)(a.hq * D > 0 ? a.hq * D : 1);
     const float inv_nk = 1.0f / (float)(a.hk * D > 0 ? a.hk * D : 1);
     const int vout_bytes = a.hv * D * OUTB;
 
     int64_t i = 0;
     bool aborted = false;
-    for (; i < n_local; ++i) {
-        const int stage = (int)(i % stages);
+    // Ring position of token i (i mod stages), the phase its buffer is in
+    // ((i / stages) mod 2), and the previous token's buffer, kept by counting.
+    int stage = 0, prev_stage = stages - 1;
+    uint32_t phase = 0;
+    int64_t t = p;
+    for (; i < n_local; ++i, t += NP) {
         const int parity = (int)(i & 1);
-        const int64_t t = p + i * NP;
-        const bool ok = mbar_wait_abortable(&full[stage], (uint32_t)((i / stages) & 1),
-                                            a.wait_limit_ns, abort_flag);
+        const bool ok = mbar_wait_abortable(&full[stage], phase, a.wait_limit_ns, abort_flag);
         const unsigned char* row = ring + (size_t)stage * row_bytes;
         if (ctid == 0 && ok && v_bulk) {
             bulk_store(a.v_out + t * vbytes, row + v_off, (uint32_t)vbytes);
@@ -439,19 +467,37 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
         // This token's cos/sin, staged per l-row: [c_0..c_7][s_0..s_7][pad].
         {
             float* cp = cst + parity * L * kCsPitch;
-            for (int j = stage_every ? my_j : ctid; j >= 0 && j < HALF;
-                 j += stage_every ? HALF : Bg) {
-                int rl, k;
-                if (NEOX) {
-                    rl = j >> 3; k = j & 7;
-                } else if (j < 4 * L) {
-                    rl = j >> 2; k = j & 3;
-                } else {
-                    rl = (j - 4 * L) >> 2; k = 4 + ((j - 4 * L) & 3);
+            if (HALF <= Bg) {
+                if (ctid < HALF) {  // whole warps: HALF is a multiple of 32
+                    const int axis = (stage_code >> 11) & 3;
+                    const int col = (int)(stage_code >> 13);
+                    float2 v;
+                    if (a.use_table) {
+                        const int base = axis == 0 ? pf * hcf
+                                                   : (axis == 1 ? nf + ph * hch : nf + nh + pw * hcw);
+                        v = tab[base + col];
+                    } else {
+                        const int pos = axis == 0 ? pf : (axis == 1 ? ph : pw);
+                        v = direct_cos_sin((uint32_t)pos, gq[ctid]);
+                    }
+                    const int dst = (int)(stage_code & 2047);
+                    cp[dst] = v.x;
+                    cp[dst + 8] = v.y;
                 }
-                const float2 v = pair_cos_sin(a, gq, tab, j, pf, ph, pw);
-                cp[rl * kCsPitch + k] = v.x;
-                cp[rl * kCsPitch + 8 + k] = v.y;
+            } else {
+                for (int j = ctid; j < HALF; j += Bg) {
+                    int rl, k;
+                    if (NEOX) {
+                        rl = j >> 3; k = j & 7;
+                    } else if (j < 4 * L) {
+                        rl = j >> 2; k = j & 3;
+                    } else {
+                        rl = (j - 4 * L) >> 2; k = 4 + ((j - 4 * L) & 3);
+                    }
+                    const float2 v = pair_cos_sin(a, gq, tab, j, pf, ph, pw);
+                    cp[rl * kCsPitch + k] = v.x;
+                    cp[rl * kCsPitch + 8 + k] = v.y;
+                }
             }
         }
         if (norm) {
@@ -466,12 +512,16 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
         }
         // Every thread of the group is past token i-1: refill its buffer.
         if (ctid == 0 && i >= 1 && i - 1 + stages < n_local) {
-            const int ps = (int)((i - 1) % stages);
             if (v_bulk) bulk_wait_read_all();
             fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&full[ps], tx);
-            bulk_load(ring + (size_t)ps * row_bytes, a.qkv + (t - NP + stages * NP) * row_bytes,
-                      row_bytes, &full[ps]);
+            mbar_arrive_expect_tx(&full[prev_stage], tx);
+            bulk_load(ring + (size_t)prev_stage * row_bytes,
+                      a.qkv + (t + (stages - 1) * NP) * row_bytes, row_bytes, &full[prev_stage]);
+        }
+        prev_stage = stage;
+        if (++stage == stages) {
+            stage = 0;
+            phase ^= 1u;
         }
         pw += dw;
         ph += dh + (pw >= a.ppw ? 1 : 0);
@@ -482,13 +532,15 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
 
         float rq = 1.0f, rk = 1.0f;
         if (norm) {
-            float tq = 0.0f, tk = 0.0f;
-            for (int w = 0; w < nwarps; ++w) {
-                const float2 v = red[parity * 32 + w];
-                tq += v.x; tk += v.y;
+            // (sum Q^2, sum K^2) partials of the warps, two warps per 16-byte read
+            const float4* r4 = reinterpret_cast<const float4*>(red + parity * 32);
+            float4 acc = r4[0];
+            for (int w = 1; w < (nwarps + 1) >> 1; ++w) {
+                const float4 v = r4[w];
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
             }
-            rq = rsqrtf(tq * inv_nq + a.eps);
-            rk = rsqrtf(tk * inv_nk + a.eps);
+            rq = rsqrtf((acc.x + acc.z) * inv_nq + a.eps);
+            rk = rsqrtf((acc.y + acc.w) * inv_nk + a.eps);
         }
         float cs[8], sn[8];
         {
