@@ -74,6 +74,10 @@ __device__ __forceinline__ uint2 pack8_e4m3(const float (&f)[8], float scale) {
                       pack_e4m3x4(f[4] * scale, f[5] * scale, f[6] * scale, f[7] * scale));
 }
 
+__device__ __forceinline__ uint2 pack8_e4m3_unscaled(const float (&f)[8]) {
+    return make_uint2(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]));
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -249,6 +253,11 @@ __device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred
         : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
         : "memory");
     return r != 0;
+}
+
+// Plain barrier over the first `nthreads` threads at named barrier `id`.
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Two-lane fp32 math. On sm_100 these map to the packed fp32x2 instructions.

@@ -179,11 +179,13 @@ __device__ __forceinline__ void apply_slot(const uint4& va, const uint4& vb, con
 
 // As apply_slot, with the weights of the slot given as fp32 from shared
 // memory: w points at float4 index (h*2 + m)*VPH + v for vector v, half m.
+// For E4M3 output the caller has already folded the output scale into r (or,
+// without the norm, into cos/sin).
 template <int D, bool NEOX, bool FP8>
 __device__ __forceinline__ void apply_slot_wf(const uint4& va, const uint4& vb,
                                               const float4* wsm_head, bool norm, float r,
                                               const float (&cs)[8], const float (&sn)[8],
-                                              uint8_t* out_head, int l, float scale) {
+                                              uint8_t* out_head, int l) {
     constexpr int L = D / 16;
     constexpr int VPH = D / 8;
     float2 xa[4] = {bf16x2_to_f2(va.x), bf16x2_to_f2(va.y), bf16x2_to_f2(va.z),
@@ -227,8 +229,8 @@ __device__ __forceinline__ void apply_slot_wf(const uint4& va, const uint4& vb,
         const float fa[8] = {oa[0].x, oa[0].y, oa[1].x, oa[1].y, oa[2].x, oa[2].y, oa[3].x, oa[3].y};
         const float fb[8] = {ob[0].x, ob[0].y, ob[1].x, ob[1].y, ob[2].x, ob[2].y, ob[3].x, ob[3].y};
         uint8_t* p = out_head + 8 * l;
-        st_v2(p, pack8_e4m3(fa, scale));
-        st_v2(p + 8 * L, pack8_e4m3(fb, scale));
+        st_v2(p, pack8_e4m3_unscaled(fa));
+        st_v2(p + 8 * L, pack8_e4m3_unscaled(fb));
     } else {
         uint8_t* p = out_head + 16 * l;
         st_v4(p, make_uint4(f2_to_bf16x2(oa[0]), f2_to_bf16x2(oa[1]), f2_to_bf16x2(oa[2]),
@@ -452,12 +454,16 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
             if (!v_bulk) {
                 const unsigned char* vrow = row + v_off;
                 uint8_t* vout = a.v_out + t * vout_bytes;
+                const float2 vs2 = make_float2(a.v_scale, a.v_scale);
                 for (int vi = ctid; vi < nv; vi += Bg) {
                     const uint4 v = reinterpret_cast<const uint4*>(vrow)[vi];
                     if constexpr (FP8) {
-                        float f[8];
-                        unpack8(v, f);
-                        st_v2(vout + (size_t)vi * 8, pack8_e4m3(f, a.v_scale));
+                        const float2 f0 = mul2(bf16x2_to_f2(v.x), vs2);
+                        const float2 f1 = mul2(bf16x2_to_f2(v.y), vs2);
+                        const float2 f2 = mul2(bf16x2_to_f2(v.z), vs2);
+                        const float2 f3 = mul2(bf16x2_to_f2(v.w), vs2);
+                        const float f[8] = {f0.x, f0.y, f1.x, f1.y, f2.x, f2.y, f3.x, f3.y};
+                        st_v2(vout + (size_t)vi * 8, pack8_e4m3_unscaled(f));
                     } else {
                         st_v4(vout + (size_t)vi * 16, v);
                     }
@@ -510,7 +516,11 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
             if (ctid == 0) *abort_flag = 1u;
             break;
         }
-        // Every thread of the group is past token i-1: refill its buffer.
+        // Every thread of the group is past token i-1 (it re-reads token i's
+        // rows after this barrier, not i-1's): refill i-1's buffer with the
+        // token `stages` after it. A second barrier at the end of each token
+        // would free the buffer earlier, but it stops warps from running
+        // ahead and measured slower.
         if (ctid == 0 && i >= 1 && i - 1 + stages < n_local) {
             if (v_bulk) bulk_wait_read_all();
             fence_proxy_async_smem();
@@ -541,6 +551,10 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
             }
             rq = rsqrtf((acc.x + acc.z) * inv_nq + a.eps);
             rk = rsqrtf((acc.y + acc.w) * inv_nk + a.eps);
+            if (FP8) {  // E4M3(value * scale): the scale rides on r
+                rq *= a.q_scale;
+                rk *= a.q_scale;
+            }
         }
         float cs[8], sn[8];
         {
@@ -550,6 +564,13 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
             cs[4] = c1.x; cs[5] = c1.y; cs[6] = c1.z; cs[7] = c1.w;
             sn[0] = s0.x; sn[1] = s0.y; sn[2] = s0.z; sn[3] = s0.w;
             sn[4] = s1.x; sn[5] = s1.y; sn[6] = s1.z; sn[7] = s1.w;
+            if (FP8 && !norm) {  // no r to carry the scale: put it on cos/sin
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    cs[k] *= a.q_scale;
+                    sn[k] *= a.q_scale;
+                }
+            }
         }
 #pragma unroll
         for (int k = 0; k < S; ++k) {
@@ -558,13 +579,12 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
             if (slot < nq) {
                 const uint4* q4 = reinterpret_cast<const uint4*>(row) + h * VPH + l;
                 apply_slot_wf<D, NEOX, FP8>(q4[0], q4[L], wsm + h * 2 * VPH, norm, rq, cs, sn,
-                                            a.q_out + (t * a.hq + h) * D * OUTB, l, a.q_scale);
+                                            a.q_out + (t * a.hq + h) * D * OUTB, l);
             }
             if (slot < nk) {
                 const uint4* k4 = reinterpret_cast<const uint4*>(row) + (a.hq + h) * VPH + l;
                 apply_slot_wf<D, NEOX, FP8>(k4[0], k4[L], wsm + (a.hq + h) * 2 * VPH, norm, rk,
-                                            cs, sn, a.k_out + (t * a.hk + h) * D * OUTB, l,
-                                            a.q_scale);
+                                            cs, sn, a.k_out + (t * a.hk + h) * D * OUTB, l);
             }
         }
     }
