@@ -12,9 +12,11 @@
 // every rotation pair sits inside the lane: half split -> vectors l and
 // l + rotary_dim/16 for l < rotary_dim/16, the pass-through vectors two by two
 // after that; interleaved -> vectors l and l + D/16. The group's sum of
-// squares is a GS-lane shuffle reduction: no shared memory, no barrier. Every
-// thread works on U heads at once so that 2U loads are in flight. The table
-// row of a token is read by all its heads and stays in L1.
+// squares is a GS-lane shuffle reduction: no shared memory, no barrier. A warp
+// item is 4 rounds of 32/GS heads of one token: the lane's cos/sin for that
+// token (the same for every head) are loaded once, together with the 8 data
+// vectors, so that one memory latency covers the item. The norm weights live
+// in shared memory as fp32.
 //
 // General kernel: one warp per head through shared memory, for the shapes and
 // alignments the fast kernel does not take.
@@ -67,14 +69,26 @@ __device__ __forceinline__ void load_cos_sin4(const uint8_t* tbl_row, int col, i
 
 template <int GS, bool IL, bool F32>
 __global__ void __launch_bounds__(kBlock) rope_table_fast(const RopeTableArgs a) {
+    constexpr int HR = 32 / GS;  // heads per warp round
     const int D = a.head_dim, R = a.rotary_dim;
     const int L = D / 16;
-    const int l = threadIdx.x % GS;
+    const int lane = threadIdx.x & 31;
+    const int l = lane % GS, sub = lane / GS;
     const bool active = l < L;
     const int H = a.hq + a.hk;
-    const int64_t ngroups = a.num_tokens * H;
-    const int gpb = kBlock / GS;  // groups per block per round
-    const int tb = F32 ? 4 : 2;   // table element bytes
+    const int per_item = kUnroll * HR;               // heads of one token per warp item
+    const int cpt = (H + per_item - 1) / per_item;   // items per token
+    const int64_t items = a.num_tokens * cpt;
+    const int tb = F32 ? 4 : 2;  // table element bytes
+
+    // Norm weights of q and k as fp32 in shared memory: [q | k][D].
+    __shared__ __align__(16) float wsm[2 * 256];
+    for (int c = threadIdx.x; c < 2 * D; c += blockDim.x) {
+        const uint16_t* w = reinterpret_cast<const uint16_t*>(c < D ? a.q_weight : a.k_weight);
+        const int cc = c < D ? c : c - D;
+        wsm[c] = ((c < D ? a.hq : a.hk) > 0) ? __uint_as_float((uint32_t)w[cc] << 16) : 0.0f;
+    }
+    __syncthreads();
 
     // Vectors of this lane inside a head and how they rotate.
     int va, vb;
@@ -90,96 +104,120 @@ __global__ void __launch_bounds__(kBlock) rope_table_fast(const RopeTableArgs a)
             va = R / 8 + 2 * (l - r16); vb = va + 1;
         }
     }
-    uint4 wqa = make_uint4(0, 0, 0, 0), wqb = wqa, wka = wqa, wkb = wqa;
-    if (active) {
-        const uint4* qw = reinterpret_cast<const uint4*>(a.q_weight);
-        const uint4* kw = reinterpret_cast<const uint4*>(a.k_weight);
-        if (a.hq > 0) { wqa = qw[va]; wqb = qw[vb]; }
-        if (a.hk > 0) { wka = kw[va]; wkb = kw[vb]; }
-    }
     const float inv_d = 1.0f / (float)D;
+    const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    // item = t * cpt + chunk; stepped by nwarps without dividing per item
+    int64_t t = warp_id / cpt;
+    int chunk = (int)(warp_id - t * cpt);
+    const int64_t dt = nwarps / cpt;
+    const int dchunk = (int)(nwarps - dt * cpt);
 
-    for (int64_t g0 = (int64_t)blockIdx.x * gpb * kUnroll; g0 < ngroups;
-         g0 += (int64_t)gridDim.x * gpb * kUnroll) {
+    for (int64_t item = warp_id; item < items; item += nwarps) {
+        const int h0 = chunk * per_item;
+        // This token's cos/sin for this lane's pairs: issued with the data loads.
+        const uint8_t* trow = a.table + (size_t)t * R * tb;
+        float c[8], s[8];
+        if (active) {
+            if (IL) {
+                if (rot_a) load_cos_sin4<F32>(trow, 4 * va, R / 2, c, s);
+                if (rot_b) load_cos_sin4<F32>(trow, 4 * vb, R / 2, c + 4, s + 4);
+            } else if (across) {
+                load_cos_sin8<F32>(trow, 8 * va, R / 2, c, s);
+            }
+        }
         uint4 xa[kUnroll], xb[kUnroll];
-        int64_t tok[kUnroll];
-        int head[kUnroll];
-        bool isk[kUnroll], ok[kUnroll];
+        bool ok[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int64_t g = g0 + (int64_t)u * gpb + threadIdx.x / GS;
-            ok[u] = active && g < ngroups;
-            tok[u] = g / H;
-            const int hh = (int)(g - tok[u] * H);
-            isk[u] = hh >= a.hq;
-            head[u] = isk[u] ? hh - a.hq : hh;
+            const int hh = h0 + u * HR + sub;
+            ok[u] = active && hh < H;
             if (ok[u]) {
-                const uint8_t* src = isk[u]
-                    ? a.k + ((size_t)tok[u] * a.k_stride + (size_t)head[u] * D) * 2
-                    : a.q + ((size_t)tok[u] * a.q_stride + (size_t)head[u] * D) * 2;
+                const bool isk = hh >= a.hq;
+                const int head = isk ? hh - a.hq : hh;
+                const uint8_t* src = isk
+                    ? a.k + ((size_t)t * a.k_stride + (size_t)head * D) * 2
+                    : a.q + ((size_t)t * a.q_stride + (size_t)head * D) * 2;
                 xa[u] = ld_cs_v4(src + (size_t)va * 16);
                 xb[u] = ld_cs_v4(src + (size_t)vb * 16);
             }
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            float fa[8], fb[8];
-            unpack8(xa[u], fa);
-            unpack8(xb[u], fb);
-            float ss = 0.0f;
+            const int hh = h0 + u * HR + sub;
+            float2 fa[4], fb[4];
+            fa[0] = bf16x2_to_f2(xa[u].x); fa[1] = bf16x2_to_f2(xa[u].y);
+            fa[2] = bf16x2_to_f2(xa[u].z); fa[3] = bf16x2_to_f2(xa[u].w);
+            fb[0] = bf16x2_to_f2(xb[u].x); fb[1] = bf16x2_to_f2(xb[u].y);
+            fb[2] = bf16x2_to_f2(xb[u].z); fb[3] = bf16x2_to_f2(xb[u].w);
+            float2 ss2 = make_float2(0.0f, 0.0f);
             if (ok[u]) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) ss += fa[e] * fa[e] + fb[e] * fb[e];
+                for (int m = 0; m < 4; ++m) {
+                    ss2 = fma2(fa[m], fa[m], ss2);
+                    ss2 = fma2(fb[m], fb[m], ss2);
+                }
             }
-            ss = group_sum<GS>(ss);
+            const float ss = group_sum<GS>(ss2.x + ss2.y);
             if (!ok[u]) continue;
+            const bool isk = hh >= a.hq;
+            const int head = isk ? hh - a.hq : hh;
             const float r = rsqrtf(ss * inv_d + a.eps);
-            float wa[8], wb[8];
-            unpack8(isk[u] ? wka : wqa, wa);
-            unpack8(isk[u] ? wkb : wqb, wb);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                fa[e] = fa[e] * r * wa[e];
-                fb[e] = fb[e] * r * wb[e];
-            }
-            const uint8_t* trow = a.table + (size_t)tok[u] * R * tb;
-            float oa[8], ob[8];
+            const float2 r2 = make_float2(r, r);
+            const float4* w4 = reinterpret_cast<const float4*>(wsm + (isk ? D : 0));
+            const float4 wa0 = w4[2 * va], wa1 = w4[2 * va + 1];
+            const float4 wb0 = w4[2 * vb], wb1 = w4[2 * vb + 1];
+            fa[0] = mul2(mul2(fa[0], r2), make_float2(wa0.x, wa0.y));
+            fa[1] = mul2(mul2(fa[1], r2), make_float2(wa0.z, wa0.w));
+            fa[2] = mul2(mul2(fa[2], r2), make_float2(wa1.x, wa1.y));
+            fa[3] = mul2(mul2(fa[3], r2), make_float2(wa1.z, wa1.w));
+            fb[0] = mul2(mul2(fb[0], r2), make_float2(wb0.x, wb0.y));
+            fb[1] = mul2(mul2(fb[1], r2), make_float2(wb0.z, wb0.w));
+            fb[2] = mul2(mul2(fb[2], r2), make_float2(wb1.x, wb1.y));
+            fb[3] = mul2(mul2(fb[3], r2), make_float2(wb1.z, wb1.w));
+            float2 oa[4], ob[4];
             if (IL) {
-                float c[8], s[8];
-                if (rot_a) load_cos_sin4<F32>(trow, 4 * va, R / 2, c, s);
-                if (rot_b) load_cos_sin4<F32>(trow, 4 * vb, R / 2, c + 4, s + 4);
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     if (rot_a) {
-                        oa[2 * m] = fa[2 * m] * c[m] - fa[2 * m + 1] * s[m];
-                        oa[2 * m + 1] = fa[2 * m + 1] * c[m] + fa[2 * m] * s[m];
+                        oa[m].x = fa[m].x * c[m] - fa[m].y * s[m];
+                        oa[m].y = fa[m].y * c[m] + fa[m].x * s[m];
                     } else {
-                        oa[2 * m] = fa[2 * m]; oa[2 * m + 1] = fa[2 * m + 1];
+                        oa[m] = fa[m];
                     }
                     if (rot_b) {
-                        ob[2 * m] = fb[2 * m] * c[4 + m] - fb[2 * m + 1] * s[4 + m];
-                        ob[2 * m + 1] = fb[2 * m + 1] * c[4 + m] + fb[2 * m] * s[4 + m];
+                        ob[m].x = fb[m].x * c[4 + m] - fb[m].y * s[4 + m];
+                        ob[m].y = fb[m].y * c[4 + m] + fb[m].x * s[4 + m];
                     } else {
-                        ob[2 * m] = fb[2 * m]; ob[2 * m + 1] = fb[2 * m + 1];
+                        ob[m] = fb[m];
                     }
                 }
             } else if (across) {
-                float c[8], s[8];
-                load_cos_sin8<F32>(trow, 8 * va, R / 2, c, s);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    oa[e] = fa[e] * c[e] - fb[e] * s[e];
-                    ob[e] = fb[e] * c[e] + fa[e] * s[e];
+                for (int m = 0; m < 4; ++m) {
+                    const float2 c2 = make_float2(c[2 * m], c[2 * m + 1]);
+                    const float2 s2 = make_float2(s[2 * m], s[2 * m + 1]);
+                    const float2 ns2 = make_float2(-s[2 * m], -s[2 * m + 1]);
+                    oa[m] = fma2(fa[m], c2, mul2(fb[m], ns2));
+                    ob[m] = fma2(fb[m], c2, mul2(fa[m], s2));
                 }
             } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) { oa[e] = fa[e]; ob[e] = fb[e]; }
+                for (int m = 0; m < 4; ++m) { oa[m] = fa[m]; ob[m] = fb[m]; }
             }
-            uint8_t* dst = isk[u]
-                ? a.k_out + ((size_t)tok[u] * a.k_out_stride + (size_t)head[u] * D) * 2
-                : a.q_out + ((size_t)tok[u] * a.q_out_stride + (size_t)head[u] * D) * 2;
-            st_v4(dst + (size_t)va * 16, pack8_bf16(oa));
-            st_v4(dst + (size_t)vb * 16, pack8_bf16(ob));
+            uint8_t* dst = isk
+                ? a.k_out + ((size_t)t * a.k_out_stride + (size_t)head * D) * 2
+                : a.q_out + ((size_t)t * a.q_out_stride + (size_t)head * D) * 2;
+            st_v4(dst + (size_t)va * 16, make_uint4(f2_to_bf16x2(oa[0]), f2_to_bf16x2(oa[1]),
+                                                    f2_to_bf16x2(oa[2]), f2_to_bf16x2(oa[3])));
+            st_v4(dst + (size_t)vb * 16, make_uint4(f2_to_bf16x2(ob[0]), f2_to_bf16x2(ob[1]),
+                                                    f2_to_bf16x2(ob[2]), f2_to_bf16x2(ob[3])));
+        }
+        t += dt;
+        chunk += dchunk;
+        if (chunk >= cpt) {
+            chunk -= cpt;
+            ++t;
         }
     }
 }
@@ -279,9 +317,10 @@ cudaError_t launch_persistent(K kern, int64_t work_blocks, const RopeTableArgs& 
 
 template <int GS>
 cudaError_t run_fast(const RopeTableArgs& a, cudaStream_t stream, LaunchInfo* info) {
-    const int64_t groups = a.num_tokens * (a.hq + a.hk);
-    const int64_t per_block = (int64_t)(kBlock / GS) * kUnroll;
-    const int64_t blocks = (groups + per_block - 1) / per_block;
+    const int H = a.hq + a.hk;
+    const int per_item = kUnroll * (32 / GS);
+    const int64_t items = a.num_tokens * ((H + per_item - 1) / per_item);
+    const int64_t blocks = (items + kBlock / 32 - 1) / (kBlock / 32);
     const int id = 1000 + GS * 10 + (a.interleaved ? 1 : 0) * 2 + (a.table_f32 ? 1 : 0);
     if (a.interleaved) {
         return a.table_f32
