@@ -31,15 +31,20 @@ METRIC = "tokens/s and achieved HBM GB/s (% of B200 peak) for fused QK-norm+RoPE
 FALLBACK_HBM_GBS = 6650.0
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu
-# capture summarised in profiles/, valid only for the kernel sources whose
-# hash is stored beside it (null otherwise).
-TRAFFIC = {}
+# capture summarised in profiles/ (rope3d_video3d.md, rope3d_fp8neox.md),
+# valid only for the 3D kernel sources whose hash is stored beside it (the
+# bench reports null otherwise).
+TRAFFIC = {
+    "video3d": (377559296 + 326729728, "7195c344e100429b"),
+    "fp8neox": (1097353216 + 516898560, "7195c344e100429b"),
+}
 
 
 def kernel_source_hash() -> str:
+    """Hash of the sources the 3D kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "qk_rmsnorm_rope_qknr_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in ("common.cuh", "launch.h", "rope3d.cu"):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
