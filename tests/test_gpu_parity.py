@@ -336,3 +336,28 @@ def test_table_outputs_written_exactly():
     torch.cuda.synchronize()
     assert torch.all(qb[T * Hq * D:] == -1) and torch.all(kb[T * Hk * D:] == -1)
     assert not torch.any(qb[:T * Hq * D] == -1) and not torch.any(kb[:T * Hk * D] == -1)
+
+
+def test_3d_sequence_shards_match_whole_call():
+    """Sequence sharding (what each rank of a multi-GPU run does): the token
+    shards of sharding.token_shard, each called with its pos_offset, give the
+    whole call's outputs bit for bit."""
+    from qk_rmsnorm_rope_qknr_b200 import sharding
+
+    w = W.WORKLOADS["video3d"]
+    T = 3 * 1000 + 7
+    inp = W.make_inputs(w, device="cpu", tokens=T)
+    qkv = inp["qkv"].to(DEV)
+    qw, kw = inp["q_weight"].to(DEV), inp["k_weight"].to(DEV)
+    whole = run_3d(qkv, qw, kw, pos_offset=11, **_p3(w))
+    P = w.ppf * w.pph * w.ppw
+    for world in (2, 3, 8):
+        parts = [[], [], []]
+        for rank in range(world):
+            s, c = sharding.token_shard(T, world, rank)
+            out = run_3d(qkv[s:s + c], qw, kw, pos_offset=sharding.shard_pos_offset(s, 11, P),
+                         **_p3(w))
+            for lst, o in zip(parts, out):
+                lst.append(o)
+        for lst, o in zip(parts, whole):
+            assert torch.equal(torch.cat(lst), o)

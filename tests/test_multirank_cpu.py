@@ -1,0 +1,103 @@
+"""The multi-rank path on CPU: world size 2 over gloo.
+
+Each rank takes its contiguous token shard of one 3D sequence (and of one
+table-form batch), runs the oracle on it with the shard's pos_offset (or table
+rows), and all_gathers the pieces; the result must equal the unsharded call
+bit for bit. This checks the sharding arithmetic with real collectives; on
+GPUs the same shards go to qknr_rope_3d / qknr_rope_table on each rank.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from qk_rmsnorm_rope_qknr_b200 import sharding
+
+WORLD = 2
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _inputs3d(T, row, seed=3):
+    g = torch.Generator().manual_seed(seed)
+    qkv = torch.randn(T, row, generator=g).to(torch.bfloat16)
+    qw = (1 + 0.1 * torch.randn(2 * 32, generator=g)).to(torch.bfloat16)
+    kw = (1 + 0.1 * torch.randn(2 * 32, generator=g)).to(torch.bfloat16)
+    return qkv, qw, kw
+
+
+P3 = dict(ppf=3, pph=2, ppw=5, num_frame_channels=8, num_height_channels=12,
+          num_width_channels=12, num_heads_q=2, num_heads_k=2, num_heads_v=1, head_dim=32,
+          eps=1e-5, interleave=False)
+
+
+def _worker(rank, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD)
+    try:
+        import oracle as O
+        from tests._util import t2u16
+
+        # --- 3D sequence of 2.4 grids, offset into the sequence by 7 tokens
+        T, P = 72, 3 * 2 * 5
+        qkv, qw, kw = _inputs3d(T, 5 * 32)
+        start, count = sharding.token_shard(T, WORLD, rank)
+        off = sharding.shard_pos_offset(start, 7, P)
+        mine = O.rope_3d(t2u16(qkv[start:start + count]), t2u16(qw), t2u16(kw), pos_offset=off,
+                         **P3)
+        for part, ref in zip(mine, O.rope_3d(t2u16(qkv), t2u16(qw), t2u16(kw), pos_offset=7,
+                                             **P3)):
+            pieces = [None] * WORLD
+            dist.all_gather_object(pieces, part)
+            assert np.array_equal(np.concatenate(pieces), ref)
+        # --- table form: 33 tokens, the shard takes its own table rows
+        g = torch.Generator().manual_seed(5)
+        q = torch.randn(33, 3, 16, generator=g).to(torch.bfloat16)
+        k = torch.randn(33, 1, 16, generator=g).to(torch.bfloat16)
+        w = (1 + 0.1 * torch.randn(16, generator=g)).to(torch.bfloat16)
+        th = torch.arange(33, dtype=torch.float64)[:, None] * 0.3 ** torch.arange(6.0)[None, :]
+        tbl = torch.cat([th.cos(), th.sin()], 1).float().numpy()
+        s, c = sharding.token_shard(33, WORLD, rank)
+        mine = O.rope_table(t2u16(q[s:s + c]), t2u16(k[s:s + c]), t2u16(w), t2u16(w),
+                            tbl[s:s + c].copy(), 1e-6, 12, interleaved=True)
+        ref = O.rope_table(t2u16(q), t2u16(k), t2u16(w), t2u16(w), tbl, 1e-6, 12,
+                           interleaved=True)
+        for part, r in zip(mine, ref):
+            pieces = [None] * WORLD
+            dist.all_gather_object(pieces, part)
+            assert np.array_equal(np.concatenate(pieces), r)
+        dist.barrier()
+        open(os.path.join(out_dir, f"ok{rank}"), "w").write("ok")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_token_shard_arithmetic():
+    for T in (0, 1, 5, 72, 15360, 59521):
+        for world in (1, 2, 3, 8):
+            spans = [sharding.token_shard(T, world, r) for r in range(world)]
+            assert spans[0][0] == 0
+            assert sum(c for _, c in spans) == T
+            for (s0, c0), (s1, _) in zip(spans, spans[1:]):
+                assert s0 + c0 == s1
+            assert max(c for _, c in spans) - min(c for _, c in spans) <= 1
+    assert sharding.shard_pos_offset(40, 7, 30) == 17
+    with pytest.raises(ValueError):
+        sharding.token_shard(4, 2, 2)
+
+
+def test_two_ranks_over_gloo(tmp_path):
+    port = _free_port()
+    mp.start_processes(_worker, args=(port, str(tmp_path)), nprocs=WORLD, join=True,
+                       start_method="spawn")
+    for r in range(WORLD):
+        assert (tmp_path / f"ok{r}").read_text() == "ok"
