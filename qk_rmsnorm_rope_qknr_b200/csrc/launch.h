@@ -49,6 +49,10 @@ struct RopeTableArgs {
     int32_t interleaved;
     int32_t in_place;  // an output aliases its input
     float eps;
+    // Pipelined (bulk-copy) kernel only:
+    int32_t stages;           // ring buffers per warp
+    uint32_t stall_tx_bytes;  // test hook: extra bytes a buffer waits for (0 in use)
+    uint64_t wait_limit_ns;   // a wait on a bulk copy gives up after this long
 };
 
 // Launch description returned for the benchmark and tests.
@@ -68,5 +72,8 @@ cudaError_t launch_rope3d(const Rope3DArgs& a, int head_dim, int neox, int fp8,
 cudaError_t read_device_status(uint32_t* out, int clear, cudaStream_t stream);
 cudaError_t launch_rope_table(const RopeTableArgs& a, int fast_path, cudaStream_t stream,
                               LaunchInfo* info);
+
+// Status word of the table kernels (bit 0 as for the 3D kernels).
+cudaError_t read_table_status(uint32_t* out, int clear, cudaStream_t stream);
 
 }  // namespace qknr

@@ -147,10 +147,12 @@ int qknr_test_set_wait_fault(uint32_t extra_bytes, uint64_t limit_ns) {
 
 int qknr_device_status(void* cuda_stream, uint32_t* status_out, int32_t clear) {
     if (!status_out) return fail(QKNR_ERR_NULL, "status_out is NULL");
-    uint32_t v = 0;
-    cudaError_t e = qknr::read_device_status(&v, clear, static_cast<cudaStream_t>(cuda_stream));
+    uint32_t v = 0, w = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    cudaError_t e = qknr::read_device_status(&v, clear, st);
+    if (e == cudaSuccess) e = qknr::read_table_status(&w, clear, st);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
-    *status_out = v;
+    *status_out = v | w;
     return ok();
 }
 
@@ -261,6 +263,8 @@ int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
     a.interleaved = interleaved ? 1 : 0;
     a.in_place = q_inplace || k_inplace;
     a.eps = eps;
+    a.stall_tx_bytes = g_fault_extra_bytes.load(std::memory_order_relaxed);
+    a.wait_limit_ns = a.stall_tx_bytes ? g_fault_limit_ns.load() : 0;
 
     // Fast kernel: 16-byte vectors everywhere and rotation pairs inside a lane.
     const bool vec_ok =

@@ -27,52 +27,61 @@
 
 namespace qknr {
 
+__device__ unsigned int g_table_status;
+
 namespace {
 
 constexpr int kBlock = 256;
 constexpr int kUnroll = 4;
 
+// The same reads from a table row staged in shared memory (plain loads: the
+// read-only global path must not see a shared address).
 template <bool F32>
-__device__ __forceinline__ void load_cos_sin8(const uint8_t* tbl_row, int col, int half,
+__device__ __forceinline__ void smem_cos_sin8(const uint8_t* row, int col, int half,
                                               float (&c)[8], float (&s)[8]) {
     if constexpr (F32) {
-        const float4* pc = reinterpret_cast<const float4*>(tbl_row + (size_t)col * 4);
-        const float4* ps = reinterpret_cast<const float4*>(tbl_row + (size_t)(half + col) * 4);
-        const float4 c0 = __ldg(pc), c1 = __ldg(pc + 1), s0 = __ldg(ps), s1 = __ldg(ps + 1);
+        const float4* pc = reinterpret_cast<const float4*>(row + (size_t)col * 4);
+        const float4* ps = reinterpret_cast<const float4*>(row + (size_t)(half + col) * 4);
+        const float4 c0 = pc[0], c1 = pc[1], s0 = ps[0], s1 = ps[1];
         c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w;
         c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
         s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w;
         s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
     } else {
-        const uint4 cv = __ldg(reinterpret_cast<const uint4*>(tbl_row + (size_t)col * 2));
-        const uint4 sv = __ldg(reinterpret_cast<const uint4*>(tbl_row + (size_t)(half + col) * 2));
+        const uint4 cv = *reinterpret_cast<const uint4*>(row + (size_t)col * 2);
+        const uint4 sv = *reinterpret_cast<const uint4*>(row + (size_t)(half + col) * 2);
         unpack8(cv, c);
         unpack8(sv, s);
     }
 }
 
 template <bool F32>
-__device__ __forceinline__ void load_cos_sin4(const uint8_t* tbl_row, int col, int half,
-                                              float* c, float* s) {
+__device__ __forceinline__ void smem_cos_sin4(const uint8_t* row, int col, int half, float* c,
+                                              float* s) {
     if constexpr (F32) {
-        const float4 cv = __ldg(reinterpret_cast<const float4*>(tbl_row + (size_t)col * 4));
-        const float4 sv = __ldg(reinterpret_cast<const float4*>(tbl_row + (size_t)(half + col) * 4));
+        const float4 cv = *reinterpret_cast<const float4*>(row + (size_t)col * 4);
+        const float4 sv = *reinterpret_cast<const float4*>(row + (size_t)(half + col) * 4);
         c[0] = cv.x; c[1] = cv.y; c[2] = cv.z; c[3] = cv.w;
         s[0] = sv.x; s[1] = sv.y; s[2] = sv.z; s[3] = sv.w;
     } else {
-        const uint2 cv = __ldg(reinterpret_cast<const uint2*>(tbl_row + (size_t)col * 2));
-        const uint2 sv = __ldg(reinterpret_cast<const uint2*>(tbl_row + (size_t)(half + col) * 2));
+        const uint2 cv = *reinterpret_cast<const uint2*>(row + (size_t)col * 2);
+        const uint2 sv = *reinterpret_cast<const uint2*>(row + (size_t)(half + col) * 2);
         c[0] = bf16_lo(cv.x); c[1] = bf16_hi(cv.x); c[2] = bf16_lo(cv.y); c[3] = bf16_hi(cv.y);
         s[0] = bf16_lo(sv.x); s[1] = bf16_hi(sv.x); s[2] = bf16_lo(sv.y); s[3] = bf16_hi(sv.y);
     }
 }
 
+// Bytes of one ring buffer: the item's heads, then the token's table row.
+__host__ __device__ inline int table_stage_bytes(int per_item, int D, int R, int tb) {
+    return (per_item * D * 2 + R * tb + 15) & ~15;
+}
+
 template <int GS, bool IL, bool F32>
-__global__ void __launch_bounds__(kBlock) rope_table_fast(const RopeTableArgs a) {
+__global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a) {
     constexpr int HR = 32 / GS;  // heads per warp round
     const int D = a.head_dim, R = a.rotary_dim;
     const int L = D / 16;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int l = lane % GS, sub = lane / GS;
     const bool active = l < L;
     const int H = a.hq + a.hk;
@@ -80,15 +89,63 @@ __global__ void __launch_bounds__(kBlock) rope_table_fast(const RopeTableArgs a)
     const int cpt = (H + per_item - 1) / per_item;   // items per token
     const int64_t items = a.num_tokens * cpt;
     const int tb = F32 ? 4 : 2;  // table element bytes
+    const int stages = a.stages;
+    const int sbytes = table_stage_bytes(per_item, D, R, tb);
 
-    // Norm weights of q and k as fp32 in shared memory: [q | k][D].
-    __shared__ __align__(16) float wsm[2 * 256];
+    extern __shared__ __align__(128) unsigned char smem[];
+    float* wsm = reinterpret_cast<float*>(smem);                       // [q | k][D] fp32
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * 256 * 4);  // [warps][stages]
+    unsigned char* rings = smem + 2 * 256 * 4 + ((kBlock / 32) * stages * 8 + 127) / 128 * 128;
+    uint64_t* full = bars + warp * stages;
+    unsigned char* ring = rings + (size_t)warp * stages * sbytes;
+
+    const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t n_local = warp_id < items ? (items - 1 - warp_id) / nwarps + 1 : 0;
+    // item -> (token, chunk), stepped by nwarps without dividing per item
+    const int64_t dt = nwarps / cpt;
+    const int dchunk = (int)(nwarps - dt * cpt);
+
+    // Issue the copies of one item into ring buffer `s` (lane 0 only).
+    auto issue = [&](int64_t t, int chunk, int s) {
+        const int h0 = chunk * per_item, h1 = min(h0 + per_item, H);
+        const int q1 = min(h1, a.hq), k0 = max(h0, a.hq);
+        const uint32_t qbytes = h0 < a.hq ? (uint32_t)(q1 - h0) * D * 2 : 0;
+        const uint32_t kbytes = h1 > a.hq ? (uint32_t)(h1 - k0) * D * 2 : 0;
+        unsigned char* dst = ring + (size_t)s * sbytes;
+        mbar_arrive_expect_tx(&full[s], qbytes + kbytes + (uint32_t)(R * tb) + a.stall_tx_bytes);
+        if (qbytes)
+            bulk_load(dst, a.q + ((size_t)t * a.q_stride + (size_t)h0 * D) * 2, qbytes, &full[s]);
+        if (kbytes)
+            bulk_load(dst + qbytes, a.k + ((size_t)t * a.k_stride + (size_t)(k0 - a.hq) * D) * 2,
+                      kbytes, &full[s]);
+        bulk_load(dst + (size_t)per_item * D * 2, a.table + (size_t)t * R * tb, (uint32_t)(R * tb),
+                  &full[s]);
+    };
+
+    if (lane == 0) {
+        for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
     for (int c = threadIdx.x; c < 2 * D; c += blockDim.x) {
         const uint16_t* w = reinterpret_cast<const uint16_t*>(c < D ? a.q_weight : a.k_weight);
         const int cc = c < D ? c : c - D;
         wsm[c] = ((c < D ? a.hq : a.hk) > 0) ? __uint_as_float((uint32_t)w[cc] << 16) : 0.0f;
     }
-    __syncthreads();
+    __syncwarp();
+    int64_t t = warp_id / cpt;
+    int chunk = (int)(warp_id - t * cpt);
+    if (lane == 0) {  // first ring of items
+        int64_t tt = t;
+        int cc = chunk;
+        for (int s = 0; s < stages && s < n_local; ++s) {
+            issue(tt, cc, s);
+            tt += dt;
+            cc += dchunk;
+            if (cc >= cpt) { cc -= cpt; ++tt; }
+        }
+    }
+    __syncthreads();  // weights
 
     // Vectors of this lane inside a head and how they rotate.
     int va, vb;
@@ -105,61 +162,60 @@ __global__ void __launch_bounds__(kBlock) rope_table_fast(const RopeTableArgs a)
         }
     }
     const float inv_d = 1.0f / (float)D;
-    const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    // item = t * cpt + chunk; stepped by nwarps without dividing per item
-    int64_t t = warp_id / cpt;
-    int chunk = (int)(warp_id - t * cpt);
-    const int64_t dt = nwarps / cpt;
-    const int dchunk = (int)(nwarps - dt * cpt);
+    // the item `stages` ahead of the current one
+    int64_t t_ahead = t, chunk_ahead = chunk;
+    for (int s = 0; s < stages; ++s) {
+        t_ahead += dt;
+        chunk_ahead += dchunk;
+        if (chunk_ahead >= cpt) { chunk_ahead -= cpt; ++t_ahead; }
+    }
 
-    for (int64_t item = warp_id; item < items; item += nwarps) {
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t i = 0;
+    bool aborted = false;
+    for (; i < n_local; ++i) {
+        const bool ok = mbar_wait_bounded(&full[stage], phase, a.wait_limit_ns);
+        if (__any_sync(0xffffffffu, !ok)) {
+            aborted = true;
+            break;
+        }
+        const unsigned char* buf = ring + (size_t)stage * sbytes;
+        const unsigned char* trow = buf + (size_t)per_item * D * 2;
         const int h0 = chunk * per_item;
-        // This token's cos/sin for this lane's pairs: issued with the data loads.
-        const uint8_t* trow = a.table + (size_t)t * R * tb;
         float c[8], s[8];
         if (active) {
             if (IL) {
-                if (rot_a) load_cos_sin4<F32>(trow, 4 * va, R / 2, c, s);
-                if (rot_b) load_cos_sin4<F32>(trow, 4 * vb, R / 2, c + 4, s + 4);
+                if (rot_a) smem_cos_sin4<F32>(trow, 4 * va, R / 2, c, s);
+                if (rot_b) smem_cos_sin4<F32>(trow, 4 * vb, R / 2, c + 4, s + 4);
             } else if (across) {
-                load_cos_sin8<F32>(trow, 8 * va, R / 2, c, s);
-            }
-        }
-        uint4 xa[kUnroll], xb[kUnroll];
-        bool ok[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int hh = h0 + u * HR + sub;
-            ok[u] = active && hh < H;
-            if (ok[u]) {
-                const bool isk = hh >= a.hq;
-                const int head = isk ? hh - a.hq : hh;
-                const uint8_t* src = isk
-                    ? a.k + ((size_t)t * a.k_stride + (size_t)head * D) * 2
-                    : a.q + ((size_t)t * a.q_stride + (size_t)head * D) * 2;
-                xa[u] = ld_cs_v4(src + (size_t)va * 16);
-                xb[u] = ld_cs_v4(src + (size_t)vb * 16);
+                smem_cos_sin8<F32>(trow, 8 * va, R / 2, c, s);
             }
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int hh = h0 + u * HR + sub;
+            const int hi = u * HR + sub;  // head index inside the item
+            const int hh = h0 + hi;
+            const bool okh = active && hh < H;
+            uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
+            if (okh) {
+                const uint4* v = reinterpret_cast<const uint4*>(buf + (size_t)hi * D * 2);
+                xa = v[va];
+                xb = v[vb];
+            }
             float2 fa[4], fb[4];
-            fa[0] = bf16x2_to_f2(xa[u].x); fa[1] = bf16x2_to_f2(xa[u].y);
-            fa[2] = bf16x2_to_f2(xa[u].z); fa[3] = bf16x2_to_f2(xa[u].w);
-            fb[0] = bf16x2_to_f2(xb[u].x); fb[1] = bf16x2_to_f2(xb[u].y);
-            fb[2] = bf16x2_to_f2(xb[u].z); fb[3] = bf16x2_to_f2(xb[u].w);
+            fa[0] = bf16x2_to_f2(xa.x); fa[1] = bf16x2_to_f2(xa.y);
+            fa[2] = bf16x2_to_f2(xa.z); fa[3] = bf16x2_to_f2(xa.w);
+            fb[0] = bf16x2_to_f2(xb.x); fb[1] = bf16x2_to_f2(xb.y);
+            fb[2] = bf16x2_to_f2(xb.z); fb[3] = bf16x2_to_f2(xb.w);
             float2 ss2 = make_float2(0.0f, 0.0f);
-            if (ok[u]) {
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    ss2 = fma2(fa[m], fa[m], ss2);
-                    ss2 = fma2(fb[m], fb[m], ss2);
-                }
+            for (int m = 0; m < 4; ++m) {
+                ss2 = fma2(fa[m], fa[m], ss2);
+                ss2 = fma2(fb[m], fb[m], ss2);
             }
             const float ss = group_sum<GS>(ss2.x + ss2.y);
-            if (!ok[u]) continue;
+            if (!okh) continue;
             const bool isk = hh >= a.hq;
             const int head = isk ? hh - a.hq : hh;
             const float r = rsqrtf(ss * inv_d + a.eps);
@@ -213,12 +269,28 @@ __global__ void __launch_bounds__(kBlock) rope_table_fast(const RopeTableArgs a)
             st_v4(dst + (size_t)vb * 16, make_uint4(f2_to_bf16x2(ob[0]), f2_to_bf16x2(ob[1]),
                                                     f2_to_bf16x2(ob[2]), f2_to_bf16x2(ob[3])));
         }
+        // Every lane is done with this buffer: refill it with the item a ring ahead.
+        __syncwarp();
+        if (lane == 0 && i + stages < n_local) {
+            fence_proxy_async_smem();
+            issue(t_ahead, (int)chunk_ahead, stage);
+        }
+        t_ahead += dt;
+        chunk_ahead += dchunk;
+        if (chunk_ahead >= cpt) { chunk_ahead -= cpt; ++t_ahead; }
         t += dt;
         chunk += dchunk;
-        if (chunk >= cpt) {
-            chunk -= cpt;
-            ++t;
+        if (chunk >= cpt) { chunk -= cpt; ++t; }
+        if (++stage == stages) {
+            stage = 0;
+            phase ^= 1u;
         }
+    }
+    if (aborted && lane == 0) {
+        atomicOr(&g_table_status, 1u);
+        // Drain this warp's copies still in flight (bounded): items i .. i+stages-1.
+        for (int64_t j = i; j < n_local && j < i + stages; ++j)
+            mbar_wait_bounded(&full[j % stages], (uint32_t)((j / stages) & 1), a.wait_limit_ns);
     }
 }
 
@@ -315,21 +387,54 @@ cudaError_t launch_persistent(K kern, int64_t work_blocks, const RopeTableArgs& 
     return cudaGetLastError();
 }
 
+template <typename K>
+cudaError_t launch_bulk(K kern, const RopeTableArgs& a0, int per_item, cudaStream_t stream,
+                        LaunchInfo* info, int id) {
+    RopeTableArgs a = a0;
+    const int tb = a.table_f32 ? 4 : 2;
+    const int sbytes = table_stage_bytes(per_item, a.head_dim, a.rotary_dim, tb);
+    const int warps = kBlock / 32;
+    // Two CTAs per SM, each warp with as many ring buffers (2..4) as fit.
+    const int fixed = 2 * 256 * 4 + 128 + warps * 4 * 8;
+    a.stages = std::max(2, std::min(4, (227 * 1024 / 2 - 1024 - fixed) / (warps * sbytes)));
+    if (a.wait_limit_ns == 0) a.wait_limit_ns = 2000000000ull;  // 2 s
+    const int smem = 2 * 256 * 4 + ((warps * a.stages * 8 + 127) / 128 * 128) +
+                     warps * a.stages * sbytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    int dev = 0, sms = 0, per_sm = 0;
+    if (e == cudaSuccess) e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBlock, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int H = a.hq + a.hk;
+    const int64_t items = a.num_tokens * ((H + per_item - 1) / per_item);
+    const int64_t want_blocks = (items + warps - 1) / warps;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * per_sm,
+                                                                 want_blocks));
+    kern<<<grid, kBlock, smem, stream>>>(a);
+    if (info) {
+        info->grid = grid;
+        info->block = kBlock;
+        info->smem = smem;
+        info->kernel_id = id;
+    }
+    return cudaGetLastError();
+}
+
 template <int GS>
 cudaError_t run_fast(const RopeTableArgs& a, cudaStream_t stream, LaunchInfo* info) {
-    const int H = a.hq + a.hk;
     const int per_item = kUnroll * (32 / GS);
-    const int64_t items = a.num_tokens * ((H + per_item - 1) / per_item);
-    const int64_t blocks = (items + kBlock / 32 - 1) / (kBlock / 32);
     const int id = 1000 + GS * 10 + (a.interleaved ? 1 : 0) * 2 + (a.table_f32 ? 1 : 0);
     if (a.interleaved) {
         return a.table_f32
-            ? launch_persistent(rope_table_fast<GS, true, true>, blocks, a, stream, info, id)
-            : launch_persistent(rope_table_fast<GS, true, false>, blocks, a, stream, info, id);
+            ? launch_bulk(rope_table_bulk<GS, true, true>, a, per_item, stream, info, id)
+            : launch_bulk(rope_table_bulk<GS, true, false>, a, per_item, stream, info, id);
     }
     return a.table_f32
-        ? launch_persistent(rope_table_fast<GS, false, true>, blocks, a, stream, info, id)
-        : launch_persistent(rope_table_fast<GS, false, false>, blocks, a, stream, info, id);
+        ? launch_bulk(rope_table_bulk<GS, false, true>, a, per_item, stream, info, id)
+        : launch_bulk(rope_table_bulk<GS, false, false>, a, per_item, stream, info, id);
 }
 
 }  // namespace
@@ -349,6 +454,19 @@ cudaError_t launch_rope_table(const RopeTableArgs& a, int fast_path, cudaStream_
     return a.table_f32
         ? launch_persistent(rope_table_general<true>, blocks, a, stream, info, 2001)
         : launch_persistent(rope_table_general<false>, blocks, a, stream, info, 2000);
+}
+
+cudaError_t read_table_status(uint32_t* out, int clear, cudaStream_t stream) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_table_status, sizeof(uint32_t), 0,
+                                              cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && clear) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_table_status, &zero, sizeof(uint32_t), 0,
+                                    cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    }
+    return e;
 }
 
 }  // namespace qknr

@@ -50,3 +50,32 @@ def test_wait_timeout_raises_status_and_context_survives():
     for a, b in zip(good, again):
         assert torch.equal(a, b)
     assert Q.qknr_device_status() == 0
+
+
+def test_table_wait_timeout_raises_status_and_context_survives():
+    w = W.WORKLOADS["table_hs"]
+    inp = {k: v.cuda() for k, v in W.make_inputs(w, tokens=64).items()}
+
+    def call(qo, ko):
+        Q.qknr_rope_table(inp["q"], inp["k"], qo, ko, inp["q_weight"], inp["k_weight"],
+                          inp["rope_table"], eps=w.eps, rotary_dim=w.rotary_dim,
+                          interleaved=w.interleaved)
+
+    good = [torch.empty_like(inp["q"]), torch.empty_like(inp["k"])]
+    call(*good)
+    torch.cuda.synchronize()
+    Q.qknr_device_status(clear=True)
+    L = Q.lib()
+    assert L.qknr_test_set_wait_fault(16, 20_000_000) == 0
+    try:
+        call(torch.zeros_like(inp["q"]), torch.zeros_like(inp["k"]))
+        torch.cuda.synchronize()
+    finally:
+        assert L.qknr_test_set_wait_fault(0, 0) == 0
+    assert Q.qknr_device_status(clear=True) & 1
+    again = [torch.empty_like(inp["q"]), torch.empty_like(inp["k"])]
+    call(*again)
+    torch.cuda.synchronize()
+    for a, b in zip(good, again):
+        assert torch.equal(a, b)
+    assert Q.qknr_device_status() == 0
