@@ -119,8 +119,8 @@ int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
  *      q*output_quant_scale, k*output_quant_scale and v*v_quant_scale.
  *      Without output_fp8, v_out is a bit copy of V.
  *
- * Validation: tokens divisible by ppf*pph*ppw (pos_offset == 0) or any count
- * (pos_offset > 0, a shard of a longer sequence); channel counts even,
+ * Validation: num_tokens divisible by ppf*pph*ppw for a whole call, any count
+ * for a sequence shard (sequence_shard = 1); channel counts even,
  * non-negative, summing to head_dim; head_dim in {64, 128, 256}; heads >= 0 and
  * Hq + Hk + Hv >= 1; factor == 1 and attention_factor == 1 (YARN is not built:
  * QKNR_ERR_UNSUPPORTED); qkv and all outputs 16-byte aligned; no output
@@ -135,7 +135,7 @@ typedef struct {
     void* k_out;        /* bf16 or E4M3 [num_tokens, Hk, head_dim]               */
     void* v_out;        /* bf16 or E4M3 [num_tokens, Hv, head_dim]               */
     int64_t num_tokens;
-    int64_t pos_offset; /* position of the first token in the patch sequence     */
+    int64_t pos_offset; /* patch position of the first token (mod ppf*pph*ppw)   */
     int32_t ppf, pph, ppw;
     int32_t num_frame_channels, num_height_channels, num_width_channels;
     int32_t num_heads_q, num_heads_k, num_heads_v, head_dim;
@@ -147,6 +147,10 @@ typedef struct {
     int32_t output_fp8;
     float output_quant_scale;
     float v_quant_scale;
+    int32_t sequence_shard; /* 0: the whole patch sequence(s), num_tokens divisible
+                               by ppf*pph*ppw; 1: a contiguous slice of a longer
+                               sequence starting at patch position pos_offset
+                               (one rank's part of a sharded call): any count */
 } qknr_rope_3d_params;
 
 int qknr_rope_3d(const qknr_rope_3d_params* params, void* cuda_stream);

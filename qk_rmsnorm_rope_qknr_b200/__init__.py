@@ -57,7 +57,7 @@ class Rope3DParams(C.Structure):
                 ("factor", C.c_float), ("low", C.c_float), ("high", C.c_float),
                 ("attention_factor", C.c_float), ("is_qk_norm", C.c_int32),
                 ("output_fp8", C.c_int32), ("output_quant_scale", C.c_float),
-                ("v_quant_scale", C.c_float)]
+                ("v_quant_scale", C.c_float), ("sequence_shard", C.c_int32)]
 
 
 _lib = None
@@ -169,8 +169,11 @@ def make_3d_params(qkv, q_weight, k_weight, q_out, k_out, v_out, *, ppf, pph, pp
                    num_frame_channels, num_height_channels, num_width_channels, num_heads_q,
                    num_heads_k, num_heads_v, head_dim, eps=1e-6, base=10000.0, interleave=True,
                    factor=1.0, low=0.0, high=0.0, attention_factor=1.0, is_qk_norm=True,
-                   output_fp8=False, output_quant_scale=1.0, v_quant_scale=1.0, pos_offset=0,
-                   num_tokens=None) -> Rope3DParams:
+                   output_fp8=False, output_quant_scale=1.0, v_quant_scale=1.0,
+                   pos_offset: Optional[int] = None, num_tokens=None) -> Rope3DParams:
+    """C parameter block. pos_offset=None is a whole call (num_tokens must be a
+    multiple of ppf*pph*ppw); an integer marks a sequence shard whose first
+    token sits at that patch position (any token count)."""
     row = (num_heads_q + num_heads_k + num_heads_v) * head_dim
     if num_tokens is None:
         if qkv.dtype != torch.bfloat16 or qkv.shape[-1] != row or not qkv.is_contiguous():
@@ -181,7 +184,9 @@ def make_3d_params(qkv, q_weight, k_weight, q_out, k_out, v_out, *, ppf, pph, pp
     p.struct_size = C.sizeof(Rope3DParams)
     p.qkv, p.q_weight, p.k_weight = _ptr(qkv), _ptr(q_weight), _ptr(k_weight)
     p.q_out, p.k_out, p.v_out = _ptr(q_out), _ptr(k_out), _ptr(v_out)
-    p.num_tokens, p.pos_offset = int(num_tokens), int(pos_offset)
+    p.num_tokens = int(num_tokens)
+    p.pos_offset = 0 if pos_offset is None else int(pos_offset)
+    p.sequence_shard = 0 if pos_offset is None else 1
     p.ppf, p.pph, p.ppw = ppf, pph, ppw
     p.num_frame_channels, p.num_height_channels = num_frame_channels, num_height_channels
     p.num_width_channels = num_width_channels
@@ -196,7 +201,8 @@ def make_3d_params(qkv, q_weight, k_weight, q_out, k_out, v_out, *, ppf, pph, pp
 
 def qknr_rope_3d(qkv, q_weight, k_weight, q_out, k_out, v_out, *, stream=None, **params) -> None:
     """3D form through the C ABI (destination passing; see include/qknr.h).
-    params are the page's keyword arguments plus pos_offset."""
+    params are the page's keyword arguments plus pos_offset (an integer marks
+    a sequence shard; see make_3d_params)."""
     p = make_3d_params(qkv, q_weight, k_weight, q_out, k_out, v_out, **params)
     odt = torch.float8_e4m3fn if params.get("output_fp8") else torch.bfloat16
     for n, o, h in (("q_out", q_out, p.num_heads_q), ("k_out", k_out, p.num_heads_k),
@@ -256,7 +262,8 @@ def fused_qk_rmsnorm_rope(qkv: torch.Tensor, q_weight: torch.Tensor, k_weight: t
                           output_quant_scale: float = 1.0, v_quant_scale: float = 1.0,
                           q_out: Optional[torch.Tensor] = None,
                           k_out: Optional[torch.Tensor] = None,
-                          v_out: Optional[torch.Tensor] = None, pos_offset: int = 0,
+                          v_out: Optional[torch.Tensor] = None,
+                          pos_offset: Optional[int] = None,
                           stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Across-heads Q/K RMSNorm + 3D RoPE + V copy (+ FP8). Outputs are
     [B, S, H, D] for a 3D qkv and [T, H, D] for a 2D one."""

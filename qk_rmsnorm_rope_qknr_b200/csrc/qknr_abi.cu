@@ -306,8 +306,10 @@ int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
         return fail(QKNR_ERR_SHAPE, "channels %d+%d+%d != head_dim %d", cf, ch, cw, D);
     if (p.num_tokens < 0) return fail(QKNR_ERR_SHAPE, "num_tokens < 0");
     if (p.pos_offset < 0) return fail(QKNR_ERR_SHAPE, "pos_offset < 0");
-    if (p.pos_offset == 0 && p.num_tokens % P != 0)
-        return fail(QKNR_ERR_SHAPE, "num_tokens %lld not divisible by ppf*pph*ppw = %lld",
+    if (!p.sequence_shard && p.num_tokens % P != 0)
+        return fail(QKNR_ERR_SHAPE,
+                    "num_tokens %lld not divisible by ppf*pph*ppw = %lld (a slice of a longer "
+                    "sequence sets sequence_shard)",
                     (long long)p.num_tokens, (long long)P);
     if (!(p.base > 0.0) || std::isinf(p.base)) return fail(QKNR_ERR_SHAPE, "base must be > 0");
     if (p.factor != 1.0f)
