@@ -156,6 +156,36 @@ typedef struct {
 int qknr_rope_3d(const qknr_rope_3d_params* params, void* cuda_stream);
 
 /*
+ * Tensor-parallel 3D form. When the Q, K and V heads of a token are split
+ * across ranks, each rank holds packed rows of its own heads only, but the
+ * RMSNorm must still run over the global channel width of Q (and of K).
+ * "vllm_omni.diffusion.models.sana_wm.ucpe" (cam_prep_func) states this rule:
+ * a tensor-parallel shard must normalise over the global channel width.
+ * The transform is the one of qknr_rope_3d ("flashinfer.norm.
+ * fused_qk_rmsnorm_rope"), split in two passes around one exchange:
+ *
+ *   1. qknr_rope_3d_partial_ssq: per token, the sums of x^2 over this call's
+ *      Q channels and over its K channels -> ssq_out, fp32 [num_tokens][2].
+ *      Only the Q and K part of each row is read; outputs, weights, eps and
+ *      the FP8 fields of params are ignored (may be NULL / anything).
+ *   2. the caller sums ssq_out over all ranks (an all-reduce).
+ *   3. qknr_rope_3d_with_ssq: the full transform of this call's heads (RoPE,
+ *      V copy, FP8 as usual) with r = 1 / sqrt(ssq[t][0] / (heads_q_total *
+ *      head_dim) + eps) for Q and likewise for K over heads_k_total.
+ *      params.is_qk_norm must be 1; heads_*_total >= this call's heads.
+ *
+ * With one rank (heads_*_total equal to the call's own heads) the passes give
+ * the same result as qknr_rope_3d up to the order of the fp32 additions.
+ * The [T][2] arrays are 8-byte aligned and must not overlap any other buffer.
+ * Both passes run on the pipelined kernel: a row that does not fit two
+ * buffers of shared memory returns QKNR_ERR_UNSUPPORTED.
+ */
+int qknr_rope_3d_partial_ssq(const qknr_rope_3d_params* params, float* ssq_out,
+                             void* cuda_stream);
+int qknr_rope_3d_with_ssq(const qknr_rope_3d_params* params, const float* ssq,
+                          int32_t heads_q_total, int32_t heads_k_total, void* cuda_stream);
+
+/*
  * Device-side status of this library's kernels on the current device, for
  * failures that can only be seen on the GPU. Bit 0: a kernel's wait on one of
  * its own bulk copies ran past its time limit (2 s), so that launch abandoned

@@ -31,8 +31,9 @@ QKNR_OK, QKNR_ERR_NULL, QKNR_ERR_SHAPE, QKNR_ERR_UNSUPPORTED = 0, 1, 2, 3
 QKNR_ERR_ALIGN, QKNR_ERR_ALIAS, QKNR_ERR_POINTER, QKNR_ERR_CUDA = 4, 5, 6, 7
 QKNR_DT_BF16, QKNR_DT_F32, QKNR_DT_E4M3 = 0, 1, 2
 
-EXPORTS = ("qknr_rope_table", "qknr_rope_3d", "qknr_device_status", "qknr_test_set_wait_fault",
-           "qknr_status_string", "qknr_last_error_detail", "qknr_abi_version")
+EXPORTS = ("qknr_rope_table", "qknr_rope_3d", "qknr_rope_3d_partial_ssq", "qknr_rope_3d_with_ssq",
+           "qknr_device_status", "qknr_test_set_wait_fault", "qknr_status_string",
+           "qknr_last_error_detail", "qknr_abi_version")
 
 
 class QknrError(RuntimeError):
@@ -77,6 +78,10 @@ def lib() -> C.CDLL:
         L.qknr_rope_table.restype = C.c_int
         L.qknr_rope_3d.argtypes = [C.POINTER(Rope3DParams), vp]
         L.qknr_rope_3d.restype = C.c_int
+        L.qknr_rope_3d_partial_ssq.argtypes = [C.POINTER(Rope3DParams), vp, vp]
+        L.qknr_rope_3d_partial_ssq.restype = C.c_int
+        L.qknr_rope_3d_with_ssq.argtypes = [C.POINTER(Rope3DParams), vp, i32, i32, vp]
+        L.qknr_rope_3d_with_ssq.restype = C.c_int
         L.qknr_status_string.argtypes = [C.c_int]
         L.qknr_status_string.restype = C.c_char_p
         L.qknr_last_error_detail.restype = C.c_char_p
@@ -221,6 +226,29 @@ def qknr_rope_3d(qkv, q_weight, k_weight, q_out, k_out, v_out, *, stream=None, *
     _check(lib().qknr_rope_3d(C.byref(p), st))
 
 
+def qknr_rope_3d_partial_ssq(qkv, ssq_out, *, stream=None, **params) -> None:
+    """Tensor-parallel pass 1 through the C ABI: per-token sums of x^2 over this
+    call's Q and K heads into ssq_out (fp32 [tokens, 2])."""
+    p = make_3d_params(qkv, None, None, None, None, None, **params)
+    if ssq_out.dtype != torch.float32 or tuple(ssq_out.shape) != (p.num_tokens, 2) or \
+            not ssq_out.is_contiguous():
+        raise QknrValueError(QKNR_ERR_SHAPE, f"ssq_out must be a dense fp32 [{p.num_tokens}, 2]")
+    _check(lib().qknr_rope_3d_partial_ssq(C.byref(p), _ptr(ssq_out), _stream(stream, qkv)))
+
+
+def qknr_rope_3d_with_ssq(qkv, q_weight, k_weight, q_out, k_out, v_out, ssq, *, heads_q_total,
+                          heads_k_total, stream=None, **params) -> None:
+    """Tensor-parallel pass 3 through the C ABI: the 3D transform of this call's
+    heads with the all-reduced sums ssq (fp32 [tokens, 2]) over heads_q_total /
+    heads_k_total heads."""
+    p = make_3d_params(qkv, q_weight, k_weight, q_out, k_out, v_out, **params)
+    if ssq.dtype != torch.float32 or tuple(ssq.shape) != (p.num_tokens, 2) or \
+            not ssq.is_contiguous():
+        raise QknrValueError(QKNR_ERR_SHAPE, f"ssq must be a dense fp32 [{p.num_tokens}, 2]")
+    _check(lib().qknr_rope_3d_with_ssq(C.byref(p), _ptr(ssq), int(heads_q_total),
+                                       int(heads_k_total), _stream(stream, qkv, q_out)))
+
+
 def qknr_device_status(clear: bool = False, stream=None, device=None) -> int:
     """Device status word (bit 0: a kernel gave up waiting on its own bulk
     copy and left its outputs incomplete). Synchronises the stream."""
@@ -284,6 +312,7 @@ def fused_qk_rmsnorm_rope(qkv: torch.Tensor, q_weight: torch.Tensor, k_weight: t
     return tuple(outs)
 
 
-__all__ = ["qknr_rope_table", "qknr_rope_3d", "qknr_device_status", "fused_qk_norm_rope", "fused_qk_rmsnorm_rope",
+__all__ = ["qknr_rope_table", "qknr_rope_3d", "qknr_rope_3d_partial_ssq", "qknr_rope_3d_with_ssq",
+           "qknr_device_status", "fused_qk_norm_rope", "fused_qk_rmsnorm_rope",
            "QknrError", "QknrValueError", "lib", "build", "make_3d_params", "Rope3DParams",
            "EXPORTS", "LIB_PATH"]

@@ -32,7 +32,15 @@ struct Rope3DArgs {
     int32_t v_bulk;          // bf16 V leaves through a bulk store
     uint32_t stall_tx_bytes; // test hook: extra bytes a stage waits for (0 in use)
     uint64_t wait_limit_ns;  // a wait on a bulk copy gives up after this long
+    // Tensor-parallel head slices (see qknr_rope_3d_partial_ssq / _with_ssq):
+    int32_t mode;            // 0 whole transform, 1 partial sums only, 2 sums supplied
+    float* ssq_out;          // mode 1: [T][2] fp32 (sum Q^2, sum K^2) of this slice
+    const float* ssq_in;     // mode 2: [T][2] fp32 sums over all heads of all slices
+    int32_t norm_q_elems;    // channels the Q mean runs over (hq*D, or all heads' in mode 2)
+    int32_t norm_k_elems;
 };
+
+enum { kModeWhole = 0, kModePartialSsq = 1, kModeSuppliedSsq = 2 };
 
 struct RopeTableArgs {
     const uint8_t* q;  // bf16 [T, hq, D], token stride q_stride elements

@@ -280,12 +280,24 @@ int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
     return ok();
 }
 
-int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
+}  // extern "C"
+
+namespace {
+
+// The three 3D entry points share one body. mode: kModeWhole (the full
+// transform), kModePartialSsq (per-token sums of squares of this call's Q and
+// K heads into ssq_out only), kModeSuppliedSsq (the full transform with the
+// per-token sums taken from ssq_in, over heads_q_total / heads_k_total heads).
+int run_3d(const qknr_rope_3d_params* prm, int mode, float* ssq_out, const float* ssq_in,
+           int32_t heads_q_total, int32_t heads_k_total, void* cuda_stream) {
     if (!prm) return fail(QKNR_ERR_NULL, "params is NULL");
     if (prm->struct_size != sizeof(qknr_rope_3d_params))
         return fail(QKNR_ERR_SHAPE, "params.struct_size %zu != %zu (header mismatch)",
                     prm->struct_size, sizeof(qknr_rope_3d_params));
     const qknr_rope_3d_params& p = *prm;
+    const bool partial = mode == qknr::kModePartialSsq;
+    const bool supplied = mode == qknr::kModeSuppliedSsq;
+    const bool norm = partial || p.is_qk_norm;
     const int D = p.head_dim;
     if (D != 64 && D != 128 && D != 256)
         return fail(QKNR_ERR_SHAPE, "head_dim %d must be 64, 128 or 256", D);
@@ -317,39 +329,54 @@ int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
                     (double)p.factor);
     if (p.attention_factor != 1.0f)
         return fail(QKNR_ERR_SHAPE, "attention_factor must be 1.0 when factor is 1.0");
-    if (p.is_qk_norm && (!(p.eps >= 0.0f) || std::isinf(p.eps)))
+    if (norm && !partial && (!(p.eps >= 0.0f) || std::isinf(p.eps)))
         return fail(QKNR_ERR_SHAPE, "eps must be >= 0");
-    if (p.output_fp8 && (!std::isfinite(p.output_quant_scale) || !std::isfinite(p.v_quant_scale)))
+    if (!partial && p.output_fp8 &&
+        (!std::isfinite(p.output_quant_scale) || !std::isfinite(p.v_quant_scale)))
         return fail(QKNR_ERR_SHAPE, "FP8 scales must be finite");
+    if (supplied) {
+        if (!p.is_qk_norm) return fail(QKNR_ERR_SHAPE, "supplied sums need is_qk_norm = 1");
+        if (heads_q_total < p.num_heads_q || heads_k_total < p.num_heads_k)
+            return fail(QKNR_ERR_SHAPE, "heads_*_total (%d, %d) below this slice's heads (%d, %d)",
+                        heads_q_total, heads_k_total, p.num_heads_q, p.num_heads_k);
+    }
     if (p.num_tokens == 0) return ok();
 
     const int64_t T = p.num_tokens;
     const int64_t row = (int64_t)(p.num_heads_q + p.num_heads_k + p.num_heads_v) * D;
     const int ob = p.output_fp8 ? 1 : 2;
-    const bool hq = p.num_heads_q > 0, hk = p.num_heads_k > 0, hv = p.num_heads_v > 0;
+    const bool hq = p.num_heads_q > 0 && !partial, hk = p.num_heads_k > 0 && !partial;
+    const bool hv = p.num_heads_v > 0 && !partial;
+    const bool wq = norm && !partial && p.num_heads_q > 0, wk = norm && !partial && p.num_heads_k > 0;
     if (!p.qkv) return fail(QKNR_ERR_NULL, "qkv is NULL");
     if ((hq && !p.q_out) || (hk && !p.k_out) || (hv && !p.v_out))
         return fail(QKNR_ERR_NULL, "an output pointer is NULL");
-    if (p.is_qk_norm && ((hq && !p.q_weight) || (hk && !p.k_weight)))
+    if ((wq && !p.q_weight) || (wk && !p.k_weight))
         return fail(QKNR_ERR_NULL, "a weight pointer is NULL with is_qk_norm");
+    if (partial && !ssq_out) return fail(QKNR_ERR_NULL, "ssq_out is NULL");
+    if (supplied && !ssq_in) return fail(QKNR_ERR_NULL, "ssq is NULL");
     const Span sin_{p.qkv, (uint64_t)T * row * 2};
-    const Span so[3] = {{p.q_out, (uint64_t)T * p.num_heads_q * D * ob},
-                        {p.k_out, (uint64_t)T * p.num_heads_k * D * ob},
-                        {p.v_out, (uint64_t)T * p.num_heads_v * D * ob}};
-    const Span sw[2] = {{p.is_qk_norm ? p.q_weight : nullptr, (uint64_t)p.num_heads_q * D * 2},
-                        {p.is_qk_norm ? p.k_weight : nullptr, (uint64_t)p.num_heads_k * D * 2}};
-    for (int i = 0; i < 3; ++i) {
+    const Span so[4] = {{hq ? p.q_out : nullptr, (uint64_t)T * p.num_heads_q * D * ob},
+                        {hk ? p.k_out : nullptr, (uint64_t)T * p.num_heads_k * D * ob},
+                        {hv ? p.v_out : nullptr, (uint64_t)T * p.num_heads_v * D * ob},
+                        {ssq_out, (uint64_t)T * 8}};
+    const Span si[3] = {{wq ? p.q_weight : nullptr, (uint64_t)p.num_heads_q * D * 2},
+                        {wk ? p.k_weight : nullptr, (uint64_t)p.num_heads_k * D * 2},
+                        {ssq_in, (uint64_t)T * 8}};
+    for (int i = 0; i < 4; ++i) {
         if (overlap(so[i], sin_)) return fail(QKNR_ERR_ALIAS, "an output overlaps qkv");
         for (int j = 0; j < i; ++j)
             if (overlap(so[i], so[j])) return fail(QKNR_ERR_ALIAS, "two outputs overlap");
-        for (int j = 0; j < 2; ++j)
-            if (overlap(so[i], sw[j])) return fail(QKNR_ERR_ALIAS, "an output overlaps a weight");
+        for (int j = 0; j < 3; ++j)
+            if (overlap(so[i], si[j])) return fail(QKNR_ERR_ALIAS, "an output overlaps an input");
     }
     if (!aligned16(p.qkv) || (hq && !aligned16(p.q_out)) || (hk && !aligned16(p.k_out)) ||
         (hv && !aligned16(p.v_out)))
         return fail(QKNR_ERR_ALIGN, "qkv and the outputs must be 16-byte aligned");
-    if (p.is_qk_norm && ((hq && !aligned16(p.q_weight)) || (hk && !aligned16(p.k_weight))))
+    if ((wq && !aligned16(p.q_weight)) || (wk && !aligned16(p.k_weight)))
         return fail(QKNR_ERR_ALIGN, "weights must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(ssq_out) | reinterpret_cast<uintptr_t>(ssq_in)) & 7u)
+        return fail(QKNR_ERR_ALIGN, "the [T][2] sums must be 8-byte aligned");
 
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -371,13 +398,21 @@ int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
         if ((rc = classify(p.v_out, "v_out", dev, &ptr))) return rc;
         a.v_out = static_cast<uint8_t*>(const_cast<void*>(ptr));
     }
-    if (p.is_qk_norm && hq) {
+    if (wq) {
         if ((rc = classify(p.q_weight, "q_weight", dev, &ptr))) return rc;
         a.q_weight = static_cast<const uint8_t*>(ptr);
     }
-    if (p.is_qk_norm && hk) {
+    if (wk) {
         if ((rc = classify(p.k_weight, "k_weight", dev, &ptr))) return rc;
         a.k_weight = static_cast<const uint8_t*>(ptr);
+    }
+    if (partial) {
+        if ((rc = classify(ssq_out, "ssq_out", dev, &ptr))) return rc;
+        a.ssq_out = static_cast<float*>(const_cast<void*>(ptr));
+    }
+    if (supplied) {
+        if ((rc = classify(ssq_in, "ssq", dev, &ptr))) return rc;
+        a.ssq_in = static_cast<const float*>(ptr);
     }
     a.num_tokens = T;
     a.pos_offset = p.pos_offset % P;
@@ -390,7 +425,7 @@ int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
     a.hq = p.num_heads_q;
     a.hk = p.num_heads_k;
     a.hv = p.num_heads_v;
-    a.is_qk_norm = p.is_qk_norm ? 1 : 0;
+    a.is_qk_norm = norm ? 1 : 0;
     const int64_t entries = (int64_t)p.ppf * (cf / 2) + (int64_t)p.pph * (ch / 2) +
                             (int64_t)p.ppw * (cw / 2);
     a.table_entries = entries > (1 << 20) ? (1 << 20) + 1 : (int32_t)entries;
@@ -398,13 +433,40 @@ int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
     a.q_scale = p.output_quant_scale;
     a.v_scale = p.v_quant_scale;
     a.base = p.base;
+    a.mode = mode;
+    a.norm_q_elems = (supplied ? heads_q_total : p.num_heads_q) * D;
+    a.norm_k_elems = (supplied ? heads_k_total : p.num_heads_k) * D;
     a.stall_tx_bytes = g_fault_extra_bytes.load(std::memory_order_relaxed);
     a.wait_limit_ns = a.stall_tx_bytes ? g_fault_limit_ns.load() : 0;
     qknr::LaunchInfo info{};
-    e = qknr::launch_rope3d(a, D, p.interleave ? 0 : 1, p.output_fp8 ? 1 : 0,
+    e = qknr::launch_rope3d(a, D, p.interleave ? 0 : 1, (p.output_fp8 && !partial) ? 1 : 0,
                             static_cast<cudaStream_t>(cuda_stream), &info);
+    if (e == cudaErrorNotSupported) {
+        cudaGetLastError();
+        return fail(QKNR_ERR_UNSUPPORTED,
+                    "a row of %lld bytes is too long for the pipelined kernel that the "
+                    "tensor-parallel passes need", (long long)(row * 2));
+    }
     if (e != cudaSuccess) return cuda_fail(e, "3D kernel launch");
     return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
+    return run_3d(prm, qknr::kModeWhole, nullptr, nullptr, 0, 0, cuda_stream);
+}
+
+int qknr_rope_3d_partial_ssq(const qknr_rope_3d_params* prm, float* ssq_out, void* cuda_stream) {
+    return run_3d(prm, qknr::kModePartialSsq, ssq_out, nullptr, 0, 0, cuda_stream);
+}
+
+int qknr_rope_3d_with_ssq(const qknr_rope_3d_params* prm, const float* ssq,
+                          int32_t heads_q_total, int32_t heads_k_total, void* cuda_stream) {
+    return run_3d(prm, qknr::kModeSuppliedSsq, nullptr, ssq, heads_q_total, heads_k_total,
+                  cuda_stream);
 }
 
 }  // extern "C"

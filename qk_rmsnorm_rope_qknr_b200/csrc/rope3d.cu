@@ -318,10 +318,15 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
 
     const int G = a.groups;
     const int Bg = blockDim.x / G;  // threads per group, a multiple of 32
-    const int row_bytes = (a.hq + a.hk + a.hv) * D * 2;
+    const bool partial = a.mode == kModePartialSsq;  // sums of squares only
+    const bool supplied = a.mode == kModeSuppliedSsq;  // sums come from ssq_in
+    const int row_bytes = (a.hq + a.hk + a.hv) * D * 2;  // token stride in qkv
+    // A partial pass needs only the Q and K part of each row.
+    const int stage_bytes = partial ? (a.hq + a.hk) * D * 2 : row_bytes;
     const int stages = a.stages;
     const bool norm = a.is_qk_norm != 0;
-    const MgLayout lay = mg_layout(D, G, stages, row_bytes, norm ? (a.hq + a.hk) * D : 0,
+    const MgLayout lay = mg_layout(D, G, stages, stage_bytes,
+                                   (norm && !partial) ? (a.hq + a.hk) * D : 0,
                                    a.use_table ? a.table_entries * 8 : 0);
     extern __shared__ __align__(128) unsigned char smem[];
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + lay.abort);
@@ -332,14 +337,14 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
     const int tid = threadIdx.x;
     const int g = tid / Bg;
     const int ctid = tid - g * Bg;
-    unsigned char* ring = smem + lay.ring + (size_t)g * stages * row_bytes;
+    unsigned char* ring = smem + lay.ring + (size_t)g * stages * stage_bytes;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.full) + g * stages;
     float* cst = reinterpret_cast<float*>(smem + lay.cst) + g * 2 * L * kCsPitch;
     float2* red = reinterpret_cast<float2*>(smem + lay.red) + g * 64;
 
     const int64_t NP = (int64_t)gridDim.x * G;  // pipelines in the grid
-    const uint32_t tx = (uint32_t)row_bytes + a.stall_tx_bytes;
-    const int vbytes = a.hv * D * 2;
+    const uint32_t tx = (uint32_t)stage_bytes + a.stall_tx_bytes;
+    const int vbytes = partial ? 0 : a.hv * D * 2;
     const bool v_bulk = a.v_bulk && vbytes > 0;
     const size_t v_off = (size_t)(a.hq + a.hk) * D * 2;  // V inside a row
 
@@ -351,16 +356,16 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
         // First `stages` rows of every pipeline.
         for (int q = 0; q < G; ++q) {
             const int64_t p = (int64_t)blockIdx.x * G + q;
-            unsigned char* rq = smem + lay.ring + (size_t)q * stages * row_bytes;
+            unsigned char* rq = smem + lay.ring + (size_t)q * stages * stage_bytes;
             uint64_t* fq = reinterpret_cast<uint64_t*>(smem + lay.full) + q * stages;
             for (int i = 0; i < stages && p + i * NP < a.num_tokens; ++i) {
                 mbar_arrive_expect_tx(&fq[i], tx);
-                bulk_load(rq + (size_t)i * row_bytes, a.qkv + (p + i * NP) * row_bytes,
-                          row_bytes, &fq[i]);
+                bulk_load(rq + (size_t)i * stage_bytes, a.qkv + (p + i * NP) * row_bytes,
+                          stage_bytes, &fq[i]);
             }
         }
     }
-    if (norm) {
+    if (norm && !partial) {
         // fp32 weights, float4 index (h*2 + m)*VPH + v for channels 8v+4m..+3 of head h.
         const int nq4 = a.hq * VPH * 2, n4 = (a.hq + a.hk) * VPH * 2;
         for (int q = tid; q < n4; q += blockDim.x) {
@@ -375,7 +380,7 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
     // Partial sums of warps a group does not have stay zero.
     for (int q = tid; q < G * 64; q += blockDim.x)
         reinterpret_cast<float2*>(smem + lay.red)[q] = make_float2(0.0f, 0.0f);
-    setup_angles<D>(a, gq, tab);
+    if (!partial) setup_angles<D>(a, gq, tab);
     __syncthreads();
 
     // ------------------------------ one pipeline ------------------------------
@@ -415,8 +420,8 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
         const int col = axis == 0 ? j : (axis == 1 ? j - hcf : j - hcf - hch);
         stage_code = (uint32_t)(rl * kCsPitch + k) | ((uint32_t)axis << 11) | ((uint32_t)col << 13);
     }
-    const float inv_nq = 1.0f / (float)(a.hq * D > 0 ? a.hq * D : 1);
-    const float inv_nk = 1.0f / (float)(a.hk * D > 0 ? a.hk * D : 1);
+    const float inv_nq = 1.0f / (float)(a.norm_q_elems > 0 ? a.norm_q_elems : 1);
+    const float inv_nk = 1.0f / (float)(a.norm_k_elems > 0 ? a.norm_k_elems : 1);
     const int vout_bytes = a.hv * D * OUTB;
 
     int64_t i = 0;
@@ -429,14 +434,14 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
     for (; i < n_local; ++i, t += NP) {
         const int parity = (int)(i & 1);
         const bool ok = mbar_wait_abortable(&full[stage], phase, a.wait_limit_ns, abort_flag);
-        const unsigned char* row = ring + (size_t)stage * row_bytes;
+        const unsigned char* row = ring + (size_t)stage * stage_bytes;
         if (ctid == 0 && ok && v_bulk) {
             bulk_store(a.v_out + t * vbytes, row + v_off, (uint32_t)vbytes);
             bulk_commit();
         }
         float2 sq2 = make_float2(0.0f, 0.0f), sk2 = make_float2(0.0f, 0.0f);
         if (ok) {
-            if (norm) {
+            if (norm && !supplied) {
 #pragma unroll
                 for (int k = 0; k < S; ++k) {
                     const int slot = ctid + k * Bg;
@@ -451,7 +456,7 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
                     }
                 }
             }
-            if (!v_bulk) {
+            if (!v_bulk && !partial) {
                 const unsigned char* vrow = row + v_off;
                 uint8_t* vout = a.v_out + t * vout_bytes;
                 const float2 vs2 = make_float2(a.v_scale, a.v_scale);
@@ -471,7 +476,7 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
             }
         }
         // This token's cos/sin, staged per l-row: [c_0..c_7][s_0..s_7][pad].
-        {
+        if (!partial) {
             float* cp = cst + parity * L * kCsPitch;
             if (HALF <= Bg) {
                 if (ctid < HALF) {  // whole warps: HALF is a multiple of 32
@@ -506,7 +511,7 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
                 }
             }
         }
-        if (norm) {
+        if (norm && !supplied) {
             const float sq = warp_sum(sq2.x + sq2.y);
             const float sk = warp_sum(sk2.x + sk2.y);
             if (lane == 0) red[parity * 32 + cwarp] = make_float2(sq, sk);
@@ -525,8 +530,8 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
             if (v_bulk) bulk_wait_read_all();
             fence_proxy_async_smem();
             mbar_arrive_expect_tx(&full[prev_stage], tx);
-            bulk_load(ring + (size_t)prev_stage * row_bytes,
-                      a.qkv + (t + (stages - 1) * NP) * row_bytes, row_bytes, &full[prev_stage]);
+            bulk_load(ring + (size_t)prev_stage * stage_bytes,
+                      a.qkv + (t + (stages - 1) * NP) * row_bytes, stage_bytes, &full[prev_stage]);
         }
         prev_stage = stage;
         if (++stage == stages) {
@@ -542,15 +547,26 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
 
         float rq = 1.0f, rk = 1.0f;
         if (norm) {
-            // (sum Q^2, sum K^2) partials of the warps, two warps per 16-byte read
-            const float4* r4 = reinterpret_cast<const float4*>(red + parity * 32);
-            float4 acc = r4[0];
-            for (int w = 1; w < (nwarps + 1) >> 1; ++w) {
-                const float4 v = r4[w];
-                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            float tq, tk;
+            if (supplied) {  // sums over every slice's heads, from the caller
+                const float2 v = reinterpret_cast<const float2*>(a.ssq_in)[t];
+                tq = v.x; tk = v.y;
+            } else {
+                // (sum Q^2, sum K^2) partials of the warps, two warps per 16-byte read
+                const float4* r4 = reinterpret_cast<const float4*>(red + parity * 32);
+                float4 acc = r4[0];
+                for (int w = 1; w < (nwarps + 1) >> 1; ++w) {
+                    const float4 v = r4[w];
+                    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+                }
+                tq = acc.x + acc.z; tk = acc.y + acc.w;
             }
-            rq = rsqrtf((acc.x + acc.z) * inv_nq + a.eps);
-            rk = rsqrtf((acc.y + acc.w) * inv_nk + a.eps);
+            if (partial) {  // this slice's sums are the whole result
+                if (ctid == 0) reinterpret_cast<float2*>(a.ssq_out)[t] = make_float2(tq, tk);
+                continue;
+            }
+            rq = rsqrtf(tq * inv_nq + a.eps);
+            rk = rsqrtf(tk * inv_nk + a.eps);
             if (FP8) {  // E4M3(value * scale): the scale rides on r
                 rq *= a.q_scale;
                 rk *= a.q_scale;
@@ -752,11 +768,14 @@ template <int D, bool NEOX, bool FP8, int S>
 cudaError_t run(const Rope3DArgs& a, int block, cudaStream_t stream, LaunchInfo* info) {
     constexpr int HALF = D / 2;
     Rope3DArgs args = a;
+    const bool partial = a.mode == kModePartialSsq;
     const int table_bytes = a.table_entries * 8;
-    args.use_table = table_bytes <= kMaxTableBytes ? 1 : 0;
+    args.use_table = (!partial && table_bytes <= kMaxTableBytes) ? 1 : 0;
     const int used_table = args.use_table ? table_bytes : 0;
-    const int row_bytes = (a.hq + a.hk + a.hv) * D * 2;
-    const int weight_floats = a.is_qk_norm ? (a.hq + a.hk) * D : 0;
+    const int row_bytes = partial ? (a.hq + a.hk) * D * 2 : (a.hq + a.hk + a.hv) * D * 2;
+    const int weight_floats = (a.is_qk_norm && !partial) ? (a.hq + a.hk) * D : 0;
+    if (args.norm_q_elems == 0) args.norm_q_elems = a.hq * D;
+    if (args.norm_k_elems == 0) args.norm_k_elems = a.hk * D;
     // Pipelines per CTA: as many groups as fit in 24 warps and in shared memory,
     // each with a ring of 3 row buffers (2 if 3 do not fit even for one group).
     const int warps = block / 32;
@@ -791,6 +810,8 @@ cudaError_t run(const Rope3DArgs& a, int block, cudaStream_t stream, LaunchInfo*
         }
         id = 3100;
         block *= groups;
+    } else if (a.mode != kModeWhole) {
+        return cudaErrorNotSupported;  // the tensor-parallel passes run on the pipelined kernel
     } else {
         smem = 2 * HALF * 8 + 64 * 8 + HALF * 8 + used_table;
         e = launch_grid(rope3d_reg_kernel<D, NEOX, FP8, S>, block, smem, a.num_tokens, args,

@@ -194,3 +194,28 @@ def test_wait_fault_hook_argument_checks(L):
     assert L.qknr_test_set_wait_fault(8, 1000) == Q.QKNR_ERR_SHAPE
     assert L.qknr_test_set_wait_fault(16, 0) == Q.QKNR_ERR_SHAPE
     assert L.qknr_test_set_wait_fault(0, 0) == Q.QKNR_OK
+
+
+def test_tensor_parallel_entry_point_checks(L):
+    p = _p3()
+    assert L.qknr_rope_3d_partial_ssq(C.byref(p), None, None) == Q.QKNR_ERR_NULL
+    assert L.qknr_rope_3d_partial_ssq(C.byref(p), A + (6 << 30) + 4, None) == Q.QKNR_ERR_ALIGN
+    assert L.qknr_rope_3d_partial_ssq(C.byref(p), A + 64, None) == Q.QKNR_ERR_ALIAS  # inside qkv
+    assert L.qknr_rope_3d_with_ssq(C.byref(p), None, 4, 4, None) == Q.QKNR_ERR_NULL
+    assert L.qknr_rope_3d_with_ssq(C.byref(p), A + (6 << 30), 3, 4, None) == Q.QKNR_ERR_SHAPE
+    p2 = _p3(is_qk_norm=False)
+    assert L.qknr_rope_3d_with_ssq(C.byref(p2), A + (6 << 30), 4, 4, None) == Q.QKNR_ERR_SHAPE
+    assert b"is_qk_norm" in L.qknr_last_error_detail()
+    p3 = _p3()
+    p3.q_out = A + (6 << 30)  # overlaps the supplied sums
+    assert L.qknr_rope_3d_with_ssq(C.byref(p3), A + (6 << 30), 4, 4, None) == Q.QKNR_ERR_ALIAS
+
+
+def test_tp_head_slices():
+    from qk_rmsnorm_rope_qknr_b200 import tp
+
+    for total in (1, 5, 24, 32):
+        for world in (1, 2, 3, 4, 8):
+            sl = [tp.head_slice(total, world, r) for r in range(world)]
+            assert sl[0][0] == 0 and sl[-1][1] == total
+            assert all(a[1] == b[0] for a, b in zip(sl, sl[1:]))

@@ -81,6 +81,60 @@ def _worker(rank, port, out_dir):
         dist.destroy_process_group()
 
 
+def _tp_worker(rank, port, out_dir):
+    """Head-sharded (tensor-parallel) exchange: each rank sums x^2 over its own
+    heads, tp.all_reduce_ssq adds the ranks' sums, and the rank's heads,
+    normalised with the global sums and rotated with the oracle's own steps,
+    equal the oracle's unsplit call."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD)
+    try:
+        import oracle as O
+        from qk_rmsnorm_rope_qknr_b200 import tp
+        from tests._util import t2u16
+
+        D, Hq, Hk, Hv, T, eps = 32, 3, 2, 1, 30, 1e-5
+        g = torch.Generator().manual_seed(11)
+        qkv = torch.randn(T, (Hq + Hk + Hv) * D, generator=g).to(torch.bfloat16)
+        qw = (1 + 0.1 * torch.randn(Hq * D, generator=g)).to(torch.bfloat16)
+        kw = (1 + 0.1 * torch.randn(Hk * D, generator=g)).to(torch.bfloat16)
+        p = dict(P3, num_heads_q=Hq, num_heads_k=Hk, num_heads_v=Hv, eps=eps)
+        full_q, full_k, _ = O.rope_3d(t2u16(qkv), t2u16(qw), t2u16(kw), exact=True, **p)
+        sq, sk = tp.head_slice(Hq, WORLD, rank), tp.head_slice(Hk, WORLD, rank)
+        x = qkv.double()
+        xq = x[:, sq[0] * D:sq[1] * D]
+        xk = x[:, (Hq + sk[0]) * D:(Hq + sk[1]) * D]
+        ssq = torch.stack([xq.pow(2).sum(1), xk.pow(2).sum(1)], 1).float()
+        tp.all_reduce_ssq(ssq)
+        want = torch.stack([x[:, :Hq * D].pow(2).sum(1), x[:, Hq * D:(Hq + Hk) * D].pow(2).sum(1)],
+                           1)
+        assert torch.allclose(ssq.double(), want, rtol=1e-6)
+        pa, pb = O.pairs_3d(8, 12, 12, False)
+        for X, xs, sl, w, tot, col, full in ((0, xq, sq, qw, Hq, 0, full_q),
+                                             (1, xk, sk, kw, Hk, 1, full_k)):
+            r = 1.0 / np.sqrt(ssq[:, col].double().numpy() / (tot * D) + eps)
+            wv = O.bf16_to_f64(t2u16(w))[sl[0] * D:sl[1] * D]
+            for t in range(T):
+                th = O.angles_3d(*O.position_3d(t, 0, 3, 2, 5), 8, 12, 12, 10000.0)
+                y = xs[t].numpy() * r[t] * wv
+                for hh in range(sl[1] - sl[0]):
+                    out = O.rotate(y[hh * D:(hh + 1) * D], pa, pb, np.cos(th), np.sin(th))
+                    assert np.allclose(out, full[t, sl[0] + hh], rtol=0, atol=1e-5), (X, t, hh)
+        dist.barrier()
+        open(os.path.join(out_dir, f"tp{rank}"), "w").write("ok")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_tensor_parallel_exchange_over_gloo(tmp_path):
+    port = _free_port()
+    mp.start_processes(_tp_worker, args=(port, str(tmp_path)), nprocs=WORLD, join=True,
+                       start_method="spawn")
+    for r in range(WORLD):
+        assert (tmp_path / f"tp{r}").read_text() == "ok"
+
+
 def test_token_shard_arithmetic():
     for T in (0, 1, 5, 72, 15360, 59521):
         for world in (1, 2, 3, 8):
