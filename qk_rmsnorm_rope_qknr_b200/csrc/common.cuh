@@ -255,6 +255,18 @@ __device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred
     return r != 0;
 }
 
+// Programmatic dependent launch. wait: block this thread until the grids this
+// launch depends on have completed and their memory is visible (a no-op when
+// the launch did not opt in). launch_dependents: let the next grid on the
+// stream start scheduling its blocks (they still wait for this grid before
+// touching memory it may write).
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Plain barrier over the first `nthreads` threads at named barrier `id`.
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -348,11 +348,15 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
     const bool v_bulk = a.v_bulk && vbytes > 0;
     const size_t v_off = (size_t)(a.hq + a.hk) * D * 2;  // V inside a row
 
+    // Everything up to griddep_wait() touches only shared memory and the
+    // arguments, so with a programmatic dependent launch it overlaps the end
+    // of the previous kernel on the stream.
     if (tid == 0) {
         for (int q = 0; q < G * stages; ++q)
             mbar_init(reinterpret_cast<uint64_t*>(smem + lay.full) + q, 1);
         *abort_flag = 0u;
         fence_mbar_init();
+        griddep_wait();
         // First `stages` rows of every pipeline.
         for (int q = 0; q < G; ++q) {
             const int64_t p = (int64_t)blockIdx.x * G + q;
@@ -365,6 +369,12 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
             }
         }
     }
+    // Partial sums of warps a group does not have stay zero.
+    for (int q = tid; q < G * 64; q += blockDim.x)
+        reinterpret_cast<float2*>(smem + lay.red)[q] = make_float2(0.0f, 0.0f);
+    if (!partial) setup_angles<D>(a, gq, tab);
+    griddep_wait();
+    griddep_launch_dependents();
     if (norm && !partial) {
         // fp32 weights, float4 index (h*2 + m)*VPH + v for channels 8v+4m..+3 of head h.
         const int nq4 = a.hq * VPH * 2, n4 = (a.hq + a.hk) * VPH * 2;
@@ -377,10 +387,6 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
             wsm[q] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
         }
     }
-    // Partial sums of warps a group does not have stay zero.
-    for (int q = tid; q < G * 64; q += blockDim.x)
-        reinterpret_cast<float2*>(smem + lay.red)[q] = make_float2(0.0f, 0.0f);
-    if (!partial) setup_angles<D>(a, gq, tab);
     __syncthreads();
 
     // ------------------------------ one pipeline ------------------------------
@@ -737,6 +743,25 @@ __global__ void __launch_bounds__(kMaxBlock) rope3d_reg_kernel(const Rope3DArgs 
     }
 }
 
+// Launch with programmatic stream serialisation: the kernel may start its
+// prologue while the previous kernel on the stream finishes (the kernel waits
+// with griddepcontrol.wait before it touches global memory).
+template <typename K, typename A>
+cudaError_t launch_overlapped(K kern, int grid, int block, int smem, cudaStream_t stream,
+                              const A& args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args);
+}
+
 int device_sms() {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -805,8 +830,7 @@ cudaError_t run(const Rope3DArgs& a, int block, cudaStream_t stream, LaunchInfo*
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e == cudaSuccess) {
             grid = (int)std::min<int64_t>(sms, (a.num_tokens + groups - 1) / groups);
-            kern<<<grid, block * groups, smem, stream>>>(args);
-            e = cudaGetLastError();
+            e = launch_overlapped(kern, grid, block * groups, smem, stream, args);
         }
         id = 3100;
         block *= groups;

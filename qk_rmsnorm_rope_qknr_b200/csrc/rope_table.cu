@@ -127,6 +127,10 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
         for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
     }
+    // Global memory only after the previous kernel on the stream is done (a
+    // no-op unless launched as a programmatic dependent launch).
+    griddep_wait();
+    griddep_launch_dependents();
     for (int c = threadIdx.x; c < 2 * D; c += blockDim.x) {
         const uint16_t* w = reinterpret_cast<const uint16_t*>(c < D ? a.q_weight : a.k_weight);
         const int cc = c < D ? c : c - D;
@@ -413,14 +417,24 @@ cudaError_t launch_bulk(K kern, const RopeTableArgs& a0, int per_item, cudaStrea
     const int64_t want_blocks = (items + warps - 1) / warps;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * per_sm,
                                                                  want_blocks));
-    kern<<<grid, kBlock, smem, stream>>>(a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kBlock);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, a);
     if (info) {
         info->grid = grid;
         info->block = kBlock;
         info->smem = smem;
         info->kernel_id = id;
     }
-    return cudaGetLastError();
+    return e;
 }
 
 template <int GS>
