@@ -6,7 +6,8 @@ shares no code with it (the C source is compiled on its own by oracle/build.py).
 
 Everything here is numpy-in / numpy-out marshalling around the C functions in
 qknr_oracle.c; the arithmetic, and the readings R1..R12 of the pages, are
-stated there. bf16 values travel as uint16 bit patterns, E4M3 as uint8.
+stated there. bf16 and binary16 values travel as uint16 bit patterns, E4M3 as
+uint8.
 
 Parity status: every function is pinned by tests/test_oracle_pins.py except
 two readings the pages cannot decide -- the 3D NeoX pair layout (whole-head
@@ -46,6 +47,13 @@ def lib(path=None):
         L.qknr_oracle_e4m3_from_double.argtypes = [f64]
         L.qknr_oracle_e4m3_from_double.restype = C.c_uint8
         L.qknr_oracle_bf16_from_double_array.argtypes = [vp, vp, i64]
+        L.qknr_oracle_f16_from_double_array.argtypes = [vp, vp, i64]
+        L.qknr_oracle_f16_to_double.argtypes = [C.c_uint16]
+        L.qknr_oracle_f16_to_double.restype = f64
+        L.qknr_oracle_rope_table_exact_act.argtypes = [vp, vp, vp, vp, vp, i32, i32, i64, i32,
+                                                       i32, i32, i32, f64, i32, vp, vp]
+        L.qknr_oracle_rope_table_act.argtypes = [vp, vp, vp, vp, vp, i32, i32, i64, i32, i32,
+                                                 i32, i32, f64, i32, vp, vp]
         L.qknr_oracle_e4m3_from_double_array.argtypes = [vp, vp, i64]
         L.qknr_oracle_rmsnorm.argtypes = [vp, i64, vp, f64, vp]
         L.qknr_oracle_rotate.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
@@ -92,6 +100,19 @@ def bf16_from_f64(x):
     out = np.empty(x.shape, np.uint16)
     lib().qknr_oracle_bf16_from_double_array(_p(x), _p(out), x.size)
     return out
+
+
+def f16_from_f64(x):
+    """One RNE rounding of float64 values to IEEE binary16 bit patterns."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, np.uint16)
+    lib().qknr_oracle_f16_from_double_array(_p(x), _p(out), x.size)
+    return out
+
+
+def f16_to_f64(bits):
+    """binary16 bit patterns -> exact float64 values."""
+    return np.ascontiguousarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
 
 
 def e4m3_from_f64(x):
@@ -159,10 +180,11 @@ def angles_3d(f, h, w, cf, ch, cw, base):
 
 # ------------------------------------------------------------- table form --
 def rope_table(q, k, q_weight, k_weight, table, eps, rotary_dim=None, interleaved=False,
-               exact=False):
-    """Table form. q [T,Hq,D], k [T,Hk,D], weights [D] (uint16 bf16 bits);
-    table [T, rotary_dim] as float32 or uint16 bf16 bits. Returns (q_out, k_out)
-    as bf16 bits, or as float64 before rounding when exact=True."""
+               exact=False, act="bf16"):
+    """Table form. q [T,Hq,D], k [T,Hk,D], weights [D] (uint16 bit patterns of
+    the activation type `act`, "bf16" or "f16"); table [T, rotary_dim] as
+    float32 or uint16 patterns of the activation type. Returns (q_out, k_out) as
+    activation-type bits, or as float64 before rounding when exact=True."""
     q, k = _u16(q), _u16(k)
     qw, kw = _u16(q_weight), _u16(k_weight)
     T, Hq, D = q.shape
@@ -172,18 +194,18 @@ def rope_table(q, k, q_weight, k_weight, table, eps, rotary_dim=None, interleave
     is_f32 = tbl.dtype == np.float32
     assert is_f32 or tbl.dtype == np.uint16
     assert tbl.shape == (T, R), (tbl.shape, T, R)
+    assert act in ("bf16", "f16")
+    f16 = int(act == "f16")
     if exact:
         qo = np.empty(q.shape, np.float64)
         ko = np.empty(k.shape, np.float64)
-        fn = lib().qknr_oracle_rope_table_exact
-        rc = fn(_p(q), _p(k), _p(qw), _p(kw), _p(tbl), int(is_f32), T, Hq, Hk, D, R, float(eps),
-                int(interleaved), _p(qo), _p(ko))
+        fn = lib().qknr_oracle_rope_table_exact_act
     else:
         qo = np.empty(q.shape, np.uint16)
         ko = np.empty(k.shape, np.uint16)
-        fn = lib().qknr_oracle_rope_table
-        rc = fn(_p(q), _p(k), _p(qw), _p(kw), _p(tbl), int(is_f32), T, Hq, Hk, D, R, float(eps),
-                int(interleaved), _p(qo), _p(ko))
+        fn = lib().qknr_oracle_rope_table_act
+    rc = fn(_p(q), _p(k), _p(qw), _p(kw), _p(tbl), int(is_f32), f16, T, Hq, Hk, D, R, float(eps),
+            int(interleaved), _p(qo), _p(ko))
     if rc != 0:
         raise ValueError("oracle rejected the table-form arguments")
     return qo, ko
@@ -235,7 +257,8 @@ def set_threads(n):
     lib().qknr_oracle_set_threads(int(n))
 
 
-__all__ = ["bf16_to_f64", "bf16_from_f64", "e4m3_from_f64", "e4m3_to_f64", "rmsnorm",
+__all__ = ["bf16_to_f64", "bf16_from_f64", "f16_from_f64", "f16_to_f64", "e4m3_from_f64",
+           "e4m3_to_f64", "rmsnorm",
            "pairs_table", "pairs_3d", "rotate", "position_3d", "angles_3d", "rope_table",
            "rope_3d", "threads", "set_threads", "lib"]
 _ = os

@@ -42,6 +42,9 @@
  *   R11 With is_qk_norm off, Q/K are only rotated (weights and eps unused).
  *   R12 Table form: channels at and beyond rotary_dim are normalised but not
  *       rotated.
+ *   R13 Table form activations may be bf16 or IEEE binary16 ([T]: the table is
+ *       "either the activation dtype or float32"); weights share the
+ *       activation type, outputs are rounded once to it.
  *
  * Threads: the per-token loops run under OpenMP when it is enabled; every
  * token is computed independently, so the results do not depend on the
@@ -139,6 +142,44 @@ uint8_t qknr_oracle_e4m3_from_double(double x)
     int E = leading_exponent(v);
     int m = (int)((v / ldexp(1.0, E) - 1.0) * 8.0);
     return (uint8_t)(sign | (uint8_t)(((E + 7) << 3) | m));
+}
+
+/* IEEE binary16 value of a 16-bit pattern, exactly (sign, 5 exponent bits with
+ * bias 15, 10 fraction bits; exponent 0 is subnormal m 2^-24; 31 is inf/NaN). */
+double qknr_oracle_f16_to_double(uint16_t b)
+{
+    double s = (b & 0x8000u) ? -1.0 : 1.0;
+    int e = (b >> 10) & 0x1F;
+    int m = b & 0x3FF;
+    if (e == 31) return m ? NAN : s * INFINITY;
+    if (e == 0) return s * ldexp((double)m, -24);
+    return s * ldexp(1.0 + m / 1024.0, e - 15);
+}
+
+/* One round-to-nearest-even rounding of x to binary16 (11 significant bits,
+ * normal exponents -14..15, subnormal spacing 2^-24; overflow gives inf). */
+uint16_t qknr_oracle_f16_from_double(double x)
+{
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    if (isnan(x)) return (uint16_t)(sign | 0x7E00u);
+    double a = fabs(x);
+    if (isinf(a)) return (uint16_t)(sign | 0x7C00u);
+    if (a == 0.0) return sign;
+    int e = leading_exponent(a);
+    if (e < -14) e = -14;
+    double quantum = ldexp(1.0, e - 10);
+    double v = round_half_even(a / quantum) * quantum;
+    if (v >= 65536.0) return (uint16_t)(sign | 0x7C00u);
+    if (v == 0.0) return sign;
+    if (v < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)(v / ldexp(1.0, -24)));
+    int E = leading_exponent(v);
+    int m = (int)((v / ldexp(1.0, E) - 1.0) * 1024.0);
+    return (uint16_t)(sign | (uint16_t)(((E + 15) << 10) | m));
+}
+
+void qknr_oracle_f16_from_double_array(const double* x, uint16_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = qknr_oracle_f16_from_double(x[i]);
 }
 
 void qknr_oracle_bf16_from_double_array(const double* x, uint16_t* out, int64_t n)
@@ -248,11 +289,18 @@ void qknr_oracle_angles_3d(int64_t f, int64_t h, int64_t w, int32_t Cf, int32_t 
  * k [T, Hk, D] bf16 inputs, [D] bf16 weights and a [T, rotary_dim] table
  * holding cos(theta) in its first rotary_dim/2 columns and sin(theta) in the
  * rest, stored as fp32 (table_is_f32) or bf16. Outputs are fp64, same layout. */
-int qknr_oracle_rope_table_exact(const uint16_t* q, const uint16_t* k, const uint16_t* q_weight,
-                                 const uint16_t* k_weight, const void* table,
-                                 int32_t table_is_f32, int64_t num_tokens, int32_t heads_q,
-                                 int32_t heads_k, int32_t head_dim, int32_t rotary_dim,
-                                 double eps, int32_t interleaved, double* q_out, double* k_out)
+/* 16-bit activation pattern -> value: bf16, or binary16 when act_is_f16. */
+static double act_to_double(uint16_t b, int32_t act_is_f16)
+{
+    return act_is_f16 ? qknr_oracle_f16_to_double(b) : qknr_oracle_bf16_to_double(b);
+}
+
+int qknr_oracle_rope_table_exact_act(const uint16_t* q, const uint16_t* k,
+                                     const uint16_t* q_weight, const uint16_t* k_weight,
+                                     const void* table, int32_t table_is_f32, int32_t act_is_f16,
+                                     int64_t num_tokens, int32_t heads_q, int32_t heads_k,
+                                     int32_t head_dim, int32_t rotary_dim, double eps,
+                                     int32_t interleaved, double* q_out, double* k_out)
 {
     int32_t D = head_dim, R = rotary_dim;
     if (D <= 0 || D > 256 || R <= 0 || R > D || (R & 1)) return 1;
@@ -261,8 +309,8 @@ int qknr_oracle_rope_table_exact(const uint16_t* q, const uint16_t* k, const uin
     int32_t* pa = malloc(sizeof(int32_t) * (R / 2));
     int32_t* pb = malloc(sizeof(int32_t) * (R / 2));
     for (int32_t d = 0; d < D; ++d) {
-        wq[d] = qknr_oracle_bf16_to_double(q_weight[d]);
-        wk[d] = qknr_oracle_bf16_to_double(k_weight[d]);
+        wq[d] = act_to_double(q_weight[d], act_is_f16);
+        wk[d] = act_to_double(k_weight[d], act_is_f16);
     }
     qknr_oracle_pairs_table(R, interleaved, pa, pb);
 
@@ -276,8 +324,8 @@ int qknr_oracle_rope_table_exact(const uint16_t* q, const uint16_t* k, const uin
                 s[j] = row[R / 2 + j];
             } else {
                 const uint16_t* row = (const uint16_t*)table + t * R;
-                c[j] = qknr_oracle_bf16_to_double(row[j]);
-                s[j] = qknr_oracle_bf16_to_double(row[R / 2 + j]);
+                c[j] = act_to_double(row[j], act_is_f16);
+                s[j] = act_to_double(row[R / 2 + j], act_is_f16);
             }
         }
         for (int pass = 0; pass < 2; ++pass) {
@@ -287,7 +335,7 @@ int qknr_oracle_rope_table_exact(const uint16_t* q, const uint16_t* k, const uin
             const double* wt = pass ? wk : wq;
             for (int32_t hh = 0; hh < H; ++hh) {
                 const uint16_t* xr = src + (t * H + hh) * D;
-                for (int32_t d = 0; d < D; ++d) x[d] = qknr_oracle_bf16_to_double(xr[d]);
+                for (int32_t d = 0; d < D; ++d) x[d] = act_to_double(xr[d], act_is_f16);
                 qknr_oracle_rmsnorm(x, D, wt, eps, y);
                 qknr_oracle_rotate(y, D, R / 2, pa, pb, c, s, dst + (t * H + hh) * D);
             }
@@ -300,26 +348,53 @@ int qknr_oracle_rope_table_exact(const uint16_t* q, const uint16_t* k, const uin
     return 0;
 }
 
-/* Table form rounded to bf16 outputs (R3). */
-int qknr_oracle_rope_table(const uint16_t* q, const uint16_t* k, const uint16_t* q_weight,
-                           const uint16_t* k_weight, const void* table, int32_t table_is_f32,
-                           int64_t num_tokens, int32_t heads_q, int32_t heads_k,
-                           int32_t head_dim, int32_t rotary_dim, double eps, int32_t interleaved,
-                           uint16_t* q_out, uint16_t* k_out)
+int qknr_oracle_rope_table_exact(const uint16_t* q, const uint16_t* k, const uint16_t* q_weight,
+                                 const uint16_t* k_weight, const void* table,
+                                 int32_t table_is_f32, int64_t num_tokens, int32_t heads_q,
+                                 int32_t heads_k, int32_t head_dim, int32_t rotary_dim,
+                                 double eps, int32_t interleaved, double* q_out, double* k_out)
+{
+    return qknr_oracle_rope_table_exact_act(q, k, q_weight, k_weight, table, table_is_f32, 0,
+                                            num_tokens, heads_q, heads_k, head_dim, rotary_dim,
+                                            eps, interleaved, q_out, k_out);
+}
+
+/* Table form rounded to the activation type (R3): bf16, or binary16 when
+ * act_is_f16 (the pages allow the table in "the activation dtype or float32",
+ * so activations other than bf16 exist; binary16 is the other 16-bit one). */
+int qknr_oracle_rope_table_act(const uint16_t* q, const uint16_t* k, const uint16_t* q_weight,
+                               const uint16_t* k_weight, const void* table, int32_t table_is_f32,
+                               int32_t act_is_f16, int64_t num_tokens, int32_t heads_q,
+                               int32_t heads_k, int32_t head_dim, int32_t rotary_dim, double eps,
+                               int32_t interleaved, uint16_t* q_out, uint16_t* k_out)
 {
     int64_t nq = num_tokens * heads_q * head_dim, nk = num_tokens * heads_k * head_dim;
     double* eq = malloc(sizeof(double) * (nq ? nq : 1));
     double* ek = malloc(sizeof(double) * (nk ? nk : 1));
-    int rc = qknr_oracle_rope_table_exact(q, k, q_weight, k_weight, table, table_is_f32,
-                                          num_tokens, heads_q, heads_k, head_dim, rotary_dim,
-                                          eps, interleaved, eq, ek);
-    if (rc == 0) {
+    int rc = qknr_oracle_rope_table_exact_act(q, k, q_weight, k_weight, table, table_is_f32,
+                                              act_is_f16, num_tokens, heads_q, heads_k, head_dim,
+                                              rotary_dim, eps, interleaved, eq, ek);
+    if (rc == 0 && act_is_f16) {
+        qknr_oracle_f16_from_double_array(eq, q_out, nq);
+        qknr_oracle_f16_from_double_array(ek, k_out, nk);
+    } else if (rc == 0) {
         qknr_oracle_bf16_from_double_array(eq, q_out, nq);
         qknr_oracle_bf16_from_double_array(ek, k_out, nk);
     }
     free(eq);
     free(ek);
     return rc;
+}
+
+int qknr_oracle_rope_table(const uint16_t* q, const uint16_t* k, const uint16_t* q_weight,
+                           const uint16_t* k_weight, const void* table, int32_t table_is_f32,
+                           int64_t num_tokens, int32_t heads_q, int32_t heads_k,
+                           int32_t head_dim, int32_t rotary_dim, double eps, int32_t interleaved,
+                           uint16_t* q_out, uint16_t* k_out)
+{
+    return qknr_oracle_rope_table_act(q, k, q_weight, k_weight, table, table_is_f32, 0,
+                                      num_tokens, heads_q, heads_k, head_dim, rotary_dim, eps,
+                                      interleaved, q_out, k_out);
 }
 
 /* ------------------------------------------------------------------------ */

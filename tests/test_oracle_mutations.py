@@ -46,6 +46,13 @@ MUTATIONS = {
                         "qknr_oracle_e4m3_from_double(ev[i] * q_scale)"),
     "norm_flag_ignored": ("if (is_qk_norm)\n            qknr_oracle_rmsnorm",
                           "if (1)\n            qknr_oracle_rmsnorm"),
+    "f16_exponent_bias": ("return s * ldexp(1.0 + m / 1024.0, e - 15);",
+                          "return s * ldexp(1.0 + m / 1024.0, e - 16);"),
+    "f16_no_subnormal_floor": ("if (e < -14) e = -14;", ""),
+    "f16_overflow_early": ("if (v >= 65536.0) return (uint16_t)(sign | 0x7C00u);",
+                           "if (v >= 65504.0) return (uint16_t)(sign | 0x7C00u);"),
+    "act_type_ignored": ("return act_is_f16 ? qknr_oracle_f16_to_double(b) : qknr_oracle_bf16_to_double(b);",
+                         "return qknr_oracle_bf16_to_double(b);"),
 }
 
 # cheap pins first, so a planted mistake is usually caught within a second

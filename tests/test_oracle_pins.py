@@ -97,6 +97,68 @@ def pin_e4m3_hand_cases():
     assert int(O.e4m3_from_f64(np.array([math.nan]))[0]) == 0x7F
 
 
+def pin_f16_rounding_vs_torch():
+    """IEEE binary16 (table-form activations may be fp16): every finite binary16
+    value, every midpoint between neighbours, and points 1/64 of a step off
+    them, rounded by the oracle from double, equal torch's float32 -> float16
+    (one RNE rounding)."""
+    allh = np.arange(1 << 16, dtype=np.uint16).view(np.float16).astype(np.float64)
+    fin = np.sort(np.unique(allh[np.isfinite(allh)]))
+    mids = (fin[:-1] + fin[1:]) / 2
+    steps = np.diff(fin)
+    f = np.concatenate([fin, mids, mids + steps / 64, mids - steps / 64, [65520.0, -65520.0,
+                                                                         70000.0, 1e-9]])
+    f32 = f.astype(np.float32)
+    want = torch.from_numpy(f32.copy()).to(torch.float16).view(torch.int16).numpy() \
+        .view(np.uint16)
+    got = O.f16_from_f64(f32.astype(np.float64))
+    assert np.array_equal(got, want)
+
+
+def pin_f16_hand_cases():
+    """binary16 by hand: 65504 is the largest finite (0x7BFF); 65520 is its tie
+    with 2^16 and rounds to even, i.e. to infinity (0x7C00); 2^-24 is the
+    smallest subnormal (0x0001) and 2^-25 its tie with zero (-> 0); 1 + 2^-11 is
+    the tie between 1 and 1 + 2^-10 (-> 1.0, 0x3C00), one 2^-40 above it goes up."""
+    cases = [(65504.0, 0x7BFF), (65520.0, 0x7C00), (-65520.0, 0xFC00), (2.0 ** -24, 0x0001),
+             (2.0 ** -25, 0x0000), (3 * 2.0 ** -26, 0x0001), (1 + 2.0 ** -11, 0x3C00),
+             (1 + 2.0 ** -11 + 2.0 ** -40, 0x3C01), (2.0 ** -14, 0x0400), (-2.0, 0xC000)]
+    for x, want in cases:
+        assert int(O.f16_from_f64(np.array([x]))[0]) == want, (x, want)
+    for bits in (0x0001, 0x03FF, 0x0400, 0x3C00, 0x7BFF, 0xC000):
+        v = O.f16_to_f64(np.array([bits], np.uint16))[0]
+        assert O.lib().qknr_oracle_f16_to_double(bits) == v
+
+
+def pin_table_f16_brute_force():
+    """Table form with binary16 activations, weights and table: per-head RMS
+    norm, weight, rotation, by numpy matrix products on the exact fp16 values."""
+    T, Hq, Hk, D, R = 4, 2, 1, 16, 12
+    h = lambda a: np.asarray(a, np.float16).view(np.uint16)  # noqa: E731
+    q = h(RNG.standard_normal((T, Hq, D)) * 30)
+    k = h(RNG.standard_normal((T, Hk, D)))
+    qw, kw = h(1 + 0.2 * RNG.standard_normal(D)), h(1 + 0.2 * RNG.standard_normal(D))
+    theta = RNG.uniform(-4, 4, (T, R // 2))
+    tbl = h(np.concatenate([np.cos(theta), np.sin(theta)], 1))
+    for il in (True, False):
+        qo, ko = O.rope_table(q, k, qw, kw, tbl, 1e-5, R, interleaved=il, exact=True, act="f16")
+        pa, pb = O.pairs_table(R, il)
+        tv = O.f16_to_f64(tbl)
+        for t in range(T):
+            M = np.eye(D)
+            for j in range(R // 2):
+                a, b = pa[j], pb[j]
+                c, s_ = tv[t, j], tv[t, R // 2 + j]
+                M[a, a], M[a, b], M[b, a], M[b, b] = c, -s_, s_, c
+            for X, src, wt in ((qo, q, qw), (ko, k, kw)):
+                xs = O.f16_to_f64(src[t])
+                for hh in range(xs.shape[0]):
+                    y = xs[hh] / np.sqrt(np.mean(xs[hh] ** 2) + 1e-5) * O.f16_to_f64(wt)
+                    assert np.allclose(X[t, hh], M @ y, rtol=1e-12, atol=1e-12)
+        qb, _ = O.rope_table(q, k, qw, kw, tbl, 1e-5, R, interleaved=il, act="f16")
+        assert np.array_equal(qb, O.f16_from_f64(qo))
+
+
 # ----------------------------------------------------------------------------
 # Steps: position, angle, norm, rotation, pair maps.
 # ----------------------------------------------------------------------------
