@@ -9,6 +9,8 @@ HBM; the 377 MB input (plus 377 MB output) exceeds the 126 MB L2, so no flush
 is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  (NAME: a 3D workload, or table_hs / table_il / table_hs_f16 for the table
+  form, timed over rotated input sets since one set fits in L2)
   python bench.py --impl reference ...   # the fp64 CPU oracle, bounded sample
 
 Under torchrun each rank processes its own batch (weak scaling, no
@@ -31,20 +33,23 @@ METRIC = "tokens/s and achieved HBM GB/s (% of B200 peak) for fused QK-norm+RoPE
 FALLBACK_HBM_GBS = 6650.0
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu
-# capture summarised in profiles/ (rope3d_video3d.md, rope3d_fp8neox.md),
-# valid only for the 3D kernel sources whose hash is stored beside it (the
-# bench reports null otherwise).
+# captures summarised in profiles/ (rope3d_video3d.md, rope3d_fp8neox.md,
+# rope_table.md), valid only for the kernel sources whose hash is stored
+# beside it (the bench reports null otherwise).
 TRAFFIC = {
-    "video3d": (377604608 + 326107904, "bd01f916b071c711"),
-    "fp8neox": (1097277184 + 517313280, "bd01f916b071c711"),
+    "video3d": (377565184 + 325254144, "3127d2c9428b44fd"),
+    "fp8neox": (1097152000 + 517399296, "3127d2c9428b44fd"),
+    "table_hs": (43553536 + 2353920, "806ac1b73bc41843"),
+    "table_il": (25727744 + 22272, "806ac1b73bc41843"),
+    "table_hs_f16": (42767104 + 2006272, "806ac1b73bc41843"),
 }
 
 
-def kernel_source_hash() -> str:
-    """Hash of the sources the 3D kernel is built from."""
+def kernel_source_hash(form: str = "3d") -> str:
+    """Hash of the sources the form's kernels are built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "qk_rmsnorm_rope_qknr_b200", "csrc")
-    for f in ("common.cuh", "launch.h", "rope3d.cu"):
+    for f in ("common.cuh", "launch.h", "rope3d.cu" if form == "3d" else "rope_table.cu"):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -135,6 +140,8 @@ def oracle_sample(w, inp_cpu, budget_s: float, chunk: int = 256):
     import oracle as O
     from tests._util import t2u16
 
+    if w.form != "3d":
+        return oracle_sample_table(w, inp_cpu, budget_s, chunk)
     qkv = inp_cpu["qkv"].reshape(-1, inp_cpu["qkv"].shape[-1])
     qw, kw = t2u16(inp_cpu["q_weight"]), t2u16(inp_cpu["k_weight"])
     p = w.params()
@@ -145,6 +152,27 @@ def oracle_sample(w, inp_cpu, budget_s: float, chunk: int = 256):
         bits = t2u16(qkv[done:done + n])
         t0 = time.perf_counter()
         O.rope_3d(bits, qw, kw, pos_offset=done, **p)
+        spent += time.perf_counter() - t0
+        done += n
+    return done, spent, O.threads()
+
+
+def oracle_sample_table(w, inp_cpu, budget_s: float, chunk: int):
+    import oracle as O
+    from tests._util import t2u16
+
+    q, k, tbl = inp_cpu["q"], inp_cpu["k"], inp_cpu["rope_table"]
+    qw, kw = t2u16(inp_cpu["q_weight"]), t2u16(inp_cpu["k_weight"])
+    done, spent = 0, 0.0
+    T = q.shape[0]
+    while spent < budget_s and done < T:
+        n = min(chunk, T - done)
+        tb = tbl[done:done + n]
+        tb = tb.numpy() if tb.dtype.is_floating_point and tb.element_size() == 4 else t2u16(tb)
+        qb, kb = t2u16(q[done:done + n]), t2u16(k[done:done + n])
+        t0 = time.perf_counter()
+        O.rope_table(qb, kb, qw, kw, tb, w.eps, w.rotary_dim, interleaved=w.interleaved,
+                     act=w.act)
         spent += time.perf_counter() - t0
         done += n
     return done, spent, O.threads()
@@ -185,11 +213,9 @@ def run_reference(args, w):
 
 
 # ------------------------------------------------------------------ GPU arm --
-def run_gpu(args, w):
+def init_gpu():
+    """This rank's device, and an NCCL group when launched with several ranks."""
     import torch
-
-    import qk_rmsnorm_rope_qknr_b200 as Q
-    from qk_rmsnorm_rope_qknr_b200 import workloads as W
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -202,6 +228,47 @@ def run_gpu(args, w):
 
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
         pg = dist
+    return rank, world, local, dev, pg
+
+
+def time_steps(step, args, stream, local, dev, pg):
+    """W untimed steps, then K back-to-back steps (one kernel launch each,
+    nothing else on the stream) between two events on the launching stream.
+    The kernels are programmatic dependent launches, so no event may sit
+    between them: the average launch duration is the region's time over K.
+    Returns (ms per step, max over ranks; the clock sampler)."""
+    import torch
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    if pg:
+        t = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = t.item()
+    return total_ms / args.steps, clocks
+
+
+def run_gpu(args, w):
+    import torch
+
+    import qk_rmsnorm_rope_qknr_b200 as Q
+    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+
+    rank, world, local, dev, pg = init_gpu()
     Q.lib()
 
     # Each rank: its own batch of the workload (seed offset by rank).
@@ -213,35 +280,10 @@ def run_gpu(args, w):
     qkv, qw, kw = inp["qkv"], inp["q_weight"], inp["k_weight"]
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def step(i):
         Q.qknr_rope_3d(qkv, qw, kw, *outs, stream=stream, **p)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-
-    # Timed region: K back-to-back steps (one kernel launch each, nothing else
-    # on the stream) between two events on the launching stream. The kernels
-    # are programmatic dependent launches, so no event may sit between them:
-    # the average launch duration is the region's time over K.
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        t_start.record(stream)
-        for _ in range(args.steps):
-            step()
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    if pg:
-        pg.barrier()
-    total_ms = t_start.elapsed_time(t_end)
-    if pg:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = t.item()
-    ms_per_step = total_ms / args.steps
+    ms_per_step, clocks = time_steps(step, args, stream, local, dev, pg)
     avg_launch_ms = ms_per_step
     tokens_per_s = world * T / (ms_per_step / 1e3)
 
@@ -292,6 +334,138 @@ def run_gpu(args, w):
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+def run_gpu_table(args, w):
+    """The table form (per-head norm + cos/sin table): one launch of
+    qknr_rope_table per step. Its inputs are smaller than L2, so the steps
+    rotate through enough input/output sets to pass 600 MB, each set evicted
+    from L2 before it comes round again."""
+    import torch
+
+    import qk_rmsnorm_rope_qknr_b200 as Q
+    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+
+    rank, world, local, dev, pg = init_gpu()
+    Q.lib()
+    T = w.tokens
+    alg_bytes = W.algorithmic_bytes(w)
+    nsets = max(3, -(-600_000_000 // alg_bytes))
+    sets = []
+    for k in range(nsets):
+        inp = W.make_inputs(w, device=dev, seed=w.seed + 1000 * rank + k)
+        inp["q_out"], inp["k_out"] = torch.empty_like(inp["q"]), torch.empty_like(inp["k"])
+        sets.append(inp)
+    stream = torch.cuda.current_stream(dev)
+
+    def run(s, st=stream):
+        Q.qknr_rope_table(s["q"], s["k"], s["q_out"], s["k_out"], s["q_weight"], s["k_weight"],
+                          s["rope_table"], eps=w.eps, rotary_dim=w.rotary_dim,
+                          interleaved=w.interleaved, stream=st)
+
+    ms_per_step, clocks = time_steps(lambda i: run(sets[i % nsets]), args, stream, local, dev, pg)
+    tokens_per_s = world * T / (ms_per_step / 1e3)
+    peak, peak_kind = measured_peaks()
+    achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+    tr = TRAFFIC.get(w.name)
+    traffic = tr[0] if tr and tr[1] == kernel_source_hash("table") else None
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e_table(args, w, sets[0], run, stream, dev, world, pg)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_cpu = min(T, 2048)
+        inp_cpu = {k: v[:n_cpu].cpu() if k in ("q", "k", "rope_table") else v.cpu()
+                   for k, v in sets[0].items() if k not in ("q_out", "k_out")}
+        n, sec, threads = oracle_sample(w, inp_cpu, args.cpu_seconds, chunk=128)
+        cpu = {"value": n / sec, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"first {n} tokens of {w.name} ({sec:.1f} s of fp64 oracle work)"}
+    if rank == 0:
+        q = sets[0]["q"]
+        line = {
+            "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.act, "data": "synthetic",
+            "config": {"workload": w.name, "tokens_per_gpu": T, "q_shape": list(q.shape),
+                       "k_shape": list(sets[0]["k"].shape), "rotary_dim": w.rotary_dim,
+                       "interleaved": w.interleaved,
+                       "table_dtype": "f32" if w.table_f32 else w.act,
+                       "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": f"{nsets} rotated input/output sets "
+                             f"({nsets * alg_bytes / 1e6:.0f} MB > 126 MB L2)"},
+            "hbm_gbs": achieved, "hbm_pct_of_peak": 100.0 * achieved / peak,
+            "kernel_us": ms_per_step * 1e3,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": alg_bytes},
+            "cpu_baseline": cpu, "clocks": clocks.summary(), "e2e": e2e,
+            "gpu_launches": args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def measure_e2e_table(args, w, dset, run, stream, dev, world, pg):
+    """End to end through the C ABI for the table form, inputs and outputs in
+    page-locked host memory: staged (copy q, k and the table in, run, copy
+    q_out and k_out back) or zero-copy (the kernel reads and writes the host
+    buffers across the bus); the faster is reported."""
+    import torch
+
+    names_in = ("q", "k", "q_weight", "k_weight", "rope_table")
+    host = {n: torch.empty(dset[n].shape, dtype=dset[n].dtype).pin_memory() for n in names_in}
+    for n in names_in:
+        host[n].copy_(dset[n].cpu())
+    for n in ("q_out", "k_out"):
+        host[n] = torch.empty(dset[n].shape, dtype=dset[n].dtype).pin_memory()
+    dev_set = {n: torch.empty_like(dset[n]) for n in dset}
+    dev_set["q_weight"], dev_set["k_weight"] = dset["q_weight"], dset["k_weight"]
+    hz = dict(host, q_weight=dset["q_weight"], k_weight=dset["k_weight"])
+    steps = max(3, min(args.e2e_steps, args.steps))
+
+    def staged():
+        for n in ("q", "k", "rope_table"):
+            dev_set[n].copy_(host[n], non_blocking=True)
+        run(dev_set)
+        for n in ("q_out", "k_out"):
+            host[n].copy_(dev_set[n], non_blocking=True)
+
+    def zero_copy():
+        run(hz)
+
+    def timed(step):
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+        if pg:
+            t = torch.tensor([ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ms = t.item()
+        return ms
+
+    ms = {"staged": timed(staged), "zero-copy": timed(zero_copy)}
+    best = min(ms, key=ms.get)
+    nbytes = lambda names: sum(dset[n].numel() * dset[n].element_size() for n in names)  # noqa
+    return {"value": world * w.tokens / (ms[best] / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": nbytes(("q", "k", "rope_table")),
+            "d2h_bytes_per_step": nbytes(("q_out", "k_out")),
+            "steps": steps, "mode": best,
+            "ms_per_step": {k: round(v, 4) for k, v in ms.items()}}
 
 
 def measure_e2e(args, w, qkv, qw, kw, outs, p, stream, dev, world, pg):
@@ -397,11 +571,9 @@ def main():
     from qk_rmsnorm_rope_qknr_b200 import workloads as W
 
     w = W.WORKLOADS[args.workload]
-    if w.form != "3d":
-        ap.error("the bench times the 3D entry point; pick a 3D workload")
     if args.impl == "reference":
         return run_reference(args, w)
-    return run_gpu(args, w)
+    return run_gpu(args, w) if w.form == "3d" else run_gpu_table(args, w)
 
 
 if __name__ == "__main__":

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define QKNR_ABI_VERSION 1
+#define QKNR_ABI_VERSION 2
 
 typedef enum {
     QKNR_OK = 0,
@@ -58,7 +58,8 @@ typedef enum {
 typedef enum {
     QKNR_DT_BF16 = 0,
     QKNR_DT_F32 = 1,
-    QKNR_DT_E4M3 = 2
+    QKNR_DT_E4M3 = 2,
+    QKNR_DT_F16 = 3 /* IEEE binary16 */
 } qknr_dtype;
 
 /*
@@ -72,15 +73,20 @@ typedef enum {
  *   c = rope_table[t][j], s = rope_table[t][rotary_dim/2 + j]
  *   out[a] = y[a] c - y[b] s,  out[b] = y[b] c + y[a] s;  channels >= rotary_dim: out = y
  *
- * q, k          bf16 [num_tokens, heads, head_dim]: heads dense inside a token,
- *               tokens q_token_stride / k_token_stride ELEMENTS apart
+ * act_dtype     QKNR_DT_BF16 or QKNR_DT_F16: the type of q, k, their outputs
+ *               and the weights (the "activation dtype").
+ * q, k          [num_tokens, heads, head_dim] of act_dtype: heads dense inside
+ *               a token, tokens q_token_stride / k_token_stride ELEMENTS apart
  *               (0 = dense, heads*head_dim). Read only.
- * q_out, k_out  bf16, same shape, their own token strides (0 = dense). May
+ * q_out, k_out  act_dtype, same shape, their own token strides (0 = dense). May
  *               equal q / k exactly (in place, then with the same stride);
  *               any other overlap with an input is QKNR_ERR_ALIAS.
- * q_weight, k_weight  bf16 [head_dim].
- * rope_table    [num_tokens, rotary_dim], dense, QKNR_DT_F32 or QKNR_DT_BF16:
+ * q_weight, k_weight  act_dtype [head_dim].
+ * rope_table    [num_tokens, rotary_dim], dense, QKNR_DT_F32 or act_dtype (the
+ *               contract bullets allow exactly these two table types):
  *               columns [0, rotary_dim/2) hold cos(theta_j), the rest sin(theta_j).
+ *               Any other act_dtype, or a 16-bit table of the other 16-bit
+ *               type, is QKNR_ERR_SHAPE.
  * head_dim      1..256; rotary_dim 0 means head_dim, else even and <= head_dim.
  * heads_q, heads_k >= 0 (a tensor with 0 heads is neither read nor written and
  *               its pointers may be NULL).
@@ -91,7 +97,8 @@ typedef enum {
  */
 int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
                     const void* q_weight, const void* k_weight, const void* rope_table,
-                    int32_t table_dtype, int64_t num_tokens, int32_t heads_q, int32_t heads_k,
+                    int32_t table_dtype, int32_t act_dtype, int64_t num_tokens, int32_t heads_q,
+                    int32_t heads_k,
                     int32_t head_dim, int32_t rotary_dim, int64_t q_token_stride,
                     int64_t k_token_stride, int64_t q_out_token_stride,
                     int64_t k_out_token_stride, float eps, int32_t interleaved,

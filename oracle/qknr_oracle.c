@@ -42,9 +42,10 @@
  *   R11 With is_qk_norm off, Q/K are only rotated (weights and eps unused).
  *   R12 Table form: channels at and beyond rotary_dim are normalised but not
  *       rotated.
- *   R13 Table form activations may be bf16 or IEEE binary16 ([T]: the table is
- *       "either the activation dtype or float32"); weights share the
- *       activation type, outputs are rounded once to it.
+ *   R13 Table form activations may be bf16 or IEEE binary16 ([T]: the table
+ *       has the activation type or is float32, so the activation type is
+ *       not fixed to bf16); weights share the activation type, outputs are
+ *       rounded once to it.
  *
  * Threads: the per-token loops run under OpenMP when it is enabled; every
  * token is computed independently, so the results do not depend on the

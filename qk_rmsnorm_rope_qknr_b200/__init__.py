@@ -29,7 +29,8 @@ LIB_PATH = os.path.join(_PKG, "libqknr.so")
 
 QKNR_OK, QKNR_ERR_NULL, QKNR_ERR_SHAPE, QKNR_ERR_UNSUPPORTED = 0, 1, 2, 3
 QKNR_ERR_ALIGN, QKNR_ERR_ALIAS, QKNR_ERR_POINTER, QKNR_ERR_CUDA = 4, 5, 6, 7
-QKNR_DT_BF16, QKNR_DT_F32, QKNR_DT_E4M3 = 0, 1, 2
+QKNR_DT_BF16, QKNR_DT_F32, QKNR_DT_E4M3, QKNR_DT_F16 = 0, 1, 2, 3
+ABI_VERSION = 2  # QKNR_ABI_VERSION the argument lists below are written for
 
 EXPORTS = ("qknr_rope_table", "qknr_rope_3d", "qknr_rope_3d_partial_ssq", "qknr_rope_3d_with_ssq",
            "qknr_device_status", "qknr_test_set_wait_fault", "qknr_status_string",
@@ -73,8 +74,8 @@ def lib() -> C.CDLL:
                               "qk_rmsnorm_rope_qknr_b200.build.build()")
         L = C.CDLL(LIB_PATH)
         vp, i32, i64 = C.c_void_p, C.c_int32, C.c_int64
-        L.qknr_rope_table.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
-                                      i64, i64, i64, i64, C.c_float, i32, vp]
+        L.qknr_rope_table.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i64, i32, i32, i32,
+                                      i32, i64, i64, i64, i64, C.c_float, i32, vp]
         L.qknr_rope_table.restype = C.c_int
         L.qknr_rope_3d.argtypes = [C.POINTER(Rope3DParams), vp]
         L.qknr_rope_3d.restype = C.c_int
@@ -86,6 +87,9 @@ def lib() -> C.CDLL:
         L.qknr_status_string.restype = C.c_char_p
         L.qknr_last_error_detail.restype = C.c_char_p
         L.qknr_abi_version.restype = C.c_int
+        if L.qknr_abi_version() != ABI_VERSION:
+            raise ImportError(f"libqknr.so has ABI version {L.qknr_abi_version()}, this binding "
+                              f"expects {ABI_VERSION}; rebuild it")
         L.qknr_device_status.argtypes = [vp, C.POINTER(C.c_uint32), i32]
         L.qknr_device_status.restype = C.c_int
         L.qknr_test_set_wait_fault.argtypes = [C.c_uint32, C.c_uint64]
@@ -125,19 +129,30 @@ def _stream(stream, *tensors) -> Optional[int]:
     return None
 
 
-def _table_dtype(t: torch.Tensor) -> int:
+_ACT_DTYPES = {torch.bfloat16: QKNR_DT_BF16, torch.float16: QKNR_DT_F16}
+
+
+def _act_dtype(q: torch.Tensor) -> int:
+    if q.dtype not in _ACT_DTYPES:
+        raise QknrValueError(QKNR_ERR_SHAPE, f"q dtype {q.dtype} is not bfloat16/float16")
+    return _ACT_DTYPES[q.dtype]
+
+
+def _table_dtype(t: torch.Tensor, act: torch.dtype) -> int:
     if t.dtype == torch.float32:
         return QKNR_DT_F32
-    if t.dtype == torch.bfloat16:
-        return QKNR_DT_BF16
-    raise QknrValueError(QKNR_ERR_SHAPE, f"rope_table dtype {t.dtype} is not float32/bfloat16")
+    if t.dtype == act:
+        return _ACT_DTYPES[act]
+    raise QknrValueError(QKNR_ERR_SHAPE,
+                         f"rope_table dtype {t.dtype} is neither float32 nor {act}")
 
 
-def _token_stride(t: torch.Tensor, name: str, heads: int, head_dim: int) -> int:
+def _token_stride(t: torch.Tensor, name: str, heads: int, head_dim: int,
+                  dtype: torch.dtype = torch.bfloat16) -> int:
     if t.dim() != 3 or t.shape[1] != heads or t.shape[2] != head_dim:
         raise QknrValueError(QKNR_ERR_SHAPE, f"{name} must be [tokens, {heads}, {head_dim}]")
-    if t.dtype != torch.bfloat16:
-        raise QknrValueError(QKNR_ERR_SHAPE, f"{name} must be bfloat16")
+    if t.dtype != dtype:
+        raise QknrValueError(QKNR_ERR_SHAPE, f"{name} must be {dtype}")
     if t.shape[0] > 0 and heads > 0 and (t.stride(2) != 1 or (heads > 1 and
                                                              t.stride(1) != head_dim)):
         raise QknrValueError(QKNR_ERR_SHAPE, f"{name}: heads must be dense inside a token")
@@ -148,24 +163,30 @@ def _token_stride(t: torch.Tensor, name: str, heads: int, head_dim: int) -> int:
 def qknr_rope_table(q, k, q_out, k_out, q_weight, k_weight, rope_table, *, eps: float,
                     rotary_dim: int = 0, interleaved: bool = False, stream=None) -> None:
     """Table form through the C ABI (destination passing; see include/qknr.h).
-    q/k/q_out/k_out are bf16 [tokens, heads, head_dim] with dense heads."""
+    q/k/q_out/k_out are [tokens, heads, head_dim] with dense heads, all bf16 or
+    all float16 (the activation dtype, taken from q); the weights have the
+    activation dtype, the table float32 or the activation dtype."""
+    if q.dim() != 3:
+        raise QknrValueError(QKNR_ERR_SHAPE, "q must be [tokens, heads, head_dim]")
+    act = _act_dtype(q)
     T, Hq, D = q.shape
-    Hk = k.shape[1]
-    qs = _token_stride(q, "q", Hq, D)
-    ks = _token_stride(k, "k", Hk, D)
-    qos = _token_stride(q_out, "q_out", Hq, D)
-    kos = _token_stride(k_out, "k_out", Hk, D)
+    Hk = k.shape[1] if k.dim() == 3 else -1
+    qs = _token_stride(q, "q", Hq, D, q.dtype)
+    ks = _token_stride(k, "k", Hk, D, q.dtype)
+    qos = _token_stride(q_out, "q_out", Hq, D, q.dtype)
+    kos = _token_stride(k_out, "k_out", Hk, D, q.dtype)
     if k.shape[0] != T or q_out.shape[0] != T or k_out.shape[0] != T:
         raise QknrValueError(QKNR_ERR_SHAPE, "q, k and outputs differ in token count")
     R = rotary_dim or D
     if rope_table.dim() != 2 or tuple(rope_table.shape) != (T, R) or not rope_table.is_contiguous():
         raise QknrValueError(QKNR_ERR_SHAPE, f"rope_table must be a dense [{T}, {R}] tensor")
     for n, w in (("q_weight", q_weight), ("k_weight", k_weight)):
-        if w.dtype != torch.bfloat16 or w.numel() != D or not w.is_contiguous():
-            raise QknrValueError(QKNR_ERR_SHAPE, f"{n} must be a dense bf16 [{D}] tensor")
+        if w.dtype != q.dtype or w.numel() != D or not w.is_contiguous():
+            raise QknrValueError(QKNR_ERR_SHAPE, f"{n} must be a dense {q.dtype} [{D}] tensor")
     st = _stream(stream, q, k, q_out, k_out)
     _check(lib().qknr_rope_table(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _ptr(q_weight),
-                                 _ptr(k_weight), _ptr(rope_table), _table_dtype(rope_table), T, Hq,
+                                 _ptr(k_weight), _ptr(rope_table),
+                                 _table_dtype(rope_table, q.dtype), act, T, Hq,
                                  Hk, D, R, qs, ks, qos, kos, float(eps), int(bool(interleaved)),
                                  st))
 

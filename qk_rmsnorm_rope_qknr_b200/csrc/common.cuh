@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -281,5 +282,45 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
 }
 
 __device__ __forceinline__ uint32_t f2_to_bf16x2(float2 v) { return pack_bf16x2(v.x, v.y); }
+
+// 16-bit activation pairs: bf16 (H16 = false) or IEEE binary16 (H16 = true).
+template <bool H16>
+__device__ __forceinline__ float2 act2_to_f2(uint32_t w) {
+    if constexpr (H16) {
+        return __half22float2(*reinterpret_cast<const __half2*>(&w));
+    } else {
+        return bf16x2_to_f2(w);
+    }
+}
+
+template <bool H16>
+__device__ __forceinline__ uint32_t f2_to_act2(float2 v) {
+    if constexpr (H16) {
+        __half2 h = __floats2half2_rn(v.x, v.y);
+        return *reinterpret_cast<uint32_t*>(&h);
+    } else {
+        return pack_bf16x2(v.x, v.y);
+    }
+}
+
+template <bool H16>
+__device__ __forceinline__ float act_to_f(uint16_t b) {
+    if constexpr (H16) {
+        return __half2float(*reinterpret_cast<const __half*>(&b));
+    } else {
+        return __uint_as_float((uint32_t)b << 16);
+    }
+}
+
+template <bool H16>
+__device__ __forceinline__ uint16_t f_to_act(float f) {
+    if constexpr (H16) {
+        __half h = __float2half_rn(f);
+        return *reinterpret_cast<uint16_t*>(&h);
+    } else {
+        __nv_bfloat16 b = __float2bfloat16_rn(f);
+        return *reinterpret_cast<uint16_t*>(&b);
+    }
+}
 
 }  // namespace qknr

@@ -54,6 +54,7 @@ struct RopeTableArgs {
     int64_t q_stride, k_stride, q_out_stride, k_out_stride;  // elements
     int32_t hq, hk, head_dim, rotary_dim;
     int32_t table_f32;
+    int32_t act_f16;  // activations (and a non-fp32 table) are binary16, else bf16
     int32_t interleaved;
     int32_t in_place;  // an output aliases its input
     float eps;

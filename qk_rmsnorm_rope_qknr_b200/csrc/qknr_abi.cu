@@ -158,8 +158,8 @@ int qknr_device_status(void* cuda_stream, uint32_t* status_out, int32_t clear) {
 
 int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
                     const void* q_weight, const void* k_weight, const void* rope_table,
-                    int32_t table_dtype, int64_t num_tokens, int32_t heads_q, int32_t heads_k,
-                    int32_t head_dim, int32_t rotary_dim, int64_t q_token_stride,
+                    int32_t table_dtype, int32_t act_dtype, int64_t num_tokens, int32_t heads_q,
+                    int32_t heads_k, int32_t head_dim, int32_t rotary_dim, int64_t q_token_stride,
                     int64_t k_token_stride, int64_t q_out_token_stride,
                     int64_t k_out_token_stride, float eps, int32_t interleaved,
                     void* cuda_stream) {
@@ -172,8 +172,10 @@ int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
     if (R < 2 || (R & 1) || R > head_dim)
         return fail(QKNR_ERR_SHAPE, "rotary_dim %d must be even and <= head_dim %d", R,
                     head_dim);
-    if (table_dtype != QKNR_DT_F32 && table_dtype != QKNR_DT_BF16)
-        return fail(QKNR_ERR_SHAPE, "rope_table dtype must be float32 or bfloat16");
+    if (act_dtype != QKNR_DT_BF16 && act_dtype != QKNR_DT_F16)
+        return fail(QKNR_ERR_SHAPE, "activation dtype must be bfloat16 or float16");
+    if (table_dtype != QKNR_DT_F32 && table_dtype != act_dtype)
+        return fail(QKNR_ERR_SHAPE, "rope_table dtype must be float32 or the activation dtype");
     if (!(eps >= 0.0f) || std::isinf(eps)) return fail(QKNR_ERR_SHAPE, "eps must be >= 0");
     const int64_t qrow = (int64_t)heads_q * head_dim, krow = (int64_t)heads_k * head_dim;
     const int64_t qs = q_token_stride ? q_token_stride : qrow;
@@ -216,12 +218,12 @@ int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
             (has_q && overlap(sko, Span{q_weight, (uint64_t)head_dim * 2})))
             return fail(QKNR_ERR_ALIAS, "k_out overlaps a weight");
     }
-    // 2-byte alignment is the minimum for bf16 / fp32 element access.
+    // 2-byte alignment is the minimum for 16-bit element access.
     const uintptr_t any = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                           reinterpret_cast<uintptr_t>(q_out) | reinterpret_cast<uintptr_t>(k_out) |
                           reinterpret_cast<uintptr_t>(q_weight) |
                           reinterpret_cast<uintptr_t>(k_weight);
-    if (any & 1u) return fail(QKNR_ERR_ALIGN, "a bf16 pointer is not 2-byte aligned");
+    if (any & 1u) return fail(QKNR_ERR_ALIGN, "a 16-bit pointer is not 2-byte aligned");
     if (reinterpret_cast<uintptr_t>(rope_table) & (uintptr_t)(tb - 1))
         return fail(QKNR_ERR_ALIGN, "rope_table is not aligned to its element size");
 
@@ -260,6 +262,7 @@ int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
     a.head_dim = head_dim;
     a.rotary_dim = R;
     a.table_f32 = table_dtype == QKNR_DT_F32;
+    a.act_f16 = act_dtype == QKNR_DT_F16;
     a.interleaved = interleaved ? 1 : 0;
     a.in_place = q_inplace || k_inplace;
     a.eps = eps;

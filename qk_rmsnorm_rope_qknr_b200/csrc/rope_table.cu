@@ -5,7 +5,8 @@
 // q [T, Hq, D] and k [T, Hk, D] is RMS-normalised over its D channels, scaled
 // by a [D] weight and rotated by the token's row of a [T, rotary_dim] cos/sin
 // table, pairs (2j, 2j+1) (interleaved) or (j, j + rotary_dim/2) (half split);
-// channels >= rotary_dim are normalised only.
+// channels >= rotary_dim are normalised only. Activations (and weights, and a
+// 16-bit table) are bf16 or IEEE binary16; the arithmetic is fp32 either way.
 //
 // Fast kernel: a head is a group of GS lanes (GS = next power of two of D/16);
 // lane l of the group owns two 16-byte vectors of the head, chosen so that
@@ -35,8 +36,9 @@ constexpr int kBlock = 256;
 constexpr int kUnroll = 4;
 
 // The same reads from a table row staged in shared memory (plain loads: the
-// read-only global path must not see a shared address).
-template <bool F32>
+// read-only global path must not see a shared address). A 16-bit table has the
+// activation type.
+template <bool F32, bool H16>
 __device__ __forceinline__ void smem_cos_sin8(const uint8_t* row, int col, int half,
                                               float (&c)[8], float (&s)[8]) {
     if constexpr (F32) {
@@ -50,12 +52,17 @@ __device__ __forceinline__ void smem_cos_sin8(const uint8_t* row, int col, int h
     } else {
         const uint4 cv = *reinterpret_cast<const uint4*>(row + (size_t)col * 2);
         const uint4 sv = *reinterpret_cast<const uint4*>(row + (size_t)(half + col) * 2);
-        unpack8(cv, c);
-        unpack8(sv, s);
+        const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w}, sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float2 c2 = act2_to_f2<H16>(cw[m]), s2 = act2_to_f2<H16>(sw[m]);
+            c[2 * m] = c2.x; c[2 * m + 1] = c2.y;
+            s[2 * m] = s2.x; s[2 * m + 1] = s2.y;
+        }
     }
 }
 
-template <bool F32>
+template <bool F32, bool H16>
 __device__ __forceinline__ void smem_cos_sin4(const uint8_t* row, int col, int half, float* c,
                                               float* s) {
     if constexpr (F32) {
@@ -66,8 +73,10 @@ __device__ __forceinline__ void smem_cos_sin4(const uint8_t* row, int col, int h
     } else {
         const uint2 cv = *reinterpret_cast<const uint2*>(row + (size_t)col * 2);
         const uint2 sv = *reinterpret_cast<const uint2*>(row + (size_t)(half + col) * 2);
-        c[0] = bf16_lo(cv.x); c[1] = bf16_hi(cv.x); c[2] = bf16_lo(cv.y); c[3] = bf16_hi(cv.y);
-        s[0] = bf16_lo(sv.x); s[1] = bf16_hi(sv.x); s[2] = bf16_lo(sv.y); s[3] = bf16_hi(sv.y);
+        const float2 c0 = act2_to_f2<H16>(cv.x), c1 = act2_to_f2<H16>(cv.y);
+        const float2 s0 = act2_to_f2<H16>(sv.x), s1 = act2_to_f2<H16>(sv.y);
+        c[0] = c0.x; c[1] = c0.y; c[2] = c1.x; c[3] = c1.y;
+        s[0] = s0.x; s[1] = s0.y; s[2] = s1.x; s[3] = s1.y;
     }
 }
 
@@ -76,7 +85,7 @@ __host__ __device__ inline int table_stage_bytes(int per_item, int D, int R, int
     return (per_item * D * 2 + R * tb + 15) & ~15;
 }
 
-template <int GS, bool IL, bool F32>
+template <int GS, bool IL, bool F32, bool H16>
 __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a) {
     constexpr int HR = 32 / GS;  // heads per warp round
     const int D = a.head_dim, R = a.rotary_dim;
@@ -134,7 +143,7 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
     for (int c = threadIdx.x; c < 2 * D; c += blockDim.x) {
         const uint16_t* w = reinterpret_cast<const uint16_t*>(c < D ? a.q_weight : a.k_weight);
         const int cc = c < D ? c : c - D;
-        wsm[c] = ((c < D ? a.hq : a.hk) > 0) ? __uint_as_float((uint32_t)w[cc] << 16) : 0.0f;
+        wsm[c] = ((c < D ? a.hq : a.hk) > 0) ? act_to_f<H16>(w[cc]) : 0.0f;
     }
     __syncwarp();
     int64_t t = warp_id / cpt;
@@ -190,10 +199,10 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
         float c[8], s[8];
         if (active) {
             if (IL) {
-                if (rot_a) smem_cos_sin4<F32>(trow, 4 * va, R / 2, c, s);
-                if (rot_b) smem_cos_sin4<F32>(trow, 4 * vb, R / 2, c + 4, s + 4);
+                if (rot_a) smem_cos_sin4<F32, H16>(trow, 4 * va, R / 2, c, s);
+                if (rot_b) smem_cos_sin4<F32, H16>(trow, 4 * vb, R / 2, c + 4, s + 4);
             } else if (across) {
-                smem_cos_sin8<F32>(trow, 8 * va, R / 2, c, s);
+                smem_cos_sin8<F32, H16>(trow, 8 * va, R / 2, c, s);
             }
         }
 #pragma unroll
@@ -208,10 +217,10 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
                 xb = v[vb];
             }
             float2 fa[4], fb[4];
-            fa[0] = bf16x2_to_f2(xa.x); fa[1] = bf16x2_to_f2(xa.y);
-            fa[2] = bf16x2_to_f2(xa.z); fa[3] = bf16x2_to_f2(xa.w);
-            fb[0] = bf16x2_to_f2(xb.x); fb[1] = bf16x2_to_f2(xb.y);
-            fb[2] = bf16x2_to_f2(xb.z); fb[3] = bf16x2_to_f2(xb.w);
+            fa[0] = act2_to_f2<H16>(xa.x); fa[1] = act2_to_f2<H16>(xa.y);
+            fa[2] = act2_to_f2<H16>(xa.z); fa[3] = act2_to_f2<H16>(xa.w);
+            fb[0] = act2_to_f2<H16>(xb.x); fb[1] = act2_to_f2<H16>(xb.y);
+            fb[2] = act2_to_f2<H16>(xb.z); fb[3] = act2_to_f2<H16>(xb.w);
             float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
@@ -268,10 +277,12 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
             uint8_t* dst = isk
                 ? a.k_out + ((size_t)t * a.k_out_stride + (size_t)head * D) * 2
                 : a.q_out + ((size_t)t * a.q_out_stride + (size_t)head * D) * 2;
-            st_v4(dst + (size_t)va * 16, make_uint4(f2_to_bf16x2(oa[0]), f2_to_bf16x2(oa[1]),
-                                                    f2_to_bf16x2(oa[2]), f2_to_bf16x2(oa[3])));
-            st_v4(dst + (size_t)vb * 16, make_uint4(f2_to_bf16x2(ob[0]), f2_to_bf16x2(ob[1]),
-                                                    f2_to_bf16x2(ob[2]), f2_to_bf16x2(ob[3])));
+            st_v4(dst + (size_t)va * 16,
+                  make_uint4(f2_to_act2<H16>(oa[0]), f2_to_act2<H16>(oa[1]),
+                             f2_to_act2<H16>(oa[2]), f2_to_act2<H16>(oa[3])));
+            st_v4(dst + (size_t)vb * 16,
+                  make_uint4(f2_to_act2<H16>(ob[0]), f2_to_act2<H16>(ob[1]),
+                             f2_to_act2<H16>(ob[2]), f2_to_act2<H16>(ob[3])));
         }
         // Every lane is done with this buffer: refill it with the item a ring ahead.
         __syncwarp();
@@ -301,7 +312,7 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
 // One warp per head; any head_dim <= 256, any even rotary_dim <= head_dim,
 // 2-byte alignment. The normalised head goes through shared memory so that
 // every lane can read its partner channel.
-template <bool F32>
+template <bool F32, bool H16>
 __global__ void __launch_bounds__(kBlock) rope_table_general(const RopeTableArgs a) {
     __shared__ float ybuf[kBlock / 32][256];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -327,7 +338,7 @@ __global__ void __launch_bounds__(kBlock) rope_table_general(const RopeTableArgs
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int d = lane + 32 * k;
-            x[k] = d < D ? __uint_as_float((uint32_t)src[d] << 16) : 0.0f;
+            x[k] = d < D ? act_to_f<H16>(src[d]) : 0.0f;
             ss += x[k] * x[k];
         }
         ss = warp_sum(ss);
@@ -335,7 +346,7 @@ __global__ void __launch_bounds__(kBlock) rope_table_general(const RopeTableArgs
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int d = lane + 32 * k;
-            if (d < D) y[d] = x[k] * r * __uint_as_float((uint32_t)__ldg(w + d) << 16);
+            if (d < D) y[d] = x[k] * r * act_to_f<H16>(__ldg(w + d));
         }
         __syncwarp();
 #pragma unroll
@@ -357,13 +368,12 @@ __global__ void __launch_bounds__(kBlock) rope_table_general(const RopeTableArgs
                     c = __ldg(tr + j); s = __ldg(tr + half + j);
                 } else {
                     const uint16_t* tr = reinterpret_cast<const uint16_t*>(a.table) + (size_t)t * R;
-                    c = __uint_as_float((uint32_t)__ldg(tr + j) << 16);
-                    s = __uint_as_float((uint32_t)__ldg(tr + half + j) << 16);
+                    c = act_to_f<H16>(__ldg(tr + j));
+                    s = act_to_f<H16>(__ldg(tr + half + j));
                 }
                 o = first ? y[d] * c - y[p] * s : y[d] * c + y[p] * s;
             }
-            __nv_bfloat16 b = __float2bfloat16_rn(o);
-            dst[d] = *reinterpret_cast<uint16_t*>(&b);
+            dst[d] = f_to_act<H16>(o);
         }
         __syncwarp();
     }
@@ -437,18 +447,25 @@ cudaError_t launch_bulk(K kern, const RopeTableArgs& a0, int per_item, cudaStrea
     return e;
 }
 
-template <int GS>
-cudaError_t run_fast(const RopeTableArgs& a, cudaStream_t stream, LaunchInfo* info) {
+template <int GS, bool H16>
+cudaError_t run_fast_act(const RopeTableArgs& a, cudaStream_t stream, LaunchInfo* info) {
     const int per_item = kUnroll * (32 / GS);
-    const int id = 1000 + GS * 10 + (a.interleaved ? 1 : 0) * 2 + (a.table_f32 ? 1 : 0);
+    const int id = 1000 + (H16 ? 500 : 0) + GS * 10 + (a.interleaved ? 1 : 0) * 2 +
+                   (a.table_f32 ? 1 : 0);
     if (a.interleaved) {
         return a.table_f32
-            ? launch_bulk(rope_table_bulk<GS, true, true>, a, per_item, stream, info, id)
-            : launch_bulk(rope_table_bulk<GS, true, false>, a, per_item, stream, info, id);
+            ? launch_bulk(rope_table_bulk<GS, true, true, H16>, a, per_item, stream, info, id)
+            : launch_bulk(rope_table_bulk<GS, true, false, H16>, a, per_item, stream, info, id);
     }
     return a.table_f32
-        ? launch_bulk(rope_table_bulk<GS, false, true>, a, per_item, stream, info, id)
-        : launch_bulk(rope_table_bulk<GS, false, false>, a, per_item, stream, info, id);
+        ? launch_bulk(rope_table_bulk<GS, false, true, H16>, a, per_item, stream, info, id)
+        : launch_bulk(rope_table_bulk<GS, false, false, H16>, a, per_item, stream, info, id);
+}
+
+template <int GS>
+cudaError_t run_fast(const RopeTableArgs& a, cudaStream_t stream, LaunchInfo* info) {
+    return a.act_f16 ? run_fast_act<GS, true>(a, stream, info)
+                     : run_fast_act<GS, false>(a, stream, info);
 }
 
 }  // namespace
@@ -465,9 +482,14 @@ cudaError_t launch_rope_table(const RopeTableArgs& a, int fast_path, cudaStream_
     }
     const int64_t groups = a.num_tokens * (a.hq + a.hk);
     const int64_t blocks = (groups + kBlock / 32 - 1) / (kBlock / 32);
+    if (a.act_f16) {
+        return a.table_f32
+            ? launch_persistent(rope_table_general<true, true>, blocks, a, stream, info, 2011)
+            : launch_persistent(rope_table_general<false, true>, blocks, a, stream, info, 2010);
+    }
     return a.table_f32
-        ? launch_persistent(rope_table_general<true>, blocks, a, stream, info, 2001)
-        : launch_persistent(rope_table_general<false>, blocks, a, stream, info, 2000);
+        ? launch_persistent(rope_table_general<true, false>, blocks, a, stream, info, 2001)
+        : launch_persistent(rope_table_general<false, false>, blocks, a, stream, info, 2000);
 }
 
 cudaError_t read_table_status(uint32_t* out, int clear, cudaStream_t stream) {

@@ -13,6 +13,7 @@ video-DiT and MiniMax-H3 geometries the pages name):
   table_hs    table form, half-split, q [4096,32,128], k [4096,8,128], rd 96, fp32 table
   table_il    table form, adjacent pairs, q,k [2048,24,128] (x3, 1% outliers x20),
               rd 128, bf16 table
+  table_hs_f16  table_hs with IEEE binary16 activations, weights and table
   video3d     3D form, [1,15360,(32+32+32)*128], grid 16x30x32, 16/56/56, bf16 out
   fp8neox     3D form, [2,29760,(24+24+24)*128] ~N(0, 2^2), grid 31x24x40,
               32/48/48, NeoX pairs, E4M3 out (scales 0.5 / 0.25)
@@ -89,7 +90,12 @@ class FormTable:
     outlier_mult: float = 1.0
     rope_base: float = 10000.0
     seed: int = 0
+    act: str = "bf16"  # activation (and 16-bit table) type: "bf16" or "f16"
     form: str = "table"
+
+    @property
+    def act_dtype(self) -> torch.dtype:
+        return torch.float16 if self.act == "f16" else torch.bfloat16
 
 
 WORKLOADS = {
@@ -100,6 +106,8 @@ WORKLOADS = {
     "table_il": FormTable("table_il", tokens=2048, hq=24, hk=24, head_dim=128, rotary_dim=128,
                           table_f32=False, interleaved=True, std=3.0, outlier_frac=0.01,
                           outlier_mult=20.0),
+    "table_hs_f16": FormTable("table_hs_f16", tokens=4096, hq=32, hk=8, head_dim=128,
+                              rotary_dim=96, table_f32=False, interleaved=False, act="f16"),
     "video3d": Form3D("video3d", batch=1, seq=15360, ppf=16, pph=30, ppw=32, cf=16, ch=56,
                       cw=56, hq=32, hk=32, hv=32, head_dim=128),
     "fp8neox": Form3D("fp8neox", batch=2, seq=29760, ppf=31, pph=24, ppw=40, cf=32, ch=48,
@@ -112,27 +120,30 @@ WORKLOADS = {
 }
 
 
-def _normal(g: torch.Generator, shape, std: float, device) -> torch.Tensor:
+def _normal(g: torch.Generator, shape, std: float, device,
+            dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
     x = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
-    return (x * std).to(torch.bfloat16) if std != 1.0 else x.to(torch.bfloat16)
+    return (x * std).to(dtype) if std != 1.0 else x.to(dtype)
 
 
-def _weight(g: torch.Generator, n: int, device) -> torch.Tensor:
+def _weight(g: torch.Generator, n: int, device, dtype: torch.dtype = torch.bfloat16
+            ) -> torch.Tensor:
     w = torch.randn(n, generator=g, dtype=torch.float32, device=device)
-    return (1.0 + 0.1 * w).to(torch.bfloat16)
+    return (1.0 + 0.1 * w).to(dtype)
 
 
 def rope_table_input(tokens: int, rotary_dim: int, base: float, f32: bool,
-                     device="cpu") -> torch.Tensor:
+                     device="cpu", act: torch.dtype = torch.bfloat16) -> torch.Tensor:
     """A caller-built [tokens, rotary_dim] table [cos(theta) | sin(theta)] with
     theta[t, i] = t * base^(-2i/rotary_dim), built in float64 and stored as
-    float32 or bfloat16 (the input the table form consumes)."""
+    float32 or as the activation dtype `act` (the input the table form
+    consumes)."""
     half = rotary_dim // 2
     pos = torch.arange(tokens, dtype=torch.float64).unsqueeze(1)
     inv = base ** (-2.0 * torch.arange(half, dtype=torch.float64) / rotary_dim)
     theta = pos * inv.unsqueeze(0)
     tbl = torch.cat([torch.cos(theta), torch.sin(theta)], dim=1)
-    return tbl.to(torch.float32 if f32 else torch.bfloat16).to(device)
+    return tbl.to(torch.float32 if f32 else act).to(device)
 
 
 def make_inputs(w, device="cpu", tokens: Optional[int] = None, seed: Optional[int] = None):
@@ -156,16 +167,17 @@ def make_inputs(w, device="cpu", tokens: Optional[int] = None, seed: Optional[in
         kw = _weight(g, w.hk * w.head_dim, device)
         return dict(qkv=qkv, q_weight=qw, k_weight=kw)
     T = w.tokens if tokens is None else tokens
-    q = _normal(g, (T, w.hq, w.head_dim), w.std, device)
-    k = _normal(g, (T, w.hk, w.head_dim), w.std, device)
-    qw = _weight(g, w.head_dim, device)
-    kw = _weight(g, w.head_dim, device)
+    act = w.act_dtype
+    q = _normal(g, (T, w.hq, w.head_dim), w.std, device, act)
+    k = _normal(g, (T, w.hk, w.head_dim), w.std, device, act)
+    qw = _weight(g, w.head_dim, device, act)
+    kw = _weight(g, w.head_dim, device, act)
     if w.outlier_frac > 0:
         mq = torch.rand(q.shape, generator=g, device=device) < w.outlier_frac
         mk = torch.rand(k.shape, generator=g, device=device) < w.outlier_frac
-        q = torch.where(mq, (q.float() * w.outlier_mult).to(torch.bfloat16), q)
-        k = torch.where(mk, (k.float() * w.outlier_mult).to(torch.bfloat16), k)
-    table = rope_table_input(T, w.rotary_dim, w.rope_base, w.table_f32, device)
+        q = torch.where(mq, (q.float() * w.outlier_mult).to(act), q)
+        k = torch.where(mk, (k.float() * w.outlier_mult).to(act), k)
+    table = rope_table_input(T, w.rotary_dim, w.rope_base, w.table_f32, device, act)
     return dict(q=q, k=k, q_weight=qw, k_weight=kw, rope_table=table)
 
 

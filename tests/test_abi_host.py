@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_strings(L):
-    assert L.qknr_abi_version() == 1
+    assert L.qknr_abi_version() == Q.ABI_VERSION == 2
     for s in range(8):
         assert L.qknr_status_string(s)
     assert L.qknr_status_string(0) == b"ok"
@@ -145,11 +145,12 @@ def test_3d_zero_tokens_is_noop(L):
 def _table(L, **over):
     kw = dict(q=A, k=A + (1 << 30), q_out=A + (2 << 30), k_out=A + (3 << 30),
               q_weight=A + (4 << 30), k_weight=A + (4 << 30) + 4096, rope_table=A + (5 << 30),
-              table_dtype=Q.QKNR_DT_F32, T=16, Hq=4, Hk=2, D=128, R=96, qs=0, ks=0, qos=0,
+              table_dtype=Q.QKNR_DT_F32, act=Q.QKNR_DT_BF16, T=16, Hq=4, Hk=2, D=128, R=96, qs=0, ks=0, qos=0,
               kos=0, eps=1e-6, il=0)
     kw.update(over)
     rc = L.qknr_rope_table(kw["q"], kw["k"], kw["q_out"], kw["k_out"], kw["q_weight"],
-                           kw["k_weight"], kw["rope_table"], kw["table_dtype"], kw["T"], kw["Hq"],
+                           kw["k_weight"], kw["rope_table"], kw["table_dtype"], kw["act"], kw["T"],
+                           kw["Hq"],
                            kw["Hk"], kw["D"], kw["R"], kw["qs"], kw["ks"], kw["qos"], kw["kos"],
                            kw["eps"], kw["il"], None)
     return rc, L.qknr_last_error_detail().decode()
@@ -159,6 +160,9 @@ def _table(L, **over):
     (dict(D=0), Q.QKNR_ERR_SHAPE), (dict(D=258, R=96), Q.QKNR_ERR_SHAPE),
     (dict(R=97), Q.QKNR_ERR_SHAPE), (dict(R=130), Q.QKNR_ERR_SHAPE),
     (dict(table_dtype=Q.QKNR_DT_E4M3), Q.QKNR_ERR_SHAPE), (dict(T=-1), Q.QKNR_ERR_SHAPE),
+    (dict(act=Q.QKNR_DT_F32), Q.QKNR_ERR_SHAPE), (dict(act=Q.QKNR_DT_E4M3), Q.QKNR_ERR_SHAPE),
+    (dict(table_dtype=Q.QKNR_DT_F16), Q.QKNR_ERR_SHAPE),             # 16-bit table of another type
+    (dict(act=Q.QKNR_DT_F16, table_dtype=Q.QKNR_DT_BF16), Q.QKNR_ERR_SHAPE),
     (dict(Hq=-2), Q.QKNR_ERR_SHAPE), (dict(eps=-1.0), Q.QKNR_ERR_SHAPE),
     (dict(qs=100), Q.QKNR_ERR_SHAPE), (dict(q=0), Q.QKNR_ERR_NULL),
     (dict(k_weight=0), Q.QKNR_ERR_NULL), (dict(rope_table=0), Q.QKNR_ERR_NULL),
@@ -188,6 +192,12 @@ def test_python_wrapper_raises_valueerror(L):
         Q.fused_qk_norm_rope(x, x, w, w, tbl[:, :63], 1e-6)
     with pytest.raises(ValueError):
         Q.fused_qk_norm_rope(x.float(), x, w, w, tbl, 1e-6)
+    with pytest.raises(ValueError):                       # q float16, k bf16
+        Q.fused_qk_norm_rope(x.half(), x, w.half(), w.half(), tbl, 1e-6)
+    with pytest.raises(ValueError):                       # float16 activations, bf16 weights
+        Q.fused_qk_norm_rope(x.half(), x.half(), w, w, tbl, 1e-6)
+    with pytest.raises(ValueError):                       # float16 activations, bf16 table
+        Q.fused_qk_norm_rope(x.half(), x.half(), w.half(), w.half(), tbl.bfloat16(), 1e-6)
 
 
 def test_wait_fault_hook_argument_checks(L):

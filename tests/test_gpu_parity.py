@@ -12,7 +12,7 @@ import torch
 import oracle as O
 import qk_rmsnorm_rope_qknr_b200 as Q
 from qk_rmsnorm_rope_qknr_b200 import workloads as W
-from tests._util import bf16_mismatch, e4m3_mismatch, t2u16, t2u8
+from tests._util import act_mismatch, bf16_mismatch, e4m3_mismatch, t2u16, t2u8
 
 pytestmark = pytest.mark.gpu
 
@@ -109,7 +109,7 @@ def test_3d_workload_full_size_sampled(name):
         assert torch.equal(v_out, v_in)
 
 
-@pytest.mark.parametrize("name", ["table_hs", "table_il"])
+@pytest.mark.parametrize("name", ["table_hs", "table_il", "table_hs_f16"])
 def test_table_workload_full(name):
     w = W.WORKLOADS[name]
     inp = W.make_inputs(w, device="cpu")
@@ -127,10 +127,11 @@ def _table_bits(t):
 def check_table_against_oracle(inp, qo, ko, eps, rd, il, what=""):
     args = (t2u16(inp["q"]), t2u16(inp["k"]), t2u16(inp["q_weight"]), t2u16(inp["k_weight"]),
             _table_bits(inp["rope_table"].cpu().contiguous()), eps, rd)
-    ex_q, ex_k = O.rope_table(*args, interleaved=il, exact=True)
-    rq, rk = O.rope_table(*args, interleaved=il)
+    act = "f16" if inp["q"].dtype == torch.float16 else "bf16"
+    ex_q, ex_k = O.rope_table(*args, interleaved=il, exact=True, act=act)
+    rq, rk = O.rope_table(*args, interleaved=il, act=act)
     for n, o, r, x in (("q", qo, rq, ex_q), ("k", ko, rk, ex_k)):
-        bad, st = bf16_mismatch(t2u16(o), r, x)
+        bad, st = act_mismatch(t2u16(o), r, x, act)
         assert len(bad) == 0, f"{what} {n}: {len(bad)} beyond tolerance {st} at {bad[:3].tolist()}"
 
 
@@ -267,13 +268,13 @@ def test_3d_batch_shape():
 
 
 # ----------------------------------------------------------- table variants --
-def _rand_table_inputs(T, Hq, Hk, D, R, f32, seed=0, std=1.0):
+def _rand_table_inputs(T, Hq, Hk, D, R, f32, seed=0, std=1.0, act=torch.bfloat16):
     g = torch.Generator(device="cpu").manual_seed(seed)
-    q = (torch.randn(T, Hq, D, generator=g) * std).to(torch.bfloat16)
-    k = (torch.randn(T, Hk, D, generator=g) * std).to(torch.bfloat16)
-    qw = (1 + 0.1 * torch.randn(D, generator=g)).to(torch.bfloat16)
-    kw = (1 + 0.1 * torch.randn(D, generator=g)).to(torch.bfloat16)
-    tbl = W.rope_table_input(T, R, 10000.0, f32)
+    q = (torch.randn(T, Hq, D, generator=g) * std).to(act)
+    k = (torch.randn(T, Hk, D, generator=g) * std).to(act)
+    qw = (1 + 0.1 * torch.randn(D, generator=g)).to(act)
+    kw = (1 + 0.1 * torch.randn(D, generator=g)).to(act)
+    tbl = W.rope_table_input(T, R, 10000.0, f32, act=act)
     return dict(q=q, k=k, q_weight=qw, k_weight=kw, rope_table=tbl)
 
 
@@ -303,14 +304,45 @@ def test_table_variants(case):
     check_table_against_oracle(inp, qo.cpu(), ko.cpu(), 1e-5, R, il, str(case))
 
 
-def test_table_strided_inplace_and_misaligned():
+@pytest.mark.parametrize("case", CASES_TABLE, ids=[str(i) for i in range(len(CASES_TABLE))])
+def test_table_variants_f16(case):
+    """The same shapes with IEEE binary16 activations and weights (the table
+    float32 or binary16 as the case says)."""
+    T, Hq, Hk, D, R, f32, il = case
+    inp = _rand_table_inputs(T, Hq, Hk, D, R, f32, seed=D + R + 1, std=2.0, act=torch.float16)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    qo, ko = Q.fused_qk_norm_rope(g["q"], g["k"], g["q_weight"], g["k_weight"], g["rope_table"],
+                                  1e-5, rotary_dim=R, interleaved=il)
+    torch.cuda.synchronize()
+    assert qo.dtype == torch.float16 and ko.dtype == torch.float16
+    check_table_against_oracle(inp, qo.cpu(), ko.cpu(), 1e-5, R, il, f"f16 {case}")
+
+
+def test_table_f16_small_and_large_magnitudes():
+    """binary16 has a narrow range: rows of 1e-3 and of 3e3 (squares past
+    binary16's range, but the sums are fp32) and a weight that sends outputs to
+    the subnormals must still match the oracle."""
+    T, H, D, R = 48, 3, 128, 128
+    for std, wscale in ((1e-3, 1.0), (3e3, 1.0), (1.0, 1e-4)):
+        inp = _rand_table_inputs(T, H, H, D, R, False, seed=17, std=std, act=torch.float16)
+        inp["q_weight"] = (inp["q_weight"].float() * wscale).half()
+        g = {k: v.to(DEV) for k, v in inp.items()}
+        qo, ko = Q.fused_qk_norm_rope(g["q"], g["k"], g["q_weight"], g["k_weight"],
+                                      g["rope_table"], 1e-6, interleaved=False)
+        torch.cuda.synchronize()
+        check_table_against_oracle(inp, qo.cpu(), ko.cpu(), 1e-6, R, False,
+                                   f"std {std} wscale {wscale}")
+
+
+@pytest.mark.parametrize("act", [torch.bfloat16, torch.float16], ids=["bf16", "f16"])
+def test_table_strided_inplace_and_misaligned(act):
     """q and k as views into a packed QKV buffer (token stride 3*H*D), updated
     in place; then the same with every pointer shifted by one element (general
     kernel); all must match the oracle on dense copies."""
     T, H, D, R = 64, 4, 128, 96
-    inp = _rand_table_inputs(T, H, H, D, R, True, seed=5)
+    inp = _rand_table_inputs(T, H, H, D, R, True, seed=5, act=act)
     for shift in (0, 1):
-        buf = torch.zeros(T * 3 * H * D + 64, dtype=torch.bfloat16, device=DEV)
+        buf = torch.zeros(T * 3 * H * D + 64, dtype=act, device=DEV)
         packed = buf[shift:shift + T * 3 * H * D].view(T, 3 * H, D)
         packed[:, :H] = inp["q"].to(DEV)
         packed[:, H:2 * H] = inp["k"].to(DEV)
