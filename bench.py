@@ -135,8 +135,9 @@ def dist_env():
 
 # --------------------------------------------------------------- oracle arm --
 def oracle_sample(w, inp_cpu, budget_s: float, chunk: int = 256):
-    """Time the fp64 oracle on consecutive token chunks of the workload until
-    budget_s of CPU work is spent; returns (tokens, seconds, threads)."""
+    """Time the fp64 oracle on consecutive token chunks of the workload,
+    cycling through it, until budget_s of CPU work is spent; returns (tokens
+    processed, seconds, threads)."""
     import oracle as O
     from tests._util import t2u16
 
@@ -147,11 +148,12 @@ def oracle_sample(w, inp_cpu, budget_s: float, chunk: int = 256):
     p = w.params()
     done, spent = 0, 0.0
     T = qkv.shape[0]
-    while spent < budget_s and done < T:
-        n = min(chunk, T - done)
-        bits = t2u16(qkv[done:done + n])
+    while spent < budget_s and T > 0:
+        s0 = done % T
+        n = min(chunk, T - s0)
+        bits = t2u16(qkv[s0:s0 + n])
         t0 = time.perf_counter()
-        O.rope_3d(bits, qw, kw, pos_offset=done, **p)
+        O.rope_3d(bits, qw, kw, pos_offset=s0, **p)
         spent += time.perf_counter() - t0
         done += n
     return done, spent, O.threads()
@@ -165,11 +167,12 @@ def oracle_sample_table(w, inp_cpu, budget_s: float, chunk: int):
     qw, kw = t2u16(inp_cpu["q_weight"]), t2u16(inp_cpu["k_weight"])
     done, spent = 0, 0.0
     T = q.shape[0]
-    while spent < budget_s and done < T:
-        n = min(chunk, T - done)
-        tb = tbl[done:done + n]
+    while spent < budget_s and T > 0:
+        s0 = done % T
+        n = min(chunk, T - s0)
+        tb = tbl[s0:s0 + n]
         tb = tb.numpy() if tb.dtype.is_floating_point and tb.element_size() == 4 else t2u16(tb)
-        qb, kb = t2u16(q[done:done + n]), t2u16(k[done:done + n])
+        qb, kb = t2u16(q[s0:s0 + n]), t2u16(k[s0:s0 + n])
         t0 = time.perf_counter()
         O.rope_table(qb, kb, qw, kw, tb, w.eps, w.rotary_dim, interleaved=w.interleaved,
                      act=w.act)
@@ -186,13 +189,16 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     inp = W.make_inputs(w, device="cpu")
-    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    # About a minute of oracle work over the whole run, whatever K and W are;
+    # a step does at least one chunk, so small per-step budgets use small ones.
+    per_step = 60.0 / max(1, args.steps + args.warmup)
+    chunk = 256 if per_step >= 0.5 else 32
     for _ in range(args.warmup):
-        oracle_sample(w, inp, min(per_step, 2.0))
+        oracle_sample(w, inp, per_step, chunk)
     toks, secs = 0, 0.0
     threads = 1
     for _ in range(args.steps):
-        n, s, threads = oracle_sample(w, inp, per_step)
+        n, s, threads = oracle_sample(w, inp, per_step, chunk)
         toks += n
         secs += s
     value = toks / secs
@@ -201,10 +207,12 @@ def run_reference(args, w):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "tokens": w.tokens, "sample": "leading tokens"},
+        "config": {"workload": w.name, "tokens": w.tokens,
+                   "sample": "token chunks in order, cycling through the workload"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{toks // max(1, args.steps)} leading tokens per step of "
-                                   f"{w.name}"},
+                         "sample": f"{toks // max(1, args.steps)} tokens per step of {w.name} "
+                                   f"(in order from its first token, cycling through its "
+                                   f"{w.tokens}; {secs / max(1, args.steps):.3f} s of oracle work per step)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -301,11 +309,11 @@ def run_gpu(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        inp_cpu = {"qkv": qkv[:, :min(T, 4096)].cpu() if qkv.dim() == 3 else qkv[:4096].cpu(),
-                   "q_weight": qw.cpu(), "k_weight": kw.cpu()}
+        inp_cpu = {"qkv": qkv.cpu(), "q_weight": qw.cpu(), "k_weight": kw.cpu()}
         n, s, threads = oracle_sample(w, inp_cpu, args.cpu_seconds)
         cpu = {"value": n / s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"first {n} tokens of {w.name} ({s:.1f} s of fp64 oracle work)"}
+               "sample": f"{n} tokens of {w.name} in order, cycling through its {T} "
+                         f"({s:.1f} s of fp64 oracle work)"}
 
     if rank == 0:
         clk = clocks.summary()
@@ -375,12 +383,11 @@ def run_gpu_table(args, w):
         e2e = measure_e2e_table(args, w, sets[0], run, stream, dev, world, pg)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_cpu = min(T, 2048)
-        inp_cpu = {k: v[:n_cpu].cpu() if k in ("q", "k", "rope_table") else v.cpu()
-                   for k, v in sets[0].items() if k not in ("q_out", "k_out")}
+        inp_cpu = {k: v.cpu() for k, v in sets[0].items() if k not in ("q_out", "k_out")}
         n, sec, threads = oracle_sample(w, inp_cpu, args.cpu_seconds, chunk=128)
         cpu = {"value": n / sec, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"first {n} tokens of {w.name} ({sec:.1f} s of fp64 oracle work)"}
+               "sample": f"{n} tokens of {w.name} in order, cycling through its {T} "
+                         f"({sec:.1f} s of fp64 oracle work)"}
     if rank == 0:
         q = sets[0]["q"]
         line = {
