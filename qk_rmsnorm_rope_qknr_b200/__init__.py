@@ -149,14 +149,15 @@ def _table_dtype(t: torch.Tensor, act: torch.dtype) -> int:
 
 def _token_stride(t: torch.Tensor, name: str, heads: int, head_dim: int,
                   dtype: torch.dtype = torch.bfloat16) -> int:
-    if t.dim() != 3 or t.shape[1] != heads or t.shape[2] != head_dim:
+    sh = t.shape  # (one shape and one stride tuple: this runs on every call)
+    if len(sh) != 3 or sh[1] != heads or sh[2] != head_dim:
         raise QknrValueError(QKNR_ERR_SHAPE, f"{name} must be [tokens, {heads}, {head_dim}]")
     if t.dtype != dtype:
         raise QknrValueError(QKNR_ERR_SHAPE, f"{name} must be {dtype}")
-    if t.shape[0] > 0 and heads > 0 and (t.stride(2) != 1 or (heads > 1 and
-                                                             t.stride(1) != head_dim)):
+    st = t.stride()
+    if sh[0] > 0 and heads > 0 and (st[2] != 1 or (heads > 1 and st[1] != head_dim)):
         raise QknrValueError(QKNR_ERR_SHAPE, f"{name}: heads must be dense inside a token")
-    return t.stride(0)
+    return st[0]
 
 
 # --------------------------------------------------------------- C-ABI names --

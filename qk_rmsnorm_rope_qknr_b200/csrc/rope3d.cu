@@ -41,6 +41,7 @@
 // loads straight into registers.
 #include "common.cuh"
 #include "launch.h"
+#include "launch_cache.h"
 
 #include <algorithm>
 
@@ -763,22 +764,16 @@ cudaError_t launch_overlapped(K kern, int grid, int block, int smem, cudaStream_
 }
 
 int device_sms() {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    return sms;
+    int sms = 0;
+    return cached_sm_count(&sms) == cudaSuccess ? sms : 0;
 }
 
 template <typename K>
 cudaError_t launch_grid(K kern, int block, int smem, int64_t tokens, const Rope3DArgs& args,
                         cudaStream_t stream, int* grid_out) {
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             smem);
-        if (e != cudaSuccess) return e;
-    }
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, smem);
+    cudaError_t e =
+        cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), block, smem, &per_sm);
     if (e != cudaSuccess) return e;
     const int sms = device_sms();
     if (sms <= 0) return cudaErrorNoDevice;
@@ -827,10 +822,20 @@ cudaError_t run(const Rope3DArgs& a, int block, cudaStream_t stream, LaunchInfo*
         if (args.wait_limit_ns == 0) args.wait_limit_ns = 2000000000ull;  // 2 s
         smem = mg_layout(D, groups, stages, row_bytes, weight_floats, used_table).total;
         auto kern = rope3d_mg_kernel<D, NEOX, FP8, S>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        int per_sm = 0;
+        e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), block * groups, smem,
+                                      &per_sm);
+        if (e == cudaSuccess && per_sm < 1) e = cudaErrorInvalidConfiguration;
         if (e == cudaSuccess) {
             grid = (int)std::min<int64_t>(sms, (a.num_tokens + groups - 1) / groups);
             e = launch_overlapped(kern, grid, block * groups, smem, stream, args);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                forget_kernel(reinterpret_cast<const void*>(kern));
+                e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), block * groups,
+                                              smem, &per_sm);
+                if (e == cudaSuccess) e = launch_overlapped(kern, grid, block * groups, smem, stream, args);
+            }
         }
         id = 3100;
         block *= groups;

@@ -23,8 +23,11 @@
 // alignments the fast kernel does not take.
 #include "common.cuh"
 #include "launch.h"
+#include "launch_cache.h"
 
 #include <algorithm>
+#include <mutex>
+#include <unordered_map>
 
 namespace qknr {
 
@@ -85,14 +88,36 @@ __host__ __device__ inline int table_stage_bytes(int per_item, int D, int R, int
     return (per_item * D * 2 + R * tb + 15) & ~15;
 }
 
+// Per-lane plan of the fast kernel, chosen on the host (make_lane_map): the
+// two 16-byte vectors of its head that a lane holds, which of them its first
+// and its second shared-memory load fetch, and how they rotate. The order is
+// picked so that the 8 lanes of each 128-bit load phase hit 8 different bank
+// groups. For a half-split pair whose loads are swapped the lane negates its
+// sines, which keeps one rotation formula for both orders.
+struct LaneMap {
+    uint32_t lane[32];
+};
+constexpr uint32_t kLmFirst = 0x1Fu;          // bits 0-4: vector of the first load
+constexpr int kLmSecondShift = 5;             // bits 5-9: vector of the second load
+constexpr uint32_t kLmSwapped = 1u << 10;     // half-split pair loaded (b, a)
+constexpr uint32_t kLmAcross = 1u << 11;      // the two vectors pair up (half split)
+constexpr uint32_t kLmRot1 = 1u << 12;        // first vector's adjacent pairs rotate
+constexpr uint32_t kLmRot2 = 1u << 13;        // second vector's adjacent pairs rotate
+constexpr uint32_t kLmActive = 1u << 14;      // the lane holds part of a head
+constexpr int kWsmBytes = 2 * 4 * 32 * 16;    // weights: [q|k][4 quarter-vectors][32 lanes] float4
+
 template <int GS, bool IL, bool F32, bool H16>
-__global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a) {
+__global__ void __launch_bounds__(kBlock)
+    rope_table_bulk(const RopeTableArgs a, const __grid_constant__ LaneMap m) {
     constexpr int HR = 32 / GS;  // heads per warp round
     const int D = a.head_dim, R = a.rotary_dim;
-    const int L = D / 16;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int l = lane % GS, sub = lane / GS;
-    const bool active = l < L;
+    const int sub = lane / GS;
+    const uint32_t plan = m.lane[lane];
+    const bool active = (plan & kLmActive) != 0;
+    const int v1 = (int)(plan & kLmFirst), v2 = (int)((plan >> kLmSecondShift) & kLmFirst);
+    const bool across = (plan & kLmAcross) != 0, swapped = (plan & kLmSwapped) != 0;
+    const bool rot1 = (plan & kLmRot1) != 0, rot2 = (plan & kLmRot2) != 0;
     const int H = a.hq + a.hk;
     const int per_item = kUnroll * HR;               // heads of one token per warp item
     const int cpt = (H + per_item - 1) / per_item;   // items per token
@@ -102,9 +127,9 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
     const int sbytes = table_stage_bytes(per_item, D, R, tb);
 
     extern __shared__ __align__(128) unsigned char smem[];
-    float* wsm = reinterpret_cast<float*>(smem);                       // [q | k][D] fp32
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * 256 * 4);  // [warps][stages]
-    unsigned char* rings = smem + 2 * 256 * 4 + ((kBlock / 32) * stages * 8 + 127) / 128 * 128;
+    float4* wsm = reinterpret_cast<float4*>(smem);                  // see kWsmBytes
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWsmBytes);  // [warps][stages]
+    unsigned char* rings = smem + kWsmBytes + ((kBlock / 32) * stages * 8 + 127) / 128 * 128;
     uint64_t* full = bars + warp * stages;
     unsigned char* ring = rings + (size_t)warp * stages * sbytes;
 
@@ -140,10 +165,22 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
     // no-op unless launched as a programmatic dependent launch).
     griddep_wait();
     griddep_launch_dependents();
-    for (int c = threadIdx.x; c < 2 * D; c += blockDim.x) {
-        const uint16_t* w = reinterpret_cast<const uint16_t*>(c < D ? a.q_weight : a.k_weight);
-        const int cc = c < D ? c : c - D;
-        wsm[c] = ((c < D ? a.hq : a.hk) > 0) ? act_to_f<H16>(w[cc]) : 0.0f;
+    // Weights as fp32, laid out per lane: entry (k, lane) of q or k holds the
+    // channels 4k'..4k'+3 of the lane's vector (k < 2 ? first : second), k' =
+    // k & 1, so that each of a lane's four weight loads reads 32 consecutive
+    // float4 across the warp.
+    for (int c = threadIdx.x; c < 2 * 4 * 32; c += blockDim.x) {
+        const int isk = c >> 7, k = (c >> 5) & 3, ln = c & 31;
+        const uint32_t pl = m.lane[ln];
+        float4 w4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if ((pl & kLmActive) && (isk ? a.hk : a.hq) > 0) {
+            const int v = k < 2 ? (int)(pl & kLmFirst) : (int)((pl >> kLmSecondShift) & kLmFirst);
+            const uint16_t* w =
+                reinterpret_cast<const uint16_t*>(isk ? a.k_weight : a.q_weight) + v * 8 + (k & 1) * 4;
+            w4 = make_float4(act_to_f<H16>(w[0]), act_to_f<H16>(w[1]), act_to_f<H16>(w[2]),
+                             act_to_f<H16>(w[3]));
+        }
+        wsm[c] = w4;
     }
     __syncwarp();
     int64_t t = warp_id / cpt;
@@ -160,20 +197,6 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
     }
     __syncthreads();  // weights
 
-    // Vectors of this lane inside a head and how they rotate.
-    int va, vb;
-    bool across = false, rot_a = false, rot_b = false;
-    if (IL) {
-        va = l; vb = l + L;
-        rot_a = va < R / 8; rot_b = vb < R / 8;
-    } else {
-        const int r16 = R / 16;
-        if (l < r16) {
-            va = l; vb = l + r16; across = true;
-        } else {
-            va = R / 8 + 2 * (l - r16); vb = va + 1;
-        }
-    }
     const float inv_d = 1.0f / (float)D;
     // the item `stages` ahead of the current one
     int64_t t_ahead = t, chunk_ahead = chunk;
@@ -199,10 +222,14 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
         float c[8], s[8];
         if (active) {
             if (IL) {
-                if (rot_a) smem_cos_sin4<F32, H16>(trow, 4 * va, R / 2, c, s);
-                if (rot_b) smem_cos_sin4<F32, H16>(trow, 4 * vb, R / 2, c + 4, s + 4);
+                if (rot1) smem_cos_sin4<F32, H16>(trow, 4 * v1, R / 2, c, s);
+                if (rot2) smem_cos_sin4<F32, H16>(trow, 4 * v2, R / 2, c + 4, s + 4);
             } else if (across) {
-                smem_cos_sin8<F32, H16>(trow, 8 * va, R / 2, c, s);
+                smem_cos_sin8<F32, H16>(trow, 8 * min(v1, v2), R / 2, c, s);
+                if (swapped) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) s[k] = -s[k];
+                }
             }
         }
 #pragma unroll
@@ -213,8 +240,8 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
             uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
             if (okh) {
                 const uint4* v = reinterpret_cast<const uint4*>(buf + (size_t)hi * D * 2);
-                xa = v[va];
-                xb = v[vb];
+                xa = v[v1];
+                xb = v[v2];
             }
             float2 fa[4], fb[4];
             fa[0] = act2_to_f2<H16>(xa.x); fa[1] = act2_to_f2<H16>(xa.y);
@@ -233,9 +260,8 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
             const int head = isk ? hh - a.hq : hh;
             const float r = rsqrtf(ss * inv_d + a.eps);
             const float2 r2 = make_float2(r, r);
-            const float4* w4 = reinterpret_cast<const float4*>(wsm + (isk ? D : 0));
-            const float4 wa0 = w4[2 * va], wa1 = w4[2 * va + 1];
-            const float4 wb0 = w4[2 * vb], wb1 = w4[2 * vb + 1];
+            const float4* w4 = wsm + (isk ? 4 * 32 : 0) + lane;
+            const float4 wa0 = w4[0], wa1 = w4[32], wb0 = w4[64], wb1 = w4[96];
             fa[0] = mul2(mul2(fa[0], r2), make_float2(wa0.x, wa0.y));
             fa[1] = mul2(mul2(fa[1], r2), make_float2(wa0.z, wa0.w));
             fa[2] = mul2(mul2(fa[2], r2), make_float2(wa1.x, wa1.y));
@@ -248,13 +274,13 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
             if (IL) {
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
-                    if (rot_a) {
+                    if (rot1) {
                         oa[m].x = fa[m].x * c[m] - fa[m].y * s[m];
                         oa[m].y = fa[m].y * c[m] + fa[m].x * s[m];
                     } else {
                         oa[m] = fa[m];
                     }
-                    if (rot_b) {
+                    if (rot2) {
                         ob[m].x = fb[m].x * c[4 + m] - fb[m].y * s[4 + m];
                         ob[m].y = fb[m].y * c[4 + m] + fb[m].x * s[4 + m];
                     } else {
@@ -277,10 +303,10 @@ __global__ void __launch_bounds__(kBlock) rope_table_bulk(const RopeTableArgs a)
             uint8_t* dst = isk
                 ? a.k_out + ((size_t)t * a.k_out_stride + (size_t)head * D) * 2
                 : a.q_out + ((size_t)t * a.q_out_stride + (size_t)head * D) * 2;
-            st_v4(dst + (size_t)va * 16,
+            st_v4(dst + (size_t)v1 * 16,
                   make_uint4(f2_to_act2<H16>(oa[0]), f2_to_act2<H16>(oa[1]),
                              f2_to_act2<H16>(oa[2]), f2_to_act2<H16>(oa[3])));
-            st_v4(dst + (size_t)vb * 16,
+            st_v4(dst + (size_t)v2 * 16,
                   make_uint4(f2_to_act2<H16>(ob[0]), f2_to_act2<H16>(ob[1]),
                              f2_to_act2<H16>(ob[2]), f2_to_act2<H16>(ob[3])));
         }
@@ -382,11 +408,10 @@ __global__ void __launch_bounds__(kBlock) rope_table_general(const RopeTableArgs
 template <typename K>
 cudaError_t launch_persistent(K kern, int64_t work_blocks, const RopeTableArgs& a,
                               cudaStream_t stream, LaunchInfo* info, int id) {
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBlock,
-                                                                            0);
+    int sms = 0, per_sm = 0;
+    cudaError_t e = cached_sm_count(&sms);
+    if (e == cudaSuccess)
+        e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), kBlock, 0, &per_sm);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * per_sm,
@@ -401,6 +426,91 @@ cudaError_t launch_persistent(K kern, int64_t work_blocks, const RopeTableArgs& 
     return cudaGetLastError();
 }
 
+// Host side of LaneMap. The lanes of a head are l < D/16; lane l holds
+// vectors (l, l + D/16) when pairs are adjacent channels, the pair
+// (l, l + rotary_dim/16) when they are half split and l < rotary_dim/16, and
+// two pass-through vectors otherwise. For each phase of 8 lanes (a 128-bit
+// shared load serves 8 lanes at a time) every choice of load order is scored
+// by its bank-group collisions over the item's 4 rounds, and the best kept.
+LaneMap make_lane_map(const RopeTableArgs& a, int GS) {
+    const int D = a.head_dim, R = a.rotary_dim;
+    const int L = D / 16, VPH = D / 8, HR = 32 / GS, r16 = R / 16, rv = R / 8;
+    int va[32], vb[32];
+    bool act[32], acr[32];
+    for (int ln = 0; ln < 32; ++ln) {
+        const int l = ln % GS;
+        act[ln] = l < L;
+        acr[ln] = false;
+        va[ln] = vb[ln] = 0;
+        if (!act[ln]) continue;
+        if (a.interleaved) {
+            va[ln] = l; vb[ln] = l + L;
+        } else if (l < r16) {
+            va[ln] = l; vb[ln] = l + r16; acr[ln] = true;
+        } else {
+            va[ln] = rv + 2 * (l - r16); vb[ln] = va[ln] + 1;
+        }
+    }
+    uint32_t order = 0;  // bit ln: lane ln loads (vb, va)
+    for (int ph = 0; ph < 4; ++ph) {
+        int best = 1 << 30, best_bits = 0;
+        for (int bits = 0; bits < 256; ++bits) {
+            int cost = 0;
+            for (int u = 0; u < kUnroll; ++u) {
+                for (int ld = 0; ld < 2; ++ld) {
+                    int count[8] = {0, 0, 0, 0, 0, 0, 0, 0}, worst = 0;
+                    for (int j = 0; j < 8; ++j) {
+                        const int ln = ph * 8 + j;
+                        if (!act[ln]) continue;
+                        const bool sw = (bits >> j) & 1;
+                        const int v = (ld == 0) != sw ? va[ln] : vb[ln];
+                        const int hi = u * HR + ln / GS;
+                        const int c = ++count[(hi * VPH + v) & 7];
+                        worst = c > worst ? c : worst;
+                    }
+                    cost += worst;
+                }
+            }
+            cost = cost * 16 + __builtin_popcount(bits);  // fewer swaps on a tie
+            if (cost < best) {
+                best = cost;
+                best_bits = bits;
+            }
+        }
+        order |= (uint32_t)best_bits << (8 * ph);
+    }
+    LaneMap m;
+    for (int ln = 0; ln < 32; ++ln) {
+        if (!act[ln]) {
+            m.lane[ln] = 0;
+            continue;
+        }
+        const bool sw = (order >> ln) & 1;
+        const int v1 = sw ? vb[ln] : va[ln], v2 = sw ? va[ln] : vb[ln];
+        uint32_t w = (uint32_t)v1 | ((uint32_t)v2 << kLmSecondShift) | kLmActive;
+        if (acr[ln]) w |= kLmAcross | (sw ? kLmSwapped : 0u);
+        if (a.interleaved && v1 < rv) w |= kLmRot1;
+        if (a.interleaved && v2 < rv) w |= kLmRot2;
+        m.lane[ln] = w;
+    }
+    return m;
+}
+
+// make_lane_map is a search (about 65 thousand steps); launches look up its
+// result per shape.
+LaneMap lane_map_cached(const RopeTableArgs& a, int GS) {
+    static std::mutex mu;
+    static std::unordered_map<uint32_t, LaneMap> cache;
+    const uint32_t key = (uint32_t)a.head_dim | ((uint32_t)a.rotary_dim << 9) |
+                         ((uint32_t)(a.interleaved != 0) << 18) | ((uint32_t)GS << 19);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    const LaneMap m = make_lane_map(a, GS);
+    cache.emplace(key, m);
+    return m;
+}
+
 template <typename K>
 cudaError_t launch_bulk(K kern, const RopeTableArgs& a0, int per_item, cudaStream_t stream,
                         LaunchInfo* info, int id) {
@@ -409,17 +519,15 @@ cudaError_t launch_bulk(K kern, const RopeTableArgs& a0, int per_item, cudaStrea
     const int sbytes = table_stage_bytes(per_item, a.head_dim, a.rotary_dim, tb);
     const int warps = kBlock / 32;
     // Two CTAs per SM, each warp with as many ring buffers (2..4) as fit.
-    const int fixed = 2 * 256 * 4 + 128 + warps * 4 * 8;
+    const int fixed = kWsmBytes + 128 + warps * 4 * 8;
     a.stages = std::max(2, std::min(4, (227 * 1024 / 2 - 1024 - fixed) / (warps * sbytes)));
     if (a.wait_limit_ns == 0) a.wait_limit_ns = 2000000000ull;  // 2 s
-    const int smem = 2 * 256 * 4 + ((warps * a.stages * 8 + 127) / 128 * 128) +
+    const int smem = kWsmBytes + ((warps * a.stages * 8 + 127) / 128 * 128) +
                      warps * a.stages * sbytes;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    int dev = 0, sms = 0, per_sm = 0;
-    if (e == cudaSuccess) e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int sms = 0, per_sm = 0;
+    cudaError_t e = cached_sm_count(&sms);
     if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBlock, smem);
+        e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), kBlock, smem, &per_sm);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int H = a.hq + a.hk;
@@ -437,7 +545,14 @@ cudaError_t launch_bulk(K kern, const RopeTableArgs& a0, int per_item, cudaStrea
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, a);
+    const LaneMap m = lane_map_cached(a, 32 / (per_item / kUnroll));
+    e = cudaLaunchKernelEx(&cfg, kern, a, m);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        forget_kernel(reinterpret_cast<const void*>(kern));
+        e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), kBlock, smem, &per_sm);
+        if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, kern, a, m);
+    }
     if (info) {
         info->grid = grid;
         info->block = kBlock;
