@@ -361,8 +361,8 @@ int qknr_oracle_rope_table_exact(const uint16_t* q, const uint16_t* k, const uin
 }
 
 /* Table form rounded to the activation type (R3): bf16, or binary16 when
- * act_is_f16 (the pages allow the table in "the activation dtype or float32",
- * so activations other than bf16 exist; binary16 is the other 16-bit one). */
+ * act_is_f16 ([T] lets the table take the activation type or fp32, so the
+ * activation type is not fixed to bf16; binary16 is the other 16-bit one). */
 int qknr_oracle_rope_table_act(const uint16_t* q, const uint16_t* k, const uint16_t* q_weight,
                                const uint16_t* k_weight, const void* table, int32_t table_is_f32,
                                int32_t act_is_f16, int64_t num_tokens, int32_t heads_q,

@@ -53,6 +53,14 @@ MUTATIONS = {
                            "if (v >= 65504.0) return (uint16_t)(sign | 0x7C00u);"),
     "act_type_ignored": ("return act_is_f16 ? qknr_oracle_f16_to_double(b) : qknr_oracle_bf16_to_double(b);",
                          "return qknr_oracle_bf16_to_double(b);"),
+    "f16_nine_bit_significand": ("double quantum = ldexp(1.0, e - 10);",
+                                 "double quantum = ldexp(1.0, e - 9);"),
+    "f16_subnormal_unit": ("ldexp(1.0, -24)", "ldexp(1.0, -23)"),
+    "f16_outputs_rounded_as_bf16": ("if (rc == 0 && act_is_f16) {", "if (rc == 0 && 0) {"),
+    "f16_weights_read_as_bf16": ("wq[d] = act_to_double(q_weight[d], act_is_f16);",
+                                 "wq[d] = act_to_double(q_weight[d], 0);"),
+    "f16_table_read_as_bf16": ("c[j] = act_to_double(row[j], act_is_f16);",
+                               "c[j] = act_to_double(row[j], 0);"),
 }
 
 # cheap pins first, so a planted mistake is usually caught within a second
