@@ -13,11 +13,14 @@
 // every rotation pair sits inside the lane: half split -> vectors l and
 // l + rotary_dim/16 for l < rotary_dim/16, the pass-through vectors two by two
 // after that; interleaved -> vectors l and l + D/16. The group's sum of
-// squares is a GS-lane shuffle reduction: no shared memory, no barrier. A warp
-// item is 4 rounds of 32/GS heads of one token: the lane's cos/sin for that
-// token (the same for every head) are loaded once, together with the 8 data
-// vectors, so that one memory latency covers the item. The norm weights live
-// in shared memory as fp32.
+// squares is a GS-lane shuffle reduction: no barrier. A warp item is 4 rounds
+// of 32/GS heads of one token. Each warp keeps a ring of shared-memory buffers
+// that its lane 0 fills with bulk asynchronous copies (the item's q heads, k
+// heads and the token's table row) a ring ahead of use; the lane's cos/sin for
+// the token (the same for every head) are read once per item. Which of a
+// lane's two vectors each shared load fetches is planned on the host so that
+// no two lanes of a load phase share a bank group (LaneMap); the norm weights
+// sit in shared memory as fp32 in the matching lane-major order.
 //
 // General kernel: one warp per head through shared memory, for the shapes and
 // alignments the fast kernel does not take.
