@@ -91,6 +91,10 @@ typedef enum {
  * heads_q, heads_k >= 0 (a tensor with 0 heads is neither read nor written and
  *               its pointers may be NULL).
  * eps           >= 0.
+ * Range: sums of squares are accumulated in fp32, so a head whose sum of
+ * squares overflows fp32 (|x| above about 1e18 at head_dim 128) comes out as
+ * zeros or NaN; with eps == 0 an all-zero head comes out as NaN (0/0), as in
+ * the definition.
  * Fast path: every pointer and token stride 16-byte aligned, head_dim a
  * multiple of 16 and rotary_dim a multiple of 16 (half-split) or 8
  * (interleaved). Other valid inputs run a general kernel (2-byte alignment).
@@ -125,6 +129,9 @@ int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
  *      [T, Hv, head_dim], dense. bf16; or with output_fp8, E4M3 of
  *      q*output_quant_scale, k*output_quant_scale and v*v_quant_scale.
  *      Without output_fp8, v_out is a bit copy of V.
+ *   Range: the sums of squares are fp32, so a row whose Q or K sum of squares
+ *      overflows fp32 (|x| above about 1e17 over 4096 channels) comes out as
+ *      zeros or NaN; with eps == 0 an all-zero Q or K comes out as NaN (0/0).
  *
  * Validation: num_tokens divisible by ppf*pph*ppw for a whole call, any count
  * for a sequence shard (sequence_shard = 1); channel counts even,

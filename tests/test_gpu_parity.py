@@ -370,6 +370,47 @@ def test_table_outputs_written_exactly():
     assert not torch.any(qb[:T * Hq * D] == -1) and not torch.any(kb[:T * Hk * D] == -1)
 
 
+def test_empty_inputs_both_forms():
+    """No tokens: both entry points succeed, return empty outputs and launch
+    nothing."""
+    w = W.WORKLOADS["tiny3d"]
+    qkv = torch.empty(0, w.row, dtype=torch.bfloat16, device=DEV)
+    qw = torch.ones(w.hq * w.head_dim, dtype=torch.bfloat16, device=DEV)
+    kw = torch.ones(w.hk * w.head_dim, dtype=torch.bfloat16, device=DEV)
+    q, k, v = run_3d(qkv, qw, kw, **w.params())
+    assert q.shape == (0, w.hq, w.head_dim) and k.shape[0] == 0 and v.shape[0] == 0
+    for act in (torch.bfloat16, torch.float16):
+        x = torch.empty(0, 4, 128, dtype=act, device=DEV)
+        wt = torch.ones(128, dtype=act, device=DEV)
+        tbl = torch.empty(0, 96, dtype=torch.float32, device=DEV)
+        qo, ko = Q.fused_qk_norm_rope(x, x[:, :2], wt, wt, tbl, 1e-6, rotary_dim=96)
+        assert qo.shape == (0, 4, 128) and ko.shape == (0, 2, 128)
+    torch.cuda.synchronize()
+
+
+def test_zero_rows_give_zero_outputs():
+    """A token whose Q (or one head) is all zeros: r = 1/sqrt(eps) is finite and
+    every output of that row is exactly zero, as in the oracle."""
+    qkv, qw, kw = _rand3d(24, 3, 3, 2, 128, seed=11)
+    qkv[5, :3 * 128] = 0          # token 5: every Q head
+    qkv[9, 3 * 128:6 * 128] = 0   # token 9: every K head
+    p = dict(ppf=2, pph=3, ppw=4, num_frame_channels=32, num_height_channels=48,
+             num_width_channels=48, num_heads_q=3, num_heads_k=3, num_heads_v=2, head_dim=128,
+             eps=1e-6)
+    q, k, _ = check_3d_case(qkv, qw, kw, **p)
+    assert torch.all(q[5].float() == 0) and torch.all(k[9].float() == 0)
+    for act in (torch.bfloat16, torch.float16):
+        inp = _rand_table_inputs(16, 3, 2, 128, 96, True, seed=12, act=act)
+        inp["q"][4, 1] = 0
+        inp["k"][7] = 0
+        g = {n: t.to(DEV) for n, t in inp.items()}
+        qo, ko = Q.fused_qk_norm_rope(g["q"], g["k"], g["q_weight"], g["k_weight"],
+                                      g["rope_table"], 1e-6, rotary_dim=96)
+        torch.cuda.synchronize()
+        check_table_against_oracle(inp, qo.cpu(), ko.cpu(), 1e-6, 96, False, f"zero rows {act}")
+        assert torch.all(qo[4, 1].float() == 0) and torch.all(ko[7].float() == 0)
+
+
 def test_3d_sequence_shards_match_whole_call():
     """Sequence sharding (what each rank of a multi-GPU run does): the token
     shards of sharding.token_shard, each called with its pos_offset, give the
