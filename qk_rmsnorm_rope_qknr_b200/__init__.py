@@ -288,8 +288,9 @@ def fused_qk_norm_rope(q: torch.Tensor, k: torch.Tensor, q_weight: torch.Tensor,
                        interleaved: bool = False, q_out: Optional[torch.Tensor] = None,
                        k_out: Optional[torch.Tensor] = None, stream=None
                        ) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Q/K RMSNorm + packed RoPE, table form. Returns new (q, k) unless outputs
-    are given (pass q_out=q, k_out=k to work in place)."""
+    """Q/K RMSNorm + packed RoPE, table form. q and k are bf16 or float16 (the
+    weights too; the table float32 or the same 16-bit type). Returns new
+    (q, k) unless outputs are given (pass q_out=q, k_out=k to work in place)."""
     D = head_dim or q.shape[-1]
     if q.shape[-1] != D or k.shape[-1] != D:
         raise QknrValueError(QKNR_ERR_SHAPE, f"last dim of q/k must be head_dim={D}")
