@@ -81,7 +81,15 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+        # nvidia-smi numbers GPUs physically; under CUDA_VISIBLE_DEVICES the
+        # CUDA ordinal can differ, so name the GPU by its UUID when torch has it.
+        self.gpu = str(gpu_index)
+        try:
+            import torch
+
+            self.gpu = f"GPU-{torch.cuda.get_device_properties(gpu_index).uuid}"
+        except Exception:  # noqa: BLE001 - fall back to the ordinal
+            pass
         self.proc = None
         self.lines = []
         self.t = None
@@ -129,9 +137,10 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "gpu": self.gpu}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "gpu": self.gpu}
 
 
 def dist_env():
