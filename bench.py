@@ -37,8 +37,8 @@ FALLBACK_HBM_GBS = 6650.0
 # rope_table.md), valid only for the kernel sources whose hash is stored
 # beside it (the bench reports null otherwise).
 TRAFFIC = {
-    "video3d": (377585408 + 325397248, "965b3476a7640b1d"),
-    "fp8neox": (1097208064 + 518009088, "965b3476a7640b1d"),
+    "video3d": (377564416 + 325334784, "f0170ddbe869b9f9"),
+    "fp8neox": (1097153280 + 517297920, "f0170ddbe869b9f9"),
     "table_hs": (43557376 + 2189312, "46fea1ecdc3d7a74"),
     "table_il": (25730560 + 2816, "46fea1ecdc3d7a74"),
     "table_hs_f16": (42769408 + 1922560, "46fea1ecdc3d7a74"),

@@ -5,9 +5,14 @@
 // byte is read once, every output byte written once, nothing else touches
 // memory.
 //
-// Thread layout. One token is worked on by a group of threads. A thread owns,
-// for S "slots" (head, l), the two 16-byte vectors l and l + D/16 of that
-// head of Q and of K (l = thread mod D/16, the same for all its slots).
+// Thread layout. One token is worked on by a group of threads. A slot is
+// (head, l): the two 16-byte vectors l and l + D/16 of one Q or K head. The
+// pipelined kernel deals a token's slots -- all Q slots, then all K slots --
+// to the group's threads S at a time (thread i takes slots i, i + Bg, ...), so
+// that Q and K head counts that differ (grouped-query attention) still give
+// every thread the same work; the fallback kernel gives a thread S Q slots and
+// the S K slots of the same index. Either way l = thread mod D/16, the same
+// for all of a thread's slots.
 // Vector l's channel e pairs with vector l + D/16's channel e in NeoX mode; in
 // interleaved mode adjacent channels of one vector pair up. Either way the 8
 // rotation pairs of a thread stay inside the thread, at fixed pair slots.
@@ -310,7 +315,10 @@ __host__ __device__ inline MgLayout mg_layout(int D, int groups, int stages, int
     return o;
 }
 
-template <int D, bool NEOX, bool FP8, int S>
+// S slots per thread. MIXED: thread i takes slots i, i + Bg, ... of the list
+// [Q slots | K slots]; otherwise slot k of a thread stands for the Q slot and
+// the K slot of index i + k * Bg (equal Q and K head counts).
+template <int D, bool NEOX, bool FP8, int S, bool MIXED>
 __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
     constexpr int L = D / 16;
     constexpr int VPH = D / 8;
@@ -452,14 +460,27 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
 #pragma unroll
                 for (int k = 0; k < S; ++k) {
                     const int slot = ctid + k * Bg;
-                    const int h = slot / L;
-                    if (slot < nq) {
-                        const uint4* q4 = reinterpret_cast<const uint4*>(row) + h * VPH + l;
-                        sq2 = ssq_pair(q4[0], q4[L], sq2);
-                    }
-                    if (slot < nk) {
-                        const uint4* k4 = reinterpret_cast<const uint4*>(row) + (a.hq + h) * VPH + l;
-                        sk2 = ssq_pair(k4[0], k4[L], sk2);
+                    if constexpr (MIXED) {  // Q slots, then K slots
+                        if (slot < nq) {
+                            const uint4* q4 =
+                                reinterpret_cast<const uint4*>(row) + (slot / L) * VPH + l;
+                            sq2 = ssq_pair(q4[0], q4[L], sq2);
+                        } else if (slot < nq + nk) {
+                            const uint4* k4 = reinterpret_cast<const uint4*>(row) +
+                                              (a.hq + (slot - nq) / L) * VPH + l;
+                            sk2 = ssq_pair(k4[0], k4[L], sk2);
+                        }
+                    } else {
+                        const int h = slot / L;
+                        if (slot < nq) {
+                            const uint4* q4 = reinterpret_cast<const uint4*>(row) + h * VPH + l;
+                            sq2 = ssq_pair(q4[0], q4[L], sq2);
+                        }
+                        if (slot < nk) {
+                            const uint4* k4 =
+                                reinterpret_cast<const uint4*>(row) + (a.hq + h) * VPH + l;
+                            sk2 = ssq_pair(k4[0], k4[L], sk2);
+                        }
                     }
                 }
             }
@@ -598,16 +619,19 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
 #pragma unroll
         for (int k = 0; k < S; ++k) {
             const int slot = ctid + k * Bg;
-            const int h = slot / L;
-            if (slot < nq) {
-                const uint4* q4 = reinterpret_cast<const uint4*>(row) + h * VPH + l;
-                apply_slot_wf<D, NEOX, FP8>(q4[0], q4[L], wsm + h * 2 * VPH, norm, rq, cs, sn,
-                                            a.q_out + (t * a.hq + h) * D * OUTB, l);
+            const bool is_q = slot < nq;
+            const bool is_k = MIXED ? (slot >= nq && slot < nq + nk) : slot < nk;
+            const int hq_i = slot / L, hk_i = MIXED ? (slot - nq) / L : slot / L;
+            if (is_q) {
+                const uint4* q4 = reinterpret_cast<const uint4*>(row) + hq_i * VPH + l;
+                apply_slot_wf<D, NEOX, FP8>(q4[0], q4[L], wsm + hq_i * 2 * VPH, norm, rq, cs, sn,
+                                            a.q_out + (t * a.hq + hq_i) * D * OUTB, l);
             }
-            if (slot < nk) {
-                const uint4* k4 = reinterpret_cast<const uint4*>(row) + (a.hq + h) * VPH + l;
-                apply_slot_wf<D, NEOX, FP8>(k4[0], k4[L], wsm + (a.hq + h) * 2 * VPH, norm, rk,
-                                            cs, sn, a.k_out + (t * a.hk + h) * D * OUTB, l);
+            if (is_k) {
+                const uint4* k4 = reinterpret_cast<const uint4*>(row) + (a.hq + hk_i) * VPH + l;
+                apply_slot_wf<D, NEOX, FP8>(k4[0], k4[L], wsm + (a.hq + hk_i) * 2 * VPH, norm,
+                                            rk, cs, sn, a.k_out + (t * a.hk + hk_i) * D * OUTB,
+                                            l);
             }
         }
     }
@@ -784,9 +808,17 @@ cudaError_t launch_grid(K kern, int block, int smem, int64_t tokens, const Rope3
     return cudaGetLastError();
 }
 
+// S: the Q slot and K slot pairs per thread at block_reg threads (the
+// fallback kernel, and the pipelined kernel when Q and K have as many heads).
+// With unequal head counts the pipelined kernel instead deals 2S slots per
+// thread from the list [Q slots | K slots] over block_mg threads, so that every
+// thread still has the same work.
 template <int D, bool NEOX, bool FP8, int S>
-cudaError_t run(const Rope3DArgs& a, int block, cudaStream_t stream, LaunchInfo* info) {
+cudaError_t run(const Rope3DArgs& a, int block_mg, int block_reg, cudaStream_t stream,
+                LaunchInfo* info) {
     constexpr int HALF = D / 2;
+    const bool mixed = a.hq != a.hk;
+    int block = mixed ? block_mg : block_reg;
     Rope3DArgs args = a;
     const bool partial = a.mode == kModePartialSsq;
     const int table_bytes = a.table_entries * 8;
@@ -821,7 +853,8 @@ cudaError_t run(const Rope3DArgs& a, int block, cudaStream_t stream, LaunchInfo*
         args.v_bulk = FP8 ? 0 : 1;
         if (args.wait_limit_ns == 0) args.wait_limit_ns = 2000000000ull;  // 2 s
         smem = mg_layout(D, groups, stages, row_bytes, weight_floats, used_table).total;
-        auto kern = rope3d_mg_kernel<D, NEOX, FP8, S>;
+        void (*kern)(const Rope3DArgs) = mixed ? rope3d_mg_kernel<D, NEOX, FP8, 2 * S, true>
+                                               : rope3d_mg_kernel<D, NEOX, FP8, S, false>;
         int per_sm = 0;
         e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), block * groups, smem,
                                       &per_sm);
@@ -843,6 +876,7 @@ cudaError_t run(const Rope3DArgs& a, int block, cudaStream_t stream, LaunchInfo*
         return cudaErrorNotSupported;  // the tensor-parallel passes run on the pipelined kernel
     } else {
         smem = 2 * HALF * 8 + 64 * 8 + HALF * 8 + used_table;
+        block = block_reg;
         e = launch_grid(rope3d_reg_kernel<D, NEOX, FP8, S>, block, smem, a.num_tokens, args,
                         stream, &grid);
         id = 3000;
@@ -863,15 +897,18 @@ cudaError_t run_s(const Rope3DArgs& a, cudaStream_t stream, LaunchInfo* info) {
     int S = (slots + kMaxBlock - 1) / kMaxBlock;
     if (S > 4) return cudaErrorInvalidValue;  // rejected earlier by the host checks
     S = S <= 1 ? 1 : (S <= 2 ? 2 : 4);
-    int block = ((slots + S - 1) / S + 31) / 32 * 32;
+    int block_reg = ((slots + S - 1) / S + 31) / 32 * 32;
+    const int all_slots = std::max(a.hq + a.hk, 1) * L;
+    int block_mg = ((all_slots + 2 * S - 1) / (2 * S) + 31) / 32 * 32;
     // With few Q/K heads, widen the block so that V and the per-token cos/sin
     // have enough threads.
     const int v_vectors = a.hv * (D / 8);
-    while (block < 256 && (block < v_vectors / 2 || block < D / 2)) block += 32;
+    for (int* b : {&block_reg, &block_mg})
+        while (*b < 256 && (*b < v_vectors / 2 || *b < D / 2)) *b += 32;
     switch (S) {
-        case 1: return run<D, NEOX, FP8, 1>(a, block, stream, info);
-        case 2: return run<D, NEOX, FP8, 2>(a, block, stream, info);
-        default: return run<D, NEOX, FP8, 4>(a, block, stream, info);
+        case 1: return run<D, NEOX, FP8, 1>(a, block_mg, block_reg, stream, info);
+        case 2: return run<D, NEOX, FP8, 2>(a, block_mg, block_reg, stream, info);
+        default: return run<D, NEOX, FP8, 4>(a, block_mg, block_reg, stream, info);
     }
 }
 

@@ -158,6 +158,8 @@ CASES_3D = [
     (10000, 2, 2, 2, 64, (1, 1, 10000), (0, 0, 64), True, False, True, 0),  # no smem table
     (257, 0, 4, 2, 128, (1, 1, 257), (32, 48, 48), True, False, True, 0),   # no Q heads
     (64, 3, 3, 0, 128, (4, 4, 4), (32, 48, 48), False, True, True, 0),      # no V heads
+    (3000, 32, 8, 8, 128, (3, 40, 25), (32, 48, 48), True, False, True, 0),  # grouped-query
+    (2048, 16, 4, 4, 128, (2, 32, 32), (32, 48, 48), False, True, True, 0),  # GQA, NeoX, E4M3
 ]
 
 
