@@ -18,6 +18,7 @@ video-DiT and MiniMax-H3 geometries the pages name):
   fp8neox     3D form, [2,29760,(24+24+24)*128] ~N(0, 2^2), grid 31x24x40,
               32/48/48, NeoX pairs, E4M3 out (scales 0.5 / 0.25)
   fp8neox_nonorm  fp8neox with is_qk_norm=False
+  gqa3d       video3d's geometry with grouped-query heads 32+8+8 (parity and TP case)
 """
 from __future__ import annotations
 
@@ -113,6 +114,8 @@ WORKLOADS = {
     "fp8neox": Form3D("fp8neox", batch=2, seq=29760, ppf=31, pph=24, ppw=40, cf=32, ch=48,
                       cw=48, hq=24, hk=24, hv=24, head_dim=128, interleave=False,
                       output_fp8=True, q_scale=0.5, v_scale=0.25, std=2.0),
+    "gqa3d": Form3D("gqa3d", batch=1, seq=15360, ppf=16, pph=30, ppw=32, cf=16, ch=56, cw=56,
+                    hq=32, hk=8, hv=8, head_dim=128),
     "fp8neox_nonorm": Form3D("fp8neox_nonorm", batch=2, seq=29760, ppf=31, pph=24, ppw=40,
                              cf=32, ch=48, cw=48, hq=24, hk=24, hv=24, head_dim=128,
                              interleave=False, is_qk_norm=False, output_fp8=True, q_scale=0.5,

@@ -66,7 +66,7 @@ def check_3d_case(qkv, qw, kw, **p):
 
 
 # --------------------------------------------------------------- workloads --
-@pytest.mark.parametrize("name", ["tiny3d", "video3d", "fp8neox", "fp8neox_nonorm"])
+@pytest.mark.parametrize("name", ["tiny3d", "video3d", "fp8neox", "fp8neox_nonorm", "gqa3d"])
 def test_3d_workload_ragged_shard(name):
     """The workload's geometry on a shard of 3001 tokens that starts mid-grid:
     several CTAs' worth of tokens per CTA, a ragged end, wrapped positions."""
@@ -78,7 +78,7 @@ def test_3d_workload_ragged_shard(name):
     check_3d_case(g["qkv"], g["q_weight"], g["k_weight"], pos_offset=off, **_p3(w))
 
 
-@pytest.mark.parametrize("name", ["video3d", "fp8neox", "fp8neox_nonorm"])
+@pytest.mark.parametrize("name", ["video3d", "fp8neox", "fp8neox_nonorm", "gqa3d"])
 def test_3d_workload_full_size_sampled(name):
     """Full-size workload in the benchmark's launch configuration; the oracle
     checks 48 sampled tokens one by one (grid corners, batch seam, random), and

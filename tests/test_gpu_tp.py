@@ -61,7 +61,7 @@ def _run_simulated(w, T, R, pos_offset=None):
     return total, qkv
 
 
-@pytest.mark.parametrize("name", ["video3d", "fp8neox"])
+@pytest.mark.parametrize("name", ["video3d", "fp8neox", "gqa3d"])
 @pytest.mark.parametrize("R", [1, 2, 3, 4])
 def test_tp_simulated_matches_oracle(name, R):
     w = W.WORKLOADS[name]
