@@ -25,9 +25,10 @@
  *     ABI and nothing is written when the status is not QKNR_OK.
  *     qknr_last_error_detail() names the argument that failed, for this thread.
  *   - num_tokens == 0 is a valid no-op (QKNR_OK, no launch).
- *   - bf16 is IEEE-style bfloat16, E4M3 is the OCP FP8 E4M3FN format (bias 7,
- *     largest finite 448, no infinities); conversions to bf16 round to nearest
- *     even, conversions to E4M3 round to nearest even and saturate to +-448.
+ *   - bf16 is bfloat16 (the upper half of an IEEE binary32), f16 is IEEE
+ *     binary16, E4M3 is the OCP FP8 E4M3FN format (bias 7, largest finite
+ *     448, no infinities); conversions to bf16 and f16 round to nearest even,
+ *     conversions to E4M3 round to nearest even and saturate to +-448.
  *   - All arithmetic is fp32; each output element is rounded once.
  *
  * Thread safety: calls may come from several host threads and streams at once.

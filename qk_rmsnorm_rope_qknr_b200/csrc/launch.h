@@ -43,13 +43,13 @@ struct Rope3DArgs {
 enum { kModeWhole = 0, kModePartialSsq = 1, kModeSuppliedSsq = 2 };
 
 struct RopeTableArgs {
-    const uint8_t* q;  // bf16 [T, hq, D], token stride q_stride elements
+    const uint8_t* q;  // 16-bit activations [T, hq, D], token stride q_stride elements
     const uint8_t* k;
     uint8_t* q_out;
     uint8_t* k_out;
-    const uint8_t* q_weight;  // bf16 [D]
+    const uint8_t* q_weight;  // [D], the activation type
     const uint8_t* k_weight;
-    const uint8_t* table;  // [T, rd] fp32 or bf16
+    const uint8_t* table;  // [T, rd] fp32 or the activation type
     int64_t num_tokens;
     int64_t q_stride, k_stride, q_out_stride, k_out_stride;  // elements
     int32_t hq, hk, head_dim, rotary_dim;
