@@ -338,6 +338,275 @@ __global__ void __launch_bounds__(kBlock)
     }
 }
 
+// Heads per item of the shared-memory kernel: about 4 KB of q/k per item.
+__host__ __device__ inline int smem_item_heads(int D) {
+    const int h = 4096 / (2 * D);
+    return h < 4 ? 4 : (h > 64 ? 64 : h);
+}
+
+// Wait until all but the most recent of this thread's committed bulk stores
+// have read their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_allbut1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+// Any head_dim that is a multiple of 8 (<= 256), any even rotary_dim <=
+// head_dim, either pairing; q/k rows and outputs 16-byte aligned. Like the fast
+// kernel, each warp streams items (heads of one token) through its own ring of
+// shared-memory buffers with bulk copies; unlike it, lanes work on the heads
+// in shared memory, so that any pairing is reachable: lane i takes the channel
+// pairs i, i + 32, ... of a head (adjacent pairs (2p, 2p+1); half split (p,
+// p + rotary_dim/2) for p < rotary_dim/2, then the pass-through channels two
+// by two), writes the results back in place and lane 0 bulk-stores the item's
+// q and k heads. cos/sin come straight from the table in global memory (read
+// before the item's copy is waited for), the weights sit in registers.
+template <bool IL, bool F32, bool H16>
+__global__ void __launch_bounds__(kBlock) rope_table_smem(const RopeTableArgs a) {
+    constexpr int kMaxPairs = 4;  // pairs per lane: head_dim <= 256
+    const int D = a.head_dim, R = a.rotary_dim, half = R / 2;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int H = a.hq + a.hk;
+    const int per_item = smem_item_heads(D);
+    const int cpt = (H + per_item - 1) / per_item;  // items per token
+    const int64_t items = a.num_tokens * cpt;
+    const int stages = a.stages;
+    const int sbytes = per_item * D * 2;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);  // [warps][stages]
+    unsigned char* rings = smem + ((kBlock / 32) * stages * 8 + 127) / 128 * 128;
+    uint64_t* full = bars + warp * stages;
+    unsigned char* ring = rings + (size_t)warp * stages * sbytes;
+
+    const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t n_local = warp_id < items ? (items - 1 - warp_id) / nwarps + 1 : 0;
+    const int64_t dt = nwarps / cpt;
+    const int dchunk = (int)(nwarps - dt * cpt);
+
+    // The lane's channel pairs (fixed for every head) and their table slots.
+    // Adjacent pairs: a head is a group of gs lanes (gs = next power of two of
+    // D/8), lane v of the group holds the 16-byte vector v (pairs 4v..4v+3),
+    // and 32/gs heads are worked on at once. Half split: lane i holds pairs
+    // i, i + 32, ... of one head at a time.
+    int gs = 1;
+    while (gs < D / 8) gs <<= 1;
+    const int v = lane % gs, sub = lane / gs;
+    const bool vact = v < D / 8;
+    int ca[kMaxPairs], cb[kMaxPairs], slot[kMaxPairs];
+    bool rot[kMaxPairs], has[kMaxPairs];
+#pragma unroll
+    for (int m = 0; m < kMaxPairs; ++m) {
+        if (IL) {
+            const int p = 4 * v + m;
+            has[m] = vact;
+            ca[m] = 8 * v + 2 * m;
+            cb[m] = ca[m] + 1;
+            slot[m] = p;
+            rot[m] = vact && p < half;
+        } else {
+            const int p = lane + 32 * m;
+            has[m] = p < D / 2;
+            rot[m] = has[m] && p < half;
+            slot[m] = p;
+            if (p < half) {
+                ca[m] = p;
+                cb[m] = p + half;
+            } else {
+                ca[m] = R + 2 * (p - half);
+                cb[m] = ca[m] + 1;
+            }
+        }
+        if (!has[m]) ca[m] = cb[m] = 0;
+    }
+
+    auto issue = [&](int64_t t, int chunk, int s) {
+        const int h0 = chunk * per_item, h1 = min(h0 + per_item, H);
+        const int q1 = min(h1, a.hq), k0 = max(h0, a.hq);
+        const uint32_t qbytes = h0 < a.hq ? (uint32_t)(q1 - h0) * D * 2 : 0;
+        const uint32_t kbytes = h1 > a.hq ? (uint32_t)(h1 - k0) * D * 2 : 0;
+        unsigned char* dst = ring + (size_t)s * sbytes;
+        mbar_arrive_expect_tx(&full[s], qbytes + kbytes + a.stall_tx_bytes);
+        if (qbytes)
+            bulk_load(dst, a.q + ((size_t)t * a.q_stride + (size_t)h0 * D) * 2, qbytes, &full[s]);
+        if (kbytes)
+            bulk_load(dst + qbytes, a.k + ((size_t)t * a.k_stride + (size_t)(k0 - a.hq) * D) * 2,
+                      kbytes, &full[s]);
+    };
+
+    if (lane == 0) {
+        for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+    float wq[kMaxPairs][2], wk[kMaxPairs][2];
+    {
+        const uint16_t* qw = reinterpret_cast<const uint16_t*>(a.q_weight);
+        const uint16_t* kw = reinterpret_cast<const uint16_t*>(a.k_weight);
+#pragma unroll
+        for (int m = 0; m < kMaxPairs; ++m) {
+            const bool okq = has[m] && a.hq > 0, okk = has[m] && a.hk > 0;
+            wq[m][0] = okq ? act_to_f<H16>(qw[ca[m]]) : 0.0f;
+            wq[m][1] = okq ? act_to_f<H16>(qw[cb[m]]) : 0.0f;
+            wk[m][0] = okk ? act_to_f<H16>(kw[ca[m]]) : 0.0f;
+            wk[m][1] = okk ? act_to_f<H16>(kw[cb[m]]) : 0.0f;
+        }
+    }
+    __syncwarp();
+    int64_t t = warp_id / cpt;
+    int chunk = (int)(warp_id - t * cpt);
+    if (lane == 0) {
+        int64_t tt = t;
+        int cc = chunk;
+        for (int s = 0; s < stages && s < n_local; ++s) {
+            issue(tt, cc, s);
+            tt += dt;
+            cc += dchunk;
+            if (cc >= cpt) { cc -= cpt; ++tt; }
+        }
+    }
+    // the next item to copy in: `stages` after the first (refills run one item
+    // behind, so after item i the copy of item i - 1 + stages is issued)
+    int64_t t_ahead = t, chunk_ahead = chunk;
+    for (int s = 0; s < stages; ++s) {
+        t_ahead += dt;
+        chunk_ahead += dchunk;
+        if (chunk_ahead >= cpt) { chunk_ahead -= cpt; ++t_ahead; }
+    }
+    const float inv_d = 1.0f / (float)D;
+
+    int stage = 0, prev_stage = stages - 1;
+    uint32_t phase = 0;
+    int64_t i = 0;
+    bool aborted = false;
+    for (; i < n_local; ++i) {
+        // This token's cos/sin for the lane's rotated pairs, before the wait.
+        float c[kMaxPairs], s[kMaxPairs];
+#pragma unroll
+        for (int m = 0; m < kMaxPairs; ++m) {
+            c[m] = 1.0f;
+            s[m] = 0.0f;
+            if (rot[m]) {
+                const int j = slot[m];
+                if (F32) {
+                    const float* tr = reinterpret_cast<const float*>(a.table) + (size_t)t * R;
+                    c[m] = __ldg(tr + j);
+                    s[m] = __ldg(tr + half + j);
+                } else {
+                    const uint16_t* tr = reinterpret_cast<const uint16_t*>(a.table) + (size_t)t * R;
+                    c[m] = act_to_f<H16>(__ldg(tr + j));
+                    s[m] = act_to_f<H16>(__ldg(tr + half + j));
+                }
+            }
+        }
+        const bool ok = mbar_wait_bounded(&full[stage], phase, a.wait_limit_ns);
+        if (__any_sync(0xffffffffu, !ok)) {
+            aborted = true;
+            break;
+        }
+        unsigned char* buf = ring + (size_t)stage * sbytes;
+        const int h0 = chunk * per_item, h1 = min(h0 + per_item, H);
+        if constexpr (IL) {
+            for (int hb = h0; hb < h1; hb += 32 / gs) {  // the same trip count in every lane
+                const int hh = hb + sub;
+                const bool okh = vact && hh < h1;
+                uint4 xv = make_uint4(0, 0, 0, 0);
+                uint4* px = reinterpret_cast<uint4*>(buf) + (size_t)(hh - h0) * (D / 8) + v;
+                if (okh) xv = *px;
+                const uint32_t w32[4] = {xv.x, xv.y, xv.z, xv.w};
+                float2 f[4];
+                float ss = 0.0f;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    f[m] = act2_to_f2<H16>(w32[m]);
+                    ss = fmaf(f[m].x, f[m].x, fmaf(f[m].y, f[m].y, ss));
+                }
+                for (int o = gs >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                if (okh) {
+                    const float r = rsqrtf(ss * inv_d + a.eps);
+                    const bool isk = hh >= a.hq;
+                    uint32_t o32[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float ya = f[m].x * r * (isk ? wk[m][0] : wq[m][0]);
+                        const float yb = f[m].y * r * (isk ? wk[m][1] : wq[m][1]);
+                        o32[m] = f2_to_act2<H16>(make_float2(ya * c[m] - yb * s[m],
+                                                             yb * c[m] + ya * s[m]));
+                    }
+                    *px = make_uint4(o32[0], o32[1], o32[2], o32[3]);
+                }
+            }
+        } else {
+            for (int hh = h0; hh < h1; ++hh) {
+                uint16_t* x = reinterpret_cast<uint16_t*>(buf + (size_t)(hh - h0) * D * 2);
+                const bool isk = hh >= a.hq;
+                float xa[kMaxPairs], xb[kMaxPairs];
+                float ss = 0.0f;
+#pragma unroll
+                for (int m = 0; m < kMaxPairs; ++m) {
+                    xa[m] = has[m] ? act_to_f<H16>(x[ca[m]]) : 0.0f;
+                    xb[m] = has[m] ? act_to_f<H16>(x[cb[m]]) : 0.0f;
+                    ss = fmaf(xa[m], xa[m], ss);
+                    ss = fmaf(xb[m], xb[m], ss);
+                }
+                const float r = rsqrtf(warp_sum(ss) * inv_d + a.eps);
+#pragma unroll
+                for (int m = 0; m < kMaxPairs; ++m) {
+                    if (!has[m]) continue;
+                    const float ya = xa[m] * r * (isk ? wk[m][0] : wq[m][0]);
+                    const float yb = xb[m] * r * (isk ? wk[m][1] : wq[m][1]);
+                    x[ca[m]] = f_to_act<H16>(ya * c[m] - yb * s[m]);
+                    x[cb[m]] = f_to_act<H16>(yb * c[m] + ya * s[m]);
+                }
+            }
+        }
+        fence_proxy_async_smem();  // each lane's writes, before the bulk engine reads them
+        __syncwarp();
+        if (lane == 0) {
+            // The item's results leave by bulk stores; the buffer of the
+            // previous item (whose stores were issued one item ago) is refilled.
+            const int q1 = min(h1, a.hq), k0 = max(h0, a.hq);
+            const uint32_t qbytes = h0 < a.hq ? (uint32_t)(q1 - h0) * D * 2 : 0;
+            const uint32_t kbytes = h1 > a.hq ? (uint32_t)(h1 - k0) * D * 2 : 0;
+            if (qbytes)
+                bulk_store(a.q_out + ((size_t)t * a.q_out_stride + (size_t)h0 * D) * 2, buf, qbytes);
+            if (kbytes)
+                bulk_store(a.k_out + ((size_t)t * a.k_out_stride + (size_t)(k0 - a.hq) * D) * 2,
+                           buf + qbytes, kbytes);
+            bulk_commit();
+            if (i >= 1 && i - 1 + stages < n_local) {
+                bulk_wait_read_allbut1();
+                issue(t_ahead, (int)chunk_ahead, prev_stage);
+            }
+        }
+        if (i >= 1) {
+            t_ahead += dt;
+            chunk_ahead += dchunk;
+            if (chunk_ahead >= cpt) { chunk_ahead -= cpt; ++t_ahead; }
+        }
+        t += dt;
+        chunk += dchunk;
+        if (chunk >= cpt) { chunk -= cpt; ++t; }
+        prev_stage = stage;
+        if (++stage == stages) {
+            stage = 0;
+            phase ^= 1u;
+        }
+    }
+    if (lane == 0) {
+        if (aborted) {
+            atomicOr(&g_table_status, 1u);
+            // Copies that may be in flight (bounded): items i .. i+stages-2, or
+            // the whole first ring if none was consumed.
+            const int64_t hi = i == 0 ? stages : i + stages - 1;
+            for (int64_t j = i; j < n_local && j < hi; ++j)
+                mbar_wait_bounded(&full[j % stages], (uint32_t)((j / stages) & 1), a.wait_limit_ns);
+        }
+        bulk_wait_all();
+    }
+}
+
 // One warp per head; any head_dim <= 256, any even rotary_dim <= head_dim,
 // 2-byte alignment. The normalised head goes through shared memory so that
 // every lane can read its partner channel.
@@ -565,6 +834,65 @@ cudaError_t launch_bulk(K kern, const RopeTableArgs& a0, int per_item, cudaStrea
     return e;
 }
 
+template <typename K>
+cudaError_t launch_smem(K kern, const RopeTableArgs& a0, cudaStream_t stream, LaunchInfo* info,
+                        int id) {
+    RopeTableArgs a = a0;
+    const int sbytes = smem_item_heads(a.head_dim) * a.head_dim * 2;
+    const int warps = kBlock / 32;
+    // Two CTAs per SM, each warp with as many ring buffers (2..4) as fit.
+    const int fixed = 128 + warps * 4 * 8;
+    a.stages = std::max(2, std::min(4, (227 * 1024 / 2 - 1024 - fixed) / (warps * sbytes)));
+    if (a.wait_limit_ns == 0) a.wait_limit_ns = 2000000000ull;  // 2 s
+    const int smem = ((warps * a.stages * 8 + 127) / 128 * 128) + warps * a.stages * sbytes;
+    int sms = 0, per_sm = 0;
+    cudaError_t e = cached_sm_count(&sms);
+    if (e == cudaSuccess)
+        e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), kBlock, smem, &per_sm);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int per_item = smem_item_heads(a.head_dim);
+    const int64_t items = a.num_tokens * ((a.hq + a.hk + per_item - 1) / per_item);
+    const int grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>((int64_t)sms * per_sm, (items + warps - 1) / warps));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kBlock);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        forget_kernel(reinterpret_cast<const void*>(kern));
+        e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), kBlock, smem, &per_sm);
+        if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, kern, a);
+    }
+    if (info) {
+        info->grid = grid;
+        info->block = kBlock;
+        info->smem = smem;
+        info->kernel_id = id;
+    }
+    return e;
+}
+
+// Whether the shared-memory kernel takes these arguments: head_dim a multiple
+// of 8 and every q/k row (input and output) on a 16-byte boundary.
+bool smem_path_ok(const RopeTableArgs& a) {
+    auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (a.head_dim % 8 != 0 || a.head_dim > 256) return false;
+    if (a.hq > 0 && !(al(a.q) && al(a.q_out) && a.q_stride % 8 == 0 && a.q_out_stride % 8 == 0))
+        return false;
+    if (a.hk > 0 && !(al(a.k) && al(a.k_out) && a.k_stride % 8 == 0 && a.k_out_stride % 8 == 0))
+        return false;
+    return true;
+}
+
 template <int GS, bool H16>
 cudaError_t run_fast_act(const RopeTableArgs& a, cudaStream_t stream, LaunchInfo* info) {
     const int per_item = kUnroll * (32 / GS);
@@ -597,6 +925,23 @@ cudaError_t launch_rope_table(const RopeTableArgs& a, int fast_path, cudaStream_
         if (L <= 4) return run_fast<4>(a, stream, info);
         if (L <= 8) return run_fast<8>(a, stream, info);
         return run_fast<16>(a, stream, info);
+    }
+    if (smem_path_ok(a)) {
+        const int id = 2100 + (a.interleaved ? 100 : 0) + (a.act_f16 ? 10 : 0) + (a.table_f32 ? 1 : 0);
+        if (a.interleaved) {
+            if (a.act_f16) {
+                return a.table_f32 ? launch_smem(rope_table_smem<true, true, true>, a, stream, info, id)
+                                   : launch_smem(rope_table_smem<true, false, true>, a, stream, info, id);
+            }
+            return a.table_f32 ? launch_smem(rope_table_smem<true, true, false>, a, stream, info, id)
+                               : launch_smem(rope_table_smem<true, false, false>, a, stream, info, id);
+        }
+        if (a.act_f16) {
+            return a.table_f32 ? launch_smem(rope_table_smem<false, true, true>, a, stream, info, id)
+                               : launch_smem(rope_table_smem<false, false, true>, a, stream, info, id);
+        }
+        return a.table_f32 ? launch_smem(rope_table_smem<false, true, false>, a, stream, info, id)
+                           : launch_smem(rope_table_smem<false, false, false>, a, stream, info, id);
     }
     const int64_t groups = a.num_tokens * (a.hq + a.hk);
     const int64_t blocks = (groups + kBlock / 32 - 1) / (kBlock / 32);

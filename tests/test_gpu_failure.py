@@ -52,14 +52,27 @@ def test_wait_timeout_raises_status_and_context_survives():
     assert Q.qknr_device_status() == 0
 
 
-def test_table_wait_timeout_raises_status_and_context_survives():
-    w = W.WORKLOADS["table_hs"]
-    inp = {k: v.cuda() for k, v in W.make_inputs(w, tokens=64).items()}
+def _table_inputs(shape):
+    if shape == "table_hs":  # the fast (register) kernel
+        w = W.WORKLOADS["table_hs"]
+        inp = {k: v.cuda() for k, v in W.make_inputs(w, tokens=64).items()}
+        return inp, w.rotary_dim, w.interleaved
+    # head_dim 72, rotary_dim 40: the shared-memory kernel
+    g = torch.Generator(device="cpu").manual_seed(3)
+    inp = dict(q=torch.randn(64, 6, 72, generator=g), k=torch.randn(64, 2, 72, generator=g),
+               q_weight=torch.ones(72), k_weight=torch.ones(72))
+    inp = {k: v.to(torch.bfloat16).cuda() for k, v in inp.items()}
+    inp["rope_table"] = W.rope_table_input(64, 40, 10000.0, True, "cuda")
+    return inp, 40, True
+
+
+@pytest.mark.parametrize("shape", ["table_hs", "d72_r40"])
+def test_table_wait_timeout_raises_status_and_context_survives(shape):
+    inp, R, il = _table_inputs(shape)
 
     def call(qo, ko):
         Q.qknr_rope_table(inp["q"], inp["k"], qo, ko, inp["q_weight"], inp["k_weight"],
-                          inp["rope_table"], eps=w.eps, rotary_dim=w.rotary_dim,
-                          interleaved=w.interleaved)
+                          inp["rope_table"], eps=1e-6, rotary_dim=R, interleaved=il)
 
     good = [torch.empty_like(inp["q"]), torch.empty_like(inp["k"])]
     call(*good)

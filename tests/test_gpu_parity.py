@@ -357,6 +357,28 @@ def test_table_strided_inplace_and_misaligned(act):
         assert torch.all(packed[:, 2 * H:] == 0)
 
 
+@pytest.mark.parametrize("act", [torch.bfloat16, torch.float16], ids=["bf16", "f16"])
+@pytest.mark.parametrize("il,R", [(True, 36), (False, 40), (False, 72)])
+def test_table_smem_path_strided_inplace(act, il, R):
+    """head_dim 72 (not a multiple of 16) with 16-byte aligned rows takes the
+    shared-memory kernel: q and k as views into a packed buffer (token stride
+    3*H*D), updated in place, over enough tokens that each warp's ring turns
+    over several times."""
+    T, H, D = 12000, 5, 72  # about 5 items per warp: the rings turn over
+    inp = _rand_table_inputs(T, H, H, D, R, True, seed=R, act=act)
+    buf = torch.zeros(T * 3 * H * D, dtype=act, device=DEV)
+    packed = buf.view(T, 3 * H, D)
+    packed[:, :H] = inp["q"].to(DEV)
+    packed[:, H:2 * H] = inp["k"].to(DEV)
+    q, k = packed[:, :H], packed[:, H:2 * H]
+    g = {n: inp[n].to(DEV) for n in ("q_weight", "k_weight", "rope_table")}
+    Q.fused_qk_norm_rope(q, k, g["q_weight"], g["k_weight"], g["rope_table"], 1e-6,
+                         rotary_dim=R, interleaved=il, q_out=q, k_out=k)
+    torch.cuda.synchronize()
+    check_table_against_oracle(inp, q.cpu(), k.cpu(), 1e-6, R, il, f"smem {act} {il} {R}")
+    assert torch.all(packed[:, 2 * H:] == 0)
+
+
 def test_table_outputs_written_exactly():
     T, Hq, Hk, D, R = 33, 3, 2, 128, 128
     inp = _rand_table_inputs(T, Hq, Hk, D, R, False, seed=9)
