@@ -236,6 +236,24 @@ def test_3d_pinned_host_buffers():
         assert torch.equal(a.cpu(), b)
 
 
+@pytest.mark.parametrize("D,R,il", [(128, 96, False), (72, 40, True)], ids=["fast", "smem"])
+def test_table_pinned_host_buffers(D, R, il):
+    """The table form on page-locked host q, k, table and outputs (the kernels'
+    bulk copies and table loads cross the bus): the same bits as on device
+    buffers, for the fast kernel and the shared-memory kernel."""
+    inp = _rand_table_inputs(256, 6, 2, D, R, True, seed=D)
+    g = {n: t.to(DEV) for n, t in inp.items()}
+    dq, dk = Q.fused_qk_norm_rope(g["q"], g["k"], g["q_weight"], g["k_weight"], g["rope_table"],
+                                  1e-6, rotary_dim=R, interleaved=il)
+    h = {n: inp[n].pin_memory() for n in ("q", "k", "rope_table")}
+    hq, hk = torch.empty_like(h["q"]).pin_memory(), torch.empty_like(h["k"]).pin_memory()
+    Q.qknr_rope_table(h["q"], h["k"], hq, hk, g["q_weight"], g["k_weight"], h["rope_table"],
+                      eps=1e-6, rotary_dim=R, interleaved=il,
+                      stream=torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert torch.equal(dq.cpu(), hq) and torch.equal(dk.cpu(), hk)
+
+
 def test_3d_pageable_host_memory_is_rejected():
     qkv, qw, kw = _rand3d(16, 4, 4, 4, 64)
     p = dict(ppf=1, pph=4, ppw=4, num_frame_channels=16, num_height_channels=24,
