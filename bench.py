@@ -302,6 +302,8 @@ def run_gpu(args, w):
     odt = torch.float8_e4m3fn if w.output_fp8 else torch.bfloat16
     outs = [torch.empty(T, h, w.head_dim, dtype=odt, device=dev) for h in (w.hq, w.hk, w.hv)]
     p = w.params()
+    if getattr(args, "tokens", None):
+        p["pos_offset"] = 0  # a sequence shard of the workload: any token count
     qkv, qw, kw = inp["qkv"], inp["q_weight"], inp["k_weight"]
     stream = torch.cuda.current_stream(dev)
 
@@ -570,7 +572,7 @@ def measure_e2e_table(args, w, dset, run, stream, dev, world, pg):
 
 def measure_e2e(args, w, qkv, qw, kw, outs, p, stream, dev, world, pg):
     """End to end through the C ABI with the step's input and outputs in
-    page-locked host memory. Two ways, both timed, the faster reported:
+    page-locked host memory. Three ways, all timed, the fastest reported:
       staged:    copy the input host -> device, run, copy the outputs back;
       zero-copy: hand the host buffers to qknr_rope_3d itself; the kernel's
                  bulk copies read the input across the bus and its stores
@@ -678,12 +680,23 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="run the workload's geometry on this many tokens instead (3D: a "
+                         "sequence shard from position 0); for profiling smaller cases")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from qk_rmsnorm_rope_qknr_b200 import workloads as W
 
     w = W.WORKLOADS[args.workload]
+    if args.tokens:
+        import dataclasses
+
+        if w.form == "3d":
+            w = dataclasses.replace(w, name=f"{w.name}[{args.tokens}]", batch=1, seq=args.tokens,
+                                    input_2d=True)
+        else:
+            w = dataclasses.replace(w, name=f"{w.name}[{args.tokens}]", tokens=args.tokens)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w) if w.form == "3d" else run_gpu_table(args, w)
