@@ -350,17 +350,17 @@ __device__ __forceinline__ void bulk_wait_read_allbut1() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
-// Any head_dim that is a multiple of 8 (<= 256), any even rotary_dim <=
-// head_dim, either pairing; q/k rows and outputs 16-byte aligned. Like the fast
+// Half-split pairs, any head_dim that is a multiple of 8 (<= 256), any even
+// rotary_dim <= head_dim; q/k rows and outputs 16-byte aligned. Like the fast
 // kernel, each warp streams items (heads of one token) through its own ring of
 // shared-memory buffers with bulk copies; unlike it, lanes work on the heads
 // in shared memory, so that any pairing is reachable: lane i takes the channel
-// pairs i, i + 32, ... of a head (adjacent pairs (2p, 2p+1); half split (p,
-// p + rotary_dim/2) for p < rotary_dim/2, then the pass-through channels two
-// by two), writes the results back in place and lane 0 bulk-stores the item's
+// pairs i, i + 32, ... of a head ((p, p + rotary_dim/2) for p < rotary_dim/2,
+// then the pass-through channels two by two), writes the results back in
+// place and lane 0 bulk-stores the item's
 // q and k heads. cos/sin come straight from the table in global memory (read
 // before the item's copy is waited for), the weights sit in registers.
-template <bool IL, bool F32, bool H16>
+template <bool F32, bool H16>
 __global__ void __launch_bounds__(kBlock) rope_table_smem(const RopeTableArgs a) {
     constexpr int kMaxPairs = 4;  // pairs per lane: head_dim <= 256
     const int D = a.head_dim, R = a.rotary_dim, half = R / 2;
@@ -384,38 +384,22 @@ __global__ void __launch_bounds__(kBlock) rope_table_smem(const RopeTableArgs a)
     const int64_t dt = nwarps / cpt;
     const int dchunk = (int)(nwarps - dt * cpt);
 
-    // The lane's channel pairs (fixed for every head) and their table slots.
-    // Adjacent pairs: a head is a group of gs lanes (gs = next power of two of
-    // D/8), lane v of the group holds the 16-byte vector v (pairs 4v..4v+3),
-    // and 32/gs heads are worked on at once. Half split: lane i holds pairs
-    // i, i + 32, ... of one head at a time.
-    int gs = 1;
-    while (gs < D / 8) gs <<= 1;
-    const int v = lane % gs, sub = lane / gs;
-    const bool vact = v < D / 8;
+    // The lane's channel pairs (fixed for every head) and their table slots:
+    // pairs i, i + 32, ... of one head at a time.
     int ca[kMaxPairs], cb[kMaxPairs], slot[kMaxPairs];
     bool rot[kMaxPairs], has[kMaxPairs];
 #pragma unroll
     for (int m = 0; m < kMaxPairs; ++m) {
-        if (IL) {
-            const int p = 4 * v + m;
-            has[m] = vact;
-            ca[m] = 8 * v + 2 * m;
-            cb[m] = ca[m] + 1;
-            slot[m] = p;
-            rot[m] = vact && p < half;
+        const int p = lane + 32 * m;
+        has[m] = p < D / 2;
+        rot[m] = has[m] && p < half;
+        slot[m] = p;
+        if (p < half) {
+            ca[m] = p;
+            cb[m] = p + half;
         } else {
-            const int p = lane + 32 * m;
-            has[m] = p < D / 2;
-            rot[m] = has[m] && p < half;
-            slot[m] = p;
-            if (p < half) {
-                ca[m] = p;
-                cb[m] = p + half;
-            } else {
-                ca[m] = R + 2 * (p - half);
-                cb[m] = ca[m] + 1;
-            }
+            ca[m] = R + 2 * (p - half);
+            cb[m] = ca[m] + 1;
         }
         if (!has[m]) ca[m] = cb[m] = 0;
     }
@@ -507,58 +491,26 @@ __global__ void __launch_bounds__(kBlock) rope_table_smem(const RopeTableArgs a)
         }
         unsigned char* buf = ring + (size_t)stage * sbytes;
         const int h0 = chunk * per_item, h1 = min(h0 + per_item, H);
-        if constexpr (IL) {
-            for (int hb = h0; hb < h1; hb += 32 / gs) {  // the same trip count in every lane
-                const int hh = hb + sub;
-                const bool okh = vact && hh < h1;
-                uint4 xv = make_uint4(0, 0, 0, 0);
-                uint4* px = reinterpret_cast<uint4*>(buf) + (size_t)(hh - h0) * (D / 8) + v;
-                if (okh) xv = *px;
-                const uint32_t w32[4] = {xv.x, xv.y, xv.z, xv.w};
-                float2 f[4];
-                float ss = 0.0f;
+        for (int hh = h0; hh < h1; ++hh) {
+            uint16_t* x = reinterpret_cast<uint16_t*>(buf + (size_t)(hh - h0) * D * 2);
+            const bool isk = hh >= a.hq;
+            float xa[kMaxPairs], xb[kMaxPairs];
+            float ss = 0.0f;
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    f[m] = act2_to_f2<H16>(w32[m]);
-                    ss = fmaf(f[m].x, f[m].x, fmaf(f[m].y, f[m].y, ss));
-                }
-                for (int o = gs >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                if (okh) {
-                    const float r = rsqrtf(ss * inv_d + a.eps);
-                    const bool isk = hh >= a.hq;
-                    uint32_t o32[4];
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const float ya = f[m].x * r * (isk ? wk[m][0] : wq[m][0]);
-                        const float yb = f[m].y * r * (isk ? wk[m][1] : wq[m][1]);
-                        o32[m] = f2_to_act2<H16>(make_float2(ya * c[m] - yb * s[m],
-                                                             yb * c[m] + ya * s[m]));
-                    }
-                    *px = make_uint4(o32[0], o32[1], o32[2], o32[3]);
-                }
+            for (int m = 0; m < kMaxPairs; ++m) {
+                xa[m] = has[m] ? act_to_f<H16>(x[ca[m]]) : 0.0f;
+                xb[m] = has[m] ? act_to_f<H16>(x[cb[m]]) : 0.0f;
+                ss = fmaf(xa[m], xa[m], ss);
+                ss = fmaf(xb[m], xb[m], ss);
             }
-        } else {
-            for (int hh = h0; hh < h1; ++hh) {
-                uint16_t* x = reinterpret_cast<uint16_t*>(buf + (size_t)(hh - h0) * D * 2);
-                const bool isk = hh >= a.hq;
-                float xa[kMaxPairs], xb[kMaxPairs];
-                float ss = 0.0f;
+            const float r = rsqrtf(warp_sum(ss) * inv_d + a.eps);
 #pragma unroll
-                for (int m = 0; m < kMaxPairs; ++m) {
-                    xa[m] = has[m] ? act_to_f<H16>(x[ca[m]]) : 0.0f;
-                    xb[m] = has[m] ? act_to_f<H16>(x[cb[m]]) : 0.0f;
-                    ss = fmaf(xa[m], xa[m], ss);
-                    ss = fmaf(xb[m], xb[m], ss);
-                }
-                const float r = rsqrtf(warp_sum(ss) * inv_d + a.eps);
-#pragma unroll
-                for (int m = 0; m < kMaxPairs; ++m) {
-                    if (!has[m]) continue;
-                    const float ya = xa[m] * r * (isk ? wk[m][0] : wq[m][0]);
-                    const float yb = xb[m] * r * (isk ? wk[m][1] : wq[m][1]);
-                    x[ca[m]] = f_to_act<H16>(ya * c[m] - yb * s[m]);
-                    x[cb[m]] = f_to_act<H16>(yb * c[m] + ya * s[m]);
-                }
+            for (int m = 0; m < kMaxPairs; ++m) {
+                if (!has[m]) continue;
+                const float ya = xa[m] * r * (isk ? wk[m][0] : wq[m][0]);
+                const float yb = xb[m] * r * (isk ? wk[m][1] : wq[m][1]);
+                x[ca[m]] = f_to_act<H16>(ya * c[m] - yb * s[m]);
+                x[cb[m]] = f_to_act<H16>(yb * c[m] + ya * s[m]);
             }
         }
         fence_proxy_async_smem();  // each lane's writes, before the bulk engine reads them
@@ -599,6 +551,247 @@ __global__ void __launch_bounds__(kBlock) rope_table_smem(const RopeTableArgs a)
             atomicOr(&g_table_status, 1u);
             // Copies that may be in flight (bounded): items i .. i+stages-2, or
             // the whole first ring if none was consumed.
+            const int64_t hi = i == 0 ? stages : i + stages - 1;
+            for (int64_t j = i; j < n_local && j < hi; ++j)
+                mbar_wait_bounded(&full[j % stages], (uint32_t)((j / stages) & 1), a.wait_limit_ns);
+        }
+        bulk_wait_all();
+    }
+}
+
+// Lanes per head (gs) and 16-byte vectors per lane (mv <= 4) for adjacent
+// pairs in shared memory: the split of a head's D/8 vectors that leaves the
+// fewest lanes idle (then the fewest vectors per lane).
+__host__ __device__ inline void il_lane_split(int D, int* gs, int* mv) {
+    const int vph = D / 8;
+    int best = 1 << 30;
+    for (int g = 1; g <= 32; g <<= 1) {
+        const int m = (vph + g - 1) / g;
+        if (m > 4) continue;
+        const int key = (g * m - vph) * 8 + m;
+        if (key < best) {
+            best = key;
+            *gs = g;
+            *mv = m;
+        }
+    }
+}
+
+// Shared-memory bytes ahead of the rings of rope_table_smem_il: mbarriers,
+// fp32 weights [q | k][256], and per warp the item's cos/sin [2][128] fp32.
+__host__ __device__ inline int smem_il_fixed_bytes(int stages) {
+    return ((kBlock / 32) * stages * 8 + 127) / 128 * 128 + 2 * 256 * 4 + (kBlock / 32) * 2 * 128 * 4;
+}
+
+// Adjacent pairs, any head_dim that is a multiple of 8 (<= 256) and any even
+// rotary_dim, q/k rows and outputs 16-byte aligned. The ring of bulk copies,
+// the in-place results and the bulk stores are those of rope_table_smem; the
+// work split differs: a head is a group of gs lanes and lane l of the group
+// holds the 16-byte vectors l, l + gs, ... (mv of them, il_lane_split), so
+// that 32/gs heads move per step with few idle lanes (head_dim 72: 4 lanes of
+// 3 vectors, 8 heads per step). Weights sit in shared memory as fp32; an
+// item's cos/sin are read from the table once per warp (before the item's
+// copy is waited for) and staged in shared memory, where lanes of the same
+// position read the same words.
+template <bool F32, bool H16>
+__global__ void __launch_bounds__(kBlock) rope_table_smem_il(const RopeTableArgs a) {
+    const int D = a.head_dim, R = a.rotary_dim, half = R / 2;
+    const int vph = D / 8;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int H = a.hq + a.hk;
+    const int per_item = smem_item_heads(D);
+    const int cpt = (H + per_item - 1) / per_item;  // items per token
+    const int64_t items = a.num_tokens * cpt;
+    const int stages = a.stages;
+    const int sbytes = per_item * D * 2;
+    int gs = 32, mv = 1;
+    il_lane_split(D, &gs, &mv);
+    const int l = lane % gs, sub = lane / gs, hps = 32 / gs;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);  // [warps][stages]
+    float* wsm = reinterpret_cast<float*>(smem + ((kBlock / 32) * stages * 8 + 127) / 128 * 128);
+    float* csm = wsm + 2 * 256 + warp * 2 * 128;  // this warp's [cos | sin] of the item
+    unsigned char* rings = smem + smem_il_fixed_bytes(stages);
+    uint64_t* full = bars + warp * stages;
+    unsigned char* ring = rings + (size_t)warp * stages * sbytes;
+
+    const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t n_local = warp_id < items ? (items - 1 - warp_id) / nwarps + 1 : 0;
+    const int64_t dt = nwarps / cpt;
+    const int dchunk = (int)(nwarps - dt * cpt);
+
+    auto issue = [&](int64_t t, int chunk, int s) {
+        const int h0 = chunk * per_item, h1 = min(h0 + per_item, H);
+        const int q1 = min(h1, a.hq), k0 = max(h0, a.hq);
+        const uint32_t qbytes = h0 < a.hq ? (uint32_t)(q1 - h0) * D * 2 : 0;
+        const uint32_t kbytes = h1 > a.hq ? (uint32_t)(h1 - k0) * D * 2 : 0;
+        unsigned char* dst = ring + (size_t)s * sbytes;
+        mbar_arrive_expect_tx(&full[s], qbytes + kbytes + a.stall_tx_bytes);
+        if (qbytes)
+            bulk_load(dst, a.q + ((size_t)t * a.q_stride + (size_t)h0 * D) * 2, qbytes, &full[s]);
+        if (kbytes)
+            bulk_load(dst + qbytes, a.k + ((size_t)t * a.k_stride + (size_t)(k0 - a.hq) * D) * 2,
+                      kbytes, &full[s]);
+    };
+
+    if (lane == 0) {
+        for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+    for (int c = threadIdx.x; c < 2 * 256; c += blockDim.x) {
+        const bool isk = c >= 256;
+        const int cc = isk ? c - 256 : c;
+        const uint16_t* w = reinterpret_cast<const uint16_t*>(isk ? a.k_weight : a.q_weight);
+        wsm[c] = (cc < D && (isk ? a.hk : a.hq) > 0) ? act_to_f<H16>(w[cc]) : 0.0f;
+    }
+    int64_t t = warp_id / cpt;
+    int chunk = (int)(warp_id - t * cpt);
+    if (lane == 0) {
+        int64_t tt = t;
+        int cc = chunk;
+        for (int s = 0; s < stages && s < n_local; ++s) {
+            issue(tt, cc, s);
+            tt += dt;
+            cc += dchunk;
+            if (cc >= cpt) { cc -= cpt; ++tt; }
+        }
+    }
+    __syncthreads();  // weights
+    // the next item to copy in (refills run one item behind)
+    int64_t t_ahead = t, chunk_ahead = chunk;
+    for (int s = 0; s < stages; ++s) {
+        t_ahead += dt;
+        chunk_ahead += dchunk;
+        if (chunk_ahead >= cpt) { chunk_ahead -= cpt; ++t_ahead; }
+    }
+    const float inv_d = 1.0f / (float)D;
+
+    int stage = 0, prev_stage = stages - 1;
+    uint32_t phase = 0;
+    int64_t i = 0;
+    bool aborted = false;
+    for (; i < n_local; ++i) {
+        // This token's cos/sin, slots lane, lane + 32, ..., read before the wait.
+        float cr[4], sr[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = lane + 32 * u;
+            cr[u] = 1.0f;
+            sr[u] = 0.0f;
+            if (j < half) {
+                if (F32) {
+                    const float* tr = reinterpret_cast<const float*>(a.table) + (size_t)t * R;
+                    cr[u] = __ldg(tr + j);
+                    sr[u] = __ldg(tr + half + j);
+                } else {
+                    const uint16_t* tr = reinterpret_cast<const uint16_t*>(a.table) + (size_t)t * R;
+                    cr[u] = act_to_f<H16>(__ldg(tr + j));
+                    sr[u] = act_to_f<H16>(__ldg(tr + half + j));
+                }
+            }
+        }
+        const bool ok = mbar_wait_bounded(&full[stage], phase, a.wait_limit_ns);
+        if (__any_sync(0xffffffffu, !ok)) {
+            aborted = true;
+            break;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = lane + 32 * u;
+            if (j < half) {
+                csm[j] = cr[u];
+                csm[128 + j] = sr[u];
+            }
+        }
+        __syncwarp();
+        unsigned char* buf = ring + (size_t)stage * sbytes;
+        const int h0 = chunk * per_item, h1 = min(h0 + per_item, H);
+        for (int hb = h0; hb < h1; hb += hps) {  // the same trip count in every lane
+            const int hh = hb + sub;
+            const bool okh = hh < h1;
+            uint4* head = reinterpret_cast<uint4*>(buf) + (size_t)(hh - h0) * vph;
+            float2 f[4][4];
+            float ss = 0.0f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int vv = l + gs * m;
+                uint4 xv = make_uint4(0, 0, 0, 0);
+                if (m < mv && okh && vv < vph) xv = head[vv];
+                f[m][0] = act2_to_f2<H16>(xv.x);
+                f[m][1] = act2_to_f2<H16>(xv.y);
+                f[m][2] = act2_to_f2<H16>(xv.z);
+                f[m][3] = act2_to_f2<H16>(xv.w);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) ss = fmaf(f[m][k].x, f[m][k].x, fmaf(f[m][k].y, f[m][k].y, ss));
+            }
+            for (int o = gs >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            if (!okh) continue;
+            const float r = rsqrtf(ss * inv_d + a.eps);
+            const float* wrow = wsm + (hh >= a.hq ? 256 : 0);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int vv = l + gs * m;
+                if (m >= mv || vv >= vph) continue;
+                const float4 w0 = reinterpret_cast<const float4*>(wrow)[2 * vv];
+                const float4 w1 = reinterpret_cast<const float4*>(wrow)[2 * vv + 1];
+                const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                float4 c4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f), s4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (4 * vv < half) {
+                    c4 = reinterpret_cast<const float4*>(csm)[vv];
+                    s4 = reinterpret_cast<const float4*>(csm + 128)[vv];
+                }
+                const float cv[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
+                uint32_t o32[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const bool rk = 4 * vv + k < half;
+                    const float ya = f[m][k].x * r * wv[2 * k], yb = f[m][k].y * r * wv[2 * k + 1];
+                    const float c = rk ? cv[k] : 1.0f, s = rk ? sv[k] : 0.0f;
+                    o32[k] = f2_to_act2<H16>(make_float2(ya * c - yb * s, yb * c + ya * s));
+                }
+                head[vv] = make_uint4(o32[0], o32[1], o32[2], o32[3]);
+            }
+        }
+        fence_proxy_async_smem();  // each lane's writes, before the bulk engine reads them
+        __syncwarp();
+        if (lane == 0) {
+            // The item's results leave by bulk stores; the buffer of the
+            // previous item (whose stores were issued one item ago) is refilled.
+            const int q1 = min(h1, a.hq), k0 = max(h0, a.hq);
+            const uint32_t qbytes = h0 < a.hq ? (uint32_t)(q1 - h0) * D * 2 : 0;
+            const uint32_t kbytes = h1 > a.hq ? (uint32_t)(h1 - k0) * D * 2 : 0;
+            if (qbytes)
+                bulk_store(a.q_out + ((size_t)t * a.q_out_stride + (size_t)h0 * D) * 2, buf, qbytes);
+            if (kbytes)
+                bulk_store(a.k_out + ((size_t)t * a.k_out_stride + (size_t)(k0 - a.hq) * D) * 2,
+                           buf + qbytes, kbytes);
+            bulk_commit();
+            if (i >= 1 && i - 1 + stages < n_local) {
+                bulk_wait_read_allbut1();
+                issue(t_ahead, (int)chunk_ahead, prev_stage);
+            }
+        }
+        if (i >= 1) {
+            t_ahead += dt;
+            chunk_ahead += dchunk;
+            if (chunk_ahead >= cpt) { chunk_ahead -= cpt; ++t_ahead; }
+        }
+        t += dt;
+        chunk += dchunk;
+        if (chunk >= cpt) { chunk -= cpt; ++t; }
+        prev_stage = stage;
+        if (++stage == stages) {
+            stage = 0;
+            phase ^= 1u;
+        }
+    }
+    if (lane == 0) {
+        if (aborted) {
+            atomicOr(&g_table_status, 1u);
             const int64_t hi = i == 0 ? stages : i + stages - 1;
             for (int64_t j = i; j < n_local && j < hi; ++j)
                 mbar_wait_bounded(&full[j % stages], (uint32_t)((j / stages) & 1), a.wait_limit_ns);
@@ -835,16 +1028,18 @@ cudaError_t launch_bulk(K kern, const RopeTableArgs& a0, int per_item, cudaStrea
 }
 
 template <typename K>
-cudaError_t launch_smem(K kern, const RopeTableArgs& a0, cudaStream_t stream, LaunchInfo* info,
-                        int id) {
+cudaError_t launch_smem(K kern, bool il, const RopeTableArgs& a0, cudaStream_t stream,
+                        LaunchInfo* info, int id) {
     RopeTableArgs a = a0;
     const int sbytes = smem_item_heads(a.head_dim) * a.head_dim * 2;
     const int warps = kBlock / 32;
     // Two CTAs per SM, each warp with as many ring buffers (2..4) as fit.
-    const int fixed = 128 + warps * 4 * 8;
-    a.stages = std::max(2, std::min(4, (227 * 1024 / 2 - 1024 - fixed) / (warps * sbytes)));
+    auto fixed_bytes = [&](int stages) {
+        return il ? smem_il_fixed_bytes(stages) : ((warps * stages * 8 + 127) / 128 * 128);
+    };
+    a.stages = std::max(2, std::min(4, (227 * 1024 / 2 - 1024 - fixed_bytes(4)) / (warps * sbytes)));
     if (a.wait_limit_ns == 0) a.wait_limit_ns = 2000000000ull;  // 2 s
-    const int smem = ((warps * a.stages * 8 + 127) / 128 * 128) + warps * a.stages * sbytes;
+    const int smem = fixed_bytes(a.stages) + warps * a.stages * sbytes;
     int sms = 0, per_sm = 0;
     cudaError_t e = cached_sm_count(&sms);
     if (e == cudaSuccess)
@@ -930,18 +1125,20 @@ cudaError_t launch_rope_table(const RopeTableArgs& a, int fast_path, cudaStream_
         const int id = 2100 + (a.interleaved ? 100 : 0) + (a.act_f16 ? 10 : 0) + (a.table_f32 ? 1 : 0);
         if (a.interleaved) {
             if (a.act_f16) {
-                return a.table_f32 ? launch_smem(rope_table_smem<true, true, true>, a, stream, info, id)
-                                   : launch_smem(rope_table_smem<true, false, true>, a, stream, info, id);
+                return a.table_f32
+                    ? launch_smem(rope_table_smem_il<true, true>, true, a, stream, info, id)
+                    : launch_smem(rope_table_smem_il<false, true>, true, a, stream, info, id);
             }
-            return a.table_f32 ? launch_smem(rope_table_smem<true, true, false>, a, stream, info, id)
-                               : launch_smem(rope_table_smem<true, false, false>, a, stream, info, id);
+            return a.table_f32
+                ? launch_smem(rope_table_smem_il<true, false>, true, a, stream, info, id)
+                : launch_smem(rope_table_smem_il<false, false>, true, a, stream, info, id);
         }
         if (a.act_f16) {
-            return a.table_f32 ? launch_smem(rope_table_smem<false, true, true>, a, stream, info, id)
-                               : launch_smem(rope_table_smem<false, false, true>, a, stream, info, id);
+            return a.table_f32 ? launch_smem(rope_table_smem<true, true>, false, a, stream, info, id)
+                               : launch_smem(rope_table_smem<false, true>, false, a, stream, info, id);
         }
-        return a.table_f32 ? launch_smem(rope_table_smem<false, true, false>, a, stream, info, id)
-                           : launch_smem(rope_table_smem<false, false, false>, a, stream, info, id);
+        return a.table_f32 ? launch_smem(rope_table_smem<true, false>, false, a, stream, info, id)
+                           : launch_smem(rope_table_smem<false, false>, false, a, stream, info, id);
     }
     const int64_t groups = a.num_tokens * (a.hq + a.hk);
     const int64_t blocks = (groups + kBlock / 32 - 1) / (kBlock / 32);
