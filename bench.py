@@ -39,9 +39,9 @@ FALLBACK_HBM_GBS = 6650.0
 TRAFFIC = {
     "video3d": (377564416 + 325334784, "f0170ddbe869b9f9"),
     "fp8neox": (1097153280 + 517297920, "f0170ddbe869b9f9"),
-    "table_hs": (43557120 + 1894912, "ad4e2e7b6e8ba1e9"),
-    "table_il": (25730560 + 12544, "ad4e2e7b6e8ba1e9"),
-    "table_hs_f16": (42769664 + 1910784, "ad4e2e7b6e8ba1e9"),
+    "table_hs": (43556608 + 1892864, "83ce825adb161bb2"),
+    "table_il": (25730560 + 25856, "83ce825adb161bb2"),
+    "table_hs_f16": (42769152 + 1915136, "83ce825adb161bb2"),
 }
 
 
