@@ -340,8 +340,9 @@ def run_gpu(args, w):
             "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic",
+            "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "tokens_per_gpu": T,
+                       "io": "bf16 in, " + ("e4m3 out" if w.output_fp8 else "bf16 out"),
                        "qkv_shape": list(qkv.shape), "grid": [w.ppf, w.pph, w.ppw],
                        "channels": [w.cf, w.ch, w.cw], "heads": [w.hq, w.hk, w.hv],
                        "head_dim": w.head_dim, "interleave": w.interleave,
@@ -445,8 +446,9 @@ def run_gpu_table(args, w):
             "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": w.act, "data": "synthetic",
-            "config": {"workload": w.name, "tokens_per_gpu": T, "q_shape": list(q.shape),
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "tokens_per_gpu": T, "io": f"{w.act} in and out",
+                       "q_shape": list(q.shape),
                        "k_shape": list(sets[0]["k"].shape), "rotary_dim": w.rotary_dim,
                        "interleaved": w.interleaved,
                        "table_dtype": "f32" if w.table_f32 else w.act,
