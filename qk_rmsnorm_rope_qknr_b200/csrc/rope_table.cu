@@ -350,14 +350,14 @@ __device__ __forceinline__ void bulk_wait_read_allbut1() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
-// Half-split pairs, any head_dim that is a multiple of 8 (<= 256), any even
-// rotary_dim <= head_dim; q/k rows and outputs 16-byte aligned. Like the fast
+// Any head_dim that is a multiple of 8 (<= 256), any even rotary_dim <=
+// head_dim, either pairing; q/k rows and outputs 16-byte aligned. Like the fast
 // kernel, each warp streams items (heads of one token) through its own ring of
 // shared-memory buffers with bulk copies; unlike it, lanes work on the heads
 // in shared memory, so that any pairing is reachable: lane i takes the channel
-// pairs i, i + 32, ... of a head ((p, p + rotary_dim/2) for p < rotary_dim/2,
-// then the pass-through channels two by two), writes the results back in
-// place and lane 0 bulk-stores the item's
+// pairs i, i + 32, ... of a head (adjacent pairs (2p, 2p+1); half split (p,
+// p + rotary_dim/2) for p < rotary_dim/2, then the pass-through channels two
+// by two), writes the results back in place and lane 0 bulk-stores the item's
 // q and k heads. cos/sin come straight from the table in global memory (read
 // before the item's copy is waited for), the weights sit in registers.
 template <bool F32, bool H16>
@@ -394,7 +394,10 @@ __global__ void __launch_bounds__(kBlock) rope_table_smem(const RopeTableArgs a)
         has[m] = p < D / 2;
         rot[m] = has[m] && p < half;
         slot[m] = p;
-        if (p < half) {
+        if (a.interleaved) {
+            ca[m] = 2 * p;
+            cb[m] = 2 * p + 1;
+        } else if (p < half) {
             ca[m] = p;
             cb[m] = p + half;
         } else {
@@ -593,7 +596,11 @@ __host__ __device__ inline int smem_il_fixed_bytes(int stages) {
 // item's cos/sin are read from the table once per warp (before the item's
 // copy is waited for) and staged in shared memory, where lanes of the same
 // position read the same words.
-template <bool F32, bool H16>
+// HS: half-split pairs with rotary_dim a multiple of 8 in the same layout:
+// chunk c of a head is pairs 4c..4c+3, i.e. channels 4c..4c+3 and
+// rotary_dim/2 + 4c..+3 (two 8-byte pieces) while 4c < rotary_dim/2, and the
+// pass-through channels 8c..8c+7 (one 16-byte vector) after that.
+template <bool HS, bool F32, bool H16>
 __global__ void __launch_bounds__(kBlock) rope_table_smem_il(const RopeTableArgs a) {
     const int D = a.head_dim, R = a.rotary_dim, half = R / 2;
     const int vph = D / 8;
@@ -719,12 +726,28 @@ __global__ void __launch_bounds__(kBlock) rope_table_smem_il(const RopeTableArgs
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int vv = l + gs * m;
-                uint4 xv = make_uint4(0, 0, 0, 0);
-                if (m < mv && okh && vv < vph) xv = head[vv];
-                f[m][0] = act2_to_f2<H16>(xv.x);
-                f[m][1] = act2_to_f2<H16>(xv.y);
-                f[m][2] = act2_to_f2<H16>(xv.z);
-                f[m][3] = act2_to_f2<H16>(xv.w);
+                const bool here = m < mv && okh && vv < vph;
+                if (HS && 4 * vv < half) {  // (a, b) of pairs 4vv..4vv+3
+                    const uint16_t* h16 = reinterpret_cast<const uint16_t*>(head);
+                    uint2 xa = make_uint2(0, 0), xb = xa;
+                    if (here) {
+                        xa = *reinterpret_cast<const uint2*>(h16 + 4 * vv);
+                        xb = *reinterpret_cast<const uint2*>(h16 + half + 4 * vv);
+                    }
+                    const float2 a01 = act2_to_f2<H16>(xa.x), a23 = act2_to_f2<H16>(xa.y);
+                    const float2 b01 = act2_to_f2<H16>(xb.x), b23 = act2_to_f2<H16>(xb.y);
+                    f[m][0] = make_float2(a01.x, b01.x);
+                    f[m][1] = make_float2(a01.y, b01.y);
+                    f[m][2] = make_float2(a23.x, b23.x);
+                    f[m][3] = make_float2(a23.y, b23.y);
+                } else {
+                    uint4 xv = make_uint4(0, 0, 0, 0);
+                    if (here) xv = head[vv];
+                    f[m][0] = act2_to_f2<H16>(xv.x);
+                    f[m][1] = act2_to_f2<H16>(xv.y);
+                    f[m][2] = act2_to_f2<H16>(xv.z);
+                    f[m][3] = act2_to_f2<H16>(xv.w);
+                }
 #pragma unroll
                 for (int k = 0; k < 4; ++k) ss = fmaf(f[m][k].x, f[m][k].x, fmaf(f[m][k].y, f[m][k].y, ss));
             }
@@ -736,8 +759,17 @@ __global__ void __launch_bounds__(kBlock) rope_table_smem_il(const RopeTableArgs
             for (int m = 0; m < 4; ++m) {
                 const int vv = l + gs * m;
                 if (m >= mv || vv >= vph) continue;
-                const float4 w0 = reinterpret_cast<const float4*>(wrow)[2 * vv];
-                const float4 w1 = reinterpret_cast<const float4*>(wrow)[2 * vv + 1];
+                const bool split = HS && 4 * vv < half;  // a rotated half-split chunk
+                float4 w0, w1;
+                if (split) {  // weights of channels 4vv.. (a) and half + 4vv.. (b)
+                    const float4 wa = reinterpret_cast<const float4*>(wrow)[vv];
+                    const float4 wb = reinterpret_cast<const float4*>(wrow + half)[vv];
+                    w0 = make_float4(wa.x, wb.x, wa.y, wb.y);
+                    w1 = make_float4(wa.z, wb.z, wa.w, wb.w);
+                } else {
+                    w0 = reinterpret_cast<const float4*>(wrow)[2 * vv];
+                    w1 = reinterpret_cast<const float4*>(wrow)[2 * vv + 1];
+                }
                 const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
                 float4 c4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f), s4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 if (4 * vv < half) {
@@ -748,12 +780,20 @@ __global__ void __launch_bounds__(kBlock) rope_table_smem_il(const RopeTableArgs
                 uint32_t o32[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const bool rk = 4 * vv + k < half;
+                    const bool rk = HS ? split : 4 * vv + k < half;
                     const float ya = f[m][k].x * r * wv[2 * k], yb = f[m][k].y * r * wv[2 * k + 1];
                     const float c = rk ? cv[k] : 1.0f, s = rk ? sv[k] : 0.0f;
                     o32[k] = f2_to_act2<H16>(make_float2(ya * c - yb * s, yb * c + ya * s));
                 }
-                head[vv] = make_uint4(o32[0], o32[1], o32[2], o32[3]);
+                if (split) {  // o32[k] = (a_k, b_k): regroup into the a and b pieces
+                    uint16_t* h16 = reinterpret_cast<uint16_t*>(head);
+                    *reinterpret_cast<uint2*>(h16 + 4 * vv) =
+                        make_uint2(__byte_perm(o32[0], o32[1], 0x5410), __byte_perm(o32[2], o32[3], 0x5410));
+                    *reinterpret_cast<uint2*>(h16 + half + 4 * vv) =
+                        make_uint2(__byte_perm(o32[0], o32[1], 0x7632), __byte_perm(o32[2], o32[3], 0x7632));
+                } else {
+                    head[vv] = make_uint4(o32[0], o32[1], o32[2], o32[3]);
+                }
             }
         }
         fence_proxy_async_smem();  // each lane's writes, before the bulk engine reads them
@@ -1123,15 +1163,40 @@ cudaError_t launch_rope_table(const RopeTableArgs& a, int fast_path, cudaStream_
     }
     if (smem_path_ok(a)) {
         const int id = 2100 + (a.interleaved ? 100 : 0) + (a.act_f16 ? 10 : 0) + (a.table_f32 ? 1 : 0);
+        // Adjacent pairs always take the vector split (measured faster at every
+        // head_dim tried, 72 to 192). Half split takes it only when rotary_dim
+        // is a multiple of 8 and a head's pairs do not fill whole warps; with a
+        // multiple of 32 pairs the pairwise lanes are busy and measured faster.
+        const bool pairwise = !a.interleaved &&
+                              (a.rotary_dim % 8 != 0 || (a.head_dim / 2) % 32 == 0);
+        if (pairwise) {
+            if (a.act_f16) {
+                return a.table_f32 ? launch_smem(rope_table_smem<true, true>, false, a, stream, info, id)
+                                   : launch_smem(rope_table_smem<false, true>, false, a, stream, info, id);
+            }
+            return a.table_f32 ? launch_smem(rope_table_smem<true, false>, false, a, stream, info, id)
+                               : launch_smem(rope_table_smem<false, false>, false, a, stream, info, id);
+        }
         if (a.interleaved) {
             if (a.act_f16) {
                 return a.table_f32
-                    ? launch_smem(rope_table_smem_il<true, true>, true, a, stream, info, id)
-                    : launch_smem(rope_table_smem_il<false, true>, true, a, stream, info, id);
+                    ? launch_smem(rope_table_smem_il<false, true, true>, true, a, stream, info, id)
+                    : launch_smem(rope_table_smem_il<false, false, true>, true, a, stream, info, id);
             }
             return a.table_f32
-                ? launch_smem(rope_table_smem_il<true, false>, true, a, stream, info, id)
-                : launch_smem(rope_table_smem_il<false, false>, true, a, stream, info, id);
+                ? launch_smem(rope_table_smem_il<false, true, false>, true, a, stream, info, id)
+                : launch_smem(rope_table_smem_il<false, false, false>, true, a, stream, info, id);
+        }
+        if (a.rotary_dim % 8 == 0) {  // half split in 8-byte pieces
+            const int idv = id + 50;
+            if (a.act_f16) {
+                return a.table_f32
+                    ? launch_smem(rope_table_smem_il<true, true, true>, true, a, stream, info, idv)
+                    : launch_smem(rope_table_smem_il<true, false, true>, true, a, stream, info, idv);
+            }
+            return a.table_f32
+                ? launch_smem(rope_table_smem_il<true, true, false>, true, a, stream, info, idv)
+                : launch_smem(rope_table_smem_il<true, false, false>, true, a, stream, info, idv);
         }
         if (a.act_f16) {
             return a.table_f32 ? launch_smem(rope_table_smem<true, true>, false, a, stream, info, id)

@@ -376,7 +376,7 @@ def test_table_strided_inplace_and_misaligned(act):
 
 
 @pytest.mark.parametrize("act", [torch.bfloat16, torch.float16], ids=["bf16", "f16"])
-@pytest.mark.parametrize("il,R", [(True, 36), (False, 40), (False, 72)])
+@pytest.mark.parametrize("il,R", [(True, 36), (False, 40), (False, 72), (False, 36)])
 def test_table_smem_path_strided_inplace(act, il, R):
     """head_dim 72 (not a multiple of 16) with 16-byte aligned rows takes the
     shared-memory kernel: q and k as views into a packed buffer (token stride
