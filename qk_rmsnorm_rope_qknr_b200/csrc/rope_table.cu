@@ -350,14 +350,14 @@ __device__ __forceinline__ void bulk_wait_read_allbut1() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
-// Any head_dim that is a multiple of 8 (<= 256), any even rotary_dim <=
-// head_dim, either pairing; q/k rows and outputs 16-byte aligned. Like the fast
+// Half-split pairs, any head_dim that is a multiple of 8 (<= 256), any even
+// rotary_dim <= head_dim; q/k rows and outputs 16-byte aligned. Like the fast
 // kernel, each warp streams items (heads of one token) through its own ring of
 // shared-memory buffers with bulk copies; unlike it, lanes work on the heads
 // in shared memory, so that any pairing is reachable: lane i takes the channel
-// pairs i, i + 32, ... of a head (adjacent pairs (2p, 2p+1); half split (p,
-// p + rotary_dim/2) for p < rotary_dim/2, then the pass-through channels two
-// by two), writes the results back in place and lane 0 bulk-stores the item's
+// pairs i, i + 32, ... of a head ((p, p + rotary_dim/2) for p < rotary_dim/2,
+// then the pass-through channels two by two), writes the results back in
+// place and lane 0 bulk-stores the item's
 // q and k heads. cos/sin come straight from the table in global memory (read
 // before the item's copy is waited for), the weights sit in registers.
 template <bool F32, bool H16>
@@ -394,10 +394,7 @@ __global__ void __launch_bounds__(kBlock) rope_table_smem(const RopeTableArgs a)
         has[m] = p < D / 2;
         rot[m] = has[m] && p < half;
         slot[m] = p;
-        if (a.interleaved) {
-            ca[m] = 2 * p;
-            cb[m] = 2 * p + 1;
-        } else if (p < half) {
+        if (p < half) {
             ca[m] = p;
             cb[m] = p + half;
         } else {
