@@ -39,9 +39,9 @@ FALLBACK_HBM_GBS = 6650.0
 TRAFFIC = {
     "video3d": (377564416 + 325334784, "f0170ddbe869b9f9"),
     "fp8neox": (1097153280 + 517297920, "f0170ddbe869b9f9"),
-    "table_hs": (43556608 + 1892864, "83ce825adb161bb2"),
-    "table_il": (25730560 + 25856, "83ce825adb161bb2"),
-    "table_hs_f16": (42769152 + 1915136, "83ce825adb161bb2"),
+    "table_hs": (43562240 + 2029568, "9230c313092c6dc7"),
+    "table_il": (25730816 + 15616, "9230c313092c6dc7"),
+    "table_hs_f16": (42770176 + 2013952, "9230c313092c6dc7"),
 }
 
 
