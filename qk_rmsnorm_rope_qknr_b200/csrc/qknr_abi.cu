@@ -331,7 +331,7 @@ int run_3d(const qknr_rope_3d_params* prm, int mode, float* ssq_out, const float
         return fail(QKNR_ERR_UNSUPPORTED, "YARN scaling (factor %g != 1) is not supported",
                     (double)p.factor);
     if (p.attention_factor != 1.0f)
-        return fail(QKNR_ERR_SHAPE, "attention_factor must be 1.0 when factor is 1.0");
+        return fail(QKNR_ERR_SHAPE, "attention_factor other than 1 needs YARN (factor != 1), which is not built");
     if (norm && !partial && (!(p.eps >= 0.0f) || std::isinf(p.eps)))
         return fail(QKNR_ERR_SHAPE, "eps must be >= 0");
     if (!partial && p.output_fp8 &&

@@ -1,9 +1,9 @@
 """Host-side dispatch policy for the fused op
 ("vllm_omni.diffusion.layers.fused_qk_norm_rope": fused_qk_norm_rope_min_tokens).
 
-A fused call costs a fixed amount of host time (argument checks, the launch),
-while the GPU time it saves grows with the tokens it covers, so below some
-token count a consumer may prefer its unfused chain. The consumer passes the
+Each fused call pays a fixed host cost (argument checks, the launch), and
+what it saves on the GPU scales with the number of tokens, so small calls may
+do better with a consumer's unfused chain. The consumer passes the
 crossover it measured on its own hardware as `default`; one environment
 variable overrides it for every consumer of a deployment. The variable is read
 at each call, so it can change without re-importing anything.
@@ -18,7 +18,7 @@ _INT = re.compile(r"[0-9]+")
 
 
 def fused_qk_norm_rope_min_tokens(default: int) -> int:
-    """Token span below which a consumer should keep its unfused chain.
+    """The smallest token count for which a consumer should take the fused op.
 
     The environment variable, when set and not blank, must be a non-negative
     decimal integer (0 = always fuse); anything else raises ValueError. Unset

@@ -2,8 +2,9 @@
 
 Each rank holds packed rows of its own heads, [tokens, (hq+hk+hv)*head_dim],
 and the [hq*head_dim] / [hk*head_dim] slices of the norm weights. The
-across-heads RMSNorm must still run over all ranks' channels ("a tensor-parallel
-shard still normalises over the global channel width"), so one call is
+across-heads RMSNorm must still run over all ranks' channels (the SANA-WM UCPE
+page, cam_prep_func: a head shard is normalised over the whole channel width,
+not its own slice), so one call is
     partial sums of x^2 (this rank's heads)  ->  all-reduce (sum)  ->
     transform with the global sums,
 the first and last step in libqknr.so's kernels, the exchange a
@@ -53,7 +54,15 @@ def fused_qk_rmsnorm_rope_tp(qkv: torch.Tensor, q_weight: torch.Tensor, k_weight
                                                         device=qkv.device))
     ssq = torch.empty(T, 2, dtype=torch.float32, device=qkv.device)
     Q.qknr_rope_3d_partial_ssq(qkv, ssq, stream=stream, **params)
-    all_reduce_ssq(ssq, group)
+    # The collective is queued behind the partial sums and ahead of the
+    # transform: on the caller's stream when one is given.
+    if stream is not None and not isinstance(stream, torch.cuda.Stream):
+        stream = torch.cuda.ExternalStream(int(stream), device=qkv.device)
+    if stream is not None:
+        with torch.cuda.stream(stream):
+            all_reduce_ssq(ssq, group)
+    else:
+        all_reduce_ssq(ssq, group)
     Q.qknr_rope_3d_with_ssq(qkv, q_weight, k_weight, *outs, ssq, heads_q_total=heads_q_total,
                             heads_k_total=heads_k_total, stream=stream, **params)
     return tuple(outs)

@@ -92,5 +92,13 @@ def test_tp_one_rank_nccl_group():
         torch.cuda.synchronize()
         ref, exact = oracle_3d(inp["qkv"].cpu(), inp["q_weight"].cpu(), inp["k_weight"].cpu(), **p)
         assert_3d_close([q, k, v], ref, exact, False, "tp world 1")
+        # on a side stream: the exchange is ordered between the two kernels there
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        q2, k2, v2 = tp.fused_qk_rmsnorm_rope_tp(inp["qkv"], inp["q_weight"], inp["k_weight"],
+                                                 heads_q_total=w.hq, heads_k_total=w.hk,
+                                                 stream=side, **p)
+        side.synchronize()
+        assert torch.equal(q, q2) and torch.equal(k, k2) and torch.equal(v, v2)
     finally:
         dist.destroy_process_group()
