@@ -215,7 +215,7 @@ def pin_rotation_is_complex_product():
 def pin_pair_maps():
     """[T] contract bullets: half-split pairs (d, d + rotary_dim/2); interleaved
     adjacent pairs (2i, 2i+1). [F] interleave=False is NeoX style: whole-head
-    half split (the reading this build takes)."""
+    half split (the reading taken here)."""
     pa, pb = O.pairs_table(8, True)
     assert pa.tolist() == [0, 2, 4, 6] and pb.tolist() == [1, 3, 5, 7]
     pa, pb = O.pairs_table(6, False)
