@@ -310,6 +310,9 @@ CASES_TABLE = [
     (30, 2, 3, 128, 40, False, False),   # half split with rd % 16 != 0: general kernel
     (30, 2, 3, 2, 2, True, True),        # smallest head
     (30, 3, 0, 64, 64, True, False),     # no K heads
+    (40, 3, 0, 72, 40, True, True),      # shared-memory (vector) kernel, no K heads
+    (40, 0, 2, 72, 40, True, False),     # shared-memory (vector, half split) kernel, no Q heads
+    (40, 2, 3, 128, 36, True, False),    # shared-memory pairwise kernel (rd % 8 != 0)
 ]
 
 
