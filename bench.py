@@ -206,9 +206,10 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     inp = W.make_inputs(w, device="cpu")
-    # About a minute of oracle work over the whole run, whatever K and W are;
-    # a step does at least one chunk, so small per-step budgets use small ones.
-    per_step = 60.0 / max(1, args.steps + args.warmup)
+    # About a minute of oracle work over the whole run (6 x --cpu-seconds),
+    # whatever K and W are; a step does at least one chunk, so small per-step
+    # budgets use small ones.
+    per_step = 6.0 * args.cpu_seconds / max(1, args.steps + args.warmup)
     chunk = 256 if per_step >= 0.5 else 32
     for _ in range(args.warmup):
         oracle_sample(w, inp, per_step, chunk)
