@@ -173,9 +173,10 @@ int qknr_rope_3d(const qknr_rope_3d_params* params, void* cuda_stream);
 /*
  * Tensor-parallel 3D form. When the Q, K and V heads of a token are split
  * across ranks, each rank holds packed rows of its own heads only, but the
- * RMSNorm must still run over the global channel width of Q (and of K).
- * "vllm_omni.diffusion.models.sana_wm.ucpe" (cam_prep_func) states this rule:
- * a tensor-parallel shard must normalise over the global channel width.
+ * across-heads RMSNorm still covers all of Q's (and all of K's) channels on
+ * every rank, not one rank's slice ("vllm_omni.diffusion.models.sana_wm.ucpe",
+ * cam_prep_func, which leaves the norm to the model's own modules for exactly
+ * this reason).
  * The transform is the one of qknr_rope_3d ("flashinfer.norm.
  * fused_qk_rmsnorm_rope"), split in two passes around one exchange:
  *
@@ -214,8 +215,9 @@ int qknr_device_status(void* cuda_stream, uint32_t* status_out, int32_t clear);
 
 /*
  * Test hook for the timeout path above (not for production use). While
- * extra_bytes is non-zero, every later 3D launch on any thread makes each
- * ring buffer wait for extra_bytes more than its copy delivers, so its waits
+ * extra_bytes is non-zero, every later launch of a bulk-copy kernel (3D and
+ * table forms) on any thread makes each ring buffer wait for extra_bytes more
+ * than its copy delivers, so its waits
  * run out after limit_ns and the launch takes the abandon path; the copies
  * themselves complete, so nothing is left in flight. extra_bytes == 0 turns
  * the hook off (limit_ns is then ignored and the 2 s limit returns).
