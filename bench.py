@@ -42,6 +42,7 @@ TRAFFIC = {
     "table_hs": (43562240 + 2029568, "9230c313092c6dc7"),
     "table_il": (25730816 + 15616, "9230c313092c6dc7"),
     "table_hs_f16": (42770176 + 2013952, "9230c313092c6dc7"),
+    "table_d72": (24805120 + 3584, "9230c313092c6dc7"),
 }
 
 

@@ -14,6 +14,8 @@ video-DiT and MiniMax-H3 geometries the pages name):
   table_il    table form, adjacent pairs, q,k [2048,24,128] (x3, 1% outliers x20),
               rd 128, bf16 table
   table_hs_f16  table_hs with IEEE binary16 activations, weights and table
+  table_d72   table form, adjacent pairs, head_dim 72 (off the register fast path:
+              the shared-memory kernel), q [4096,32,72], k [4096,8,72], rd 72
   video3d     3D form, [1,15360,(32+32+32)*128], grid 16x30x32, 16/56/56, bf16 out
   fp8neox     3D form, [2,29760,(24+24+24)*128] ~N(0, 2^2), grid 31x24x40,
               32/48/48, NeoX pairs, E4M3 out (scales 0.5 / 0.25)
@@ -109,6 +111,8 @@ WORKLOADS = {
                           outlier_mult=20.0),
     "table_hs_f16": FormTable("table_hs_f16", tokens=4096, hq=32, hk=8, head_dim=128,
                               rotary_dim=96, table_f32=False, interleaved=False, act="f16"),
+    "table_d72": FormTable("table_d72", tokens=4096, hq=32, hk=8, head_dim=72, rotary_dim=72,
+                           table_f32=True, interleaved=True),
     "video3d": Form3D("video3d", batch=1, seq=15360, ppf=16, pph=30, ppw=32, cf=16, ch=56,
                       cw=56, hq=32, hk=32, hv=32, head_dim=128),
     "fp8neox": Form3D("fp8neox", batch=2, seq=29760, ppf=31, pph=24, ppw=40, cf=32, ch=48,

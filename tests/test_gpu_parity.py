@@ -109,7 +109,7 @@ def test_3d_workload_full_size_sampled(name):
         assert torch.equal(v_out, v_in)
 
 
-@pytest.mark.parametrize("name", ["table_hs", "table_il", "table_hs_f16"])
+@pytest.mark.parametrize("name", ["table_hs", "table_il", "table_hs_f16", "table_d72"])
 def test_table_workload_full(name):
     w = W.WORKLOADS[name]
     inp = W.make_inputs(w, device="cpu")
