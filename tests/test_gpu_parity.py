@@ -313,6 +313,9 @@ CASES_TABLE = [
     (40, 3, 0, 72, 40, True, True),      # shared-memory (vector) kernel, no K heads
     (40, 0, 2, 72, 40, True, False),     # shared-memory (vector, half split) kernel, no Q heads
     (40, 2, 3, 128, 36, True, False),    # shared-memory pairwise kernel (rd % 8 != 0)
+    (70, 5, 3, 8, 8, True, True),        # vector kernel, head_dim 8: 32 heads per warp step
+    (70, 5, 3, 24, 16, False, False),    # vector kernel, half split, 3 chunks per head
+    (70, 5, 3, 200, 104, True, True),    # vector kernel, head_dim 200: 25 chunks over 32 lanes
 ]
 
 
