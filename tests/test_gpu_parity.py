@@ -482,3 +482,53 @@ def test_3d_sequence_shards_match_whole_call():
                 lst.append(o)
         for lst, o in zip(parts, whole):
             assert torch.equal(torch.cat(lst), o)
+
+
+def test_concurrent_host_threads_match_serial():
+    """Several host threads calling both entry points at once, each on its own
+    stream and with its own shapes (the launch caches and lane plans are shared
+    state), give the bits of the same calls made one after another."""
+    import threading
+
+    jobs = []
+    for i in range(4):
+        qkv, qw, kw = _rand3d(48, 2 + i, 2, 1, 64, seed=20 + i)
+        p3 = dict(ppf=2, pph=4, ppw=6, num_frame_channels=16, num_height_channels=24,
+                  num_width_channels=24, num_heads_q=2 + i, num_heads_k=2, num_heads_v=1,
+                  head_dim=64)
+        D, R = (128, 96) if i % 2 == 0 else (72, 40)
+        t = {n: v.to(DEV) for n, v in _rand_table_inputs(64, 3, 1 + i, D, R, True,
+                                                          seed=30 + i).items()}
+        jobs.append((qkv, qw, kw, p3, t, R, bool(i % 2)))
+
+    def run(job, stream):
+        qkv, qw, kw, p3, t, R, il = job
+        outs = []
+        for _ in range(10):
+            a = run_3d(qkv, qw, kw, stream=stream, **p3)
+            b = Q.fused_qk_norm_rope(t["q"], t["k"], t["q_weight"], t["k_weight"], t["rope_table"],
+                                     1e-6, rotary_dim=R, interleaved=il, stream=stream)
+            outs.append([x.clone() for x in (*a, *b)])
+        return outs
+
+    serial = [run(j, torch.cuda.current_stream()) for j in jobs]
+    torch.cuda.synchronize()
+    results = [None] * len(jobs)
+    streams = [torch.cuda.Stream() for _ in jobs]
+    for s in streams:
+        s.wait_stream(torch.cuda.current_stream())
+
+    def worker(i):
+        with torch.cuda.stream(streams[i]):
+            results[i] = run(jobs[i], streams[i])
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(len(jobs))]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    torch.cuda.synchronize()
+    for i in range(len(jobs)):
+        for rep_s, rep_c in zip(serial[i], results[i]):
+            for x, y in zip(rep_s, rep_c):
+                assert torch.equal(x, y)
