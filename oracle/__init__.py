@@ -5,14 +5,15 @@ bench.py may import this package. The product library never imports it and
 shares no code with it (the C source is compiled on its own by oracle/build.py).
 
 Everything here is numpy-in / numpy-out marshalling around the C functions in
-qknr_oracle.c; the arithmetic, and the readings R1..R12 of the pages, are
+qknr_oracle.c; the arithmetic, and the readings R1..R13 and U1..U6 of the pages, are
 stated there. bf16 and binary16 values travel as uint16 bit patterns, E4M3 as
 uint8.
 
 Parity status: every function is pinned by tests/test_oracle_pins.py except
-two readings the pages cannot decide -- the 3D NeoX pair layout (whole-head
-pairs vs per-axis-group pairs, R8) and the direction of the FP8 scale (R9):
-"parity unpinned" for those two choices.
+three readings the pages cannot decide -- the 3D NeoX pair layout (whole-head
+pairs vs per-axis-group pairs, R8), the direction of the FP8 scale (R9) and
+the definition of the camera prep's inflation_sq output (U6): "parity
+unpinned" for those three choices.
 """
 import ctypes as C
 import os
@@ -71,6 +72,12 @@ def lib(path=None):
         L.qknr_oracle_rope_3d.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, i32, i32, i32,
                                           i32, i32, i32, i32, f64, f64, i32, i32, i32, i32, f64,
                                           f64, vp, vp, vp]
+        L.qknr_oracle_relu.argtypes = [vp, i64, vp]
+        L.qknr_oracle_ray_project.argtypes = [vp, vp, i64, vp]
+        L.qknr_oracle_ucpe_exact.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i64, i32,
+                                             i32, f64, vp, vp, vp, vp]
+        L.qknr_oracle_ucpe.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i64, i32, i32, f64,
+                                       vp, vp, vp, vp]
         L.qknr_oracle_threads.restype = C.c_int
         L.qknr_oracle_set_threads.argtypes = [C.c_int]
         _lib = L
@@ -249,6 +256,54 @@ def rope_3d(qkv, q_weight, k_weight, *, ppf, pph, ppw, num_frame_channels, num_h
     return qo, ko, vo
 
 
+# ------------------------------------------------------ UCPE camera prep --
+def relu(x):
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.empty_like(x)
+    lib().qknr_oracle_relu(_p(x), x.size, _p(y))
+    return y
+
+
+def ray_project(m, x):
+    """Every block of four consecutive values of x times the 4x4 matrix m."""
+    m = np.ascontiguousarray(m, dtype=np.float64).reshape(16)
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    assert x.size % 4 == 0
+    y = np.empty_like(x)
+    lib().qknr_oracle_ray_project(_p(m), _p(x), x.size, _p(y))
+    return y
+
+
+def ucpe_cam_prep(q, k, v, proj_q, proj_kv, rope_cos, rope_sin, k_scale, exact=False,
+                  act="bf16"):
+    """UCPE camera prep. q, k, v [B,N,H,D] uint16 patterns of the activation type
+    `act` ("bf16" or "f16"); proj_q, proj_kv [B,N,4,4] float32; rope_cos,
+    rope_sin [N, D/2] float32. Returns (q_trans, k_trans, v_trans) [B,H,D,N] as
+    activation-type bits (float64 before rounding when exact=True) and
+    inflation_sq [B,H,N] float64."""
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    assert q.shape == k.shape == v.shape and q.ndim == 4, (q.shape, k.shape, v.shape)
+    B, N, H, D = q.shape
+    pq = np.ascontiguousarray(proj_q, np.float32)
+    pkv = np.ascontiguousarray(proj_kv, np.float32)
+    assert pq.shape == pkv.shape == (B, N, 4, 4), (pq.shape, pkv.shape)
+    cs = np.ascontiguousarray(rope_cos, np.float32)
+    sn = np.ascontiguousarray(rope_sin, np.float32)
+    assert cs.shape == sn.shape == (N, D // 2), (cs.shape, sn.shape)
+    assert act in ("bf16", "f16")
+    dt = np.float64 if exact else np.uint16
+    qo = np.empty((B, H, D, N), dt)
+    ko = np.empty((B, H, D, N), dt)
+    vo = np.empty((B, H, D, N), dt)
+    infl = np.empty((B, H, N), np.float64)
+    fn = lib().qknr_oracle_ucpe_exact if exact else lib().qknr_oracle_ucpe
+    rc = fn(_p(q), _p(k), _p(v), _p(pq), _p(pkv), _p(cs), _p(sn), int(act == "f16"), B, N, H, D,
+            float(k_scale), _p(qo), _p(ko), _p(vo), _p(infl))
+    if rc != 0:
+        raise ValueError("oracle rejected the camera-prep arguments")
+    return qo, ko, vo, infl
+
+
 def threads():
     return lib().qknr_oracle_threads()
 
@@ -260,5 +315,5 @@ def set_threads(n):
 __all__ = ["bf16_to_f64", "bf16_from_f64", "f16_from_f64", "f16_to_f64", "e4m3_from_f64",
            "e4m3_to_f64", "rmsnorm",
            "pairs_table", "pairs_3d", "rotate", "position_3d", "angles_3d", "rope_table",
-           "rope_3d", "threads", "set_threads", "lib"]
+           "rope_3d", "relu", "ray_project", "ucpe_cam_prep", "threads", "set_threads", "lib"]
 _ = os

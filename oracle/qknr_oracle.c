@@ -12,6 +12,8 @@
  *       signature of fused_qk_norm_rope.
  *   [F] "flashinfer.norm.fused_qk_rmsnorm_rope" (FlashInfer API docs): the
  *       summary paragraph, "Parameters" and "Returns".
+ *   [U] "vllm_omni.diffusion.models.sana_wm.ucpe" (vLLM-Omni API docs):
+ *       cam_prep_func, its description, "Parameters" and "Returns".
  *
  * The pages give signatures and prose but print no formula. Where they leave a
  * step open this file takes the plainest reading and says so next to the step:
@@ -46,6 +48,32 @@
  *       has the activation type or is float32, so the activation type is
  *       not fixed to bf16); weights share the activation type, outputs are
  *       rounded once to it.
+ *
+ * The camera prep of [U] lists its steps (ReLU, the K scale, the ray
+ * projection, RoPE) and its shapes but no formula. Readings taken:
+ *   U1  ReLU is the feature map of Q and K and comes first; V is not passed
+ *       through it ([U] takes V un-normalised and names no V step but the
+ *       projection).
+ *   U2  The K scale multiplies K alone, after its ReLU.
+ *   U3  The ray projection splits each head's channels into blocks of four
+ *       consecutive channels and multiplies every block, as a column vector,
+ *       by the token's 4x4 matrix read row by row: y_i = sum_j M[i][j] x_j.
+ *       Q takes proj_q; K and V take proj_kv ([U] gives proj_kv for both).
+ *   U4  RoPE follows the projection, on Q and K only, with adjacent pairs
+ *       (2j, 2j+1) ([U]: the tables are for interleaved pairs and have D/2
+ *       columns, so they cover the whole head), column j of the token's row of rope_cos
+ *       and rope_sin, and the rotation of R4. V is not rotated, as in the
+ *       other two contracts.
+ *   U5  Outputs are laid out [B, H, D, N] ([U], "Returns"): the value for
+ *       batch b, token n, head h, channel d is stored at [b][h][d][n], rounded
+ *       once to the activation type (bf16 or binary16, as R13). Projection
+ *       matrices and RoPE tables are float32, used as stored.
+ *   U6  inflation_sq [B, H, N] is the factor by which the ray projection
+ *       multiplies the squared norm of the scaled key: |M_kv k'|^2 / |k'|^2,
+ *       k' = k_scale * ReLU(k) of that token and head (RoPE keeps the norm,
+ *       so before or after the rotation is the same), and 1 where k' = 0.
+ *       PARITY UNPINNED: [U] names this output but does not define it; the
+ *       same ratio for Q is the other plain reading.
  *
  * Threads: the per-token loops run under OpenMP when it is enabled; every
  * token is computed independently, so the results do not depend on the
@@ -516,6 +544,131 @@ int qknr_oracle_rope_3d(const uint16_t* qkv, const uint16_t* q_weight, const uin
             qknr_oracle_bf16_from_double_array(ek, (uint16_t*)k_out, nk);
             qknr_oracle_bf16_from_double_array(ev, (uint16_t*)v_out, nv);
         }
+    }
+    free(eq);
+    free(ek);
+    free(ev);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* UCPE camera prep ([U] cam_prep_func)                                      */
+/* ------------------------------------------------------------------------ */
+
+/* U1: the feature map of the camera branch, max(x, 0) per element. */
+void qknr_oracle_relu(const double* x, int64_t n, double* y)
+{
+    for (int64_t i = 0; i < n; ++i) y[i] = x[i] > 0.0 ? x[i] : 0.0;
+}
+
+/* U3: ray projection of one head. Every block of four consecutive channels
+ * (x[4b], ..., x[4b+3]) is replaced by m times it, m a 4x4 matrix stored row
+ * by row: y[4b+i] = sum_j m[4i+j] x[4b+j]. n must be a multiple of 4. */
+void qknr_oracle_ray_project(const double* m, const double* x, int64_t n, double* y)
+{
+    for (int64_t b = 0; b + 4 <= n; b += 4)
+        for (int i = 0; i < 4; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < 4; ++j) acc += m[4 * i + j] * x[b + j];
+            y[b + i] = acc;
+        }
+}
+
+/* Exact (pre-rounding) results of the camera prep for dense inputs
+ * q, k, v [B, N, H, D] (16-bit activation patterns, binary16 when act_is_f16),
+ * fp32 projection matrices proj_q, proj_kv [B, N, 4, 4] and fp32 rope_cos,
+ * rope_sin [N, D/2]. Outputs q_out, k_out, v_out are fp64 in [B, H, D, N]
+ * layout (U5) and inflation_sq is fp64 [B, H, N] (U6). Per token n and head h:
+ *   Q: ReLU (U1), projection by proj_q (U3), rotation (U4);
+ *   K: ReLU (U1), times k_scale (U2), projection by proj_kv (U3), rotation (U4);
+ *   V: projection by proj_kv only (U1, U4).
+ * Returns 1, writing nothing, when head_dim is not a positive multiple of 4
+ * up to 512 or a size is negative. */
+int qknr_oracle_ucpe_exact(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const float* proj_q, const float* proj_kv, const float* rope_cos,
+                           const float* rope_sin, int32_t act_is_f16, int64_t batch,
+                           int64_t num_tokens, int32_t heads, int32_t head_dim, double k_scale,
+                           double* q_out, double* k_out, double* v_out, double* inflation_sq)
+{
+    const int32_t D = head_dim;
+    const int64_t B = batch, N = num_tokens, H = heads;
+    if (B < 0 || N < 0 || H < 0 || D <= 0 || D > 512 || (D % 4)) return 1;
+    int32_t* pa = malloc(sizeof(int32_t) * (D / 2));
+    int32_t* pb = malloc(sizeof(int32_t) * (D / 2));
+    qknr_oracle_pairs_table(D, 1, pa, pb); /* U4: adjacent pairs (2j, 2j+1) */
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 16)
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t n = 0; n < N; ++n) {
+            double mq[16], mkv[16], c[256], s[256];
+            double x[512], r[512], y[512], o[512];
+            for (int i = 0; i < 16; ++i) {
+                mq[i] = proj_q[(b * N + n) * 16 + i];
+                mkv[i] = proj_kv[(b * N + n) * 16 + i];
+            }
+            for (int32_t j = 0; j < D / 2; ++j) {
+                c[j] = rope_cos[n * (D / 2) + j];
+                s[j] = rope_sin[n * (D / 2) + j];
+            }
+            for (int64_t h = 0; h < H; ++h) {
+                const int64_t in = ((b * N + n) * H + h) * D;
+                const int64_t out = (b * H + h) * D * N + n; /* channel d at out + d * N */
+
+                /* Q */
+                for (int32_t d = 0; d < D; ++d) x[d] = act_to_double(q[in + d], act_is_f16);
+                qknr_oracle_relu(x, D, r);
+                qknr_oracle_ray_project(mq, r, D, y);
+                qknr_oracle_rotate(y, D, D / 2, pa, pb, c, s, o);
+                for (int32_t d = 0; d < D; ++d) q_out[out + (int64_t)d * N] = o[d];
+
+                /* K, and the squared-norm gain of its projection */
+                for (int32_t d = 0; d < D; ++d) x[d] = act_to_double(k[in + d], act_is_f16);
+                qknr_oracle_relu(x, D, r);
+                for (int32_t d = 0; d < D; ++d) r[d] *= k_scale;
+                qknr_oracle_ray_project(mkv, r, D, y);
+                double before = 0.0, after = 0.0;
+                for (int32_t d = 0; d < D; ++d) {
+                    before += r[d] * r[d];
+                    after += y[d] * y[d];
+                }
+                inflation_sq[(b * H + h) * N + n] = before > 0.0 ? after / before : 1.0;
+                qknr_oracle_rotate(y, D, D / 2, pa, pb, c, s, o);
+                for (int32_t d = 0; d < D; ++d) k_out[out + (int64_t)d * N] = o[d];
+
+                /* V */
+                for (int32_t d = 0; d < D; ++d) x[d] = act_to_double(v[in + d], act_is_f16);
+                qknr_oracle_ray_project(mkv, x, D, y);
+                for (int32_t d = 0; d < D; ++d) v_out[out + (int64_t)d * N] = y[d];
+            }
+        }
+    free(pa);
+    free(pb);
+    return 0;
+}
+
+/* Camera prep with its output rounding (U5): q/k/v results rounded once to
+ * the activation type (bf16, or binary16 when act_is_f16); inflation_sq is
+ * returned in fp64. */
+int qknr_oracle_ucpe(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                     const float* proj_q, const float* proj_kv, const float* rope_cos,
+                     const float* rope_sin, int32_t act_is_f16, int64_t batch, int64_t num_tokens,
+                     int32_t heads, int32_t head_dim, double k_scale, uint16_t* q_out,
+                     uint16_t* k_out, uint16_t* v_out, double* inflation_sq)
+{
+    int64_t n = batch * num_tokens * heads * head_dim;
+    if (n < 0) return 1;
+    double* eq = malloc(sizeof(double) * (n + 1));
+    double* ek = malloc(sizeof(double) * (n + 1));
+    double* ev = malloc(sizeof(double) * (n + 1));
+    int rc = qknr_oracle_ucpe_exact(q, k, v, proj_q, proj_kv, rope_cos, rope_sin, act_is_f16,
+                                    batch, num_tokens, heads, head_dim, k_scale, eq, ek, ev,
+                                    inflation_sq);
+    if (rc == 0) {
+        void (*round_to)(const double*, uint16_t*, int64_t) =
+            act_is_f16 ? qknr_oracle_f16_from_double_array : qknr_oracle_bf16_from_double_array;
+        round_to(eq, q_out, n);
+        round_to(ek, k_out, n);
+        round_to(ev, v_out, n);
     }
     free(eq);
     free(ek);

@@ -71,6 +71,43 @@ def case_table(name, seed, T, hq, hk, D, R, interleaved, table_f32, act):
                              "k_weight": arr(kw), "rope_table": arr(tbl)},
                   "expected": {"q": arr(qo), "k": arr(ko)}}
 
+CITE_UCPE = ('"vllm_omni.diffusion.models.sana_wm.ucpe" (vLLM-Omni API docs): cam_prep_func, '
+             'Parameters, Returns')
+
+
+def _camera_matrices(g, B, N):
+    """Per-token rigid motions G = [[R, t], [0, 1]] (R a random rotation, t ~
+    N(0, 0.5^2)); proj_q = G^T and proj_kv = G^-1, as float32."""
+    pq = np.empty((B, N, 4, 4), np.float32)
+    pkv = np.empty((B, N, 4, 4), np.float32)
+    for b in range(B):
+        for n in range(N):
+            m, r = np.linalg.qr(g.standard_normal((3, 3)))
+            G = np.eye(4)
+            G[:3, :3] = m * np.sign(np.diag(r))
+            G[:3, 3] = 0.5 * g.standard_normal(3)
+            pq[b, n] = G.T
+            pkv[b, n] = np.linalg.inv(G)
+    return pq, pkv
+
+
+def case_ucpe(name, seed, B, N, H, D, act):
+    g = np.random.default_rng(seed)
+    to = O.f16_from_f64 if act == "f16" else O.bf16_from_f64
+    q, k, v = (to(g.standard_normal((B, N, H, D))) for _ in range(3))
+    pq, pkv = _camera_matrices(g, B, N)
+    theta = np.arange(N)[:, None] * 10000.0 ** (-2.0 * np.arange(D // 2) / D)[None, :]
+    cos_t, sin_t = np.cos(theta).astype(np.float32), np.sin(theta).astype(np.float32)
+    k_scale = D ** -0.5 * 4 ** -0.5
+    qo, ko, vo, infl = O.ucpe_cam_prep(q, k, v, pq, pkv, cos_t, sin_t, k_scale, act=act)
+    p = dict(k_scale=k_scale, act=act)
+    return name, {"form": "ucpe", "cite": CITE_UCPE, "params": p,
+                  "inputs": {"q": arr(q), "k": arr(k), "v": arr(v), "proj_q": arr(pq),
+                             "proj_kv": arr(pkv), "rope_cos": arr(cos_t),
+                             "rope_sin": arr(sin_t)},
+                  "expected": {"q": arr(qo), "k": arr(ko), "v": arr(vo),
+                               "inflation_sq": arr(infl)}}
+
 
 def cases():
     return [
@@ -83,6 +120,8 @@ def cases():
     case_table("oracle_table_halfsplit_f32", 4, 6, 2, 1, 64, 48, False, True, "bf16"),
     case_table("oracle_table_interleaved_bf16", 5, 6, 1, 2, 64, 64, True, False, "bf16"),
     case_table("oracle_table_halfsplit_f16", 6, 6, 2, 1, 64, 32, False, False, "f16"),
+    case_ucpe("oracle_ucpe_bf16", 7, 2, 12, 2, 16, "bf16"),
+    case_ucpe("oracle_ucpe_f16", 8, 1, 9, 3, 24, "f16"),
     ]
 
 

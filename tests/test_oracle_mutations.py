@@ -61,6 +61,32 @@ MUTATIONS = {
                                  "wq[d] = act_to_double(q_weight[d], 0);"),
     "f16_table_read_as_bf16": ("c[j] = act_to_double(row[j], act_is_f16);",
                                "c[j] = act_to_double(row[j], 0);"),
+    "ucpe_relu_dropped": ("y[i] = x[i] > 0.0 ? x[i] : 0.0;", "y[i] = x[i];"),
+    "ucpe_relu_leaky": ("y[i] = x[i] > 0.0 ? x[i] : 0.0;", "y[i] = x[i] > 0.0 ? x[i] : 0.01 * x[i];"),
+    "ucpe_projection_transposed": ("acc += m[4 * i + j] * x[b + j];",
+                                   "acc += m[4 * j + i] * x[b + j];"),
+    "ucpe_k_scale_dropped": ("for (int32_t d = 0; d < D; ++d) r[d] *= k_scale;", ""),
+    "ucpe_v_through_relu": ("qknr_oracle_ray_project(mkv, x, D, y);",
+                            "qknr_oracle_relu(x, D, r); qknr_oracle_ray_project(mkv, r, D, y);"),
+    "ucpe_v_rotated": ("for (int32_t d = 0; d < D; ++d) v_out[out + (int64_t)d * N] = y[d];",
+                       "qknr_oracle_rotate(y, D, D / 2, pa, pb, c, s, o); "
+                       "for (int32_t d = 0; d < D; ++d) v_out[out + (int64_t)d * N] = o[d];"),
+    "ucpe_q_takes_kv_matrix": ("qknr_oracle_ray_project(mq, r, D, y);",
+                               "qknr_oracle_ray_project(mkv, r, D, y);"),
+    "ucpe_half_split_pairs": ("qknr_oracle_pairs_table(D, 1, pa, pb); /* U4",
+                              "qknr_oracle_pairs_table(D, 0, pa, pb); /* U4"),
+    "ucpe_heads_batch_swapped": ("const int64_t out = (b * H + h) * D * N + n;",
+                                 "const int64_t out = (h * B + b) * D * N + n;"),
+    "ucpe_table_row_ignored": ("c[j] = rope_cos[n * (D / 2) + j];", "c[j] = rope_cos[j];"),
+    "ucpe_matrix_of_first_token": ("mq[i] = proj_q[(b * N + n) * 16 + i];",
+                                   "mq[i] = proj_q[(b * N) * 16 + i];"),
+    "ucpe_inflation_inverted": ("before > 0.0 ? after / before : 1.0",
+                                "before > 0.0 ? before / (after > 0.0 ? after : 1.0) : 1.0"),
+    "ucpe_inflation_zero_key": ("before > 0.0 ? after / before : 1.0",
+                                "before > 0.0 ? after / before : 0.0"),
+    "ucpe_f16_outputs_as_bf16": ("act_is_f16 ? qknr_oracle_f16_from_double_array : "
+                                 "qknr_oracle_bf16_from_double_array;",
+                                 "qknr_oracle_bf16_from_double_array;"),
 }
 
 # cheap pins first, so a planted mistake is usually caught within a second

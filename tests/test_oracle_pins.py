@@ -5,6 +5,7 @@ an invariant of the mathematics, or a tiny case worked out by hand in the
 comments. Pages cited by title:
   [T] "vllm_omni.diffusion.layers.fused_qk_norm_rope" -- contract bullets
   [F] "flashinfer.norm.fused_qk_rmsnorm_rope" -- summary, Parameters, Returns
+  [U] "vllm_omni.diffusion.models.sana_wm.ucpe" -- cam_prep_func
 The pin_* functions are also run by test_oracle_mutations.py against copies of
 the oracle with planted mistakes, each of which must fail at least one pin.
 """
@@ -508,6 +509,218 @@ def pin_offset_and_batch_repeat():
     qkv2[16:] = qkv2[:16]
     q, k, v = O.rope_3d(qkv2, qw, kw, **p)
     assert np.array_equal(q[:16], q[16:]) and np.array_equal(k[:16], k[16:])
+
+
+# ----------------------------------------------------------------------------
+# UCPE camera prep ([U] cam_prep_func), readings U1..U6 of the oracle.
+# ----------------------------------------------------------------------------
+def _ucpe_inputs(B, N, H, D, rng=RNG):
+    q, k, v = (_rand_bf16((B, N, H, D), rng=rng) for _ in range(3))
+    return q, k, v
+
+
+def _bf16_value_bits(x):
+    """bf16 bit patterns of values that are exactly representable in bf16."""
+    b = _bf16_bits(x)
+    assert np.array_equal(O.bf16_to_f64(b), np.asarray(x, np.float64)), "not exact in bf16"
+    return b
+
+
+def pin_ucpe_identity_geometry():
+    """Identity matrices and zero angles leave only the element steps and the
+    layout: q_trans = ReLU(q), k_trans = k_scale * ReLU(k), v_trans = v, each
+    moved from [B,N,H,D] to [B,H,D,N] (U5), all exact in bf16 because k_scale
+    is a power of two; inflation_sq = 1 (an identity projection keeps every
+    norm). Sizes differ in every axis so that a swapped index shows."""
+    B, N, H, D = 2, 5, 3, 8
+    q, k, v = _ucpe_inputs(B, N, H, D)
+    eye = np.broadcast_to(np.eye(4, dtype=np.float32), (B, N, 4, 4))
+    c = np.ones((N, D // 2), np.float32)
+    s = np.zeros((N, D // 2), np.float32)
+    qo, ko, vo, infl = O.ucpe_cam_prep(q, k, v, eye, eye, c, s, 0.25)
+    t = (0, 2, 3, 1)
+    xq, xk = O.bf16_to_f64(q), O.bf16_to_f64(k)
+    assert np.array_equal(qo, _bf16_value_bits(np.maximum(xq, 0)).transpose(t))
+    assert np.array_equal(ko, _bf16_value_bits(0.25 * np.maximum(xk, 0)).transpose(t))
+    assert np.array_equal(vo, v.transpose(t))
+    assert np.array_equal(infl, np.ones((B, H, N)))
+
+
+def pin_ucpe_projection_orientation():
+    """Permutation matrices move channels inside each block of four (U3):
+    with y_i = sum_j M[i][j] x_j, row i of M having its 1 in column p(i) gives
+    y_i = x_p(i). proj_q uses the 3-cycle p = (1, 2, 0, 3), proj_kv p = (3, 1,
+    0, 2); neither equals its own transpose, and they differ from each other,
+    so a transposed matrix or a swapped Q/KV matrix moves the wrong channel.
+    Positive inputs and zero angles keep every value exact."""
+    B, N, H, D = 1, 3, 2, 12
+    rng = np.random.default_rng(7)
+    q, k, v = (_bf16_bits(np.abs(rng.standard_normal((B, N, H, D))) + 0.1) for _ in range(3))
+    pq_map, pkv_map = (1, 2, 0, 3), (3, 1, 0, 2)
+    mq = np.zeros((4, 4), np.float32)
+    mkv = np.zeros((4, 4), np.float32)
+    for i in range(4):
+        mq[i, pq_map[i]] = 1.0
+        mkv[i, pkv_map[i]] = 1.0
+    c = np.ones((N, D // 2), np.float32)
+    s = np.zeros((N, D // 2), np.float32)
+    qo, ko, vo, infl = O.ucpe_cam_prep(q, k, v, np.broadcast_to(mq, (B, N, 4, 4)),
+                                       np.broadcast_to(mkv, (B, N, 4, 4)), c, s, 1.0)
+    perm_q = np.array([4 * (d // 4) + pq_map[d % 4] for d in range(D)])
+    perm_kv = np.array([4 * (d // 4) + pkv_map[d % 4] for d in range(D)])
+    t = (0, 2, 3, 1)
+    assert np.array_equal(qo, q[..., perm_q].transpose(t))
+    assert np.array_equal(ko, k[..., perm_kv].transpose(t))
+    assert np.array_equal(vo, v[..., perm_kv].transpose(t))
+    assert np.allclose(infl, 1.0, rtol=0, atol=1e-15)
+
+
+def pin_ucpe_hand_case():
+    """One head of four channels, two tokens, worked by hand (k_scale 0.25).
+    Token 0, angles 90 deg (pair 0: cos 0, sin 1) and 180 deg (pair 1):
+      q = (1, -2, 3, 0.5): ReLU (1, 0, 3, 0.5); proj_q rows (1,0,0,0),
+        (2,1,0,0), (0,0,1,0), (0,0,-1,2) give (1, 2, 3, -2); rotation:
+        pair (1, 2) -> (1*0 - 2*1, 2*0 + 1*1) = (-2, 1); pair (3, -2) ->
+        (-3, 2). q_trans = (-2, 1, -3, 2).
+      k = (-1, 4, 2, 2): ReLU and scale (0, 1, 0.5, 0.5); proj_kv rows
+        (0,1,0,0), (0,0,1,0), (1,0,0,0), (0,0,0,3) give (1, 0.5, 0, 1.5);
+        |k'|^2 = 1.5, |y|^2 = 3.5, inflation_sq = 7/3; rotation: (1, 0.5) ->
+        (-0.5, 1), (0, 1.5) -> (0, -1.5). k_trans = (-0.5, 1, 0, -1.5).
+      v = (1, 2, 3, 4): proj_kv gives (2, 3, 1, 12), not rotated.
+    Token 1, identity matrices, pair 0 at cos 0.6, sin 0.8 (as float32),
+    pair 1 at 0 deg:
+      q = (2, 1, -1, 1): ReLU (2, 1, 0, 1); pair (2, 1) -> (2*0.6 - 0.8,
+        1*0.6 + 2*0.8) = (0.4, 2.2); q_trans = (0.4, 2.2, 0, 1).
+      k = (1, 1, 1, 1): k' = 0.25 each, inflation_sq = 1; pair 0 ->
+        (0.25*0.6 - 0.25*0.8, 0.25*0.6 + 0.25*0.8) = (-0.05, 0.35);
+        k_trans = (-0.05, 0.35, 0.25, 0.25).
+      v = (-1, 0, 5, 7) unchanged."""
+    q = _bf16_bits([[[[1, -2, 3, 0.5]], [[2, 1, -1, 1]]]])
+    k = _bf16_bits([[[[-1, 4, 2, 2]], [[1, 1, 1, 1]]]])
+    v = _bf16_bits([[[[1, 2, 3, 4]], [[-1, 0, 5, 7]]]])
+    eye = np.eye(4, dtype=np.float32)
+    pq = np.stack([np.array([[1, 0, 0, 0], [2, 1, 0, 0], [0, 0, 1, 0], [0, 0, -1, 2]],
+                            np.float32), eye])[None]
+    pkv = np.stack([np.array([[0, 1, 0, 0], [0, 0, 1, 0], [1, 0, 0, 0], [0, 0, 0, 3]],
+                             np.float32), eye])[None]
+    c = np.array([[0, -1], [0.6, 1]], np.float32)
+    s = np.array([[1, 0], [0.8, 0]], np.float32)
+    qo, ko, vo, infl = O.ucpe_cam_prep(q, k, v, pq, pkv, c, s, 0.25, exact=True)
+    c06, s08 = float(np.float32(0.6)), float(np.float32(0.8))
+    want_q = [[-2, 1, -3, 2], [2 * c06 - s08, 1 * c06 + 2 * s08, 0, 1]]
+    want_k = [[-0.5, 1, 0, -1.5], [0.25 * (c06 - s08), 0.25 * (c06 + s08), 0.25, 0.25]]
+    want_v = [[2, 3, 1, 12], [-1, 0, 5, 7]]
+    for got, want in ((qo, want_q), (ko, want_k), (vo, want_v)):
+        assert got.shape == (1, 1, 4, 2)
+        assert np.allclose(got[0, 0].T, want, rtol=1e-15, atol=1e-15), (got[0, 0].T, want)
+    assert np.allclose(infl[0, 0], [7 / 3, 1.0], rtol=1e-15, atol=0)
+    # rounded: token 1 of q is (0.4, 2.2, 0, 1) to bf16's precision
+    qr = O.ucpe_cam_prep(q, k, v, pq, pkv, c, s, 0.25)[0]
+    assert np.array_equal(O.bf16_to_f64(qr[0, 0, :, 1]),
+                          O.bf16_to_f64(_bf16_bits([0.4, 2.2, 0.0, 1.0])))
+
+
+def _random_rotation4(rng):
+    m, r = np.linalg.qr(rng.standard_normal((4, 4)))
+    return m * np.sign(np.diag(r))
+
+
+def pin_ucpe_orthogonal_geometry_keeps_norms():
+    """Orthogonal ray projections and rotations keep the Euclidean norm of
+    every (token, head) vector: |q_trans| = |ReLU(q)|, |k_trans| = k_scale *
+    |ReLU(k)|, |v_trans| = |v|, and inflation_sq = 1. The float32 matrices and
+    cos/sin are orthogonal only to about 1e-7, hence the tolerance."""
+    B, N, H, D = 2, 4, 3, 16
+    rng = np.random.default_rng(11)
+    q, k, v = _ucpe_inputs(B, N, H, D, rng)
+    pq = np.stack([[_random_rotation4(rng) for _ in range(N)] for _ in range(B)]).astype(np.float32)
+    pkv = np.stack([[_random_rotation4(rng) for _ in range(N)] for _ in range(B)]).astype(np.float32)
+    th = rng.uniform(-np.pi, np.pi, (N, D // 2))
+    c, s = np.cos(th).astype(np.float32), np.sin(th).astype(np.float32)
+    qo, ko, vo, infl = O.ucpe_cam_prep(q, k, v, pq, pkv, c, s, 0.3, exact=True)
+    t = (0, 2, 3, 1)
+    for got, x in ((qo, np.maximum(O.bf16_to_f64(q), 0)),
+                   (ko, 0.3 * np.maximum(O.bf16_to_f64(k), 0)),
+                   (vo, O.bf16_to_f64(v))):
+        want = np.linalg.norm(x.transpose(t), axis=2)
+        assert np.allclose(np.linalg.norm(got, axis=2), want, rtol=1e-6, atol=1e-12)
+    assert np.allclose(infl, 1.0, rtol=0, atol=1e-6)
+
+
+def pin_ucpe_scaled_identity_inflation():
+    """proj_kv = c_n * I multiplies every key by c_n, so inflation_sq = c_n^2
+    for every head (U6), whatever proj_q is; a key whose ReLU is all zero has
+    inflation_sq = 1."""
+    B, N, H, D = 1, 6, 2, 8
+    rng = np.random.default_rng(5)
+    q, k, v = _ucpe_inputs(B, N, H, D, rng)
+    k = k.copy()
+    k[0, 2, 1] = _bf16_bits(-np.abs(rng.standard_normal(D)) - 0.5)  # ReLU(k) = 0 here
+    cn = np.arange(1, N + 1, dtype=np.float32) * 0.5
+    pkv = (cn[:, None, None] * np.eye(4, dtype=np.float32))[None]
+    pq = np.stack([_random_rotation4(rng) * 3 for _ in range(N)]).astype(np.float32)[None]
+    th = rng.uniform(-np.pi, np.pi, (N, D // 2))
+    c, s = np.cos(th).astype(np.float32), np.sin(th).astype(np.float32)
+    _, _, _, infl = O.ucpe_cam_prep(q, k, v, pq, pkv, c, s, 0.7, exact=True)
+    want = np.broadcast_to((cn.astype(np.float64) ** 2)[None, None, :], (B, H, N)).copy()
+    want[0, 1, 2] = 1.0
+    assert np.allclose(infl, want, rtol=1e-14, atol=0)
+
+
+def pin_ucpe_complex_brute_force():
+    """Random everything, checked against a restatement in other terms: the
+    projection as a batched matrix product over blocks (numpy einsum), the
+    rotation as multiplication of z_j = y_2j + i y_2j+1 by cos_j + i sin_j
+    (numpy complex128), the layout by transposing the result."""
+    B, N, H, D = 2, 3, 2, 12
+    rng = np.random.default_rng(3)
+    q, k, v = _ucpe_inputs(B, N, H, D, rng)
+    pq = rng.standard_normal((B, N, 4, 4)).astype(np.float32)
+    pkv = rng.standard_normal((B, N, 4, 4)).astype(np.float32)
+    th = rng.uniform(-np.pi, np.pi, (N, D // 2))
+    c, s = np.cos(th).astype(np.float32), np.sin(th).astype(np.float32)
+    ks = 0.37
+    qo, ko, vo, infl = O.ucpe_cam_prep(q, k, v, pq, pkv, c, s, ks, exact=True)
+
+    def project(m, x):  # x [B,N,H,D], m [B,N,4,4]
+        blocks = x.reshape(B, N, H, D // 4, 4)
+        return np.einsum("bnij,bnhcj->bnhci", m.astype(np.float64), blocks).reshape(B, N, H, D)
+
+    def rope(y):
+        z = (y[..., 0::2] + 1j * y[..., 1::2]) * (c + 1j * s).astype(np.complex128)[None, :, None]
+        out = np.empty_like(y)
+        out[..., 0::2], out[..., 1::2] = z.real, z.imag
+        return out
+
+    xq, xk, xv = (O.bf16_to_f64(a) for a in (q, k, v))
+    kk = ks * np.maximum(xk, 0)
+    yk = project(pkv, kk)
+    t = (0, 2, 3, 1)
+    assert np.allclose(qo, rope(project(pq, np.maximum(xq, 0))).transpose(t), rtol=1e-12,
+                       atol=1e-12)
+    assert np.allclose(ko, rope(yk).transpose(t), rtol=1e-12, atol=1e-12)
+    assert np.allclose(vo, project(pkv, xv).transpose(t), rtol=1e-12, atol=1e-12)
+    want = np.where((kk ** 2).sum(-1) > 0, (yk ** 2).sum(-1) / np.maximum((kk ** 2).sum(-1), 1e-300), 1.0)
+    assert np.allclose(infl, want.transpose(0, 2, 1), rtol=1e-12, atol=0)
+
+
+def pin_ucpe_f16_activations():
+    """binary16 activations (as R13): the same steps on binary16 inputs, each
+    result rounded once to binary16; identity geometry and a power-of-two
+    k_scale keep every value exact, so the results are the inputs' ReLU (and
+    scale) in binary16, checked against numpy's float16 conversion."""
+    B, N, H, D = 1, 3, 2, 8
+    rng = np.random.default_rng(9)
+    xs = [rng.standard_normal((B, N, H, D)).astype(np.float16) for _ in range(3)]
+    q, k, v = (x.view(np.uint16) for x in xs)
+    eye = np.broadcast_to(np.eye(4, dtype=np.float32), (B, N, 4, 4))
+    c = np.ones((N, D // 2), np.float32)
+    s = np.zeros((N, D // 2), np.float32)
+    qo, ko, vo, _ = O.ucpe_cam_prep(q, k, v, eye, eye, c, s, 2.0, act="f16")
+    t = (0, 2, 3, 1)
+    assert np.array_equal(qo, np.maximum(xs[0], 0).astype(np.float16).view(np.uint16).transpose(t))
+    assert np.array_equal(ko, (2 * np.maximum(xs[1], 0)).astype(np.float16).view(np.uint16).transpose(t))
+    assert np.array_equal(vo, v.transpose(t))
 
 
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_") and callable(v)]
