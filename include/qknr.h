@@ -10,6 +10,12 @@
  *   qknr_rope_3d     -- "flashinfer.norm.fused_qk_rmsnorm_rope" (FlashInfer
  *                       API docs): summary, Parameters, Returns.
  *
+ * and the camera-branch transform that runs beside them in the same block:
+ *
+ *   qknr_ucpe_cam_prep -- "vllm_omni.diffusion.models.sana_wm.ucpe"
+ *                       (vLLM-Omni API docs): cam_prep_func, its
+ *                       description, Parameters and Returns.
+ *
  * Common rules
  *   - Pointers are plain addresses that the current CUDA device can read or
  *     write: device memory of that device, managed memory, or page-locked host
@@ -43,7 +49,7 @@
 extern "C" {
 #endif
 
-#define QKNR_ABI_VERSION 2
+#define QKNR_ABI_VERSION 3
 
 typedef enum {
     QKNR_OK = 0,
@@ -200,6 +206,53 @@ int qknr_rope_3d_partial_ssq(const qknr_rope_3d_params* params, float* ssq_out,
                              void* cuda_stream);
 int qknr_rope_3d_with_ssq(const qknr_rope_3d_params* params, const float* ssq,
                           int32_t heads_q_total, int32_t heads_k_total, void* cuda_stream);
+
+/*
+ * UCPE camera prep ("vllm_omni.diffusion.models.sana_wm.ucpe": cam_prep_func).
+ * The page lists the steps (ReLU, the K scale, the ray projection, RoPE) and
+ * the shapes but no formula; the readings taken are these. For batch b, token
+ * n, head h, with x the head_dim channels of that (b, n, h):
+ *   Q: x' = max(x, 0); y = proj_q[b][n] applied to every block of four
+ *      channels, y[4i'+i] = sum_j M[i][j] x'[4i'+j] (M row-major);
+ *      out[2j]   = y[2j] c_j - y[2j+1] s_j,
+ *      out[2j+1] = y[2j+1] c_j + y[2j] s_j,
+ *      c_j = rope_cos[n][j], s_j = rope_sin[n][j], j < head_dim/2.
+ *   K: k' = k_scale * max(x, 0); y = proj_kv[b][n] blockwise; rotated as Q.
+ *      inflation_sq[b][h][n] = |y|^2 / |k'|^2, or 1 when k' is all zero.
+ *   V: y = proj_kv[b][n] blockwise, not rotated.
+ *   Outputs are stored transposed: q_trans[b][h][d][n] = out[d], likewise
+ *   k_trans and v_trans; each value rounded once to act_dtype.
+ * The definition of inflation_sq is not on the page (it names the output
+ * only); this squared-norm gain of the key is a reading, as is which tensors
+ * take ReLU and RoPE.
+ *
+ * act_dtype        QKNR_DT_BF16 or QKNR_DT_F16: q_normed, k_normed, v_raw and
+ *                  the three outputs.
+ * q_normed, k_normed, v_raw  [batch, num_tokens, num_heads, head_dim], dense,
+ *                  read only (Q and K already RMS-normalised by the caller).
+ * proj_q, proj_kv  float32 [batch, num_tokens, 4, 4], dense, row-major.
+ * rope_cos, rope_sin  float32 [num_tokens, head_dim/2], dense, shared by the
+ *                  batch.
+ * q_trans, k_trans, v_trans  act_dtype [batch, num_heads, head_dim, num_tokens],
+ *                  dense; written only. None may overlap an input or another
+ *                  output (QKNR_ERR_ALIAS).
+ * inflation_sq     float32 [batch, num_heads, num_tokens], or NULL to skip it.
+ * head_dim         a multiple of 8 from 8 to 256; batch, num_tokens,
+ *                  num_heads >= 0 (any of them 0: a no-op).
+ * k_scale          any finite float (the page's value is
+ *                  head_dim^-0.5 * spatial_tokens^-0.5).
+ * Alignment: every pointer 16-byte aligned (QKNR_ERR_ALIGN otherwise).
+ * num_tokens that is not a multiple of 8 is allowed; the output rows then
+ * are not 16-byte aligned and are written two bytes at a time.
+ * Range: |k'|^2 and |y|^2 are fp32 sums, so keys whose squares underflow
+ * fp32 (|k'| below about 1e-19) count as zero keys (inflation_sq 1).
+ */
+int qknr_ucpe_cam_prep(const void* q_normed, const void* k_normed, const void* v_raw,
+                       const float* proj_q, const float* proj_kv, const float* rope_cos,
+                       const float* rope_sin, void* q_trans, void* k_trans, void* v_trans,
+                       float* inflation_sq, int32_t act_dtype, int64_t batch,
+                       int64_t num_tokens, int32_t num_heads, int32_t head_dim, float k_scale,
+                       void* cuda_stream);
 
 /*
  * Device-side status of this library's kernels on the current device, for

@@ -6,8 +6,9 @@ tensors into pointers, sizes and a stream. There is no CPU or eager fallback:
 if libqknr.so is missing or cannot load, every call raises.
 
 Low-level names mirror the C entry points:
-  qknr_rope_table(...)  table-driven per-head form
-  qknr_rope_3d(...)     packed-QKV across-heads 3D form
+  qknr_rope_table(...)     table-driven per-head form
+  qknr_rope_3d(...)        packed-QKV across-heads 3D form
+  qknr_ucpe_cam_prep(...)  UCPE camera prep (ReLU, K scale, ray projection, RoPE)
 Page-shaped wrappers allocate missing outputs and return them:
   fused_qk_norm_rope(q, k, q_weight, k_weight, rope_table, eps, *, head_dim=None,
                      rotary_dim=None, interleaved=False) -> (q, k)
@@ -15,6 +16,9 @@ Page-shaped wrappers allocate missing outputs and return them:
   fused_qk_rmsnorm_rope(qkv, q_weight, k_weight, *, ppf, pph, ppw, ...,
                         q_out=None, k_out=None, v_out=None) -> (q, k, v)
       ("flashinfer.norm.fused_qk_rmsnorm_rope", Parameters / Returns)
+  cam_prep_func(q_normed, k_normed, v_raw, *, proj_q, proj_kv, rope_cos, rope_sin,
+                k_scale) -> (q_trans, k_trans, v_trans, inflation_sq)
+      ("vllm_omni.diffusion.models.sana_wm.ucpe", cam_prep_func)
 """
 from __future__ import annotations
 
@@ -30,10 +34,10 @@ LIB_PATH = os.path.join(_PKG, "libqknr.so")
 QKNR_OK, QKNR_ERR_NULL, QKNR_ERR_SHAPE, QKNR_ERR_UNSUPPORTED = 0, 1, 2, 3
 QKNR_ERR_ALIGN, QKNR_ERR_ALIAS, QKNR_ERR_POINTER, QKNR_ERR_CUDA = 4, 5, 6, 7
 QKNR_DT_BF16, QKNR_DT_F32, QKNR_DT_E4M3, QKNR_DT_F16 = 0, 1, 2, 3
-ABI_VERSION = 2  # QKNR_ABI_VERSION the argument lists below are written for
+ABI_VERSION = 3  # QKNR_ABI_VERSION the argument lists below are written for
 
 EXPORTS = ("qknr_rope_table", "qknr_rope_3d", "qknr_rope_3d_partial_ssq", "qknr_rope_3d_with_ssq",
-           "qknr_device_status", "qknr_test_set_wait_fault", "qknr_status_string",
+           "qknr_ucpe_cam_prep", "qknr_device_status", "qknr_test_set_wait_fault", "qknr_status_string",
            "qknr_last_error_detail", "qknr_abi_version")
 
 
@@ -83,6 +87,9 @@ def lib() -> C.CDLL:
         L.qknr_rope_3d_partial_ssq.restype = C.c_int
         L.qknr_rope_3d_with_ssq.argtypes = [C.POINTER(Rope3DParams), vp, i32, i32, vp]
         L.qknr_rope_3d_with_ssq.restype = C.c_int
+        L.qknr_ucpe_cam_prep.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64,
+                                         i64, i32, i32, C.c_float, vp]
+        L.qknr_ucpe_cam_prep.restype = C.c_int
         L.qknr_status_string.argtypes = [C.c_int]
         L.qknr_status_string.restype = C.c_char_p
         L.qknr_last_error_detail.restype = C.c_char_p
@@ -271,6 +278,42 @@ def qknr_rope_3d_with_ssq(qkv, q_weight, k_weight, q_out, k_out, v_out, ssq, *, 
                                        int(heads_k_total), _stream(stream, qkv, q_out)))
 
 
+def qknr_ucpe_cam_prep(q_normed, k_normed, v_raw, proj_q, proj_kv, rope_cos, rope_sin, q_trans,
+                       k_trans, v_trans, inflation_sq, *, k_scale: float, stream=None) -> None:
+    """UCPE camera prep through the C ABI (destination passing; see
+    include/qknr.h). q_normed/k_normed/v_raw dense [B, N, H, D] bf16 or float16;
+    proj_q/proj_kv dense fp32 [B, N, 4, 4]; rope_cos/rope_sin dense fp32
+    [N, D/2]; outputs dense [B, H, D, N] of the activation dtype; inflation_sq
+    dense fp32 [B, H, N] or None."""
+    if q_normed.dim() != 4:
+        raise QknrValueError(QKNR_ERR_SHAPE, "q_normed must be [B, N, H, D]")
+    act = _act_dtype(q_normed)
+    B, N, H, D = q_normed.shape
+    for n, t in (("k_normed", k_normed), ("v_raw", v_raw)):
+        if tuple(t.shape) != (B, N, H, D) or t.dtype != q_normed.dtype:
+            raise QknrValueError(QKNR_ERR_SHAPE, f"{n} must match q_normed's shape and dtype")
+    for n, t, shape, dt in (("q_normed", q_normed, (B, N, H, D), q_normed.dtype),
+                            ("k_normed", k_normed, (B, N, H, D), q_normed.dtype),
+                            ("v_raw", v_raw, (B, N, H, D), q_normed.dtype),
+                            ("proj_q", proj_q, (B, N, 4, 4), torch.float32),
+                            ("proj_kv", proj_kv, (B, N, 4, 4), torch.float32),
+                            ("rope_cos", rope_cos, (N, D // 2), torch.float32),
+                            ("rope_sin", rope_sin, (N, D // 2), torch.float32),
+                            ("q_trans", q_trans, (B, H, D, N), q_normed.dtype),
+                            ("k_trans", k_trans, (B, H, D, N), q_normed.dtype),
+                            ("v_trans", v_trans, (B, H, D, N), q_normed.dtype),
+                            ("inflation_sq", inflation_sq, (B, H, N), torch.float32)):
+        if t is None and n == "inflation_sq":
+            continue
+        if tuple(t.shape) != shape or t.dtype != dt or not t.is_contiguous():
+            raise QknrValueError(QKNR_ERR_SHAPE, f"{n} must be a dense {dt} tensor {list(shape)}")
+    st = _stream(stream, q_normed, q_trans)
+    _check(lib().qknr_ucpe_cam_prep(_ptr(q_normed), _ptr(k_normed), _ptr(v_raw), _ptr(proj_q),
+                                    _ptr(proj_kv), _ptr(rope_cos), _ptr(rope_sin),
+                                    _ptr(q_trans), _ptr(k_trans), _ptr(v_trans),
+                                    _ptr(inflation_sq), act, B, N, H, D, float(k_scale), st))
+
+
 def qknr_device_status(clear: bool = False, stream=None, device=None) -> int:
     """Device status word (bit 0: a kernel gave up waiting on its own bulk
     copy and left its outputs incomplete). Synchronises the stream."""
@@ -335,7 +378,26 @@ def fused_qk_rmsnorm_rope(qkv: torch.Tensor, q_weight: torch.Tensor, k_weight: t
     return tuple(outs)
 
 
+def cam_prep_func(q_normed: torch.Tensor, k_normed: torch.Tensor, v_raw: torch.Tensor, *,
+                  proj_q: torch.Tensor, proj_kv: torch.Tensor, rope_cos: torch.Tensor,
+                  rope_sin: torch.Tensor, k_scale: float, stream=None
+                  ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
+    """UCPE camera prep: ReLU, the K scale, the 4x4 ray projections and
+    adjacent-pair RoPE of camera Q/K (projection only for V), from [B, N, H, D]
+    inputs. Returns q_trans, k_trans, v_trans [B, H, D, N] (the inputs' dtype)
+    and inflation_sq [B, H, N] float32, the squared-norm gain of each key under
+    its projection."""
+    B, N, H, D = q_normed.shape
+    outs = [torch.empty((B, H, D, N), dtype=q_normed.dtype, device=q_normed.device)
+            for _ in range(3)]
+    infl = torch.empty((B, H, N), dtype=torch.float32, device=q_normed.device)
+    qknr_ucpe_cam_prep(q_normed, k_normed, v_raw, proj_q, proj_kv, rope_cos, rope_sin, *outs,
+                       infl, k_scale=k_scale, stream=stream)
+    return outs[0], outs[1], outs[2], infl
+
+
 __all__ = ["qknr_rope_table", "qknr_rope_3d", "qknr_rope_3d_partial_ssq", "qknr_rope_3d_with_ssq",
+           "qknr_ucpe_cam_prep", "cam_prep_func",
            "qknr_device_status", "fused_qk_norm_rope", "fused_qk_rmsnorm_rope",
            "QknrError", "QknrValueError", "lib", "build", "make_3d_params", "Rope3DParams",
            "EXPORTS", "LIB_PATH"]

@@ -458,6 +458,91 @@ int run_3d(const qknr_rope_3d_params* prm, int mode, float* ssq_out, const float
 
 extern "C" {
 
+int qknr_ucpe_cam_prep(const void* q_normed, const void* k_normed, const void* v_raw,
+                       const float* proj_q, const float* proj_kv, const float* rope_cos,
+                       const float* rope_sin, void* q_trans, void* k_trans, void* v_trans,
+                       float* inflation_sq, int32_t act_dtype, int64_t batch,
+                       int64_t num_tokens, int32_t num_heads, int32_t head_dim, float k_scale,
+                       void* cuda_stream) {
+    // ---- shape checks (host only) ----
+    if (batch < 0 || num_tokens < 0 || num_heads < 0)
+        return fail(QKNR_ERR_SHAPE, "batch, num_tokens and num_heads must be >= 0");
+    if (head_dim < 8 || head_dim > 256 || head_dim % 8 != 0)
+        return fail(QKNR_ERR_SHAPE, "head_dim %d must be a multiple of 8 from 8 to 256",
+                    head_dim);
+    if (act_dtype != QKNR_DT_BF16 && act_dtype != QKNR_DT_F16)
+        return fail(QKNR_ERR_SHAPE, "activation dtype must be bfloat16 or float16");
+    if (!std::isfinite(k_scale)) return fail(QKNR_ERR_SHAPE, "k_scale must be finite");
+    // Element counts must fit int64 comfortably (the kernel indexes in int64).
+    const int64_t kLimit = (int64_t)1 << 50;
+    if (batch > 0 && num_tokens > 0 && num_heads > 0 &&
+        (double)batch * (double)num_tokens * (double)num_heads * (double)head_dim > (double)kLimit)
+        return fail(QKNR_ERR_SHAPE, "tensor too large");
+    if (batch == 0 || num_tokens == 0 || num_heads == 0) return ok();
+
+    // ---- pointers ----
+    if (!q_normed || !k_normed || !v_raw) return fail(QKNR_ERR_NULL, "q_normed, k_normed or v_raw is NULL");
+    if (!proj_q || !proj_kv) return fail(QKNR_ERR_NULL, "proj_q or proj_kv is NULL");
+    if (!rope_cos || !rope_sin) return fail(QKNR_ERR_NULL, "rope_cos or rope_sin is NULL");
+    if (!q_trans || !k_trans || !v_trans) return fail(QKNR_ERR_NULL, "q_trans, k_trans or v_trans is NULL");
+    const void* all[] = {q_normed, k_normed, v_raw, proj_q, proj_kv, rope_cos, rope_sin,
+                         q_trans, k_trans, v_trans, inflation_sq};
+    for (const void* ptr : all)
+        if (ptr && !aligned16(ptr)) return fail(QKNR_ERR_ALIGN, "a pointer is not 16-byte aligned");
+    const uint64_t act_bytes = (uint64_t)batch * num_tokens * num_heads * head_dim * 2;
+    const uint64_t proj_bytes = (uint64_t)batch * num_tokens * 64;
+    const uint64_t rope_bytes = (uint64_t)num_tokens * (head_dim / 2) * 4;
+    const Span ins[] = {{q_normed, act_bytes}, {k_normed, act_bytes}, {v_raw, act_bytes},
+                        {proj_q, proj_bytes},  {proj_kv, proj_bytes}, {rope_cos, rope_bytes},
+                        {rope_sin, rope_bytes}};
+    const Span outs[] = {{q_trans, act_bytes},
+                         {k_trans, act_bytes},
+                         {v_trans, act_bytes},
+                         {inflation_sq, (uint64_t)batch * num_heads * num_tokens * 4}};
+    for (int i = 0; i < 4; ++i) {
+        for (const Span& in : ins)
+            if (overlap(outs[i], in)) return fail(QKNR_ERR_ALIAS, "an output overlaps an input");
+        for (int j = 0; j < i; ++j)
+            if (overlap(outs[i], outs[j])) return fail(QKNR_ERR_ALIAS, "two outputs overlap");
+    }
+
+    // ---- device access ----
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    const char* names[] = {"q_normed", "k_normed", "v_raw", "proj_q", "proj_kv", "rope_cos",
+                           "rope_sin", "q_trans", "k_trans", "v_trans", "inflation_sq"};
+    const void* dp[11] = {};
+    for (int i = 0; i < 11; ++i) {
+        if (!all[i]) continue;
+        int rc = classify(all[i], names[i], dev, &dp[i]);
+        if (rc) return rc;
+        if (!aligned16(dp[i])) return fail(QKNR_ERR_ALIGN, "%s: device address not 16-byte aligned", names[i]);
+    }
+    qknr::UcpeArgs a{};
+    a.q = static_cast<const uint8_t*>(dp[0]);
+    a.k = static_cast<const uint8_t*>(dp[1]);
+    a.v = static_cast<const uint8_t*>(dp[2]);
+    a.proj_q = static_cast<const float*>(dp[3]);
+    a.proj_kv = static_cast<const float*>(dp[4]);
+    a.rope_cos = static_cast<const float*>(dp[5]);
+    a.rope_sin = static_cast<const float*>(dp[6]);
+    a.q_out = static_cast<uint8_t*>(const_cast<void*>(dp[7]));
+    a.k_out = static_cast<uint8_t*>(const_cast<void*>(dp[8]));
+    a.v_out = static_cast<uint8_t*>(const_cast<void*>(dp[9]));
+    a.inflation_sq = static_cast<float*>(const_cast<void*>(dp[10]));
+    a.batch = batch;
+    a.num_tokens = num_tokens;
+    a.heads = num_heads;
+    a.head_dim = head_dim;
+    a.act_f16 = act_dtype == QKNR_DT_F16;
+    a.k_scale = k_scale;
+    qknr::LaunchInfo info{};
+    e = qknr::launch_ucpe(a, static_cast<cudaStream_t>(cuda_stream), &info);
+    if (e != cudaSuccess) return cuda_fail(e, "camera prep kernel launch");
+    return ok();
+}
+
 int qknr_rope_3d(const qknr_rope_3d_params* prm, void* cuda_stream) {
     return run_3d(prm, qknr::kModeWhole, nullptr, nullptr, 0, 0, cuda_stream);
 }

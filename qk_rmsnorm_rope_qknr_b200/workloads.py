@@ -1,4 +1,5 @@
-"""Seeded synthetic inputs for the fused Q/K RMSNorm + RoPE workloads.
+"""Seeded synthetic inputs for the fused Q/K RMSNorm + RoPE workloads and the
+UCPE camera prep.
 
 This module only draws inputs (and counts their bytes); it holds none of the
 transform's arithmetic, and both the CUDA path and the oracle consume the very
@@ -21,6 +22,11 @@ video-DiT and MiniMax-H3 geometries the pages name):
               32/48/48, NeoX pairs, E4M3 out (scales 0.5 / 0.25)
   fp8neox_nonorm  fp8neox with is_qk_norm=False
   gqa3d       video3d's geometry with grouped-query heads 32+8+8 (parity and TP case)
+  ucpe        UCPE camera prep: camera Q, K, V [1, 18480, 20, 112] ~N(0,1) (the SANA-WM
+              page's 18480-token ray grid, taken as 21 latent frames of 22x40 tokens;
+              20 heads of 112, a 2240-wide model, are not on the page), per-token rigid
+              motions G as proj_q = G^T and proj_kv = G^-1, cos/sin of
+              n * 10000^(-2j/112), k_scale = 112^-0.5 * 880^-0.5
 """
 from __future__ import annotations
 
@@ -101,6 +107,34 @@ class FormTable:
         return torch.float16 if self.act == "f16" else torch.bfloat16
 
 
+@dataclasses.dataclass(frozen=True)
+class FormUcpe:
+    name: str
+    batch: int
+    seq: int       # tokens N of the ray grid (latent frames x spatial tokens)
+    heads: int
+    head_dim: int
+    spatial: int   # tokens per latent frame (the spatial_tokens of k_scale)
+    rope_base: float = 10000.0
+    std: float = 1.0
+    translation_std: float = 0.5
+    seed: int = 0
+    act: str = "bf16"
+    form: str = "ucpe"
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seq
+
+    @property
+    def k_scale(self) -> float:
+        return self.head_dim ** -0.5 * self.spatial ** -0.5
+
+    @property
+    def act_dtype(self) -> torch.dtype:
+        return torch.float16 if self.act == "f16" else torch.bfloat16
+
+
 WORKLOADS = {
     "tiny3d": Form3D("tiny3d", batch=1, seq=32, ppf=2, pph=4, ppw=4, cf=16, ch=24, cw=24, hq=4,
                      hk=4, hv=4, head_dim=64, input_2d=True),
@@ -124,6 +158,7 @@ WORKLOADS = {
                              cf=32, ch=48, cw=48, hq=24, hk=24, hv=24, head_dim=128,
                              interleave=False, is_qk_norm=False, output_fp8=True, q_scale=0.5,
                              v_scale=0.25, std=2.0),
+    "ucpe": FormUcpe("ucpe", batch=1, seq=18480, heads=20, head_dim=112, spatial=880),
 }
 
 
@@ -153,6 +188,38 @@ def rope_table_input(tokens: int, rotary_dim: int, base: float, f32: bool,
     return tbl.to(torch.float32 if f32 else act).to(device)
 
 
+def camera_matrices(g: torch.Generator, batch: int, tokens: int, translation_std: float,
+                    device="cpu"):
+    """Per-token rigid motions G = [[R, t], [0, 1]]: R a random rotation (the Q
+    factor of a Gaussian 3x3 matrix, column signs fixed), t ~ N(0,
+    translation_std^2). Returns (G^T, G^-1) as float32 [batch, tokens, 4, 4]: the
+    Q and K/V matrices of a camera pair whose relative motion the attention
+    sees (inputs only: the camera prep multiplies by whatever it is given)."""
+    a = torch.randn((batch, tokens, 3, 3), generator=g, dtype=torch.float64, device=device)
+    rot, r = torch.linalg.qr(a)
+    rot = rot * torch.sign(torch.diagonal(r, dim1=-2, dim2=-1)).unsqueeze(-2)
+    t = torch.randn((batch, tokens, 3), generator=g, dtype=torch.float64, device=device)
+    t = t * translation_std
+    G = torch.zeros((batch, tokens, 4, 4), dtype=torch.float64, device=device)
+    G[..., :3, :3] = rot
+    G[..., :3, 3] = t
+    G[..., 3, 3] = 1.0
+    inv = torch.zeros_like(G)
+    inv[..., :3, :3] = rot.transpose(-1, -2)
+    inv[..., :3, 3] = -(rot.transpose(-1, -2) @ t.unsqueeze(-1)).squeeze(-1)
+    inv[..., 3, 3] = 1.0
+    return G.transpose(-1, -2).contiguous().float(), inv.float()
+
+
+def ucpe_rope_tables(tokens: int, head_dim: int, base: float, device="cpu"):
+    """cos and sin [tokens, head_dim/2] of theta[n, j] = n * base^(-2j/head_dim),
+    built in float64 and stored as float32 (the tables the camera prep reads)."""
+    pos = torch.arange(tokens, dtype=torch.float64).unsqueeze(1)
+    inv = base ** (-2.0 * torch.arange(head_dim // 2, dtype=torch.float64) / head_dim)
+    theta = pos * inv.unsqueeze(0)
+    return torch.cos(theta).float().to(device), torch.sin(theta).float().to(device)
+
+
 def make_inputs(w, device="cpu", tokens: Optional[int] = None, seed: Optional[int] = None):
     """Inputs of workload `w` (a Form3D / FormTable or its name) on `device`.
 
@@ -164,6 +231,14 @@ def make_inputs(w, device="cpu", tokens: Optional[int] = None, seed: Optional[in
         w = WORKLOADS[w]
     g = torch.Generator(device=device)
     g.manual_seed(w.seed if seed is None else seed)
+    if w.form == "ucpe":
+        N = w.seq if tokens is None else tokens
+        shape = (w.batch, N, w.heads, w.head_dim)
+        q, k, v = (_normal(g, shape, w.std, device, w.act_dtype) for _ in range(3))
+        pq, pkv = camera_matrices(g, w.batch, N, w.translation_std, device)
+        cos_t, sin_t = ucpe_rope_tables(N, w.head_dim, w.rope_base, device)
+        return dict(q_normed=q, k_normed=k, v_raw=v, proj_q=pq, proj_kv=pkv, rope_cos=cos_t,
+                    rope_sin=sin_t)
     if w.form == "3d":
         if tokens is None:
             shape = (w.seq, w.row) if w.input_2d else (w.batch, w.seq, w.row)
@@ -193,6 +268,12 @@ def algorithmic_bytes(w, tokens: Optional[int] = None) -> int:
     output written once, the weights (and table) read once."""
     if isinstance(w, str):
         w = WORKLOADS[w]
+    if w.form == "ucpe":
+        # tokens: the sequence length N (per batch element)
+        N = w.seq if tokens is None else tokens
+        per_tok_head = 3 * 2 * w.head_dim * 2 + 4   # q, k, v in and out; inflation_sq
+        return (w.batch * N * (w.heads * per_tok_head + 2 * 64)   # + proj_q, proj_kv
+                + N * w.head_dim * 4)                              # cos, sin [N, D/2] fp32
     if w.form == "3d":
         T = w.tokens if tokens is None else tokens
         out_b = 1 if w.output_fp8 else 2

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_strings(L):
-    assert L.qknr_abi_version() == Q.ABI_VERSION == 2
+    assert L.qknr_abi_version() == Q.ABI_VERSION == 3
     for s in range(8):
         assert L.qknr_status_string(s)
     assert L.qknr_status_string(0) == b"ok"
@@ -229,3 +229,64 @@ def test_tp_head_slices():
             sl = [tp.head_slice(total, world, r) for r in range(world)]
             assert sl[0][0] == 0 and sl[-1][1] == total
             assert all(a[1] == b[0] for a, b in zip(sl, sl[1:]))
+
+
+# ---------------------------------------------------------- UCPE camera prep --
+def _ucpe(L, **over):
+    kw = dict(q=A, k=A + (1 << 30), v=A + (2 << 30), pq=A + (3 << 30), pkv=A + (4 << 30),
+              cos=A + (5 << 30), sin=A + (6 << 30), qo=A + (7 << 30), ko=A + (8 << 30),
+              vo=A + (9 << 30), infl=A + (10 << 30), act=Q.QKNR_DT_BF16, B=1, N=64, H=2, D=112,
+              k_scale=0.1)
+    kw.update(over)
+    rc = L.qknr_ucpe_cam_prep(kw["q"], kw["k"], kw["v"], kw["pq"], kw["pkv"], kw["cos"],
+                              kw["sin"], kw["qo"], kw["ko"], kw["vo"], kw["infl"], kw["act"],
+                              kw["B"], kw["N"], kw["H"], kw["D"], kw["k_scale"], None)
+    return rc, L.qknr_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("over,code,needle", [
+    (dict(D=100), Q.QKNR_ERR_SHAPE, "multiple of 8"),
+    (dict(D=0), Q.QKNR_ERR_SHAPE, "multiple of 8"),
+    (dict(D=264), Q.QKNR_ERR_SHAPE, "multiple of 8"),
+    (dict(N=-1), Q.QKNR_ERR_SHAPE, ">= 0"),
+    (dict(act=Q.QKNR_DT_F32), Q.QKNR_ERR_SHAPE, "dtype"),
+    (dict(act=Q.QKNR_DT_E4M3), Q.QKNR_ERR_SHAPE, "dtype"),
+    (dict(k_scale=float("inf")), Q.QKNR_ERR_SHAPE, "k_scale"),
+    (dict(k_scale=float("nan")), Q.QKNR_ERR_SHAPE, "k_scale"),
+    (dict(B=1 << 20, N=1 << 20, H=64, D=256), Q.QKNR_ERR_SHAPE, "too large"),
+    (dict(q=None), Q.QKNR_ERR_NULL, "q_normed"),
+    (dict(pkv=None), Q.QKNR_ERR_NULL, "proj"),
+    (dict(sin=None), Q.QKNR_ERR_NULL, "rope"),
+    (dict(vo=None), Q.QKNR_ERR_NULL, "v_trans"),
+    (dict(k=A + (1 << 30) + 8), Q.QKNR_ERR_ALIGN, "16-byte"),
+    (dict(pq=A + (3 << 30) + 4), Q.QKNR_ERR_ALIGN, "16-byte"),
+    (dict(infl=A + (10 << 30) + 4), Q.QKNR_ERR_ALIGN, "16-byte"),
+    (dict(qo=A), Q.QKNR_ERR_ALIAS, "overlaps an input"),
+    (dict(ko=A + (7 << 30) + 16), Q.QKNR_ERR_ALIAS, "outputs overlap"),
+    (dict(infl=A + (6 << 30) + 64), Q.QKNR_ERR_ALIAS, "overlaps an input"),
+])
+def test_ucpe_host_validation(L, over, code, needle):
+    rc, detail = _ucpe(L, **over)
+    assert rc == code and needle in detail, (rc, detail)
+
+
+@pytest.mark.parametrize("over", [dict(B=0), dict(N=0), dict(H=0)])
+def test_ucpe_empty_is_a_no_op(L, over):
+    # nothing is launched, so the fake addresses are never used
+    assert _ucpe(L, **over) == (Q.QKNR_OK, "")
+
+
+def test_ucpe_binding_checks_shapes(L):
+    import torch
+    x = torch.zeros(1, 8, 2, 16, dtype=torch.bfloat16)
+    good = dict(proj_q=torch.zeros(1, 8, 4, 4), proj_kv=torch.zeros(1, 8, 4, 4),
+                rope_cos=torch.zeros(8, 8), rope_sin=torch.zeros(8, 8), k_scale=1.0)
+    with pytest.raises(Q.QknrValueError, match="rope_cos"):
+        Q.cam_prep_func(x, x, x, **dict(good, rope_cos=torch.zeros(8, 16)))
+    with pytest.raises(Q.QknrValueError, match="proj_kv"):
+        Q.cam_prep_func(x, x, x, **dict(good, proj_kv=torch.zeros(1, 8, 4, 4,
+                                                                  dtype=torch.float64)))
+    with pytest.raises(Q.QknrValueError, match="k_normed"):
+        Q.cam_prep_func(x, x.float(), x, **good)
+    with pytest.raises(Q.QknrValueError, match="bfloat16/float16"):
+        Q.cam_prep_func(x.float(), x.float(), x.float(), **good)

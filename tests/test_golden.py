@@ -47,7 +47,7 @@ def _bits(values, act="bf16") -> np.ndarray:
 
 
 def test_fixture_set_present():
-    assert len(FIXTURES) >= 6, FIXTURES
+    assert len(FIXTURES) >= 8, FIXTURES
 
 
 @pytest.mark.parametrize("ex", _load("worked_examples")["examples"],
@@ -80,6 +80,11 @@ def test_oracle_reproduces_stored_bits(name):
                         _unhex(inp["k_weight"]) if norm else None,
                         **dict(p, pos_offset=p["pos_offset"] or 0))
         names = ("q", "k", "v")
+    elif fx["form"] == "ucpe":
+        got = O.ucpe_cam_prep(*(_unhex(inp[n]) for n in ("q", "k", "v", "proj_q", "proj_kv",
+                                                          "rope_cos", "rope_sin")),
+                              p["k_scale"], act=p["act"])
+        names = ("q", "k", "v", "inflation_sq")
     else:
         tbl = _unhex(inp["rope_table"])
         got = O.rope_table(_unhex(inp["q"]), _unhex(inp["k"]), _unhex(inp["q_weight"]),
@@ -111,6 +116,21 @@ def test_cuda_path_matches_stored_bits(name):
         kw = dev(inp["k_weight"], torch.bfloat16) if norm else None
         outs = Q.fused_qk_rmsnorm_rope(qkv, qw, kw, **p)
         names = ("q", "k", "v")
+    elif fx["form"] == "ucpe":
+        act = torch.float16 if p["act"] == "f16" else torch.bfloat16
+        f32 = {n: torch.from_numpy(_unhex(inp[n]).copy()).cuda()
+               for n in ("proj_q", "proj_kv", "rope_cos", "rope_sin")}
+        outs = Q.cam_prep_func(dev(inp["q"], act), dev(inp["k"], act), dev(inp["v"], act),
+                               k_scale=p["k_scale"], **f32)
+        torch.cuda.synchronize()
+        want = _unhex(fx["expected"]["inflation_sq"])
+        np.testing.assert_allclose(outs[3].cpu().double().numpy(), want, rtol=2.0 ** -14, atol=0)
+        # the tolerance's rows are the head vectors: compare as [B, H, N, D]
+        outs = tuple(o.transpose(2, 3) for o in outs[:3])
+        fx = dict(fx, expected={n: dict(fx["expected"][n], hex=None,
+                                        arr=_unhex(fx["expected"][n]).transpose(0, 1, 3, 2))
+                                for n in ("q", "k", "v")})
+        names = ("q", "k", "v")
     else:
         act = torch.float16 if p["act"] == "f16" else torch.bfloat16
         tbl_np = _unhex(inp["rope_table"])
@@ -123,7 +143,8 @@ def test_cuda_path_matches_stored_bits(name):
         names = ("q", "k")
     torch.cuda.synchronize()
     for n, o in zip(names, outs):
-        want = _unhex(fx["expected"][n])
+        e = fx["expected"][n]
+        want = e["arr"] if "arr" in e else _unhex(e)
         got = o.cpu().contiguous()
         if want.dtype == np.uint8:
             bad, st = e4m3_mismatch(got.view(torch.uint8).numpy(), want)

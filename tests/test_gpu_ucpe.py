@@ -1,0 +1,207 @@
+"""UCPE camera prep ("vllm_omni.diffusion.models.sana_wm.ucpe", cam_prep_func):
+the CUDA path through the C ABI against the fp64 oracle, element by element.
+
+Tolerances:
+  q_trans, k_trans, v_trans: the table form's rule (tests/_util.py) on each
+      (token, head) vector of D channels: 2 ulp of the activation type at
+      max(|ref|, 2^-8 rms) for bf16 (2^-11 for binary16).
+  inflation_sq: relative 2^-14. The kernel forms |k'|^2 and |M k'|^2 as fp32
+      sums of D <= 256 terms (relative error below D * 2^-24 = 1.5e-5 each,
+      and far less for sums of this many positive terms), each y = M k' with
+      fp32 products (a few 2^-24 of |M| |k'|); a ratio of two such sums is good
+      to about 3e-5 in the worst case, so 2^-14 = 6.1e-5 bounds it while a
+      wrong definition (another tensor, another ratio) misses by orders of
+      magnitude.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import qk_rmsnorm_rope_qknr_b200 as Q
+from qk_rmsnorm_rope_qknr_b200 import workloads as W
+from tests._util import act_mismatch, t2u16
+
+pytestmark = pytest.mark.gpu
+
+INFL_RTOL = 2.0 ** -14
+
+
+def _case(B, N, H, D, act="bf16", seed=0, device="cuda"):
+    w = W.FormUcpe("case", batch=B, seq=N, heads=H, head_dim=D, spatial=max(1, N // 4),
+                   seed=seed, act=act)
+    return w, W.make_inputs(w, device=device)
+
+
+def _oracle(inp, k_scale, act, exact=False):
+    def bits(t):
+        return t2u16(t)
+
+    return O.ucpe_cam_prep(bits(inp["q_normed"]), bits(inp["k_normed"]), bits(inp["v_raw"]),
+                           inp["proj_q"].cpu().numpy(), inp["proj_kv"].cpu().numpy(),
+                           inp["rope_cos"].cpu().numpy(), inp["rope_sin"].cpu().numpy(),
+                           k_scale, exact=exact, act=act)
+
+
+def _compare(outs, ref, ref_exact, act, where=""):
+    """outs: the four device results; ref/ref_exact: the oracle's rounded and
+    exact results. Output arrays are [B, H, D, N]; the tolerance's rows are the
+    D-vectors, so compare as [B, H, N, D]."""
+    for name, got, want, exact in zip(("q", "k", "v"), outs[:3], ref[:3], ref_exact[:3]):
+        g = t2u16(got).transpose(0, 1, 3, 2)
+        bad, st = act_mismatch(g, want.transpose(0, 1, 3, 2), exact.transpose(0, 1, 3, 2), act)
+        assert len(bad) == 0, f"{where} {name}_trans: {len(bad)} beyond tolerance {st}, first {bad[:3]}"
+    if outs[3] is not None:
+        g = outs[3].cpu().double().numpy()
+        np.testing.assert_allclose(g, ref[3], rtol=INFL_RTOL, atol=0, err_msg=f"{where} inflation_sq")
+
+
+CASES = [
+    # B, N, H, D, act: tiles of 64 tokens with ragged tails (N not a multiple
+    # of 64, and of 8: the two-byte store path), every chunk count parity
+    (1, 64, 1, 8, "bf16"),
+    (1, 200, 3, 16, "bf16"),
+    (2, 130, 2, 24, "bf16"),
+    (1, 301, 2, 64, "bf16"),
+    (2, 96, 3, 112, "bf16"),
+    (1, 77, 5, 112, "bf16"),
+    (1, 256, 2, 128, "bf16"),
+    (2, 72, 2, 200, "bf16"),
+    (1, 129, 2, 256, "bf16"),
+    (1, 150, 3, 112, "f16"),
+    (2, 64, 2, 40, "f16"),
+]
+
+
+@pytest.mark.parametrize("B,N,H,D,act", CASES)
+def test_ucpe_matches_oracle(B, N, H, D, act):
+    w, inp = _case(B, N, H, D, act, seed=B * 1000 + N + D)
+    outs = Q.cam_prep_func(inp["q_normed"], inp["k_normed"], inp["v_raw"], proj_q=inp["proj_q"],
+                           proj_kv=inp["proj_kv"], rope_cos=inp["rope_cos"],
+                           rope_sin=inp["rope_sin"], k_scale=w.k_scale)
+    torch.cuda.synchronize()
+    ref = _oracle(inp, w.k_scale, act)
+    ref_exact = _oracle(inp, w.k_scale, act, exact=True)
+    _compare(outs, ref, ref_exact, act, where=f"B{B} N{N} H{H} D{D} {act}")
+
+
+def test_ucpe_identity_geometry_is_exact():
+    """Identity matrices, zero angles and k_scale 0.5: every output is its
+    input's ReLU (and halving) moved to [B, H, D, N], exactly."""
+    B, N, H, D = 2, 100, 3, 32
+    _, inp = _case(B, N, H, D, seed=5)
+    eye = torch.eye(4, device="cuda").expand(B, N, 4, 4).contiguous()
+    c = torch.ones(N, D // 2, device="cuda")
+    s = torch.zeros(N, D // 2, device="cuda")
+    q, k, v, infl = Q.cam_prep_func(inp["q_normed"], inp["k_normed"], inp["v_raw"], proj_q=eye,
+                                    proj_kv=eye, rope_cos=c, rope_sin=s, k_scale=0.5)
+    torch.cuda.synchronize()
+    t = (0, 2, 3, 1)
+    assert torch.equal(q.float(), inp["q_normed"].float().clamp_min(0).permute(t))
+    assert torch.equal(k.float(), (0.5 * inp["k_normed"].float().clamp_min(0)).permute(t))
+    assert torch.equal(v, inp["v_raw"].permute(t).contiguous())
+    assert torch.equal(infl, torch.ones_like(infl))
+
+
+def test_ucpe_zero_keys_and_extreme_values():
+    """Keys that ReLU zeroes give inflation_sq = 1; large and tiny values stay
+    inside the tolerance."""
+    B, N, H, D = 1, 70, 2, 64
+    w, inp = _case(B, N, H, D, seed=9)
+    k = inp["k_normed"].clone()
+    k[0, 3, 1] = -k[0, 3, 1].abs() - 0.25          # ReLU(k) = 0 for this (token, head)
+    k[0, 10] *= 1000.0
+    q = inp["q_normed"].clone()
+    q[0, 20] *= 1e-3
+    inp = dict(inp, q_normed=q, k_normed=k.to(torch.bfloat16))
+    outs = Q.cam_prep_func(inp["q_normed"], inp["k_normed"], inp["v_raw"], proj_q=inp["proj_q"],
+                           proj_kv=inp["proj_kv"], rope_cos=inp["rope_cos"],
+                           rope_sin=inp["rope_sin"], k_scale=w.k_scale)
+    torch.cuda.synchronize()
+    assert outs[3][0, 1, 3].item() == 1.0
+    _compare(outs, _oracle(inp, w.k_scale, "bf16"), _oracle(inp, w.k_scale, "bf16", exact=True),
+             "bf16", where="extremes")
+
+
+def test_ucpe_inflation_optional_and_deterministic():
+    B, N, H, D = 1, 190, 4, 112
+    w, inp = _case(B, N, H, D, seed=2)
+    args = (inp["q_normed"], inp["k_normed"], inp["v_raw"], inp["proj_q"], inp["proj_kv"],
+            inp["rope_cos"], inp["rope_sin"])
+    a = [torch.empty(B, H, D, N, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    b = [torch.empty_like(x) for x in a]
+    infl = torch.empty(B, H, N, device="cuda")
+    Q.qknr_ucpe_cam_prep(*args, *a, infl, k_scale=w.k_scale)
+    Q.qknr_ucpe_cam_prep(*args, *b, None, k_scale=w.k_scale)
+    s = torch.cuda.Stream()
+    c = [torch.empty_like(x) for x in a]
+    infl2 = torch.empty_like(infl)
+    Q.qknr_ucpe_cam_prep(*args, *c, infl2, k_scale=w.k_scale, stream=s)
+    torch.cuda.synchronize()
+    for x, y, z in zip(a, b, c):
+        assert torch.equal(x, y) and torch.equal(x, z)
+    assert torch.equal(infl, infl2)
+
+
+def test_ucpe_empty_inputs_are_no_ops():
+    for B, N, H in ((0, 64, 2), (1, 0, 2), (1, 64, 0)):
+        x = torch.empty(B, N, H, 16, dtype=torch.bfloat16, device="cuda")
+        pq = torch.empty(B, N, 4, 4, device="cuda")
+        cs = torch.empty(N, 8, device="cuda")
+        outs = Q.cam_prep_func(x, x, x, proj_q=pq, proj_kv=pq, rope_cos=cs, rope_sin=cs,
+                               k_scale=1.0)
+        torch.cuda.synchronize()
+        assert [tuple(o.shape) for o in outs] == [(B, H, 16, N)] * 3 + [(B, H, N)]
+
+
+def test_ucpe_pinned_host_buffers():
+    """Inputs and outputs in page-locked host memory: the kernel reads and
+    writes them across the bus, with the same results as device buffers."""
+    B, N, H, D = 1, 96, 2, 64
+    w, inp = _case(B, N, H, D, seed=4)
+    dev = Q.cam_prep_func(inp["q_normed"], inp["k_normed"], inp["v_raw"], proj_q=inp["proj_q"],
+                          proj_kv=inp["proj_kv"], rope_cos=inp["rope_cos"],
+                          rope_sin=inp["rope_sin"], k_scale=w.k_scale)
+    host = {k: v.cpu().pin_memory() for k, v in inp.items()}
+    outs = [torch.empty(B, H, D, N, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    infl = torch.empty(B, H, N).pin_memory()
+    st = torch.cuda.current_stream()
+    Q.qknr_ucpe_cam_prep(host["q_normed"], host["k_normed"], host["v_raw"], host["proj_q"],
+                         host["proj_kv"], host["rope_cos"], host["rope_sin"], *outs, infl,
+                         k_scale=w.k_scale, stream=st)
+    torch.cuda.synchronize()
+    for a, b in zip(dev, outs + [infl]):
+        assert torch.equal(a.cpu(), b)
+
+
+def test_ucpe_rejects_pageable_host_memory():
+    B, N, H, D = 1, 8, 1, 8
+    x = torch.zeros(B, N, H, D, dtype=torch.bfloat16)
+    pq = torch.zeros(B, N, 4, 4)
+    cs = torch.zeros(N, D // 2)
+    with pytest.raises(Q.QknrValueError):
+        Q.cam_prep_func(x, x, x, proj_q=pq, proj_kv=pq, rope_cos=cs, rope_sin=cs, k_scale=1.0)
+
+
+def test_ucpe_workload_full_size_sampled():
+    """The benchmark's workload at full size, in the launch the benchmark times;
+    the oracle recomputes a sample of tokens (every token is independent: its
+    rows, its matrices and its table rows), spread over the tiles and including
+    the ragged last tile."""
+    w = W.WORKLOADS["ucpe"]
+    inp = W.make_inputs(w, device="cuda")
+    outs = Q.cam_prep_func(inp["q_normed"], inp["k_normed"], inp["v_raw"], proj_q=inp["proj_q"],
+                           proj_kv=inp["proj_kv"], rope_cos=inp["rope_cos"],
+                           rope_sin=inp["rope_sin"], k_scale=w.k_scale)
+    torch.cuda.synchronize()
+    g = np.random.default_rng(0)
+    idx = np.unique(np.concatenate([g.integers(0, w.seq, 96), [0, 63, 64, w.seq - 1,
+                                                               w.seq - 49]]))
+    it = torch.as_tensor(idx, device="cuda")
+    sub = {k: (v[:, it] if k in ("q_normed", "k_normed", "v_raw", "proj_q", "proj_kv")
+               else v[it]).contiguous() for k, v in inp.items()}
+    ref = _oracle(sub, w.k_scale, "bf16")
+    ref_exact = _oracle(sub, w.k_scale, "bf16", exact=True)
+    got = [o[..., it] for o in outs[:3]] + [outs[3][..., it]]
+    _compare(got, ref, ref_exact, "bf16", where="ucpe full size")
+    assert torch.isfinite(outs[3]).all()
