@@ -9,8 +9,9 @@ HBM; the 377 MB input (plus 377 MB output) exceeds the 126 MB L2, so no flush
 is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-  (NAME: a 3D workload, or table_hs / table_il / table_hs_f16 for the table
-  form, timed over rotated input sets since one set fits in L2)
+  (NAME: a 3D workload, or table_hs / table_il / table_hs_f16 / table_d72 for
+  the table form, timed over rotated input sets since one set fits in L2, or
+  ucpe for the UCPE camera prep)
   python bench.py --impl reference ...   # the fp64 CPU oracle, bounded sample
 
 Under torchrun each rank processes its own batch (weak scaling, no
@@ -44,6 +45,7 @@ TRAFFIC = {
     "table_hs_f16": (42770176 + 2013952, "9230c313092c6dc7"),
     "table_d72": (24805120 + 3584, "9230c313092c6dc7"),
 }
+KERNEL_FILES = {"3d": "rope3d.cu", "table": "rope_table.cu", "ucpe": "ucpe.cu"}
 
 
 def kernel_source_hash(form: str = "3d") -> str:
@@ -54,8 +56,7 @@ def kernel_source_hash(form: str = "3d") -> str:
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "qk_rmsnorm_rope_qknr_b200", "csrc")
-    for f in ("common.cuh", "launch.h", "launch_cache.h",
-              "rope3d.cu" if form == "3d" else "rope_table.cu"):
+    for f in ("common.cuh", "launch.h", "launch_cache.h", KERNEL_FILES[form]):
         with open(os.path.join(csrc, f)) as fh:
             code = fh.read()
         code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)
@@ -159,6 +160,8 @@ def oracle_sample(w, inp_cpu, budget_s: float, chunk: int = 256):
     import oracle as O
     from tests._util import t2u16
 
+    if w.form == "ucpe":
+        return oracle_sample_ucpe(w, inp_cpu, budget_s, chunk)
     if w.form != "3d":
         return oracle_sample_table(w, inp_cpu, budget_s, chunk)
     qkv = inp_cpu["qkv"].reshape(-1, inp_cpu["qkv"].shape[-1])
@@ -194,6 +197,30 @@ def oracle_sample_table(w, inp_cpu, budget_s: float, chunk: int):
         t0 = time.perf_counter()
         O.rope_table(qb, kb, qw, kw, tb, w.eps, w.rotary_dim, interleaved=w.interleaved,
                      act=w.act)
+        spent += time.perf_counter() - t0
+        done += n
+    return done, spent, O.threads()
+
+
+def oracle_sample_ucpe(w, inp_cpu, budget_s: float, chunk: int):
+    """The camera prep's oracle on consecutive token chunks (every head of each
+    token, each batch element in turn), cycling through the workload."""
+    import oracle as O
+    from tests._util import t2u16
+
+    done, spent = 0, 0.0
+    B, N = w.batch, w.seq
+    while spent < budget_s and B * N > 0:
+        pos = done % (B * N)
+        b, s0 = pos // N, pos % N
+        n = min(chunk, N - s0)
+        sl = slice(s0, s0 + n)
+        args = (t2u16(inp_cpu["q_normed"][b:b + 1, sl]), t2u16(inp_cpu["k_normed"][b:b + 1, sl]),
+                t2u16(inp_cpu["v_raw"][b:b + 1, sl]), inp_cpu["proj_q"][b:b + 1, sl].numpy(),
+                inp_cpu["proj_kv"][b:b + 1, sl].numpy(), inp_cpu["rope_cos"][sl].numpy(),
+                inp_cpu["rope_sin"][sl].numpy(), w.k_scale)
+        t0 = time.perf_counter()
+        O.ucpe_cam_prep(*args, act=w.act)
         spent += time.perf_counter() - t0
         done += n
     return done, spent, O.threads()
@@ -673,6 +700,159 @@ def measure_e2e(args, w, qkv, qw, kw, outs, p, stream, dev, world, pg):
             "frac_of_copies_only": round(bus_ms / ms[best], 4)}
 
 
+UCPE_INPUTS = ("q_normed", "k_normed", "v_raw", "proj_q", "proj_kv", "rope_cos", "rope_sin")
+
+
+def run_gpu_ucpe(args, w):
+    """The UCPE camera prep: one launch of qknr_ucpe_cam_prep per step, through
+    the C ABI with the pointers prepared once. Inputs (254 MB for the ucpe
+    workload) and outputs exceed L2, so no flush is needed."""
+    import ctypes as C
+
+    import torch
+
+    import qk_rmsnorm_rope_qknr_b200 as Q
+    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+
+    rank, world, local, dev, pg = init_gpu()
+    L = Q.lib()
+    inp = W.make_inputs(w, device=dev, seed=w.seed + rank)
+    B, N, H, D = w.batch, w.seq, w.heads, w.head_dim
+    act = inp["q_normed"].dtype
+    outs = [torch.empty(B, H, D, N, dtype=act, device=dev) for _ in range(3)]
+    infl = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    # the binding's checks once, then the bare C call for the timed steps
+    Q.qknr_ucpe_cam_prep(*(inp[n] for n in UCPE_INPUTS), *outs, infl, k_scale=w.k_scale,
+                         stream=stream)
+    ptrs = [inp[n].data_ptr() for n in UCPE_INPUTS] + [o.data_ptr() for o in outs] + \
+        [infl.data_ptr()]
+    cargs = ptrs + [Q.QKNR_DT_F16 if w.act == "f16" else Q.QKNR_DT_BF16, B, N, H, D,
+                    C.c_float(w.k_scale), stream.cuda_stream]
+
+    def step(i):
+        rc = L.qknr_ucpe_cam_prep(*cargs)
+        if rc:
+            Q._check(rc)
+
+    ms_per_step, clocks = time_steps(step, args, stream, local, dev, pg)
+    tokens_per_s = world * B * N / (ms_per_step / 1e3)
+    alg_bytes = W.algorithmic_bytes(w)
+    peak, peak_kind = measured_peaks()
+    achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+    tr = TRAFFIC.get(w.name)
+    traffic = tr[0] if tr and tr[1] == kernel_source_hash("ucpe") else None
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e_ucpe(args, w, inp, outs, infl, stream, dev, world, pg)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = {k: v.cpu() for k, v in inp.items()}
+        n, sec, threads = oracle_sample(w, inp_cpu, args.cpu_seconds, chunk=64)
+        cpu = {"value": n / sec, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} tokens (all {H} heads each) of {w.name} in order, cycling "
+                         f"through its {B * N} ({sec:.1f} s of fp64 oracle work)"}
+    if rank == 0:
+        in_mb = sum(inp[n].numel() * inp[n].element_size() for n in UCPE_INPUTS) / 1e6
+        line = {
+            "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "tokens_per_gpu": B * N, "io": f"{w.act} in and out, "
+                       "f32 matrices, tables and inflation_sq",
+                       "shape_in": [B, N, H, D], "shape_out": [B, H, D, N],
+                       "k_scale": w.k_scale,
+                       "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": f"no flush: inputs {in_mb:.0f} MB > 126 MB L2"},
+            "hbm_gbs": achieved, "hbm_pct_of_peak": 100.0 * achieved / peak,
+            "kernel_us": ms_per_step * 1e3,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": alg_bytes},
+            "cpu_baseline": cpu, "clocks": clocks.summary(), "e2e": e2e,
+            "gpu_launches": args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def measure_e2e_ucpe(args, w, inp, outs, infl, stream, dev, world, pg):
+    """End to end through the C ABI for the camera prep, inputs and outputs in
+    page-locked host memory: staged (copy the seven inputs in, run, copy the
+    four outputs back) or zero-copy (the kernel reads and writes the host
+    buffers across the bus); the faster is reported, beside the copies alone.
+    (Token chunks are not pipelined: a chunk's outputs are strided in the
+    [B, H, D, N] layout.)"""
+    import torch
+
+    import qk_rmsnorm_rope_qknr_b200 as Q
+
+    host = {n: torch.empty(inp[n].shape, dtype=inp[n].dtype).pin_memory() for n in UCPE_INPUTS}
+    for n in UCPE_INPUTS:
+        host[n].copy_(inp[n].cpu())
+    h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs + [infl]]
+    d_in = {n: torch.empty_like(inp[n]) for n in UCPE_INPUTS}
+    steps = max(3, min(args.e2e_steps, args.steps))
+
+    def staged():
+        for n in UCPE_INPUTS:
+            d_in[n].copy_(host[n], non_blocking=True)
+        Q.qknr_ucpe_cam_prep(*(d_in[n] for n in UCPE_INPUTS), *outs, infl, k_scale=w.k_scale,
+                             stream=stream)
+        for h, o in zip(h_out, outs + [infl]):
+            h.copy_(o, non_blocking=True)
+
+    def zero_copy():
+        Q.qknr_ucpe_cam_prep(*(host[n] for n in UCPE_INPUTS), *h_out, k_scale=w.k_scale,
+                             stream=stream)
+
+    def timed(step):
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+        if pg:
+            t = torch.tensor([ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ms = t.item()
+        return ms
+
+    s_copy = torch.cuda.Stream(dev)
+
+    def copies_only():
+        for n in UCPE_INPUTS:
+            d_in[n].copy_(host[n], non_blocking=True)
+        with torch.cuda.stream(s_copy):
+            for h, o in zip(h_out, outs + [infl]):
+                h.copy_(o, non_blocking=True)
+        stream.wait_stream(s_copy)
+
+    ms = {"staged": timed(staged), "zero-copy": timed(zero_copy)}
+    best = min(ms, key=ms.get)
+    bus_ms = timed(copies_only)
+    return {"value": world * w.tokens / (ms[best] / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": sum(inp[n].numel() * inp[n].element_size() for n in UCPE_INPUTS),
+            "d2h_bytes_per_step": sum(o.numel() * o.element_size() for o in outs + [infl]),
+            "steps": steps, "mode": best,
+            "ms_per_step": {k: round(v, 4) for k, v in ms.items()},
+            "copies_only_ms_per_step": round(bus_ms, 4),
+            "frac_of_copies_only": round(bus_ms / ms[best], 4)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -699,10 +879,14 @@ def main():
         if w.form == "3d":
             w = dataclasses.replace(w, name=f"{w.name}[{args.tokens}]", batch=1, seq=args.tokens,
                                     input_2d=True)
+        elif w.form == "ucpe":
+            w = dataclasses.replace(w, name=f"{w.name}[{args.tokens}]", seq=args.tokens)
         else:
             w = dataclasses.replace(w, name=f"{w.name}[{args.tokens}]", tokens=args.tokens)
     if args.impl == "reference":
         return run_reference(args, w)
+    if w.form == "ucpe":
+        return run_gpu_ucpe(args, w)
     return run_gpu(args, w) if w.form == "3d" else run_gpu_table(args, w)
 
 

@@ -45,7 +45,8 @@ constexpr int kProjStride = 36;  // floats per token in the staged matrices (32 
 int ucpe_block(int D) { return ((kTile / 4) * (D / 8) + 31) / 32 * 32; }
 
 int ucpe_smem(int D) {
-    return 3 * D * kTile * 2 + kTile * kProjStride * 4 + kTile * (D / 8) * 8;
+    return 3 * D * kTile * 2 + kTile * kProjStride * 4 + 2 * kTile * (D / 2) * 4 +
+           kTile * (D / 8) * 8;
 }
 
 // Byte offset of (channel d, tile token t) inside one tensor's staging tile.
@@ -62,6 +63,158 @@ __device__ __forceinline__ void project_block(const float* m, const float* x, fl
     }
 }
 
+// 16-byte asynchronous copy global -> shared; with valid == false the 16
+// bytes are zero-filled and nothing is read.
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst_smem)),
+                 "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// The tile's per-token inputs that every head shares, copied asynchronously
+// into shared memory: the two 4x4 matrices ([kTile][kProjStride] floats,
+// proj_q then proj_kv) and the cos and sin rows ([kTile][D/2] floats each).
+__device__ __forceinline__ void stage_token_inputs(const UcpeArgs& a, int64_t b, int64_t n0,
+                                                   int tv, int tid, int nthr, float* proj,
+                                                   float* cosr, float* sinr) {
+    for (int f = tid; f < kTile * 8; f += nthr) {
+        const int t = f >> 3, r = f & 7;
+        const bool ok = t < tv;
+        const float* src = (r < 4 ? a.proj_q : a.proj_kv) +
+                           (ok ? (b * a.num_tokens + n0 + t) * 16 + (r & 3) * 4 : 0);
+        cp_async16(proj + t * kProjStride + r * 4, src, ok);
+    }
+    const int q4 = a.head_dim / 8;  // float4 per token row of a table
+    for (int f = tid; f < kTile * q4 * 2; f += nthr) {
+        const int which = f >= kTile * q4;  // 0: cos, 1: sin
+        const int g = f - which * kTile * q4;
+        const int t = g / q4, k4 = g - (g / q4) * q4;
+        const bool ok = t < tv;
+        const float* src = (which ? a.rope_sin : a.rope_cos) +
+                           (ok ? (n0 + t) * (a.head_dim / 2) + 4 * k4 : 0);
+        cp_async16((which ? sinr : cosr) + g * 4, src, ok);
+    }
+    cp_async_commit();
+}
+
+// Q, K and V chunks of four tokens (one item), held in registers.
+__device__ __forceinline__ void load_item(const UcpeArgs& a, int64_t b, int64_t n0, int h, int tv,
+                                          int p, int c, uint4 (&raw)[3][4]) {
+    const int D = a.head_dim;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int t = 4 * p + u;
+        if (t < tv) {
+            const int64_t row = ((b * a.num_tokens + n0 + t) * a.heads + h) * D + 8 * c;
+            raw[0][u] = ld_nc_v4(a.q + row * 2);
+            raw[1][u] = ld_nc_v4(a.k + row * 2);
+            raw[2][u] = ld_nc_v4(a.v + row * 2);
+        } else {
+            raw[0][u] = raw[1][u] = raw[2][u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+}
+
+// One token's 8 channels of tensor X (0 = Q, 1 = K, 2 = V): element steps,
+// projection, rotation; for K also the two sums of squares.
+template <bool H16, int X>
+__device__ __forceinline__ void transform8(const uint4& raw, const float* m, const float* cr,
+                                           const float* sr, float k_scale, float* y, float& si,
+                                           float& so) {
+    float x[8];
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = act2_to_f2<H16>(w[e]);
+        x[2 * e] = f.x;
+        x[2 * e + 1] = f.y;
+    }
+    if (X < 2) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = fmaxf(x[e], 0.0f);
+    }
+    if (X == 1) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] *= k_scale;
+    }
+    project_block(m, x, y);
+    project_block(m, x + 4, y + 4);
+    if (X == 1) {
+        float a = 0.f, b = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            a = fmaf(x[e], x[e], a);
+            b = fmaf(y[e], y[e], b);
+        }
+        si = a;
+        so = b;
+    }
+    if (X < 2) {
+        const float4 cs = *reinterpret_cast<const float4*>(cr);
+        const float4 sn = *reinterpret_cast<const float4*>(sr);
+        const float cj[4] = {cs.x, cs.y, cs.z, cs.w};
+        const float sj[4] = {sn.x, sn.y, sn.z, sn.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float ya = y[2 * j], yb = y[2 * j + 1];
+            y[2 * j] = fmaf(ya, cj[j], -yb * sj[j]);
+            y[2 * j + 1] = fmaf(yb, cj[j], ya * sj[j]);
+        }
+    }
+}
+
+// Tensor X of the item: four tokens, results packed two tokens to a word (the
+// lower token in the low half) and written to the staging tile as one 8-byte
+// word per channel.
+template <bool H16, int X>
+__device__ __forceinline__ void item_tensor(const uint4 (&raw)[3][4], const float* proj,
+                                            const float* cosr, const float* sinr, int D, int p,
+                                            int c, float k_scale, unsigned char* tile_x,
+                                            float* si, float* so) {
+    uint32_t packed[8][2];
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+        float y0[8], y1[8];
+        const int u0 = 2 * pr, u1 = 2 * pr + 1;
+        const int t0 = 4 * p + u0, t1 = 4 * p + u1;
+        const int moff = X == 0 ? 0 : 16;
+        const int roff = 4 * c;
+        transform8<H16, X>(raw[X][u0], proj + t0 * kProjStride + moff, cosr + t0 * (D / 2) + roff,
+                           sinr + t0 * (D / 2) + roff, k_scale, y0, si[u0], so[u0]);
+        transform8<H16, X>(raw[X][u1], proj + t1 * kProjStride + moff, cosr + t1 * (D / 2) + roff,
+                           sinr + t1 * (D / 2) + roff, k_scale, y1, si[u1], so[u1]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) packed[e][pr] = f2_to_act2<H16>(make_float2(y0[e], y1[e]));
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        *reinterpret_cast<uint2*>(tile_x + stage_offset(8 * c + e, 4 * p)) =
+            make_uint2(packed[e][0], packed[e][1]);
+    }
+}
+
+// Position of a tile in the (batch, token tile, head) order, head fastest,
+// advanced by a fixed stride without divisions.
+struct TileCursor {
+    int64_t b, tn;
+    int h;
+    __device__ __forceinline__ void advance(int64_t step_bt, int step_h, int H, int64_t tiles_n) {
+        h += step_h;
+        int64_t dbt = step_bt;
+        if (h >= H) {
+            h -= H;
+            ++dbt;
+        }
+        tn += dbt;
+        while (tn >= tiles_n) {
+            tn -= tiles_n;
+            ++b;
+        }
+    }
+};
+
 template <bool H16>
 __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
     const int D = a.head_dim, C = D / 8, H = a.heads;
@@ -69,143 +222,91 @@ __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
     const int64_t tiles_n = (N + kTile - 1) / kTile;
     const int64_t ntiles = a.batch * tiles_n * H;
     const int tid = threadIdx.x, nthr = blockDim.x;
-    const int items = (kTile / 4) * C;
     const bool vec_out = (N & 7) == 0;
 
     extern __shared__ __align__(16) unsigned char smem[];
     unsigned char* stage = smem;  // [3][D][kTile] 16-bit, swizzled rows
     float* proj = reinterpret_cast<float*>(smem + 3 * D * kTile * 2);  // [kTile][kProjStride]
-    float2* part = reinterpret_cast<float2*>(proj + kTile * kProjStride);  // [kTile][C]
+    float* cosr = proj + kTile * kProjStride;                            // [kTile][D/2]
+    float* sinr = cosr + kTile * (D / 2);                                // [kTile][D/2]
+    float2* part = reinterpret_cast<float2*>(sinr + kTile * (D / 2));   // [kTile][C]
 
     // This thread's item: tokens 4p..4p+3 of the tile, channels 8c..8c+7.
     const int p = tid / C, c = tid - (tid / C) * C;
-    const bool has_item = tid < items;
+    const bool has_item = tid < (kTile / 4) * C;
+
+    int64_t tile = blockIdx.x;
+    if (tile >= ntiles) return;
+    const int64_t step_bt = (int64_t)gridDim.x / H;
+    const int step_h = (int)((int64_t)gridDim.x - step_bt * H);
+    TileCursor cur;
+    cur.h = (int)(tile % H);
+    cur.tn = tile / H;
+    cur.b = cur.tn / tiles_n;
+    cur.tn -= cur.b * tiles_n;
 
     griddep_wait();
     griddep_launch_dependents();
 
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int h = (int)(tile % H);
-        const int64_t bt = tile / H;
-        const int64_t b = bt / tiles_n;
-        const int64_t n0 = (bt - b * tiles_n) * kTile;
-        const int tv = (int)min((int64_t)kTile, N - n0);  // tokens of this tile
+    // Prologue: the first tile's inputs.
+    uint4 raw[3][4];
+    {
+        const int64_t n0 = cur.tn * kTile;
+        const int tv = (int)min((int64_t)kTile, N - n0);
+        stage_token_inputs(a, cur.b, n0, tv, tid, nthr, proj, cosr, sinr);
+        if (has_item) load_item(a, cur.b, n0, cur.h, tv, p, c, raw);
+        cp_async_wait_all();
+    }
+    __syncthreads();
 
-        // The tile's matrices: 8 float4 per token (proj_q, then proj_kv).
-        for (int i = tid; i < kTile * 8; i += nthr) {
-            const int t = i >> 3, r = i & 7;
-            float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (t < tv) {
-                const float* src = (r < 4 ? a.proj_q : a.proj_kv) + (b * N + n0 + t) * 16 + (r & 3) * 4;
-                m = __ldg(reinterpret_cast<const float4*>(src));
-            }
-            *reinterpret_cast<float4*>(proj + t * kProjStride + r * 4) = m;
-        }
-        __syncthreads();
+    while (true) {
+        const int64_t b = cur.b, n0 = cur.tn * kTile;
+        const int h = cur.h;
+        const int tv = (int)min((int64_t)kTile, N - n0);
 
         if (has_item) {
-            // Every load of the item first, so that they are all in flight together.
-            uint4 raw[3][4];
-            float4 cs[4], sn[4];
+            float si[4], so[4];
+            item_tensor<H16, 0>(raw, proj, cosr, sinr, D, p, c, a.k_scale, stage, si, so);
+            item_tensor<H16, 1>(raw, proj, cosr, sinr, D, p, c, a.k_scale, stage + D * kTile * 2,
+                                si, so);
+            item_tensor<H16, 2>(raw, proj, cosr, sinr, D, p, c, a.k_scale,
+                                stage + 2 * D * kTile * 2, si, so);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int t = 4 * p + u;
-                if (t < tv) {
-                    const int64_t row = ((b * N + n0 + t) * H + h) * D + 8 * c;
-                    raw[0][u] = ld_nc_v4(a.q + row * 2);
-                    raw[1][u] = ld_nc_v4(a.k + row * 2);
-                    raw[2][u] = ld_nc_v4(a.v + row * 2);
-                    const int64_t tr = (n0 + t) * (D / 2) + 4 * c;
-                    cs[u] = __ldg(reinterpret_cast<const float4*>(a.rope_cos + tr));
-                    sn[u] = __ldg(reinterpret_cast<const float4*>(a.rope_sin + tr));
-                } else {
-                    raw[0][u] = raw[1][u] = raw[2][u] = make_uint4(0u, 0u, 0u, 0u);
-                    cs[u] = sn[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
-            float ssq_in[4], ssq_out[4];
-#pragma unroll
-            for (int X = 0; X < 3; ++X) {
-                uint32_t packed[8][2];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    float x[8], y[8];
-                    const uint32_t w[4] = {raw[X][u].x, raw[X][u].y, raw[X][u].z, raw[X][u].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = act2_to_f2<H16>(w[e]);
-                        x[2 * e] = f.x;
-                        x[2 * e + 1] = f.y;
-                    }
-                    if (X < 2) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = fmaxf(x[e], 0.0f);
-                    }
-                    if (X == 1) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] *= a.k_scale;
-                    }
-                    const float* m = proj + (4 * p + u) * kProjStride + (X == 0 ? 0 : 16);
-                    project_block(m, x, y);
-                    project_block(m, x + 4, y + 4);
-                    if (X == 1) {
-                        float si = 0.f, so = 0.f;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            si = fmaf(x[e], x[e], si);
-                            so = fmaf(y[e], y[e], so);
-                        }
-                        ssq_in[u] = si;
-                        ssq_out[u] = so;
-                    }
-                    if (X < 2) {
-                        const float cj[4] = {cs[u].x, cs[u].y, cs[u].z, cs[u].w};
-                        const float sj[4] = {sn[u].x, sn[u].y, sn[u].z, sn[u].w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float ya = y[2 * j], yb = y[2 * j + 1];
-                            y[2 * j] = fmaf(ya, cj[j], -yb * sj[j]);
-                            y[2 * j + 1] = fmaf(yb, cj[j], ya * sj[j]);
-                        }
-                    }
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const uint32_t o = f_to_act<H16>(y[e]);
-                        if (u & 1) {
-                            packed[e][u >> 1] |= o << 16;
-                        } else {
-                            packed[e][u >> 1] = o;
-                        }
-                    }
-                }
-                unsigned char* tile_x = stage + X * D * kTile * 2;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    *reinterpret_cast<uint2*>(tile_x + stage_offset(8 * c + e, 4 * p)) =
-                        make_uint2(packed[e][0], packed[e][1]);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) part[(4 * p + u) * C + c] = make_float2(ssq_in[u], ssq_out[u]);
+            for (int u = 0; u < 4; ++u) part[(4 * p + u) * C + c] = make_float2(si[u], so[u]);
         }
         __syncthreads();
+
+        // The next tile's inputs go out before this tile's stores.
+        tile += gridDim.x;
+        const bool more = tile < ntiles;
+        if (more) {
+            cur.advance(step_bt, step_h, H, tiles_n);
+            const int64_t nn0 = cur.tn * kTile;
+            const int ntv = (int)min((int64_t)kTile, N - nn0);
+            stage_token_inputs(a, cur.b, nn0, ntv, tid, nthr, proj, cosr, sinr);
+            if (has_item) load_item(a, cur.b, nn0, cur.h, ntv, p, c, raw);
+        }
 
         // The staged tile leaves as whole 128-byte output rows.
         const int64_t out_head = (b * H + h) * (int64_t)D;
-        for (int i = tid; i < 3 * D * 8; i += nthr) {
-            const int row = i >> 3, j = i & 7;
-            const int X = row / D, d = row - X * D;
-            const uint4 val = *reinterpret_cast<const uint4*>(
-                stage + X * D * kTile * 2 + d * (kTile * 2) + (((j ^ (d >> 3)) & 7) << 4));
+#pragma unroll
+        for (int X = 0; X < 3; ++X) {
             uint8_t* out = X == 0 ? a.q_out : (X == 1 ? a.k_out : a.v_out);
-            const int64_t n = n0 + 8 * j;
-            uint8_t* dst = out + ((out_head + d) * N + n) * 2;
-            if (vec_out && n + 8 <= N) {
-                st_v4(dst, val);
-            } else {
-                const uint32_t w[4] = {val.x, val.y, val.z, val.w};
-                for (int e = 0; e < 8 && n + e < N; ++e)
-                    reinterpret_cast<uint16_t*>(dst)[e] = (uint16_t)(w[e >> 1] >> ((e & 1) * 16));
+            const unsigned char* tile_x = stage + X * D * kTile * 2;
+            for (int i = tid; i < D * 8; i += nthr) {
+                const int d = i >> 3, j = i & 7;
+                const uint4 val = *reinterpret_cast<const uint4*>(
+                    tile_x + d * (kTile * 2) + (((j ^ (d >> 3)) & 7) << 4));
+                const int64_t n = n0 + 8 * j;
+                uint8_t* dst = out + ((out_head + d) * N + n) * 2;
+                if (vec_out && n + 8 <= N) {
+                    st_v4(dst, val);
+                } else {
+                    const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+                    for (int e = 0; e < 8 && n + e < N; ++e)
+                        reinterpret_cast<uint16_t*>(dst)[e] =
+                            (uint16_t)(w[e >> 1] >> ((e & 1) * 16));
+                }
             }
         }
         if (a.inflation_sq) {
@@ -219,6 +320,9 @@ __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
                 a.inflation_sq[(b * H + h) * N + n0 + t] = si > 0.f ? so / si : 1.0f;
             }
         }
+        if (!more) break;
+        cp_async_wait_all();
+        __syncthreads();
     }
 }
 
