@@ -39,6 +39,7 @@ namespace qknr {
 namespace {
 
 constexpr int kTile = 64;        // tokens per tile (one 128-byte output row)
+constexpr int kPairs = kTile / 2;
 constexpr int kProjStride = 36;  // floats per token in the staged matrices (32 used)
 
 // Threads per CTA: one per (4-token group, 8-channel chunk) of a tile.
@@ -70,6 +71,42 @@ __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src, bool
                  "l"(src), "r"(valid ? 16 : 0)
                  : "memory");
 }
+// 4-byte asynchronous copy global -> shared; with valid == false the 4 bytes
+// are zero-filled and nothing is read.
+__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst_smem)),
+                 "l"(src), "r"(valid ? 4 : 0)
+                 : "memory");
+}
+
+// max(x, 0) on both 16-bit halves of a word.
+template <bool H16>
+__device__ __forceinline__ uint32_t relu2(uint32_t w) {
+    if constexpr (H16) {
+        __half2 h = __hmax2(*reinterpret_cast<const __half2*>(&w), __float2half2_rn(0.0f));
+        return *reinterpret_cast<uint32_t*>(&h);
+    } else {
+        __nv_bfloat162 h = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&w),
+                                   __float2bfloat162_rn(0.0f));
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+}
+
+// Channels 2e and 2e+1 of a token pair: (lower-channel value of token A, of
+// token B) and the same for the upper channel.
+template <bool H16>
+__device__ __forceinline__ void widen_pair(uint32_t wa, uint32_t wb, float2& lo, float2& hi) {
+    if constexpr (H16) {
+        const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&wa));
+        const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&wb));
+        lo = make_float2(fa.x, fb.x);
+        hi = make_float2(fa.y, fb.y);
+    } else {
+        lo = make_float2(bf16_lo(wa), bf16_lo(wb));
+        hi = make_float2(bf16_hi(wa), bf16_hi(wb));
+    }
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
@@ -224,7 +261,7 @@ __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
     const int tid = threadIdx.x, nthr = blockDim.x;
     const bool vec_out = (N & 7) == 0;
 
-    extern __shared__ __align__(16) unsigned char smem[];
+    extern __shared__ __align__(128) unsigned char smem[];
     unsigned char* stage = smem;  // [3][D][kTile] 16-bit, swizzled rows
     float* proj = reinterpret_cast<float*>(smem + 3 * D * kTile * 2);  // [kTile][kProjStride]
     float* cosr = proj + kTile * kProjStride;                            // [kTile][D/2]
@@ -326,6 +363,319 @@ __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Fast kernel: head_dim <= 128, num_tokens a multiple of 8.
+//
+// Work unit: a tile of 64 tokens of one batch element, all heads in turn.
+// Lane i of every warp owns the token pair (2i, 2i+1) of the tile; warp w owns
+// the 8-channel chunk w. For each head:
+//   - its Q, K, V rows (64 tokens x D, three tensors) arrive by 16-byte
+//     cp.async into one stage of a ring of shared-memory stages (consecutive
+//     threads copy consecutive chunks of a row), issued several heads ahead so
+//     that about 100 KB per SM are in flight;
+//   - each thread widens, projects, rotates and rounds its two tokens x eight
+//     channels of each tensor with packed fp32x2 instructions (the tile's
+//     matrices are staged in shared memory interleaved by token pairs, its
+//     cos/sin values sit in registers for all heads) and stores one 32-bit word
+//     (both tokens) per channel straight to [B, H, D, N]: the 32 lanes of a
+//     warp write one whole 128-byte row;
+//   - the per-chunk key sums go to shared memory and are added per token, in a
+//     fixed order, one head later (so one barrier per head suffices).
+// Padding: a token pair's two rows take 2D*2 + 16 bytes of a stage, so that
+// the 16-byte chunks that eight consecutive lanes read fall in distinct banks;
+// a pair's interleaved matrices take 144 bytes for the same reason.
+constexpr int kFastMaxD = 128;
+constexpr int kMatStride = 36;  // floats per token pair per matrix (32 used)
+
+__host__ __device__ inline int fast_pair_stride(int D) { return 4 * D + 16; }  // bytes
+__host__ __device__ inline int fast_stage_bytes(int D) { return 3 * kPairs * fast_pair_stride(D); }
+
+struct FastLayout {
+    int ring, mats, part, total, stages;
+};
+
+// Stages: as many as fit (at most 4) beside two matrix and two key-sum buffers.
+__host__ __device__ inline FastLayout fast_layout(int D, int stages) {
+    FastLayout L;
+    const int C = D / 8;
+    L.stages = stages;
+    L.ring = 0;
+    L.mats = stages * fast_stage_bytes(D);            // [2][2][32][kMatStride] f32
+    L.part = L.mats + 2 * 2 * kPairs * kMatStride * 4;  // [2][C][64] float2
+    L.total = L.part + 2 * C * kTile * 8;
+    return L;
+}
+
+__device__ __forceinline__ void cp_async16z(void* dst_smem, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst_smem)),
+                 "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+template <int K>
+__device__ __forceinline__ void cp_async_wait_pending() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(K) : "memory");
+}
+
+// A step of this CTA: head h of its ti-th tile (tile blockIdx.x + ti * grid),
+// advanced one head at a time (the division runs once per tile).
+struct FastStep {
+    int64_t ti, b, n0;
+    int h, tv;
+    bool valid;
+
+    __device__ __forceinline__ void locate(const UcpeArgs& a, int64_t tiles_n, int64_t ntiles) {
+        const int64_t tile = blockIdx.x + ti * (int64_t)gridDim.x;
+        valid = tile < ntiles;
+        b = valid ? tile / tiles_n : 0;
+        n0 = valid ? (tile - b * tiles_n) * kTile : 0;
+        tv = valid ? (int)min((int64_t)kTile, a.num_tokens - n0) : 0;
+    }
+    __device__ __forceinline__ void next(const UcpeArgs& a, int64_t tiles_n, int64_t ntiles) {
+        if (++h == a.heads) {
+            h = 0;
+            ++ti;
+            locate(a, tiles_n, ntiles);
+        }
+    }
+};
+
+// The matrices of a tile's tokens into matrix buffer `mats`, interleaved by
+// token pairs (4-byte copies; tokens past the tile's end read as zeros).
+__device__ __forceinline__ void fast_stage_mats(const UcpeArgs& a, const FastStep& st, float* mats) {
+    for (int f = threadIdx.x; f < kTile * 32; f += blockDim.x) {
+        const int e = f & 15, m = (f >> 4) & 1, t = f >> 5;
+        const bool ok = t < st.tv;
+        const float* src =
+            (m ? a.proj_kv : a.proj_q) + (ok ? (st.b * a.num_tokens + st.n0 + t) * 16 + e : 0);
+        cp_async4(mats + (m * kPairs + (t >> 1)) * kMatStride + e * 2 + (t & 1), src, ok);
+    }
+}
+
+// One head's Q, K, V rows of a tile into ring stage `buf` (16-byte copies;
+// sixteen lanes per token row, lane k copying chunk k of that token's Q, K and
+// V rows; a lane takes tokens t0, t0 + 2 * warps, ...; tokens past the tile's
+// end read as zeros). `off` is the byte offset of chunk k of token t0's row at
+// head 0 of the tile (fast_row_offset); successive tokens of the lane are
+// 2 * warps rows apart.
+__device__ __forceinline__ void fast_stage_head(const UcpeArgs& a, const FastStep& st, int64_t off,
+                                                unsigned char* buf) {
+    const int D = a.head_dim, C = D / 8;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int ps = fast_pair_stride(D);
+    const int k4 = lane & 15;
+    if (k4 >= C) return;
+    const int64_t step = (int64_t)2 * nwarps * a.heads * D * 2;
+    int64_t o = off + (int64_t)st.h * D * 2;
+    for (int t = 2 * warp + (lane >> 4); t < kTile; t += 2 * nwarps, o += step) {
+        const bool ok = t < st.tv;
+        const int64_t src = ok ? o : 0;
+        unsigned char* dst = buf + (t >> 1) * ps + (t & 1) * 2 * D + 16 * k4;
+        cp_async16z(dst, a.q + src, ok);
+        cp_async16z(dst + kPairs * ps, a.k + src, ok);
+        cp_async16z(dst + 2 * kPairs * ps, a.v + src, ok);
+    }
+}
+
+// Byte offset (from the tensor base) of chunk k4 of this lane's first token
+// row at head 0 of the tile.
+__device__ __forceinline__ int64_t fast_row_offset(const UcpeArgs& a, const FastStep& st) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t0 = 2 * warp + (lane >> 4);
+    return ((st.b * a.num_tokens + st.n0 + t0) * a.heads * a.head_dim + 8 * (lane & 15)) * 2;
+}
+
+// Issue the copies of step `st` into ring stage `slot` (its head's rows; at a
+// tile's first head also the tile's matrices) and commit them as one group,
+// empty if the step is past the end.
+__device__ __forceinline__ void fast_issue(const UcpeArgs& a, const FastStep& st, int64_t off,
+                                           int slot,
+                                           unsigned char* smem, const FastLayout& L) {
+    if (st.valid) {
+        fast_stage_head(a, st, off, smem + L.ring + slot * fast_stage_bytes(a.head_dim));
+        if (st.h == 0)
+            fast_stage_mats(a, st, reinterpret_cast<float*>(smem + L.mats) +
+                                       (st.ti & 1) * 2 * kPairs * kMatStride);
+    }
+    cp_async_commit();
+}
+
+// Tensor X of this thread's token pair and chunk: widen, ReLU (Q, K), project,
+// rotate (Q, K), scale (K), round; one packed word per channel stored straight
+// to the output. For K, the pair's sums of squares go to si/so.
+template <bool H16, int X>
+__device__ __forceinline__ void fast_tensor(const unsigned char* in, const float* mats,
+                                            const float2 (&cj)[4], const float2 (&sj)[4],
+                                            int D, int pp, int c, float k_scale, uint8_t* out_row0,
+                                            int64_t row_bytes, float2& si, float2& so) {
+    const int ps = fast_pair_stride(D);
+    const uint4 ra = *reinterpret_cast<const uint4*>(in + (X * kPairs + pp) * ps + 16 * c);
+    const uint4 rb = *reinterpret_cast<const uint4*>(in + (X * kPairs + pp) * ps + 2 * D + 16 * c);
+    uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+    uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+    if (X < 2) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            wa[e] = relu2<H16>(wa[e]);
+            wb[e] = relu2<H16>(wb[e]);
+        }
+    }
+    float2 x[8], y[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) widen_pair<H16>(wa[e], wb[e], x[2 * e], x[2 * e + 1]);
+    const float* m = mats + ((X == 0 ? 0 : kPairs) + pp) * kMatStride;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 r01 = *reinterpret_cast<const float4*>(m + 8 * i);
+        const float4 r23 = *reinterpret_cast<const float4*>(m + 8 * i + 4);
+        const float2 m0 = make_float2(r01.x, r01.y), m1 = make_float2(r01.z, r01.w);
+        const float2 m2 = make_float2(r23.x, r23.y), m3 = make_float2(r23.z, r23.w);
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+            const float2* xb = x + 4 * blk;
+            y[4 * blk + i] = fma2(m3, xb[3], fma2(m2, xb[2], fma2(m1, xb[1], mul2(m0, xb[0]))));
+        }
+    }
+    if (X == 1) {
+        float2 a2 = make_float2(0.f, 0.f), b2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            a2 = fma2(x[e], x[e], a2);
+            b2 = fma2(y[e], y[e], b2);
+        }
+        si = a2;
+        so = b2;
+    }
+    if (X < 2) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 ya = y[2 * j], yb = y[2 * j + 1];
+            const float2 bs = mul2(yb, sj[j]);
+            y[2 * j] = fma2(ya, cj[j], make_float2(-bs.x, -bs.y));
+            y[2 * j + 1] = fma2(yb, cj[j], mul2(ya, sj[j]));
+        }
+    }
+    if (X == 1) {
+        const float2 ks = make_float2(k_scale, k_scale);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = mul2(y[e], ks);
+    }
+    uint8_t* o = out_row0 + 4 * pp;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        *reinterpret_cast<uint32_t*>(o + (int64_t)e * row_bytes) = f2_to_act2<H16>(y[e]);
+}
+
+template <bool H16, int STAGES>
+__global__ void __launch_bounds__(512, 1) ucpe_fast_kernel(const UcpeArgs a) {
+    const int D = a.head_dim, C = D / 8, H = a.heads;
+    const int64_t N = a.num_tokens;
+    const int64_t tiles_n = (N + kTile - 1) / kTile;
+    const int64_t ntiles = a.batch * tiles_n;
+    const int tid = threadIdx.x;
+    const int pp = tid & 31, c = tid >> 5;  // token pair, chunk
+    const bool key_scaled = a.k_scale != 0.0f;
+    const FastLayout L = fast_layout(D, STAGES);
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    float2* part = reinterpret_cast<float2*>(smem + L.part);  // [2][C][64]
+
+    if ((int64_t)blockIdx.x >= ntiles) return;
+    // this CTA's steps: its tiles x heads
+    const int64_t my_tiles = (ntiles - 1 - blockIdx.x) / gridDim.x + 1;
+    const int64_t nsteps = my_tiles * H;
+    const int64_t row_bytes = N * 2;
+
+    griddep_wait();
+    griddep_launch_dependents();
+
+    FastStep st{}, ahead{};
+    st.locate(a, tiles_n, ntiles);
+    ahead = st;
+    int64_t off = fast_row_offset(a, ahead);  // of the tile `ahead` is in
+    for (int k = 0; k < STAGES - 1; ++k) {
+        fast_issue(a, ahead, off, k, smem, L);
+        ahead.next(a, tiles_n, ntiles);
+        if (ahead.h == 0) off = fast_row_offset(a, ahead);
+    }
+
+    float2 cj[4], sj[4];
+    FastStep prev{};
+    for (int64_t s = 0; s < nsteps; ++s) {
+        cp_async_wait_pending<STAGES - 2>();  // this step's group is complete
+        __syncthreads();
+        // The stage of step s - 1 is free now: refill it with step s + STAGES - 1.
+        fast_issue(a, ahead, off, (int)((s + STAGES - 1) % STAGES), smem, L);
+        ahead.next(a, tiles_n, ntiles);
+        if (ahead.h == 0) off = fast_row_offset(a, ahead);
+
+        // Key sums of the previous step (written before the barrier above).
+        if (s > 0 && a.inflation_sq) {
+            const float2* pprev = part + ((s - 1) & 1) * C * kTile;
+            for (int t = tid; t < prev.tv; t += blockDim.x) {
+                float s_in = 0.f, s_out = 0.f;
+                for (int cc = 0; cc < C; ++cc) {
+                    const float2 v = pprev[cc * kTile + t];
+                    s_in += v.x;
+                    s_out += v.y;
+                }
+                a.inflation_sq[(prev.b * H + prev.h) * N + prev.n0 + t] =
+                    (s_in > 0.f && key_scaled) ? s_out / s_in : 1.0f;
+            }
+        }
+
+        const int64_t ti = st.ti;
+        if (st.h == 0) {
+            // this tile's cos/sin for the thread's pair and chunk, for all heads
+            const int half = D / 2;
+            const int64_t r0 = (st.n0 + 2 * pp) * half + 4 * c;
+            const bool ok0 = 2 * pp < st.tv, ok1 = 2 * pp + 1 < st.tv;
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 c0 = ok0 ? __ldg(reinterpret_cast<const float4*>(a.rope_cos + r0)) : z;
+            const float4 c1 = ok1 ? __ldg(reinterpret_cast<const float4*>(a.rope_cos + r0 + half)) : z;
+            const float4 s0 = ok0 ? __ldg(reinterpret_cast<const float4*>(a.rope_sin + r0)) : z;
+            const float4 s1 = ok1 ? __ldg(reinterpret_cast<const float4*>(a.rope_sin + r0 + half)) : z;
+            cj[0] = make_float2(c0.x, c1.x); cj[1] = make_float2(c0.y, c1.y);
+            cj[2] = make_float2(c0.z, c1.z); cj[3] = make_float2(c0.w, c1.w);
+            sj[0] = make_float2(s0.x, s1.x); sj[1] = make_float2(s0.y, s1.y);
+            sj[2] = make_float2(s0.z, s1.z); sj[3] = make_float2(s0.w, s1.w);
+        }
+        const unsigned char* in = smem + L.ring + (int)(s % STAGES) * fast_stage_bytes(D);
+        const float* mats = reinterpret_cast<const float*>(smem + L.mats) + (ti & 1) * 2 * kPairs * kMatStride;
+        const int64_t head_row0 = (st.b * H + st.h) * (int64_t)D + 8 * c;  // first output row
+        const int64_t col = st.n0 * 2;
+        float2 si = make_float2(0.f, 0.f), so = si;
+        if (2 * pp < st.tv) {
+            fast_tensor<H16, 0>(in, mats, cj, sj, D, pp, c, a.k_scale,
+                                a.q_out + head_row0 * row_bytes + col, row_bytes, si, so);
+            fast_tensor<H16, 1>(in, mats, cj, sj, D, pp, c, a.k_scale,
+                                a.k_out + head_row0 * row_bytes + col, row_bytes, si, so);
+            fast_tensor<H16, 2>(in, mats, cj, sj, D, pp, c, a.k_scale,
+                                a.v_out + head_row0 * row_bytes + col, row_bytes, si, so);
+        }
+        *reinterpret_cast<float4*>(part + (s & 1) * C * kTile + c * kTile + 2 * pp) =
+            make_float4(si.x, so.x, si.y, so.y);
+        prev = st;
+        st.next(a, tiles_n, ntiles);
+    }
+    // The last step's key sums.
+    __syncthreads();
+    if (nsteps > 0 && a.inflation_sq) {
+        const float2* pprev = part + ((nsteps - 1) & 1) * C * kTile;
+        for (int t = tid; t < prev.tv; t += blockDim.x) {
+            float s_in = 0.f, s_out = 0.f;
+            for (int cc = 0; cc < C; ++cc) {
+                const float2 v = pprev[cc * kTile + t];
+                s_in += v.x;
+                s_out += v.y;
+            }
+            a.inflation_sq[(prev.b * H + prev.h) * N + prev.n0 + t] =
+                (s_in > 0.f && key_scaled) ? s_out / s_in : 1.0f;
+        }
+    }
+    cp_async_wait_all();
+}
+
 template <typename K>
 cudaError_t launch_pdl(K kern, int grid, int block, int smem, cudaStream_t stream,
                        const UcpeArgs& args) {
@@ -344,9 +694,70 @@ cudaError_t launch_pdl(K kern, int grid, int block, int smem, cudaStream_t strea
 
 }  // namespace
 
+cudaError_t launch_fast(const UcpeArgs& a, cudaStream_t stream, LaunchInfo* info, bool* used) {
+    *used = false;
+    const int D = a.head_dim;
+    const int block = 4 * D;  // 32 token pairs x D/8 chunks
+    int sms = 0, optin = 0, dev = 0;
+    cudaError_t e = cached_sm_count(&sms);
+    if (e != cudaSuccess) return e;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    // A tile's matrices are double-buffered, so the ring may run at most
+    // heads + 1 steps ahead (the next-but-one tile's matrices must not land
+    // while a tile still reads its own). Of the ring depths that fit, take the
+    // one that keeps the most head stages in flight per SM (CTAs per SM x
+    // (depth - 1)), the deeper ring on a tie.
+    int stages = 0, per_sm = 0, best = 0;
+    void (*kern)(const UcpeArgs) = nullptr;
+    for (int s = std::min(4, a.heads + 1); s >= 3; --s) {
+        if (fast_layout(D, s).total > optin) continue;
+        void (*k)(const UcpeArgs) =
+            s == 4 ? (a.act_f16 ? ucpe_fast_kernel<true, 4> : ucpe_fast_kernel<false, 4>)
+                   : (a.act_f16 ? ucpe_fast_kernel<true, 3> : ucpe_fast_kernel<false, 3>);
+        int n = 0;
+        if (cached_smem_and_occupancy(reinterpret_cast<const void*>(k), block,
+                                      fast_layout(D, s).total, &n) != cudaSuccess) {
+            cudaGetLastError();
+            continue;
+        }
+        if (n * (s - 1) > best) {
+            best = n * (s - 1);
+            stages = s;
+            per_sm = n;
+            kern = k;
+        }
+    }
+    if (!kern) return cudaSuccess;  // does not fit: the general kernel runs instead
+    const FastLayout L = fast_layout(D, stages);
+    const int64_t tiles = a.batch * ((a.num_tokens + kTile - 1) / kTile);
+    const int grid = (int)std::min<int64_t>((int64_t)sms * per_sm, tiles);
+    e = launch_pdl(kern, grid, block, L.total, stream, a);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        forget_kernel(reinterpret_cast<const void*>(kern));
+        e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), block, L.total, &per_sm);
+        if (e == cudaSuccess) e = launch_pdl(kern, grid, block, L.total, stream, a);
+    }
+    *used = true;
+    if (info) {
+        info->grid = grid;
+        info->block = block;
+        info->smem = L.total;
+        info->kernel_id = 5100 + 10 * stages + (a.act_f16 ? 1 : 0);
+    }
+    return e;
+}
+
 cudaError_t launch_ucpe(const UcpeArgs& a, cudaStream_t stream, LaunchInfo* info) {
     const int D = a.head_dim;
     if (D < 8 || D > 256 || D % 8 != 0) return cudaErrorInvalidValue;
+    if (D <= kFastMaxD && a.num_tokens % 8 == 0) {
+        bool used = false;
+        const cudaError_t e = launch_fast(a, stream, info, &used);
+        if (used || e != cudaSuccess) return e;
+    }
     const int block = ucpe_block(D), smem = ucpe_smem(D);
     void (*kern)(const UcpeArgs) = a.act_f16 ? ucpe_prep_kernel<true> : ucpe_prep_kernel<false>;
     int sms = 0, per_sm = 0;

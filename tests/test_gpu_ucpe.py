@@ -57,8 +57,20 @@ def _compare(outs, ref, ref_exact, act, where=""):
 
 
 CASES = [
-    # B, N, H, D, act: tiles of 64 tokens with ragged tails (N not a multiple
-    # of 64, and of 8: the two-byte store path), every chunk count parity
+    # B, N, H, D, act. The pipelined kernel takes head_dim <= 128, N a multiple
+    # of 8 and at least two heads: ring depths 3 (two heads, or head_dim 128)
+    # and 4, ragged last tiles, a single 8-token tile, several tiles per CTA.
+    (1, 64, 3, 8, "bf16"),
+    (2, 128, 4, 16, "bf16"),
+    (1, 200, 5, 56, "bf16"),
+    (1, 136, 2, 112, "bf16"),
+    (1, 8, 3, 112, "bf16"),
+    (3, 64, 3, 128, "bf16"),
+    (1, 1000, 20, 112, "bf16"),
+    (1, 192, 4, 64, "f16"),
+    # The general kernel: one head, N not a multiple of 8 (two-byte stores),
+    # head_dim above 128; tiles of 64 tokens with ragged tails, every chunk
+    # count parity
     (1, 64, 1, 8, "bf16"),
     (1, 200, 3, 16, "bf16"),
     (2, 130, 2, 24, "bf16"),
@@ -85,10 +97,11 @@ def test_ucpe_matches_oracle(B, N, H, D, act):
     _compare(outs, ref, ref_exact, act, where=f"B{B} N{N} H{H} D{D} {act}")
 
 
-def test_ucpe_identity_geometry_is_exact():
+@pytest.mark.parametrize("N", [100, 96])  # general kernel, pipelined kernel
+def test_ucpe_identity_geometry_is_exact(N):
     """Identity matrices, zero angles and k_scale 0.5: every output is its
     input's ReLU (and halving) moved to [B, H, D, N], exactly."""
-    B, N, H, D = 2, 100, 3, 32
+    B, H, D = 2, 3, 32
     _, inp = _case(B, N, H, D, seed=5)
     eye = torch.eye(4, device="cuda").expand(B, N, 4, 4).contiguous()
     c = torch.ones(N, D // 2, device="cuda")
@@ -103,10 +116,11 @@ def test_ucpe_identity_geometry_is_exact():
     assert torch.equal(infl, torch.ones_like(infl))
 
 
-def test_ucpe_zero_keys_and_extreme_values():
+@pytest.mark.parametrize("N", [70, 72])  # general kernel, pipelined kernel
+def test_ucpe_zero_keys_and_extreme_values(N):
     """Keys that ReLU zeroes give inflation_sq = 1; large and tiny values stay
     inside the tolerance."""
-    B, N, H, D = 1, 70, 2, 64
+    B, H, D = 1, 2, 64
     w, inp = _case(B, N, H, D, seed=9)
     k = inp["k_normed"].clone()
     k[0, 3, 1] = -k[0, 3, 1].abs() - 0.25          # ReLU(k) = 0 for this (token, head)
@@ -123,8 +137,25 @@ def test_ucpe_zero_keys_and_extreme_values():
              "bf16", where="extremes")
 
 
-def test_ucpe_inflation_optional_and_deterministic():
-    B, N, H, D = 1, 190, 4, 112
+@pytest.mark.parametrize("N", [60, 64])  # general kernel, pipelined kernel
+def test_ucpe_zero_k_scale(N):
+    """k_scale = 0 makes every scaled key zero: k_trans is zero and
+    inflation_sq is 1 everywhere (a zero key has no gain), as in the oracle."""
+    B, H, D = 1, 3, 48
+    w, inp = _case(B, N, H, D, seed=12)
+    outs = Q.cam_prep_func(inp["q_normed"], inp["k_normed"], inp["v_raw"], proj_q=inp["proj_q"],
+                           proj_kv=inp["proj_kv"], rope_cos=inp["rope_cos"],
+                           rope_sin=inp["rope_sin"], k_scale=0.0)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[1].float().abs(), torch.zeros_like(outs[1], dtype=torch.float32))
+    assert torch.equal(outs[3], torch.ones_like(outs[3]))
+    _compare(outs, _oracle(inp, 0.0, "bf16"), _oracle(inp, 0.0, "bf16", exact=True), "bf16",
+             where="k_scale 0")
+
+
+@pytest.mark.parametrize("N", [190, 192])  # general kernel, pipelined kernel
+def test_ucpe_inflation_optional_and_deterministic(N):
+    B, H, D = 1, 4, 112
     w, inp = _case(B, N, H, D, seed=2)
     args = (inp["q_normed"], inp["k_normed"], inp["v_raw"], inp["proj_q"], inp["proj_kv"],
             inp["rope_cos"], inp["rope_sin"])
