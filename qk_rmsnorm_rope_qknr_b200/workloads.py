@@ -190,14 +190,20 @@ def rope_table_input(tokens: int, rotary_dim: int, base: float, f32: bool,
 
 def camera_matrices(g: torch.Generator, batch: int, tokens: int, translation_std: float,
                     device="cpu"):
-    """Per-token rigid motions G = [[R, t], [0, 1]]: R a random rotation (the Q
-    factor of a Gaussian 3x3 matrix, column signs fixed), t ~ N(0,
-    translation_std^2). Returns (G^T, G^-1) as float32 [batch, tokens, 4, 4]: the
-    Q and K/V matrices of a camera pair whose relative motion the attention
-    sees (inputs only: the camera prep multiplies by whatever it is given)."""
-    a = torch.randn((batch, tokens, 3, 3), generator=g, dtype=torch.float64, device=device)
-    rot, r = torch.linalg.qr(a)
-    rot = rot * torch.sign(torch.diagonal(r, dim1=-2, dim2=-1)).unsqueeze(-2)
+    """Per-token rigid motions G = [[R, t], [0, 1]]: R the rotation of a random
+    unit quaternion (a normalised Gaussian 4-vector, so R is uniform over the
+    rotations), t ~ N(0, translation_std^2). Returns (G^T, G^-1) as float32
+    [batch, tokens, 4, 4]: the Q and K/V matrices of a camera pair whose
+    relative motion the attention sees (inputs only: the camera prep multiplies
+    by whatever it is given)."""
+    qv = torch.randn((batch, tokens, 4), generator=g, dtype=torch.float64, device=device)
+    qv = qv / qv.norm(dim=-1, keepdim=True)
+    w, x, y, z = qv.unbind(-1)
+    rot = torch.stack([
+        torch.stack([1 - 2 * (y * y + z * z), 2 * (x * y - z * w), 2 * (x * z + y * w)], -1),
+        torch.stack([2 * (x * y + z * w), 1 - 2 * (x * x + z * z), 2 * (y * z - x * w)], -1),
+        torch.stack([2 * (x * z - y * w), 2 * (y * z + x * w), 1 - 2 * (x * x + y * y)], -1),
+    ], -2)
     t = torch.randn((batch, tokens, 3), generator=g, dtype=torch.float64, device=device)
     t = t * translation_std
     G = torch.zeros((batch, tokens, 4, 4), dtype=torch.float64, device=device)
