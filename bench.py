@@ -35,8 +35,8 @@ FALLBACK_HBM_GBS = 6650.0
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu
 # captures summarised in profiles/ (rope3d_video3d.md, rope3d_fp8neox.md,
-# rope_table.md), valid only for the kernel sources whose hash is stored
-# beside it (the bench reports null otherwise).
+# rope_table.md, ucpe_cam_prep.md), valid only for the kernel sources whose
+# hash is stored beside it (the bench reports null otherwise).
 TRAFFIC = {
     "video3d": (377564416 + 325334784, "f0170ddbe869b9f9"),
     "fp8neox": (1097153280 + 517297920, "f0170ddbe869b9f9"),
@@ -44,6 +44,7 @@ TRAFFIC = {
     "table_il": (25730816 + 15616, "9230c313092c6dc7"),
     "table_hs_f16": (42770176 + 2013952, "9230c313092c6dc7"),
     "table_d72": (24805120 + 3584, "9230c313092c6dc7"),
+    "ucpe": (259080000 + 202420000, "5fc2b64ced912874"),  # ncu's MB, rounded to 10 kB
 }
 KERNEL_FILES = {"3d": "rope3d.cu", "table": "rope_table.cu", "ucpe": "ucpe.cu"}
 
