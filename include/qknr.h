@@ -244,8 +244,14 @@ int qknr_rope_3d_with_ssq(const qknr_rope_3d_params* params, const float* ssq,
  * Alignment: every pointer 16-byte aligned (QKNR_ERR_ALIGN otherwise).
  * num_tokens that is not a multiple of 8 is allowed; the output rows then
  * are not 16-byte aligned and are written two bytes at a time.
- * Range: |k'|^2 and |y|^2 are fp32 sums, so keys whose squares underflow
- * fp32 (|k'| below about 1e-19) count as zero keys (inflation_sq 1).
+ * Range: the two sums of squares are fp32, taken over the key before the
+ * scale (head_dim <= 128 with num_tokens a multiple of 8) or after it (other
+ * shapes; the ratio is the same), so a key whose squares all underflow fp32
+ * (every channel below about 1e-19 in magnitude) counts as a zero key
+ * (inflation_sq 1).
+ * The kernels wait only on their own cp.async groups and bulk stores, which
+ * always complete, so they have no timeout path and do not set the device
+ * status word.
  */
 int qknr_ucpe_cam_prep(const void* q_normed, const void* k_normed, const void* v_raw,
                        const float* proj_q, const float* proj_kv, const float* rope_cos,
