@@ -236,3 +236,43 @@ def test_ucpe_workload_full_size_sampled():
     got = [o[..., it] for o in outs[:3]] + [outs[3][..., it]]
     _compare(got, ref, ref_exact, "bf16", where="ucpe full size")
     assert torch.isfinite(outs[3]).all()
+
+
+@pytest.mark.parametrize("N,cuts", [(192, [64, 136]), (150, [40, 97])])
+def test_ucpe_token_shards_match_whole_call(N, cuts):
+    """Sequence shards need no exchange: every token's result depends only on
+    its own rows, matrices and table row, so shards [n0, n1) (each with its
+    rows of the inputs, matrices and tables) reproduce the whole call's
+    columns n0..n1. N = 192: whole call and shards all take the pipelined
+    kernel, bit for bit. N = 150: the whole call takes the general kernel and
+    the first shard the pipelined one, which apply K's scale at another point,
+    so those may differ by the rounding of that step."""
+    B, H, D = 2, 3, 64
+    w, inp = _case(B, N, H, D, seed=21)
+    whole = Q.cam_prep_func(inp["q_normed"], inp["k_normed"], inp["v_raw"], proj_q=inp["proj_q"],
+                            proj_kv=inp["proj_kv"], rope_cos=inp["rope_cos"],
+                            rope_sin=inp["rope_sin"], k_scale=w.k_scale)
+    bounds = [0] + cuts + [N]
+    for n0, n1 in zip(bounds[:-1], bounds[1:]):
+        sl = slice(n0, n1)
+        part = Q.cam_prep_func(*(inp[k][:, sl].contiguous() for k in ("q_normed", "k_normed", "v_raw")),
+                               proj_q=inp["proj_q"][:, sl].contiguous(),
+                               proj_kv=inp["proj_kv"][:, sl].contiguous(),
+                               rope_cos=inp["rope_cos"][sl].contiguous(),
+                               rope_sin=inp["rope_sin"][sl].contiguous(), k_scale=w.k_scale)
+        torch.cuda.synchronize()
+        same_kernel = N % 8 == 0 and (n1 - n0) % 8 == 0
+        for a, b in zip(whole[:3], part[:3]):
+            if same_kernel:
+                assert torch.equal(a[..., sl], b)
+            else:
+                assert _same_within_rounding(a[..., sl], b)
+        torch.testing.assert_close(whole[3][..., sl], part[3], rtol=INFL_RTOL, atol=0)
+
+
+def _same_within_rounding(a, b):
+    """The two kernels may differ in the last bit where K's scale is applied
+    at a different point; 1 bf16 ulp at the row scale is allowed between them."""
+    x, y = a.float(), b.float()
+    scale = x.abs().amax(dim=2, keepdim=True).clamp_min(1e-30)
+    return bool(((x - y).abs() <= scale * 2.0 ** -7).all())
