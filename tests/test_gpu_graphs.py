@@ -1,4 +1,4 @@
-"""Both entry points can be captured in a CUDA graph and replayed: the library
+"""Every entry point can be captured in a CUDA graph and replayed: the library
 neither allocates nor synchronises, and its host-side checks are not stream
 work. Replays must match eager calls bit for bit, also after the inputs change
 in place."""
@@ -57,3 +57,32 @@ def test_table_graph_replay():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(eq, qo) and torch.equal(ek, ko)
+
+
+@pytest.mark.parametrize("N", [192, 150])  # pipelined kernel, general kernel
+def test_ucpe_graph_replay(N):
+    w = W.FormUcpe("g", batch=1, seq=N, heads=4, head_dim=112, spatial=N // 4)
+    inp = {k: v.cuda() for k, v in W.make_inputs(w).items()}
+    names = ("q_normed", "k_normed", "v_raw", "proj_q", "proj_kv", "rope_cos", "rope_sin")
+    outs = [torch.empty(1, 4, 112, N, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    infl = torch.empty(1, 4, N, device="cuda")
+    s = torch.cuda.Stream()
+
+    def call(o, f, stream=None):
+        Q.qknr_ucpe_cam_prep(*(inp[n] for n in names), *o, f, k_scale=w.k_scale, stream=stream)
+
+    with torch.cuda.stream(s):
+        call(outs, infl, s)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        call(outs, infl, s)
+    inp["k_normed"].mul_(-0.5)
+    inp["proj_kv"].mul_(2.0)
+    eager = [torch.empty_like(o) for o in outs]
+    einfl = torch.empty_like(infl)
+    call(eager, einfl)
+    g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(eager + [einfl], outs + [infl]):
+        assert torch.equal(a, b)

@@ -485,7 +485,7 @@ def test_3d_sequence_shards_match_whole_call():
 
 
 def test_concurrent_host_threads_match_serial():
-    """Several host threads calling both entry points at once, each on its own
+    """Several host threads calling the entry points at once, each on its own
     stream and with its own shapes (the launch caches and lane plans are shared
     state), give the bits of the same calls made one after another."""
     import threading
@@ -499,16 +499,22 @@ def test_concurrent_host_threads_match_serial():
         D, R = (128, 96) if i % 2 == 0 else (72, 40)
         t = {n: v.to(DEV) for n, v in _rand_table_inputs(64, 3, 1 + i, D, R, True,
                                                           seed=30 + i).items()}
-        jobs.append((qkv, qw, kw, p3, t, R, bool(i % 2)))
+        wu = W.FormUcpe("u", batch=1, seq=(96, 150, 64, 130)[i], heads=2 + i,
+                        head_dim=(112, 64, 128, 48)[i], spatial=16, seed=40 + i)
+        u = {n: v.to(DEV) for n, v in W.make_inputs(wu).items()}
+        jobs.append((qkv, qw, kw, p3, t, R, bool(i % 2), u, wu.k_scale))
 
     def run(job, stream):
-        qkv, qw, kw, p3, t, R, il = job
+        qkv, qw, kw, p3, t, R, il, u, ks = job
         outs = []
         for _ in range(10):
             a = run_3d(qkv, qw, kw, stream=stream, **p3)
             b = Q.fused_qk_norm_rope(t["q"], t["k"], t["q_weight"], t["k_weight"], t["rope_table"],
                                      1e-6, rotary_dim=R, interleaved=il, stream=stream)
-            outs.append([x.clone() for x in (*a, *b)])
+            c = Q.cam_prep_func(u["q_normed"], u["k_normed"], u["v_raw"], proj_q=u["proj_q"],
+                                proj_kv=u["proj_kv"], rope_cos=u["rope_cos"],
+                                rope_sin=u["rope_sin"], k_scale=ks, stream=stream)
+            outs.append([x.clone() for x in (*a, *b, *c)])
         return outs
 
     serial = [run(j, torch.cuda.current_stream()) for j in jobs]
