@@ -242,11 +242,12 @@ int qknr_rope_3d_with_ssq(const qknr_rope_3d_params* params, const float* ssq,
  * k_scale          any finite float (the page's value is
  *                  head_dim^-0.5 * spatial_tokens^-0.5).
  * Alignment: every pointer 16-byte aligned (QKNR_ERR_ALIGN otherwise).
- * num_tokens that is not a multiple of 8 is allowed; the output rows then
- * are not 16-byte aligned and are written two bytes at a time.
+ * Any num_tokens is allowed. head_dim <= 128 with an even num_tokens and at
+ * least two heads runs the pipelined kernel; other shapes run a general one,
+ * which writes two bytes at a time when num_tokens is not a multiple of 8.
  * Range: the two sums of squares are fp32, taken over the key before the
- * scale (head_dim <= 128 with num_tokens a multiple of 8) or after it (other
- * shapes; the ratio is the same), so a key whose squares all underflow fp32
+ * scale (the pipelined kernel) or after it (the general one; the ratio is
+ * the same), so a key whose squares all underflow fp32
  * (every channel below about 1e-19 in magnitude) counts as a zero key
  * (inflation_sq 1).
  * The kernels wait only on their own cp.async groups and bulk stores, which

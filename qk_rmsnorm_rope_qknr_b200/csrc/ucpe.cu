@@ -364,7 +364,8 @@ __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Fast kernel: head_dim <= 128, num_tokens a multiple of 8.
+// Fast kernel: head_dim <= 128, num_tokens even (whole token pairs, 4-byte
+// aligned output rows), at least two heads.
 //
 // Work unit: a tile of 64 tokens of one batch element, all heads in turn.
 // Lane i of every warp owns the token pair (2i, 2i+1) of the tile; warp w owns
@@ -753,7 +754,7 @@ cudaError_t launch_fast(const UcpeArgs& a, cudaStream_t stream, LaunchInfo* info
 cudaError_t launch_ucpe(const UcpeArgs& a, cudaStream_t stream, LaunchInfo* info) {
     const int D = a.head_dim;
     if (D < 8 || D > 256 || D % 8 != 0) return cudaErrorInvalidValue;
-    if (D <= kFastMaxD && a.num_tokens % 8 == 0) {
+    if (D <= kFastMaxD && a.num_tokens % 2 == 0) {
         bool used = false;
         const cudaError_t e = launch_fast(a, stream, info, &used);
         if (used || e != cudaSuccess) return e;
