@@ -453,10 +453,18 @@ __device__ __forceinline__ void fast_stage_mats(const UcpeArgs& a, const FastSte
     }
 }
 
+// The warp rank that decides which token rows a warp copies. 64 rows over
+// 2 * warps half-warps leave some half-warps one row more than others; the
+// rotation gives the longer share to warps 4.. and keeps it off warps 0 and 1,
+// which also add up the key sums, so that no warp is late at the barrier.
+__device__ __forceinline__ int copy_rank(int warp, int nwarps) {
+    return nwarps > 4 ? (warp + nwarps - 4) % nwarps : warp;
+}
+
 // One head's Q, K, V rows of a tile into ring stage `buf` (16-byte copies;
 // sixteen lanes per token row, lane k copying chunk k of that token's Q, K and
-// V rows; a lane takes tokens t0, t0 + 2 * warps, ...; tokens past the tile's
-// end read as zeros). `off` is the byte offset of chunk k of token t0's row at
+// V rows; a lane takes tokens t0, t0 + 2 * warps, ... with t0 from its warp's
+// copy rank; tokens past the tile's end read as zeros). `off` is the byte offset of chunk k of token t0's row at
 // head 0 of the tile (fast_row_offset); successive tokens of the lane are
 // 2 * warps rows apart.
 __device__ __forceinline__ void fast_stage_head(const UcpeArgs& a, const FastStep& st, int64_t off,
@@ -468,7 +476,7 @@ __device__ __forceinline__ void fast_stage_head(const UcpeArgs& a, const FastSte
     if (k4 >= C) return;
     const int64_t step = (int64_t)2 * nwarps * a.heads * D * 2;
     int64_t o = off + (int64_t)st.h * D * 2;
-    for (int t = 2 * warp + (lane >> 4); t < kTile; t += 2 * nwarps, o += step) {
+    for (int t = 2 * copy_rank(warp, nwarps) + (lane >> 4); t < kTile; t += 2 * nwarps, o += step) {
         const bool ok = t < st.tv;
         const int64_t src = ok ? o : 0;
         unsigned char* dst = buf + (t >> 1) * ps + (t & 1) * 2 * D + 16 * k4;
@@ -481,8 +489,8 @@ __device__ __forceinline__ void fast_stage_head(const UcpeArgs& a, const FastSte
 // Byte offset (from the tensor base) of chunk k4 of this lane's first token
 // row at head 0 of the tile.
 __device__ __forceinline__ int64_t fast_row_offset(const UcpeArgs& a, const FastStep& st) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int t0 = 2 * warp + (lane >> 4);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int t0 = 2 * copy_rank(warp, nwarps) + (lane >> 4);
     return ((st.b * a.num_tokens + st.n0 + t0) * a.heads * a.head_dim + 8 * (lane & 15)) * 2;
 }
 
