@@ -214,7 +214,7 @@ def pin_rotation_is_complex_product():
 
 
 def pin_pair_maps():
-    """[T] contract bullets: half-split pairs (d, d + rotary_dim/2); interleaved
+    """[T] contract bullets: half-split pairing of channel d with d + rotary_dim/2; interleaved
     adjacent pairs (2i, 2i+1). [F] interleave=False is NeoX style: whole-head
     half split (the reading taken here)."""
     pa, pb = O.pairs_table(8, True)
@@ -251,7 +251,7 @@ def pin_table_hand_case():
 
 
 def pin_weight_before_rotation():
-    """[T] 'Q/K RMSNorm followed by packed RoPE': the weight scales the channel
+    """[T] (contract bullets: the norm comes first, then the rotation): the weight scales the channel
     before it turns. D = 2, x = (1, 1): mean square 1, so y = (w0, w1) = (2, 0.5);
     a 90-degree turn gives (-0.5, 2). (Weighting after the turn would give
     (-1, 1) * (2, 0.5) = (-2, 0.5).)"""
