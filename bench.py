@@ -46,7 +46,8 @@ TRAFFIC = {
     "table_d72": (24805120 + 3584, "9230c313092c6dc7"),
     "ucpe": (259065344 + 204187904, "f45904e98df57c00"),
 }
-KERNEL_FILES = {"3d": "rope3d.cu", "table": "rope_table.cu", "ucpe": "ucpe.cu"}
+KERNEL_FILES = {"3d": ("rope3d.cu",), "table": ("rope_table.cu",),
+                "ucpe": ("ucpe_launch.h", "ucpe.cu")}
 
 
 def kernel_source_hash(form: str = "3d") -> str:
@@ -57,7 +58,7 @@ def kernel_source_hash(form: str = "3d") -> str:
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "qk_rmsnorm_rope_qknr_b200", "csrc")
-    for f in ("common.cuh", "launch.h", "launch_cache.h", KERNEL_FILES[form]):
+    for f in ("common.cuh", "launch.h", "launch_cache.h") + KERNEL_FILES[form]:
         with open(os.path.join(csrc, f)) as fh:
             code = fh.read()
         code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)

@@ -1,5 +1,5 @@
 // Internal interface between the C-ABI layer (qknr_abi.cu) and the kernel
-// launchers (rope3d.cu, rope_table.cu, ucpe.cu). Arguments are already validated.
+// launchers (rope3d.cu, rope_table.cu). Arguments are already validated.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -64,24 +64,6 @@ struct RopeTableArgs {
     uint64_t wait_limit_ns;   // a wait on a bulk copy gives up after this long
 };
 
-struct UcpeArgs {
-    const uint8_t* q;  // 16-bit activations [B, N, H, D], dense
-    const uint8_t* k;
-    const uint8_t* v;
-    const float* proj_q;   // [B, N, 4, 4] row-major
-    const float* proj_kv;  // [B, N, 4, 4]
-    const float* rope_cos; // [N, D/2]
-    const float* rope_sin; // [N, D/2]
-    uint8_t* q_out;        // 16-bit [B, H, D, N]
-    uint8_t* k_out;
-    uint8_t* v_out;
-    float* inflation_sq;   // [B, H, N] or null (not computed)
-    int64_t batch, num_tokens;
-    int32_t heads, head_dim;
-    int32_t act_f16;  // activations are binary16, else bf16
-    float k_scale;
-};
-
 // Launch description returned for the benchmark and tests.
 struct LaunchInfo {
     int grid;
@@ -99,10 +81,6 @@ cudaError_t launch_rope3d(const Rope3DArgs& a, int head_dim, int neox, int fp8,
 cudaError_t read_device_status(uint32_t* out, int clear, cudaStream_t stream);
 cudaError_t launch_rope_table(const RopeTableArgs& a, int fast_path, cudaStream_t stream,
                               LaunchInfo* info);
-
-// UCPE camera prep (head_dim a multiple of 8 up to 256; pointers 16-byte
-// aligned; sizes already checked).
-cudaError_t launch_ucpe(const UcpeArgs& a, cudaStream_t stream, LaunchInfo* info);
 
 // Status word of the table kernels (bit 0 as for the 3D kernels).
 cudaError_t read_table_status(uint32_t* out, int clear, cudaStream_t stream);

@@ -4,6 +4,7 @@
 #include "qknr.h"
 
 #include "launch.h"
+#include "ucpe_launch.h"
 
 #include <cuda_runtime.h>
 

@@ -30,7 +30,7 @@
 // tile; the per-chunk key sums are summed per token in a fixed order, so the
 // results do not depend on the launch shape.
 #include "common.cuh"
-#include "launch.h"
+#include "ucpe_launch.h"
 #include "launch_cache.h"
 
 #include <algorithm>
