@@ -10,7 +10,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-@pytest.mark.parametrize("workload", ["tiny3d", "table_il"])
+@pytest.mark.parametrize("workload", ["tiny3d", "table_il", "ucpe"])
 def test_reference_arm_json_line(workload):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                         "--workload", workload, "--steps", "3", "--warmup", "3",
