@@ -228,6 +228,20 @@ def oracle_sample_ucpe(w, inp_cpu, budget_s: float, chunk: int):
     return done, spent, O.threads()
 
 
+def one_core(w, inp_cpu, budget_s: float, chunk: int):
+    """The oracle on one host thread, for the single-core figure beside the
+    all-core one; returns tokens/s."""
+    import oracle as O
+
+    before = O.threads()
+    O.set_threads(1)
+    try:
+        n, sec, _ = oracle_sample(w, inp_cpu, budget_s, chunk)
+    finally:
+        O.set_threads(before)
+    return n / sec
+
+
 def run_reference(args, w):
     """--impl reference: the oracle as it stands, on the host cores."""
     from qk_rmsnorm_rope_qknr_b200 import workloads as W
@@ -363,7 +377,8 @@ def run_gpu(args, w):
         n, s, threads = oracle_sample(w, inp_cpu, args.cpu_seconds)
         cpu = {"value": n / s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} tokens of {w.name} in order, cycling through its {T} "
-                         f"({s:.1f} s of fp64 oracle work)"}
+                         f"({s:.1f} s of fp64 oracle work)",
+               "value_1core": one_core(w, inp_cpu, args.cpu_seconds / 4, 256)}
 
     if rank == 0:
         clk = clocks.summary()
@@ -470,7 +485,8 @@ def run_gpu_table(args, w):
         n, sec, threads = oracle_sample(w, inp_cpu, args.cpu_seconds, chunk=128)
         cpu = {"value": n / sec, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} tokens of {w.name} in order, cycling through its {T} "
-                         f"({sec:.1f} s of fp64 oracle work)"}
+                         f"({sec:.1f} s of fp64 oracle work)",
+               "value_1core": one_core(w, inp_cpu, args.cpu_seconds / 4, 128)}
     if rank == 0:
         q = sets[0]["q"]
         line = {
@@ -754,7 +770,8 @@ def run_gpu_ucpe(args, w):
         n, sec, threads = oracle_sample(w, inp_cpu, args.cpu_seconds, chunk=64)
         cpu = {"value": n / sec, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} tokens (all {H} heads each) of {w.name} in order, cycling "
-                         f"through its {B * N} ({sec:.1f} s of fp64 oracle work)"}
+                         f"through its {B * N} ({sec:.1f} s of fp64 oracle work)",
+               "value_1core": one_core(w, inp_cpu, args.cpu_seconds / 4, 16)}
     if rank == 0:
         in_mb = sum(inp[n].numel() * inp[n].element_size() for n in UCPE_INPUTS) / 1e6
         line = {

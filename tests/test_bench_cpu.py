@@ -43,3 +43,22 @@ def test_kernel_hash_ignores_comments(tmp_path, monkeypatch):
     assert bench.kernel_source_hash("3d") == h0
     p.write_text(p.read_text().replace("kMaxGroups = 15", "kMaxGroups = 14"))
     assert bench.kernel_source_hash("3d") != h0
+
+
+def test_one_core_figure_restores_threads():
+    """The single-thread oracle figure beside the all-core one: positive, and
+    the oracle's thread count is as before afterwards."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle as O
+    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+
+    before = O.threads()
+    for name, chunk in (("tiny3d", 16), ("table_il", 16)):
+        w = W.WORKLOADS[name]
+        inp = W.make_inputs(w, device="cpu", tokens=64 if name == "table_il" else None)
+        if name == "table_il":
+            import dataclasses
+            w = dataclasses.replace(w, tokens=64)
+        assert bench.one_core(w, inp, 0.05, chunk) > 0
+        assert O.threads() == before
