@@ -524,8 +524,10 @@ def measure_e2e_table(args, w, dset, run, stream, dev, world, pg):
     """End to end through the C ABI for the table form, inputs and outputs in
     page-locked host memory: staged (copy q, k and the table in, run, copy
     q_out and k_out back), zero-copy (the kernel reads and writes the host
-    buffers across the bus) or pipelined (8 token chunks on three streams);
-    the fastest is reported, beside the time of the copies alone."""
+    buffers across the bus), pipelined (8 token chunks on three streams) or
+    across-steps (two device sets, step i's outputs leaving while step i+1's
+    inputs arrive); the fastest is reported, beside the time of the copies
+    alone. Every step moves all of its inputs in and its outputs back."""
     import torch
 
     names_in = ("q", "k", "q_weight", "k_weight", "rope_table")
@@ -595,6 +597,57 @@ def measure_e2e_table(args, w, dset, run, stream, dev, world, pg):
             ms = t.item()
         return ms
 
+    # across steps: two device sets on two copy streams, so that step i's
+    # outputs go back while step i+1's inputs come in
+    sets2 = [dev_set, {n: torch.empty_like(dset[n]) for n in dset}]
+    sets2[1]["q_weight"], sets2[1]["k_weight"] = dset["q_weight"], dset["k_weight"]
+    x_in, x_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    xe_in = [torch.cuda.Event() for _ in range(2)]
+    xe_k = [torch.cuda.Event() for _ in range(2)]
+    xe_out = [torch.cuda.Event() for _ in range(2)]
+    for e in xe_out:
+        e.record(x_out)
+    xstep = [0]
+
+    def across_steps():
+        k = xstep[0] % 2
+        xstep[0] += 1
+        dv = sets2[k]
+        with torch.cuda.stream(x_in):
+            x_in.wait_event(xe_k[k])       # the kernel two steps back has read these
+            for n in ("q", "k", "rope_table"):
+                dv[n].copy_(host[n], non_blocking=True)
+            xe_in[k].record(x_in)
+        stream.wait_event(xe_in[k])
+        stream.wait_event(xe_out[k])       # its outputs of two steps back have left
+        run(dv)
+        xe_k[k].record(stream)
+        with torch.cuda.stream(x_out):
+            x_out.wait_event(xe_k[k])
+            for n in ("q_out", "k_out"):
+                host[n].copy_(dv[n], non_blocking=True)
+            xe_out[k].record(x_out)
+
+    def timed_across():
+        for _ in range(2):
+            across_steps()
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            across_steps()
+        stream.wait_stream(x_out)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms_ = a.elapsed_time(b) / steps
+        if pg:
+            t = torch.tensor([ms_], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ms_ = t.item()
+        return ms_
+
     # The bus alone: the same bytes copied in and out at once, no kernel.
     s_copy = torch.cuda.Stream(dev)
 
@@ -606,7 +659,8 @@ def measure_e2e_table(args, w, dset, run, stream, dev, world, pg):
                 host[n].copy_(dset[n], non_blocking=True)
         stream.wait_stream(s_copy)
 
-    ms = {"staged": timed(staged), "zero-copy": timed(zero_copy), "pipelined": timed(pipelined)}
+    ms = {"staged": timed(staged), "zero-copy": timed(zero_copy), "pipelined": timed(pipelined),
+          "across-steps": timed_across()}
     best = min(ms, key=ms.get)
     bus_ms = timed(copies_only)
     nbytes = lambda names: sum(dset[n].numel() * dset[n].element_size() for n in names)  # noqa
