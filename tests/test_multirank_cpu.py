@@ -1,9 +1,10 @@
 """The multi-rank path on CPU: world size 2 over gloo.
 
 Each rank takes its contiguous token shard of one 3D sequence (and of one
-table-form batch), runs the oracle on it with the shard's pos_offset (or table
-rows), and all_gathers the pieces; the result must equal the unsharded call
-bit for bit. This checks the sharding arithmetic with real collectives; on
+table-form batch, and of one camera-prep call), runs the oracle on it with the
+shard's pos_offset (or table rows, or rows of every per-token input), and
+all_gathers the pieces; the result must equal the unsharded call bit for
+bit. This checks the sharding arithmetic with real collectives; on
 GPUs the same shards go to qknr_rope_3d / qknr_rope_table on each rank.
 """
 import os
@@ -75,6 +76,27 @@ def _worker(rank, port, out_dir):
             pieces = [None] * WORLD
             dist.all_gather_object(pieces, part)
             assert np.array_equal(np.concatenate(pieces), r)
+        # --- camera prep: 37 tokens of 2 batch elements; the shard takes its
+        # rows of q/k/v and of the matrices and tables, and its outputs are the
+        # whole call's columns ([B, H, D, N]: the token axis is the last)
+        from qk_rmsnorm_rope_qknr_b200 import workloads as W
+
+        wu = W.FormUcpe("mr", batch=2, seq=37, heads=3, head_dim=16, spatial=9, seed=6)
+        u = W.make_inputs(wu, device="cpu")
+        s, c = sharding.token_shard(37, WORLD, rank)
+        sl = slice(s, s + c)
+
+        def cam(inp, rows):
+            return O.ucpe_cam_prep(t2u16(inp["q_normed"][:, rows]), t2u16(inp["k_normed"][:, rows]),
+                                   t2u16(inp["v_raw"][:, rows]), inp["proj_q"][:, rows].numpy(),
+                                   inp["proj_kv"][:, rows].numpy(), inp["rope_cos"][rows].numpy(),
+                                   inp["rope_sin"][rows].numpy(), wu.k_scale)
+
+        mine, ref = cam(u, sl), cam(u, slice(0, 37))
+        for part, r in zip(mine, ref):
+            pieces = [None] * WORLD
+            dist.all_gather_object(pieces, part)
+            assert np.array_equal(np.concatenate(pieces, axis=-1), r)
         dist.barrier()
         open(os.path.join(out_dir, f"ok{rank}"), "w").write("ok")
     finally:
