@@ -11,8 +11,10 @@
 //   V: times proj_kv blockwise;
 // and the three results are stored transposed, [B, H, D, N].
 //
-// The work is a stream over HBM (about 1.5 flops per byte), so the kernel is
-// built for coalescing on both sides of the transpose:
+// The work is a stream over HBM (about 1.5 flops per byte). Two kernels do it:
+// ucpe_fast_kernel (further down) for head_dim <= 128, an even token count and
+// at least two heads, and ucpe_prep_kernel for every other shape. Both are
+// built for coalescing on both sides of the transpose. The general kernel:
 //   - work unit: a tile of 64 consecutive tokens of one (batch, head), tiles
 //     numbered with the head fastest, so that the tiles in flight at once
 //     share their tokens' cos/sin rows and matrices in L2;
@@ -26,9 +28,10 @@
 //     still reads back as eight whole chunks;
 //   - the tile leaves with 16-byte stores, eight threads per output row: each
 //     row's 64 tokens are one 128-byte line of the [B, H, D, N] output.
-// The 4x4 matrices of the tile's tokens are staged in shared memory once per
-// tile; the per-chunk key sums are summed per token in a fixed order, so the
-// results do not depend on the launch shape.
+// The 4x4 matrices and the cos/sin rows of the tile's tokens are copied into
+// shared memory with cp.async (the next tile's while this one's results leave);
+// the per-chunk key sums are added per token in a fixed order, so the results
+// do not depend on the launch shape.
 #include "common.cuh"
 #include "ucpe_launch.h"
 #include "launch_cache.h"
