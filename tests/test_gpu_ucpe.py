@@ -69,6 +69,8 @@ CASES = [
     (3, 64, 3, 128, "bf16"),
     (1, 1000, 20, 112, "bf16"),
     (1, 192, 4, 64, "f16"),
+    (1, 266, 3, 104, "bf16"),   # 13 warps
+    (2, 130, 5, 120, "bf16"),   # 15 warps; the 4-stage ring needs 224 KB, at the opt-in limit
     (2, 130, 2, 24, "bf16"),
     (1, 150, 3, 112, "f16"),
     (2, 64, 2, 40, "f16"),
