@@ -44,7 +44,7 @@ TRAFFIC = {
     "table_il": (25730816 + 15616, "9230c313092c6dc7"),
     "table_hs_f16": (42770176 + 2013952, "9230c313092c6dc7"),
     "table_d72": (24805120 + 3584, "9230c313092c6dc7"),
-    "ucpe": (259065344 + 202497280, "455bbd5c9475b036"),
+    "ucpe": (259064832 + 202290688, "a8106b18f58c9fbf"),
 }
 KERNEL_FILES = {"3d": ("rope3d.cu",), "table": ("rope_table.cu",),
                 "ucpe": ("ucpe_launch.h", "ucpe.cu")}

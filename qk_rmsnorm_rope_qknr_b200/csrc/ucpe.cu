@@ -614,6 +614,23 @@ __global__ void __launch_bounds__(512, 1) ucpe_fast_kernel(const UcpeArgs a) {
     float2 cj[4], sj[4];
     FastStep prev{};
     for (int64_t s = 0; s < nsteps; ++s) {
+        // At a tile's first head its cos/sin go out first: they do not depend
+        // on shared memory, so their latency overlaps the wait and the barrier.
+        if (st.h == 0) {
+            // this tile's cos/sin for the thread's pair and chunk, for all heads
+            const int half = D / 2;
+            const int64_t r0 = (st.n0 + 2 * pp) * half + 4 * c;
+            const bool ok0 = 2 * pp < st.tv, ok1 = 2 * pp + 1 < st.tv;
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 c0 = ok0 ? __ldg(reinterpret_cast<const float4*>(a.rope_cos + r0)) : z;
+            const float4 c1 = ok1 ? __ldg(reinterpret_cast<const float4*>(a.rope_cos + r0 + half)) : z;
+            const float4 s0 = ok0 ? __ldg(reinterpret_cast<const float4*>(a.rope_sin + r0)) : z;
+            const float4 s1 = ok1 ? __ldg(reinterpret_cast<const float4*>(a.rope_sin + r0 + half)) : z;
+            cj[0] = make_float2(c0.x, c1.x); cj[1] = make_float2(c0.y, c1.y);
+            cj[2] = make_float2(c0.z, c1.z); cj[3] = make_float2(c0.w, c1.w);
+            sj[0] = make_float2(s0.x, s1.x); sj[1] = make_float2(s0.y, s1.y);
+            sj[2] = make_float2(s0.z, s1.z); sj[3] = make_float2(s0.w, s1.w);
+        }
         cp_async_wait_pending<STAGES - 2>();  // this step's group is complete
         __syncthreads();
         // The stage of step s - 1 is free now: refill it with step s + STAGES - 1.
@@ -637,21 +654,6 @@ __global__ void __launch_bounds__(512, 1) ucpe_fast_kernel(const UcpeArgs a) {
         }
 
         const int64_t ti = st.ti;
-        if (st.h == 0) {
-            // this tile's cos/sin for the thread's pair and chunk, for all heads
-            const int half = D / 2;
-            const int64_t r0 = (st.n0 + 2 * pp) * half + 4 * c;
-            const bool ok0 = 2 * pp < st.tv, ok1 = 2 * pp + 1 < st.tv;
-            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 c0 = ok0 ? __ldg(reinterpret_cast<const float4*>(a.rope_cos + r0)) : z;
-            const float4 c1 = ok1 ? __ldg(reinterpret_cast<const float4*>(a.rope_cos + r0 + half)) : z;
-            const float4 s0 = ok0 ? __ldg(reinterpret_cast<const float4*>(a.rope_sin + r0)) : z;
-            const float4 s1 = ok1 ? __ldg(reinterpret_cast<const float4*>(a.rope_sin + r0 + half)) : z;
-            cj[0] = make_float2(c0.x, c1.x); cj[1] = make_float2(c0.y, c1.y);
-            cj[2] = make_float2(c0.z, c1.z); cj[3] = make_float2(c0.w, c1.w);
-            sj[0] = make_float2(s0.x, s1.x); sj[1] = make_float2(s0.y, s1.y);
-            sj[2] = make_float2(s0.z, s1.z); sj[3] = make_float2(s0.w, s1.w);
-        }
         const unsigned char* in = smem + L.ring + (int)(s % STAGES) * fast_stage_bytes(D);
         const float* mats = reinterpret_cast<const float*>(smem + L.mats) + (ti & 1) * 2 * kPairs * kMatStride;
         const int64_t head_row0 = (st.b * H + st.h) * (int64_t)D + 8 * c;  // first output row
