@@ -40,6 +40,8 @@ FALLBACK_HBM_GBS = 6650.0
 TRAFFIC = {
     "video3d": (377564416 + 325334784, "f0170ddbe869b9f9"),
     "fp8neox": (1097153280 + 517297920, "f0170ddbe869b9f9"),
+    "fp8neox_nonorm": (1097140224 + 517154816, "f0170ddbe869b9f9"),
+    "gqa3d": (189662976 + 139130624, "f0170ddbe869b9f9"),
     "table_hs": (43562240 + 2029568, "9230c313092c6dc7"),
     "table_il": (25730816 + 15616, "9230c313092c6dc7"),
     "table_hs_f16": (42770176 + 2013952, "9230c313092c6dc7"),
