@@ -246,7 +246,7 @@ def one_core(w, inp_cpu, budget_s: float, chunk: int):
 
 def run_reference(args, w):
     """--impl reference: the oracle as it stands, on the host cores."""
-    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+    import workloads as W
 
     rank, world, _ = dist_env()
     if rank != 0:
@@ -338,7 +338,7 @@ def run_gpu(args, w):
     import torch
 
     import qk_rmsnorm_rope_qknr_b200 as Q
-    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+    import workloads as W
 
     rank, world, local, dev, pg = init_gpu()
     Q.lib()
@@ -420,7 +420,7 @@ def run_gpu_table(args, w):
     import torch
 
     import qk_rmsnorm_rope_qknr_b200 as Q
-    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+    import workloads as W
 
     rank, world, local, dev, pg = init_gpu()
     Q.lib()
@@ -786,7 +786,7 @@ def run_gpu_ucpe(args, w):
     import torch
 
     import qk_rmsnorm_rope_qknr_b200 as Q
-    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+    import workloads as W
 
     rank, world, local, dev, pg = init_gpu()
     L = Q.lib()
@@ -1003,7 +1003,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+    import workloads as W
 
     w = W.WORKLOADS[args.workload]
     if args.tokens:

@@ -16,7 +16,6 @@ the definition of the camera prep's inflation_sq output (U6): "parity
 unpinned" for those three choices.
 """
 import ctypes as C
-import os
 
 import numpy as np
 
@@ -316,4 +315,3 @@ __all__ = ["bf16_to_f64", "bf16_from_f64", "f16_from_f64", "f16_to_f64", "e4m3_f
            "e4m3_to_f64", "rmsnorm",
            "pairs_table", "pairs_3d", "rotate", "position_3d", "angles_3d", "rope_table",
            "rope_3d", "relu", "ray_project", "ucpe_cam_prep", "threads", "set_threads", "lib"]
-_ = os

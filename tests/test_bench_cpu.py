@@ -51,7 +51,7 @@ def test_one_core_figure_restores_threads():
     sys.path.insert(0, ROOT)
     import bench
     import oracle as O
-    from qk_rmsnorm_rope_qknr_b200 import workloads as W
+    import workloads as W
 
     before = O.threads()
     for name, chunk in (("tiny3d", 16), ("table_il", 16)):

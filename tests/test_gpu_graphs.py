@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import qk_rmsnorm_rope_qknr_b200 as Q
-from qk_rmsnorm_rope_qknr_b200 import workloads as W
+import workloads as W
 
 pytestmark = pytest.mark.gpu
 

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import qk_rmsnorm_rope_qknr_b200 as Q
-from qk_rmsnorm_rope_qknr_b200 import workloads as W
+import workloads as W
 from tests._util import bf16_mismatch, t2u16
 from tests.test_gpu_parity import assert_3d_close, check_table_against_oracle, oracle_3d
 

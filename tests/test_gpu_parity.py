@@ -11,7 +11,7 @@ import torch
 
 import oracle as O
 import qk_rmsnorm_rope_qknr_b200 as Q
-from qk_rmsnorm_rope_qknr_b200 import workloads as W
+import workloads as W
 from tests._util import act_mismatch, bf16_mismatch, e4m3_mismatch, t2u16, t2u8
 
 pytestmark = pytest.mark.gpu

@@ -12,7 +12,7 @@ import torch
 
 import qk_rmsnorm_rope_qknr_b200 as Q
 from qk_rmsnorm_rope_qknr_b200 import tp
-from qk_rmsnorm_rope_qknr_b200 import workloads as W
+import workloads as W
 from tests.test_gpu_parity import assert_3d_close, oracle_3d
 
 pytestmark = pytest.mark.gpu

@@ -79,7 +79,7 @@ def _worker(rank, port, out_dir):
         # --- camera prep: 37 tokens of 2 batch elements; the shard takes its
         # rows of q/k/v and of the matrices and tables, and its outputs are the
         # whole call's columns ([B, H, D, N]: the token axis is the last)
-        from qk_rmsnorm_rope_qknr_b200 import workloads as W
+        import workloads as W
 
         wu = W.FormUcpe("mr", batch=2, seq=37, heads=3, head_dim=16, spatial=9, seed=6)
         u = W.make_inputs(wu, device="cpu")

@@ -6,7 +6,7 @@ import math
 
 import torch
 
-from qk_rmsnorm_rope_qknr_b200 import workloads as W
+import workloads as W
 
 
 def test_camera_matrices_are_rigid_motion_pairs():

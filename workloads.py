@@ -31,7 +31,6 @@ video-DiT and MiniMax-H3 geometries the pages name):
 from __future__ import annotations
 
 import dataclasses
-import math
 from typing import Optional
 
 import torch
@@ -297,4 +296,3 @@ def bytes_per_token(w) -> float:
     return algorithmic_bytes(w) / w.tokens
 
 
-_ = math
