@@ -99,6 +99,7 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         self.t = None
+        self.load_from = self.load_to = None
 
     def __enter__(self):
         try:
@@ -115,7 +116,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.perf_counter(), line.strip()))
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -128,9 +129,16 @@ class ClockSampler:
             self.t.join(timeout=2)
 
     def summary(self):
+        """Median SM clock and the throttle reasons seen while the GPU was
+        under load: from the start of the spin-up to the end of the timed
+        region (samples of the idle start-up are left out)."""
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for t, ln in self.lines:
+            if self.load_from is not None and t < self.load_from:
+                continue
+            if self.load_to is not None and t > self.load_to + 0.15:
+                continue
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -304,26 +312,43 @@ def init_gpu():
 
 
 def time_steps(step, args, stream, local, dev, pg):
-    """W untimed steps, then K back-to-back steps (one kernel launch each,
-    nothing else on the stream) between two events on the launching stream.
-    The kernels are programmatic dependent launches, so no event may sit
-    between them: the average launch duration is the region's time over K.
+    """A spin-up, W untimed steps, then K back-to-back steps (one kernel launch
+    each, nothing else on the stream) between two events on the launching
+    stream. The kernels are programmatic dependent launches, so no event may
+    sit between them: the average launch duration is the region's time over K.
+
+    The optional spin-up (--spin-ms, off by default) runs untimed steps for
+    that long with the clock sampler already running, so that the region
+    starts at the clock the GPU holds under sustained load. On a 1 kW B200
+    that is the power-capped clock: after 500 ms of this load the SM clock
+    sits near 1750-1850 MHz with sw_power_cap active, where a short region
+    that starts from a cool GPU runs at 1965 MHz. Both are real operating
+    points; the bench line carries the sampled clock and the time normalised
+    to the top clock, so either can be compared.
     Returns (ms per step, max over ranks; the clock sampler)."""
     import torch
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
+        clocks.load_from = time.perf_counter()
+        n = 0
+        while (time.perf_counter() - clocks.load_from) * 1e3 < args.spin_ms:
+            step(n)
+            n += 1
+            if n % 16 == 0:  # keep the queue short, so the spin-up ends on time
+                torch.cuda.synchronize()
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
         t_start.record(stream)
         for i in range(args.steps):
             step(i)
         t_end.record(stream)
         torch.cuda.synchronize()
+        clocks.load_to = time.perf_counter()
     if pg:
         pg.barrier()
     total_ms = t_start.elapsed_time(t_end)
@@ -332,6 +357,17 @@ def time_steps(step, args, stream, local, dev, pg):
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
         total_ms = t.item()
     return total_ms / args.steps, clocks
+
+
+def clock_normalised(us_per_launch, clk):
+    """The launch time in SM cycles at the median sampled clock, and that many
+    cycles at the GPU's top clock: what the launch would take had the clock not
+    dropped (the kernels here are partly issue-bound, so their time follows
+    the SM clock). None without clock samples."""
+    if not clk.get("sm_mhz") or not clk.get("sm_max_mhz"):
+        return None
+    cycles = us_per_launch * clk["sm_mhz"]
+    return {"sm_cycles_per_launch": cycles, "us_at_sm_max": cycles / clk["sm_max_mhz"]}
 
 
 def run_gpu(args, w):
@@ -396,7 +432,8 @@ def run_gpu(args, w):
                        "head_dim": w.head_dim, "interleave": w.interleave,
                        "is_qk_norm": w.is_qk_norm, "output_fp8": w.output_fp8,
                        "parallelism": f"dp{world}" if world > 1 else "single",
-                       "l2": f"no flush: inputs {qkv.numel() * 2 / 1e6:.0f} MB > 126 MB L2"},
+                       "l2": f"no flush: inputs {qkv.numel() * 2 / 1e6:.0f} MB > 126 MB L2",
+                       "spin_up_ms": args.spin_ms},
             "hbm_gbs": achieved, "hbm_pct_of_peak": 100.0 * achieved / peak,
             "kernel_us": avg_launch_ms * 1e3,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -404,6 +441,7 @@ def run_gpu(args, w):
                          "peak_source": f"{peak_kind} hbm_gbs",
                          "algorithmic_bytes_per_launch": alg_bytes},
             "cpu_baseline": cpu, "clocks": clk, "e2e": e2e, "gpu_launches": args.steps,
+            "clock_normalised": clock_normalised(avg_launch_ms * 1e3, clk),
         }
         print(json.dumps(line), flush=True)
     if pg:
@@ -469,7 +507,7 @@ def run_gpu_table(args, w):
         if rest is not None:
             rest.replay()
 
-    graph_args = argparse.Namespace(steps=1, warmup=0)
+    graph_args = argparse.Namespace(steps=1, warmup=0, spin_ms=args.spin_ms)
     ms_region, clocks = time_steps(region, graph_args, stream, local, dev, pg)
     ms_per_step = ms_region / args.steps
     tokens_per_s = world * T / (ms_per_step / 1e3)
@@ -490,6 +528,7 @@ def run_gpu_table(args, w):
                          f"({sec:.1f} s of fp64 oracle work)",
                "value_1core": one_core(w, inp_cpu, args.cpu_seconds / 4, 128)}
     if rank == 0:
+        clk = clocks.summary()
         q = sets[0]["q"]
         line = {
             "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
@@ -505,15 +544,16 @@ def run_gpu_table(args, w):
                        "l2": f"{nsets} rotated input/output sets "
                              f"({nsets * alg_bytes / 1e6:.0f} MB > 126 MB L2)",
                        "launch": f"CUDA graphs of {nsets} launches (one per set), replayed "
-                                 f"for exactly K launches"},
+                                 f"for exactly K launches",
+                       "spin_up_ms": args.spin_ms},
             "hbm_gbs": achieved, "hbm_pct_of_peak": 100.0 * achieved / peak,
             "kernel_us": ms_per_step * 1e3,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} hbm_gbs",
                          "algorithmic_bytes_per_launch": alg_bytes},
-            "cpu_baseline": cpu, "clocks": clocks.summary(), "e2e": e2e,
-            "gpu_launches": args.steps,
+            "cpu_baseline": cpu, "clocks": clk, "e2e": e2e,
+            "gpu_launches": args.steps, "clock_normalised": clock_normalised(ms_per_step * 1e3, clk),
         }
         print(json.dumps(line), flush=True)
     if pg:
@@ -829,6 +869,7 @@ def run_gpu_ucpe(args, w):
                          f"through its {B * N} ({sec:.1f} s of fp64 oracle work)",
                "value_1core": one_core(w, inp_cpu, args.cpu_seconds / 4, 16)}
     if rank == 0:
+        clk = clocks.summary()
         in_mb = sum(inp[n].numel() * inp[n].element_size() for n in UCPE_INPUTS) / 1e6
         line = {
             "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
@@ -840,15 +881,16 @@ def run_gpu_ucpe(args, w):
                        "shape_in": [B, N, H, D], "shape_out": [B, H, D, N],
                        "k_scale": w.k_scale,
                        "parallelism": f"dp{world}" if world > 1 else "single",
-                       "l2": f"no flush: inputs {in_mb:.0f} MB > 126 MB L2"},
+                       "l2": f"no flush: inputs {in_mb:.0f} MB > 126 MB L2",
+                       "spin_up_ms": args.spin_ms},
             "hbm_gbs": achieved, "hbm_pct_of_peak": 100.0 * achieved / peak,
             "kernel_us": ms_per_step * 1e3,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} hbm_gbs",
                          "algorithmic_bytes_per_launch": alg_bytes},
-            "cpu_baseline": cpu, "clocks": clocks.summary(), "e2e": e2e,
-            "gpu_launches": args.steps,
+            "cpu_baseline": cpu, "clocks": clk, "e2e": e2e,
+            "gpu_launches": args.steps, "clock_normalised": clock_normalised(ms_per_step * 1e3, clk),
         }
         print(json.dumps(line), flush=True)
     if pg:
@@ -992,7 +1034,10 @@ def main():
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="qknr", choices=["qknr", "reference"])
-    ap.add_argument("--workload", default="video3d")
+    ap.add_argument("--workload", default="fp8neox")
+    ap.add_argument("--spin-ms", type=float, default=0.0,
+                    help="untimed steps for this long before the warm-up, with the clock "
+                         "sampler running")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")

@@ -245,11 +245,14 @@ int qknr_rope_3d_with_ssq(const qknr_rope_3d_params* params, const float* ssq,
  * Any num_tokens is allowed. head_dim <= 128 with an even num_tokens and at
  * least two heads runs the pipelined kernel; other shapes run a general one,
  * which writes two bytes at a time when num_tokens is not a multiple of 8.
- * Range: the two sums of squares are fp32, taken over the key before the
- * scale (the pipelined kernel) or after it (the general one; the ratio is
- * the same), so a key whose squares all underflow fp32
- * (every channel below about 1e-19 in magnitude) counts as a zero key
- * (inflation_sq 1).
+ * Range: both kernels apply k_scale to K's rotated result (the projection
+ * and the rotation are linear) and take the two fp32 sums of squares over the
+ * unscaled ReLU key, so the scale itself never underflows or overflows them.
+ * A key whose squares all underflow fp32 (every channel below about 1e-19 in
+ * magnitude) counts as a zero key (inflation_sq 1); a key whose sum of
+ * squares overflows fp32 (channels above about 1e18 at head_dim 256, 1.8e19
+ * for one channel) gives inflation_sq NaN, where the fp64 definition stays
+ * finite.
  * The kernels wait only on their own cp.async groups and bulk stores, which
  * always complete, so they have no timeout path and do not set the device
  * status word.

@@ -175,10 +175,6 @@ __device__ __forceinline__ void transform8(const uint4& raw, const float* m, con
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] = fmaxf(x[e], 0.0f);
     }
-    if (X == 1) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] *= k_scale;
-    }
     project_block(m, x, y);
     project_block(m, x + 4, y + 4);
     if (X == 1) {
@@ -202,6 +198,13 @@ __device__ __forceinline__ void transform8(const uint4& raw, const float* m, con
             y[2 * j] = fmaf(ya, cj[j], -yb * sj[j]);
             y[2 * j + 1] = fmaf(yb, cj[j], ya * sj[j]);
         }
+    }
+    // K's scale goes on the rotated result: the projection and the rotation
+    // are linear, and the sums above are of the unscaled key, whose gain is
+    // the scaled key's (no underflow or overflow from the scale in them).
+    if (X == 1) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] *= k_scale;
     }
 }
 
@@ -357,7 +360,8 @@ __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
                     si += v.x;
                     so += v.y;
                 }
-                a.inflation_sq[(b * H + h) * N + n0 + t] = si > 0.f ? so / si : 1.0f;
+                a.inflation_sq[(b * H + h) * N + n0 + t] =
+                    (si > 0.f && a.k_scale != 0.0f) ? so / si : 1.0f;
             }
         }
         if (!more) break;

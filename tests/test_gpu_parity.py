@@ -79,10 +79,12 @@ def test_3d_workload_ragged_shard(name):
 
 
 @pytest.mark.parametrize("name", ["video3d", "fp8neox", "fp8neox_nonorm", "gqa3d"])
-def test_3d_workload_full_size_sampled(name):
-    """Full-size workload in the benchmark's launch configuration; the oracle
-    checks 48 sampled tokens one by one (grid corners, batch seam, random), and
-    the V output is checked in full against torch's own conversion."""
+def test_3d_workload_full_size_every_token(name, capsys):
+    """Full-size workload in the benchmark's launch configuration, every
+    element of q_out, k_out and v_out against the oracle. The oracle runs over
+    the whole call in chunks of tokens (a chunk starting at token t0 is the
+    same call's tokens with pos_offset t0), so the kernel's long rings (tens of
+    tokens per pipeline, thousands of parity flips) are compared in full."""
     w = W.WORKLOADS[name]
     inp = W.make_inputs(w, device=DEV)
     qkv = inp["qkv"]
@@ -90,23 +92,46 @@ def test_3d_workload_full_size_sampled(name):
     outs = run_3d(qkv, inp["q_weight"], inp["k_weight"], **p)
     torch.cuda.synchronize()
     T = w.tokens
-    P = w.ppf * w.pph * w.ppw
-    rng = np.random.default_rng(7)
-    picks = sorted(set([0, 1, w.ppw, w.pph * w.ppw, P - 1, T - 1] + ([P, P + 1] if T > P else [])
-                       + rng.integers(0, T, 40).tolist()))
-    flat = qkv.reshape(T, -1)
-    qw_cpu, kw_cpu = inp["q_weight"].cpu(), inp["k_weight"].cpu()
-    for t in picks:
-        ref, exact = oracle_3d(flat[t:t + 1].cpu(), qw_cpu, kw_cpu, pos_offset=t, **p)
-        got = [o.reshape(T, -1, w.head_dim)[t:t + 1] for o in outs]
-        assert_3d_close(got, ref, exact, w.output_fp8, f"{name} token {t}")
-    v_in = flat[:, (w.hq + w.hk) * w.head_dim:]
-    v_out = outs[2].reshape(T, -1)
-    if w.output_fp8:
-        want = (v_in.float() * w.v_scale).to(torch.float8_e4m3fn)
-        assert torch.equal(v_out.view(torch.uint8), want.view(torch.uint8))
-    else:
-        assert torch.equal(v_out, v_in)
+    flat = qkv.reshape(T, -1).cpu()
+    got = [o.reshape(T, -1, w.head_dim).cpu() for o in outs]
+    cpu = lambda t: None if t is None else t.cpu()  # noqa: E731
+    qw_cpu, kw_cpu = cpu(inp["q_weight"]), cpu(inp["k_weight"])
+    bits = lambda t: None if t is None else t2u16(t)  # noqa: E731
+    del outs, inp, qkv
+    stats = {n: dict(n=0, exact=0, max_err=0.0) for n in "qkv"}
+    chunk = 4096
+    for t0 in range(0, T, chunk):
+        t1 = min(T, t0 + chunk)
+        rows = flat[t0:t1]
+        if w.output_fp8:
+            ref = O.rope_3d(t2u16(rows), bits(qw_cpu), bits(kw_cpu), pos_offset=t0, **p)
+            exact = (None, None, None)
+        else:
+            ref, exact = oracle_3d(rows, qw_cpu, kw_cpu, pos_offset=t0, **p)
+        for n, g, r, x in zip("qkv", got, ref, exact):
+            gs = g[t0:t1]
+            if w.output_fp8:
+                bad, st = e4m3_mismatch(t2u8(gs).reshape(r.shape), r)
+                err = st["max_steps"]
+            elif n == "v":
+                gb = t2u16(gs).reshape(r.shape)
+                bad = np.argwhere(gb != r)
+                st = dict(exact_frac=float(np.mean(gb == r)), n=int(r.size))
+                err = 0.0 if len(bad) == 0 else float("inf")
+            else:
+                bad, st = bf16_mismatch(t2u16(gs).reshape(r.shape), r, x)
+                err = st["max_err_ulps"]
+            assert len(bad) == 0, (f"{name} {n}: {len(bad)} of {r.size} beyond tolerance in "
+                                   f"tokens [{t0}, {t1}) {st}, first at {bad[:3].tolist()}")
+            s = stats[n]
+            s["exact"] += st["exact_frac"] * st["n"]
+            s["n"] += st["n"]
+            s["max_err"] = max(s["max_err"], err)
+    unit = "E4M3 steps" if w.output_fp8 else "bf16 ulp"
+    with capsys.disabled():
+        print(f"\n[every-token parity] {name} ({T} tokens): " + "; ".join(
+            f"{n}_out exact_frac {s['exact'] / s['n']:.6f}, max {s['max_err']:.3g} {unit}"
+            for n, s in stats.items()))
 
 
 @pytest.mark.parametrize("name", ["table_hs", "table_il", "table_hs_f16", "table_d72"])

@@ -158,6 +158,23 @@ def test_ucpe_zero_k_scale(N):
              where="k_scale 0")
 
 
+@pytest.mark.parametrize("k_scale", [1e-20, 1e20])
+@pytest.mark.parametrize("N", [61, 64])  # general kernel, pipelined kernel
+def test_ucpe_extreme_k_scale(N, k_scale):
+    """A tiny or huge K scale: both kernels take the sums of squares over the
+    unscaled key (the scale cancels in the gain), so inflation_sq neither
+    underflows to 1 nor overflows to NaN, and k_trans carries the scale."""
+    B, H, D = 1, 3, 48
+    w, inp = _case(B, N, H, D, seed=13)
+    outs = Q.cam_prep_func(inp["q_normed"], inp["k_normed"], inp["v_raw"], proj_q=inp["proj_q"],
+                           proj_kv=inp["proj_kv"], rope_cos=inp["rope_cos"],
+                           rope_sin=inp["rope_sin"], k_scale=k_scale)
+    torch.cuda.synchronize()
+    assert torch.isfinite(outs[3]).all()
+    _compare(outs, _oracle(inp, k_scale, "bf16"), _oracle(inp, k_scale, "bf16", exact=True),
+             "bf16", where=f"k_scale {k_scale:g}")
+
+
 @pytest.mark.parametrize("N", [191, 192])  # general kernel, pipelined kernel
 def test_ucpe_inflation_optional_and_deterministic(N):
     B, H, D = 1, 4, 112
@@ -219,28 +236,50 @@ def test_ucpe_rejects_pageable_host_memory():
         Q.cam_prep_func(x, x, x, proj_q=pq, proj_kv=pq, rope_cos=cs, rope_sin=cs, k_scale=1.0)
 
 
-def test_ucpe_workload_full_size_sampled():
-    """The benchmark's workload at full size, in the launch the benchmark times;
-    the oracle recomputes a sample of tokens (every token is independent: its
-    rows, its matrices and its table rows), spread over the tiles and including
-    the ragged last tile."""
+def test_ucpe_workload_full_size_every_token(capsys):
+    """The benchmark's workload at full size, in the launch the benchmark times,
+    every element of the four outputs against the oracle. The oracle runs over
+    token chunks (every token is independent: its rows, its matrices and its
+    table rows), so every tile of every CTA, the ragged last tile and the
+    matrix double buffer's parity flips over the whole run are compared."""
     w = W.WORKLOADS["ucpe"]
     inp = W.make_inputs(w, device="cuda")
     outs = Q.cam_prep_func(inp["q_normed"], inp["k_normed"], inp["v_raw"], proj_q=inp["proj_q"],
                            proj_kv=inp["proj_kv"], rope_cos=inp["rope_cos"],
                            rope_sin=inp["rope_sin"], k_scale=w.k_scale)
     torch.cuda.synchronize()
-    g = np.random.default_rng(0)
-    idx = np.unique(np.concatenate([g.integers(0, w.seq, 96), [0, 63, 64, w.seq - 1,
-                                                               w.seq - 49]]))
-    it = torch.as_tensor(idx, device="cuda")
-    sub = {k: (v[:, it] if k in ("q_normed", "k_normed", "v_raw", "proj_q", "proj_kv")
-               else v[it]).contiguous() for k, v in inp.items()}
-    ref = _oracle(sub, w.k_scale, "bf16")
-    ref_exact = _oracle(sub, w.k_scale, "bf16", exact=True)
-    got = [o[..., it] for o in outs[:3]] + [outs[3][..., it]]
-    _compare(got, ref, ref_exact, "bf16", where="ucpe full size")
-    assert torch.isfinite(outs[3]).all()
+    host = {k: v.cpu() for k, v in inp.items()}
+    got = [o.cpu() for o in outs]
+    del outs, inp
+    assert torch.isfinite(got[3]).all()
+    N = w.seq
+    stats = {n: dict(n=0, exact=0.0, max_err=0.0) for n in ("q", "k", "v")}
+    infl_rel = 0.0
+    chunk = 4096
+    for n0 in range(0, N, chunk):
+        n1 = min(N, n0 + chunk)
+        sub = {k: (v[:, n0:n1] if k in ("q_normed", "k_normed", "v_raw", "proj_q", "proj_kv")
+                   else v[n0:n1]).contiguous() for k, v in host.items()}
+        ref = _oracle(sub, w.k_scale, "bf16")
+        ref_exact = _oracle(sub, w.k_scale, "bf16", exact=True)
+        part = [o[..., n0:n1] for o in got]
+        for name, g, r, x in zip(("q", "k", "v"), part[:3], ref[:3], ref_exact[:3]):
+            bad, st = act_mismatch(t2u16(g).transpose(0, 1, 3, 2), r.transpose(0, 1, 3, 2),
+                                   x.transpose(0, 1, 3, 2), "bf16")
+            assert len(bad) == 0, (f"ucpe full size, tokens [{n0}, {n1}): {name}_trans "
+                                   f"{len(bad)} beyond tolerance {st}, first {bad[:3]}")
+            s = stats[name]
+            s["exact"] += st["exact_frac"] * st["n"]
+            s["n"] += st["n"]
+            s["max_err"] = max(s["max_err"], st["max_err_ulps"])
+        np.testing.assert_allclose(part[3].double().numpy(), ref[3], rtol=INFL_RTOL, atol=0,
+                                   err_msg=f"ucpe full size, tokens [{n0}, {n1}): inflation_sq")
+        infl_rel = max(infl_rel, float(np.max(np.abs(part[3].double().numpy() / ref[3] - 1.0))))
+    with capsys.disabled():
+        print(f"\n[every-token parity] ucpe ({N} tokens, {w.heads} heads of {w.head_dim}): "
+              + "; ".join(f"{n}_trans exact_frac {s['exact'] / s['n']:.6f}, max "
+                          f"{s['max_err']:.3g} bf16 ulp" for n, s in stats.items())
+              + f"; inflation_sq max rel err {infl_rel:.3g}")
 
 
 @pytest.mark.parametrize("N,cuts", [(192, [64, 136]), (151, [40, 97])])
