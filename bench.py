@@ -2,17 +2,19 @@
 """Benchmark of the fused Q/K RMSNorm + RoPE hot path on B200.
 
 One step = one call of the 3D entry point (across-heads RMSNorm + 3D RoPE +
-V copy) over one batch of the video-DiT workload: packed bf16 QKV
-[1, 15360, (32+32+32)*128], patch grid 16x30x32, channels 16/56/56,
-interleaved pairs, bf16 out. Inputs are seeded synthetic tensors resident in
-HBM; the 377 MB input (plus 377 MB output) exceeds the 126 MB L2, so no flush
-is needed between steps.
+V copy, FP8 E4M3 out) over one batch of the largest workload, the FP8 NeoX
+video geometry: packed bf16 QKV [2, 29760, (24+24+24)*128], patch grid
+31x24x40, channels 32/48/48, NeoX pairs, E4M3 outputs with scales 0.5 / 0.25.
+Inputs are seeded synthetic tensors resident in HBM; the 1.1 GB input exceeds
+the 126 MB L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-  (NAME: a 3D workload, or table_hs / table_il / table_hs_f16 / table_d72 for
-  the table form, timed over rotated input sets since one set fits in L2, or
-  ucpe for the UCPE camera prep)
+  (NAME: a 3D workload such as video3d, or table_hs / table_il / table_hs_f16 /
+  table_d72 for the table form, timed over rotated input sets since one set
+  fits in L2, or ucpe for the UCPE camera prep)
   python bench.py --impl reference ...   # the fp64 CPU oracle, bounded sample
+  python bench.py --host-sweep           # host cost per call against device
+                                         # time, 64 to 8192 tokens (C ABI)
 
 Under torchrun each rank processes its own batch (weak scaling, no
 collective on the data path); rank 0 prints one JSON line.
@@ -155,6 +157,65 @@ class ClockSampler:
                     "gpu": self.gpu}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
                 "reasons": sorted(reasons), "samples": len(sm), "gpu": self.gpu}
+
+
+def host_cost_exe():
+    """tests/host_cost.c built against the in-tree libqknr.so (gcc, once)."""
+    pkg = os.path.join(ROOT, "qk_rmsnorm_rope_qknr_b200")
+    src = os.path.join(ROOT, "tests", "host_cost.c")
+    exe = os.path.join(pkg, "_build", "host_cost")
+    lib = os.path.join(pkg, "libqknr.so")
+    if os.path.exists(exe) and os.path.getmtime(exe) >= max(os.path.getmtime(src),
+                                                             os.path.getmtime(lib)):
+        return exe
+    os.makedirs(os.path.dirname(exe), exist_ok=True)
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    subprocess.run(["gcc", "-O2", src, "-I", os.path.join(ROOT, "include"),
+                    "-I", os.path.join(cuda, "include"), "-L", pkg, "-lqknr",
+                    "-L", os.path.join(cuda, "lib64"), "-lcudart", f"-Wl,-rpath,{pkg}",
+                    f"-Wl,-rpath,{os.path.join(cuda, 'lib64')}", "-o", exe], check=True)
+    return exe
+
+
+def host_cost(form: str, tokens: int, calls: int = 200):
+    """One run of the C host-cost program: host, device and wall us per call."""
+    r = subprocess.run([host_cost_exe(), form, str(tokens), str(calls)], capture_output=True,
+                       text=True, timeout=300)
+    if r.returncode != 0:
+        raise RuntimeError(f"host_cost {form} {tokens}: {r.stderr.strip()}")
+    return json.loads(r.stdout.strip().splitlines()[-1])
+
+
+def python_call_us(call, n: int = 200) -> float:
+    """Host us per call of a Python binding call queued back to back (no sync)."""
+    import torch
+
+    for _ in range(10):
+        call()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(n):
+        call()
+    us = (time.perf_counter() - t0) * 1e6 / n
+    torch.cuda.synchronize()
+    return us
+
+
+def run_host_sweep(args):
+    """Host cost against device time per call of both contract entry points
+    from C, 64 to 8192 tokens: below the crossover (the first size whose
+    device time reaches its host time) back-to-back calls leave the GPU
+    waiting on the host."""
+    rows = {}
+    for form in ("3d", "table"):
+        rows[form] = [host_cost(form, t) for t in (64, 128, 256, 512, 1024, 2048, 4096, 8192)]
+    cross = {f: next((r["tokens"] for r in v if r["device_us_per_call"] >= r["host_us_per_call"]),
+                     None) for f, v in rows.items()}
+    print(json.dumps({"host_sweep": rows, "crossover_tokens": cross,
+                      "shapes": {"3d": "24+24+24 heads of 128, E4M3 out (fp8neox per token)",
+                                 "table": "32+8 heads of 128, rotary_dim 96, fp32 table "
+                                          "(table_hs per token)"}}), flush=True)
+    return 0
 
 
 def dist_env():
@@ -403,6 +464,16 @@ def run_gpu(args, w):
     tr = TRAFFIC.get(w.name)
     traffic = tr[0] if tr and tr[1] == kernel_source_hash() else None
 
+    host_us = None
+    if rank == 0 and world == 1 and not args.no_e2e:
+        # host cost of one call: through the Python binding (argument checks
+        # and ctypes) and from C through the ABI, with the launch
+        host_us = {"python_binding": python_call_us(lambda: step(0))}
+        if not getattr(args, "tokens", None) and w.name == "fp8neox":
+            hc = host_cost("3d", T)
+            host_us.update({"c_abi": hc["host_us_per_call"],
+                            "c_abi_device_us": hc["device_us_per_call"]})
+
     # End to end through the C ABI with host buffers: copy the step's input
     # from pinned host memory, run, copy the outputs back, every step.
     e2e = None
@@ -442,6 +513,7 @@ def run_gpu(args, w):
                          "algorithmic_bytes_per_launch": alg_bytes},
             "cpu_baseline": cpu, "clocks": clk, "e2e": e2e, "gpu_launches": args.steps,
             "clock_normalised": clock_normalised(avg_launch_ms * 1e3, clk),
+            "host_us_per_call": host_us,
         }
         print(json.dumps(line), flush=True)
     if pg:
@@ -1042,6 +1114,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--host-sweep", action="store_true",
+                    help="print host cost against device time per call, 64-8192 tokens")
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the workload's geometry on this many tokens instead (3D: a "
                          "sequence shard from position 0); for profiling smaller cases")
@@ -1063,6 +1137,8 @@ def main():
             w = dataclasses.replace(w, name=f"{w.name}[{args.tokens}]", tokens=args.tokens)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.host_sweep:
+        return run_host_sweep(args)
     if w.form == "ucpe":
         return run_gpu_ucpe(args, w)
     return run_gpu(args, w) if w.form == "3d" else run_gpu_table(args, w)

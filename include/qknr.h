@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define QKNR_ABI_VERSION 3
+#define QKNR_ABI_VERSION 4
 
 typedef enum {
     QKNR_OK = 0,
@@ -132,6 +132,14 @@ int qknr_rope_table(const void* q, const void* k, void* q_out, void* k_out,
  *      theta_j = pos_axis * base^(-2i/C).
  *   Each Q and K head rotates its pairs: (2j, 2j+1) if interleave, else
  *      (j, j + head_dim/2) (NeoX), by theta_j as in qknr_rope_table.
+ *   NeoX per axis (neox_per_axis = 1, interleave = 0): the page says only
+ *      "NeoX-style" for interleave=False, which also reads as NeoX halves
+ *      inside each axis group: with o the group's first channel and C its
+ *      channel count, the pairs are (o + i, o + i + C/2), i < C/2, rotated by
+ *      pos_axis * base^(-2i/C). The default (0) is the whole-head layout
+ *      above; both give the same result for interleave == 1. This layout is
+ *      built for channel groups that are multiples of 16 (else
+ *      QKNR_ERR_UNSUPPORTED).
  *   Outputs: q_out [T, Hq, head_dim], k_out [T, Hk, head_dim], v_out
  *      [T, Hv, head_dim], dense. bf16; or with output_fp8, E4M3 of
  *      q*output_quant_scale, k*output_quant_scale and v*v_quant_scale.
@@ -172,6 +180,9 @@ typedef struct {
                                by ppf*pph*ppw; 1: a contiguous slice of a longer
                                sequence starting at patch position pos_offset
                                (one rank's part of a sharded call): any count */
+    int32_t neox_per_axis;  /* NeoX pairs (interleave == 0) inside each axis group
+                               instead of across the whole head; see below.
+                               Ignored with interleave == 1. */
 } qknr_rope_3d_params;
 
 int qknr_rope_3d(const qknr_rope_3d_params* params, void* cuda_stream);

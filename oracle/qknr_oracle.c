@@ -35,8 +35,9 @@
  *       pair j taking the frequency of pair slot j in the frame/height/width
  *       order (the 3D analogue of the half-split pairs of [T]). The other
  *       reading, NeoX inside each axis group, is kept behind a flag
- *       (neox_per_axis) and is NOT what the CUDA path computes.
- *       PARITY UNPINNED between the two readings: the pages cannot decide it.
+ *       (neox_per_axis); the library offers it behind the same flag, off by
+ *       default. PARITY UNPINNED between the two readings: the pages cannot
+ *       decide it (each is pinned to its own textbook form).
  *   R9  FP8 output is E4M3(value * scale): the quantisation scale multiplies.
  *       PARITY UNPINNED against the reading that divides.
  *   R10 E4M3 is the OCP E4M3FN format (bias 7, largest finite 448, no

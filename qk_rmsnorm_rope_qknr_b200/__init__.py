@@ -34,7 +34,7 @@ LIB_PATH = os.path.join(_PKG, "libqknr.so")
 QKNR_OK, QKNR_ERR_NULL, QKNR_ERR_SHAPE, QKNR_ERR_UNSUPPORTED = 0, 1, 2, 3
 QKNR_ERR_ALIGN, QKNR_ERR_ALIAS, QKNR_ERR_POINTER, QKNR_ERR_CUDA = 4, 5, 6, 7
 QKNR_DT_BF16, QKNR_DT_F32, QKNR_DT_E4M3, QKNR_DT_F16 = 0, 1, 2, 3
-ABI_VERSION = 3  # QKNR_ABI_VERSION the argument lists below are written for
+ABI_VERSION = 4  # QKNR_ABI_VERSION the argument lists below are written for
 
 EXPORTS = ("qknr_rope_table", "qknr_rope_3d", "qknr_rope_3d_partial_ssq", "qknr_rope_3d_with_ssq",
            "qknr_ucpe_cam_prep", "qknr_device_status", "qknr_test_set_wait_fault", "qknr_status_string",
@@ -63,7 +63,8 @@ class Rope3DParams(C.Structure):
                 ("factor", C.c_float), ("low", C.c_float), ("high", C.c_float),
                 ("attention_factor", C.c_float), ("is_qk_norm", C.c_int32),
                 ("output_fp8", C.c_int32), ("output_quant_scale", C.c_float),
-                ("v_quant_scale", C.c_float), ("sequence_shard", C.c_int32)]
+                ("v_quant_scale", C.c_float), ("sequence_shard", C.c_int32),
+                ("neox_per_axis", C.c_int32)]
 
 
 _lib = None
@@ -204,10 +205,12 @@ def make_3d_params(qkv, q_weight, k_weight, q_out, k_out, v_out, *, ppf, pph, pp
                    num_heads_k, num_heads_v, head_dim, eps=1e-6, base=10000.0, interleave=True,
                    factor=1.0, low=0.0, high=0.0, attention_factor=1.0, is_qk_norm=True,
                    output_fp8=False, output_quant_scale=1.0, v_quant_scale=1.0,
-                   pos_offset: Optional[int] = None, num_tokens=None) -> Rope3DParams:
+                   pos_offset: Optional[int] = None, num_tokens=None,
+                   neox_per_axis=False) -> Rope3DParams:
     """C parameter block. pos_offset=None is a whole call (num_tokens must be a
     multiple of ppf*pph*ppw); an integer marks a sequence shard whose first
-    token sits at that patch position (any token count)."""
+    token sits at that patch position (any token count). neox_per_axis picks
+    the NeoX pairs inside each axis group (see include/qknr.h)."""
     row = (num_heads_q + num_heads_k + num_heads_v) * head_dim
     if num_tokens is None:
         if qkv.dtype != torch.bfloat16 or qkv.shape[-1] != row or not qkv.is_contiguous():
@@ -230,6 +233,7 @@ def make_3d_params(qkv, q_weight, k_weight, q_out, k_out, v_out, *, ppf, pph, pp
     p.factor, p.low, p.high, p.attention_factor = factor, low, high, attention_factor
     p.is_qk_norm, p.output_fp8 = int(bool(is_qk_norm)), int(bool(output_fp8))
     p.output_quant_scale, p.v_quant_scale = output_quant_scale, v_quant_scale
+    p.neox_per_axis = int(bool(neox_per_axis))
     return p
 
 
@@ -357,10 +361,12 @@ def fused_qk_rmsnorm_rope(qkv: torch.Tensor, q_weight: torch.Tensor, k_weight: t
                           q_out: Optional[torch.Tensor] = None,
                           k_out: Optional[torch.Tensor] = None,
                           v_out: Optional[torch.Tensor] = None,
-                          pos_offset: Optional[int] = None,
+                          pos_offset: Optional[int] = None, neox_per_axis: bool = False,
                           stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Across-heads Q/K RMSNorm + 3D RoPE + V copy (+ FP8). Outputs are
-    [B, S, H, D] for a 3D qkv and [T, H, D] for a 2D one."""
+    [B, S, H, D] for a 3D qkv and [T, H, D] for a 2D one. neox_per_axis (with
+    interleave=False) takes the NeoX halves inside each axis group instead of
+    across the whole head; the page does not say which is meant."""
     lead = tuple(qkv.shape[:-1])
     odt = torch.float8_e4m3fn if output_fp8 else torch.bfloat16
     outs = []
@@ -374,7 +380,8 @@ def fused_qk_rmsnorm_rope(qkv: torch.Tensor, q_weight: torch.Tensor, k_weight: t
                  base=base, interleave=interleave, factor=factor, low=low, high=high,
                  attention_factor=attention_factor, is_qk_norm=is_qk_norm,
                  output_fp8=output_fp8, output_quant_scale=output_quant_scale,
-                 v_quant_scale=v_quant_scale, pos_offset=pos_offset)
+                 v_quant_scale=v_quant_scale, pos_offset=pos_offset,
+                 neox_per_axis=neox_per_axis)
     return tuple(outs)
 
 

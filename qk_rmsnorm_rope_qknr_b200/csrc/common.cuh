@@ -64,10 +64,17 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&f)[8]) {
 }
 
 // E4M3 (OCP E4M3FN), round to nearest even, saturating to +-448.
+// Bytes a, b, c, d from the low end; two cvt.rn.satfinite.e4m3x2.f32 (the
+// first source lands in the upper byte) joined as halves of one register.
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
-    uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-    uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
-    return lo | (hi << 16);
+    uint32_t r;
+    asm("{\n.reg .b16 lo, hi;\n"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n"
+        "mov.b32 %0, {lo, hi};\n}"
+        : "=r"(r)
+        : "f"(a), "f"(b), "f"(c), "f"(d));
+    return r;
 }
 
 __device__ __forceinline__ uint2 pack8_e4m3(const float (&f)[8], float scale) {

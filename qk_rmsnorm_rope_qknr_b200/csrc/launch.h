@@ -38,6 +38,7 @@ struct Rope3DArgs {
     const float* ssq_in;     // mode 2: [T][2] fp32 sums over all heads of all slices
     int32_t norm_q_elems;    // channels the Q mean runs over (hq*D, or all heads' in mode 2)
     int32_t norm_k_elems;
+    int32_t neox_per_axis;   // NeoX halves inside each axis group (groups multiples of 16)
 };
 
 enum { kModeWhole = 0, kModePartialSsq = 1, kModeSuppliedSsq = 2 };

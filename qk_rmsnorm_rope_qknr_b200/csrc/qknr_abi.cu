@@ -328,6 +328,11 @@ int run_3d(const qknr_rope_3d_params* prm, int mode, float* ssq_out, const float
                     "sequence sets sequence_shard)",
                     (long long)p.num_tokens, (long long)P);
     if (!(p.base > 0.0) || std::isinf(p.base)) return fail(QKNR_ERR_SHAPE, "base must be > 0");
+    const bool per_axis = p.neox_per_axis && !p.interleave;
+    if (per_axis && ((cf | ch | cw) & 15))
+        return fail(QKNR_ERR_UNSUPPORTED,
+                    "NeoX pairs per axis group are built for channel groups that are multiples "
+                    "of 16 (%d/%d/%d)", cf, ch, cw);
     if (p.factor != 1.0f)
         return fail(QKNR_ERR_UNSUPPORTED, "YARN scaling (factor %g != 1) is not supported",
                     (double)p.factor);
@@ -438,6 +443,7 @@ int run_3d(const qknr_rope_3d_params* prm, int mode, float* ssq_out, const float
     a.v_scale = p.v_quant_scale;
     a.base = p.base;
     a.mode = mode;
+    a.neox_per_axis = per_axis ? 1 : 0;
     a.norm_q_elems = (supplied ? heads_q_total : p.num_heads_q) * D;
     a.norm_k_elems = (supplied ? heads_k_total : p.num_heads_k) * D;
     a.stall_tx_bytes = g_fault_extra_bytes.load(std::memory_order_relaxed);
@@ -445,6 +451,13 @@ int run_3d(const qknr_rope_3d_params* prm, int mode, float* ssq_out, const float
     qknr::LaunchInfo info{};
     e = qknr::launch_rope3d(a, D, p.interleave ? 0 : 1, (p.output_fp8 && !partial) ? 1 : 0,
                             static_cast<cudaStream_t>(cuda_stream), &info);
+    if (e == cudaErrorNotSupported && per_axis) {
+        cudaGetLastError();
+        return fail(QKNR_ERR_UNSUPPORTED,
+                    "the per-axis NeoX layout runs on the register-resident kernel, which does "
+                    "not take %d + %d heads of %d (a row of %lld bytes)",
+                    p.num_heads_q, p.num_heads_k, D, (long long)(row * 2));
+    }
     if (e == cudaErrorNotSupported) {
         cudaGetLastError();
         return fail(QKNR_ERR_UNSUPPORTED,

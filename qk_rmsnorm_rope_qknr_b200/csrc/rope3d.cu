@@ -122,6 +122,26 @@ __device__ __forceinline__ float2 pair_cos_sin(const Rope3DArgs& a, const uint64
     return direct_cos_sin((uint32_t)pos, gq[j]);
 }
 
+// Row vectors of a thread's two slot halves, as (va, dv): the first half is
+// vector va of the head, the second vector va + dv. Whole-head NeoX and
+// interleaved pairs: vectors l and l + D/16. NeoX per axis group: the thread's
+// pair slots 8l..8l+7 lie in one axis group (the groups are multiples of 16
+// channels), with first channel o and C channels, and slot 8l + e pairs
+// channels o + i and o + C/2 + i (i = 8l + e - o/2): vectors o/16 + l and
+// o/16 + C/16 + l. The slots keep their frequencies, so cos/sin are unchanged.
+template <int D, bool NEOX>
+__device__ __forceinline__ void slot_vectors(const Rope3DArgs& a, int l, int& va, int& dv) {
+    va = l;
+    dv = D / 16;
+    if (NEOX && a.neox_per_axis) {
+        const int j0 = 8 * l, hcf = a.cf >> 1, hch = a.ch >> 1;
+        const int o = j0 < hcf ? 0 : (j0 < hcf + hch ? a.cf : a.cf + a.ch);
+        const int C = j0 < hcf ? a.cf : (j0 < hcf + hch ? a.ch : a.cw);
+        va = o / 16 + l;
+        dv = C / 16;
+    }
+}
+
 // Scale by r * weight, rotate the thread's 8 pairs, convert, store one slot.
 // Channel pairs travel as float2 so that the scaling (and the NeoX rotation,
 // whose partners sit in the two vectors) use the packed fp32x2 instructions.
@@ -651,6 +671,409 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Register-resident pipelined kernel: as rope3d_mg_kernel (G token pipelines
+// per CTA, bulk-copy rings, shared angle table and fp32 weights), but each
+// thread keeps its NS slots in registers, widened to fp32, from the sums of
+// squares to the stores. A token therefore needs NS/2 times fewer threads,
+// every slot is read from shared memory and widened once, and the token's
+// own ring buffer is free at the token's barrier: it is refilled there, one
+// and a half tokens of copy time ahead of its next use. The per-token work
+// that every warp repeats (the wait, the reductions, the barrier, r, the
+// cos/sin reads, the loop) is spread over NS slots per thread instead of two.
+//
+// Slots of a thread: without MIXED, slots k < NS/2 are the Q slots
+// ctid + k*Bg and slots NS/2 + k the K slots of the same indices (equal Q and
+// K head counts); with MIXED, slot k is entry ctid + k*Bg of the list
+// [Q slots | K slots]. Either way l = ctid mod D/16 for all of them.
+// ---------------------------------------------------------------------------
+template <int NS>
+constexpr int rr_max_threads() {
+    return NS >= 4 ? 384 : 768;
+}
+
+template <int D, bool NEOX, bool FP8, int NS, bool MIXED>
+__global__ void __launch_bounds__(rr_max_threads<NS>(), 1) rope3d_rr_kernel(const Rope3DArgs a) {
+    constexpr int L = D / 16;
+    constexpr int VPH = D / 8;
+    constexpr int HALF = D / 2;
+    constexpr int OUTB = FP8 ? 1 : 2;
+    constexpr int S = NS / 2;
+
+    const int G = a.groups;
+    const int Bg = blockDim.x / G;
+    const int row_bytes = (a.hq + a.hk + a.hv) * D * 2;
+    const int stages = a.stages;
+    const bool norm = a.is_qk_norm != 0;
+    const bool supplied = a.mode == kModeSuppliedSsq;  // sums come from ssq_in
+    const MgLayout lay = mg_layout(D, G, stages, row_bytes, norm ? (a.hq + a.hk) * D : 0,
+                                   a.use_table ? a.table_entries * 8 : 0);
+    extern __shared__ __align__(128) unsigned char smem[];
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + lay.abort);
+    float4* wsm = reinterpret_cast<float4*>(smem + lay.wts);
+    uint64_t* gq = reinterpret_cast<uint64_t*>(smem + lay.gq);
+    float2* tab = reinterpret_cast<float2*>(smem + lay.tab);
+
+    const int tid = threadIdx.x;
+    const int g = tid / Bg;
+    const int ctid = tid - g * Bg;
+    unsigned char* ring = smem + lay.ring + (size_t)g * stages * row_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.full) + g * stages;
+    float* cst = reinterpret_cast<float*>(smem + lay.cst) + g * 2 * L * kCsPitch;
+    float2* red = reinterpret_cast<float2*>(smem + lay.red) + g * 64;
+
+    const int64_t NP = (int64_t)gridDim.x * G;
+    const uint32_t tx = (uint32_t)row_bytes + a.stall_tx_bytes;
+    const int vbytes = a.hv * D * 2;
+    const bool v_bulk = a.v_bulk && vbytes > 0;
+    const size_t v_off = (size_t)(a.hq + a.hk) * D * 2;
+
+    // Up to griddep_wait() only shared memory and the arguments are touched.
+    if (tid == 0) {
+        for (int q = 0; q < G * stages; ++q)
+            mbar_init(reinterpret_cast<uint64_t*>(smem + lay.full) + q, 1);
+        *abort_flag = 0u;
+        fence_mbar_init();
+        griddep_wait();
+        for (int q = 0; q < G; ++q) {
+            const int64_t p = (int64_t)blockIdx.x * G + q;
+            unsigned char* rq = smem + lay.ring + (size_t)q * stages * row_bytes;
+            uint64_t* fq = reinterpret_cast<uint64_t*>(smem + lay.full) + q * stages;
+            for (int i = 0; i < stages && p + i * NP < a.num_tokens; ++i) {
+                mbar_arrive_expect_tx(&fq[i], tx);
+                bulk_load(rq + (size_t)i * row_bytes, a.qkv + (p + i * NP) * row_bytes,
+                          row_bytes, &fq[i]);
+            }
+        }
+    }
+    for (int q = tid; q < G * 64; q += blockDim.x)
+        reinterpret_cast<float2*>(smem + lay.red)[q] = make_float2(0.0f, 0.0f);
+    setup_angles<D>(a, gq, tab);
+    griddep_wait();
+    griddep_launch_dependents();
+    if (norm) {
+        const int nq4 = a.hq * VPH * 2, n4 = (a.hq + a.hk) * VPH * 2;
+        for (int q = tid; q < n4; q += blockDim.x) {
+            const bool isk = q >= nq4;
+            const int r = isk ? q - nq4 : q;
+            const int h = r / (2 * VPH), m = (r / VPH) & 1, v = r % VPH;
+            const uint2 w = reinterpret_cast<const uint2*>(isk ? a.k_weight : a.q_weight)
+                [((size_t)h * VPH + v) * 2 + m];
+            wsm[q] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+        }
+    }
+    __syncthreads();
+
+    const int64_t p = (int64_t)blockIdx.x * G + g;
+    const int64_t n_local = p < a.num_tokens ? (a.num_tokens - 1 - p) / NP + 1 : 0;
+    const int lane = tid & 31, cwarp = ctid >> 5, nwarps = Bg >> 5;
+    const int l = ctid % L;
+    int va, dv;  // the row vectors of the thread's slot halves
+    slot_vectors<D, NEOX>(a, l, va, dv);
+    const int nq = a.hq * L, nk = a.hk * L, nv = a.hv * VPH;
+
+    // The thread's slots: the row vector of their first half (uint4 index in a
+    // row, -1 for none), their head's weights (float4 index in wsm), their
+    // byte offset in the output token row, and whether they are Q slots.
+    int roff[NS], woff[NS], ooff[NS];
+    bool isq[NS];
+#pragma unroll
+    for (int k = 0; k < NS; ++k) {
+        bool q, valid;
+        int hh;
+        if constexpr (MIXED) {
+            const int idx = ctid + k * Bg;
+            q = idx < nq;
+            valid = idx < nq + nk;
+            hh = q ? idx / L : (idx - nq) / L;
+        } else {
+            q = k < S;
+            const int idx = ctid + (q ? k : k - S) * Bg;
+            valid = idx < (q ? nq : nk);
+            hh = idx / L;
+        }
+        const int hg = q ? hh : a.hq + hh;
+        isq[k] = q;
+        roff[k] = valid ? hg * VPH + va : -1;
+        woff[k] = hg * 2 * VPH;
+        ooff[k] = hh * D * OUTB + (FP8 ? 8 : 16) * va;
+    }
+
+    // Patch of the current token, stepped by the pipeline stride.
+    const int hw = a.pph * a.ppw;
+    const int P = a.ppf * hw;
+    int pf, ph, pw, df, dh, dw;
+    {
+        const int s0 = (int)((p + a.pos_offset) % P);
+        pf = s0 / hw; ph = (s0 - pf * hw) / a.ppw; pw = s0 - pf * hw - ph * a.ppw;
+        const int st = (int)(NP % P);
+        df = st / hw; dh = (st - df * hw) / a.ppw; dw = st - df * hw - dh * a.ppw;
+    }
+    const int hcf = a.cf >> 1, hch = a.ch >> 1, hcw = a.cw >> 1;
+    const int nf = a.ppf * hcf, nh = a.pph * hch;
+    uint32_t stage_code = 0;
+    if (HALF <= Bg && ctid < HALF) {
+        const int j = ctid;
+        int rl, k;
+        if (NEOX) {
+            rl = j >> 3; k = j & 7;
+        } else if (j < 4 * L) {
+            rl = j >> 2; k = j & 3;
+        } else {
+            rl = (j - 4 * L) >> 2; k = 4 + ((j - 4 * L) & 3);
+        }
+        const int axis = j < hcf ? 0 : (j < hcf + hch ? 1 : 2);
+        const int col = axis == 0 ? j : (axis == 1 ? j - hcf : j - hcf - hch);
+        stage_code = (uint32_t)(rl * kCsPitch + k) | ((uint32_t)axis << 11) | ((uint32_t)col << 13);
+    }
+    const float inv_nq = 1.0f / (float)(a.norm_q_elems > 0 ? a.norm_q_elems : 1);
+    const float inv_nk = 1.0f / (float)(a.norm_k_elems > 0 ? a.norm_k_elems : 1);
+    const int64_t q_tok = (int64_t)a.hq * D * OUTB, k_tok = (int64_t)a.hk * D * OUTB;
+    const int vout_bytes = a.hv * D * OUTB;
+
+    int64_t i = 0;
+    bool aborted = false;
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t t = p;
+    for (; i < n_local; ++i, t += NP) {
+        const int parity = (int)(i & 1);
+        const bool ok = mbar_wait_abortable(&full[stage], phase, a.wait_limit_ns, abort_flag);
+        const unsigned char* row = ring + (size_t)stage * row_bytes;
+        if (ctid == 0 && ok && v_bulk) {
+            bulk_store(a.v_out + t * vbytes, row + v_off, (uint32_t)vbytes);
+            bulk_commit();
+        }
+        float2 x[NS][8];
+        float2 sq2 = make_float2(0.0f, 0.0f), sk2 = make_float2(0.0f, 0.0f);
+        if (ok) {
+#pragma unroll
+            for (int k = 0; k < NS; ++k) {
+                if (roff[k] < 0) continue;
+                const uint4* v4 = reinterpret_cast<const uint4*>(row) + roff[k];
+                const uint4 ra = v4[0], rb = v4[dv];
+                x[k][0] = bf16x2_to_f2(ra.x); x[k][1] = bf16x2_to_f2(ra.y);
+                x[k][2] = bf16x2_to_f2(ra.z); x[k][3] = bf16x2_to_f2(ra.w);
+                x[k][4] = bf16x2_to_f2(rb.x); x[k][5] = bf16x2_to_f2(rb.y);
+                x[k][6] = bf16x2_to_f2(rb.z); x[k][7] = bf16x2_to_f2(rb.w);
+                if (norm && !supplied) {
+                    float2 acc = isq[k] ? sq2 : sk2;
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) acc = fma2(x[k][m], x[k][m], acc);
+                    if (isq[k]) sq2 = acc; else sk2 = acc;
+                }
+            }
+            if (!v_bulk) {
+                const unsigned char* vrow = row + v_off;
+                uint8_t* vout = a.v_out + t * vout_bytes;
+                const float2 vs2 = make_float2(a.v_scale, a.v_scale);
+                for (int vi = ctid; vi < nv; vi += Bg) {
+                    const uint4 v = reinterpret_cast<const uint4*>(vrow)[vi];
+                    if constexpr (FP8) {
+                        const float2 f0 = mul2(bf16x2_to_f2(v.x), vs2);
+                        const float2 f1 = mul2(bf16x2_to_f2(v.y), vs2);
+                        const float2 f2 = mul2(bf16x2_to_f2(v.z), vs2);
+                        const float2 f3 = mul2(bf16x2_to_f2(v.w), vs2);
+                        const float f[8] = {f0.x, f0.y, f1.x, f1.y, f2.x, f2.y, f3.x, f3.y};
+                        st_v2(vout + (size_t)vi * 8, pack8_e4m3_unscaled(f));
+                    } else {
+                        st_v4(vout + (size_t)vi * 16, v);
+                    }
+                }
+            }
+        }
+        // This token's cos/sin, staged per l-row: [c_0..c_7][s_0..s_7][pad].
+        {
+            float* cp = cst + parity * L * kCsPitch;
+            if (HALF <= Bg) {
+                if (ctid < HALF) {
+                    const int axis = (stage_code >> 11) & 3;
+                    const int col = (int)(stage_code >> 13);
+                    float2 v;
+                    if (a.use_table) {
+                        const int base = axis == 0 ? pf * hcf
+                                                   : (axis == 1 ? nf + ph * hch : nf + nh + pw * hcw);
+                        v = tab[base + col];
+                    } else {
+                        const int pos = axis == 0 ? pf : (axis == 1 ? ph : pw);
+                        v = direct_cos_sin((uint32_t)pos, gq[ctid]);
+                    }
+                    const int dst = (int)(stage_code & 2047);
+                    cp[dst] = v.x;
+                    cp[dst + 8] = v.y;
+                }
+            } else {
+                for (int j = ctid; j < HALF; j += Bg) {
+                    int rl, k;
+                    if (NEOX) {
+                        rl = j >> 3; k = j & 7;
+                    } else if (j < 4 * L) {
+                        rl = j >> 2; k = j & 3;
+                    } else {
+                        rl = (j - 4 * L) >> 2; k = 4 + ((j - 4 * L) & 3);
+                    }
+                    const float2 v = pair_cos_sin(a, gq, tab, j, pf, ph, pw);
+                    cp[rl * kCsPitch + k] = v.x;
+                    cp[rl * kCsPitch + 8 + k] = v.y;
+                }
+            }
+        }
+        if (norm && !supplied) {
+            const float sq = warp_sum(sq2.x + sq2.y);
+            const float sk = warp_sum(sk2.x + sk2.y);
+            if (lane == 0) red[parity * 32 + cwarp] = make_float2(sq, sk);
+        }
+        if (named_barrier_or(1 + g, Bg, !ok)) {
+            aborted = true;
+            if (ctid == 0) *abort_flag = 1u;
+            break;
+        }
+        // Every thread holds this token's slots in registers and has read its
+        // V: the buffer takes the token `stages` after this one.
+        if (ctid == 0 && i + stages < n_local) {
+            if (v_bulk) bulk_wait_read_all();
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&full[stage], tx);
+            bulk_load(ring + (size_t)stage * row_bytes, a.qkv + (t + stages * NP) * row_bytes,
+                      row_bytes, &full[stage]);
+        }
+        if (++stage == stages) {
+            stage = 0;
+            phase ^= 1u;
+        }
+        pw += dw;
+        ph += dh + (pw >= a.ppw ? 1 : 0);
+        pw -= pw >= a.ppw ? a.ppw : 0;
+        pf += df + (ph >= a.pph ? 1 : 0);
+        ph -= ph >= a.pph ? a.pph : 0;
+        pf -= pf >= a.ppf ? a.ppf : 0;
+
+        float rq = 1.0f, rk = 1.0f;
+        if (norm) {
+            float tq, tk;
+            if (supplied) {  // sums over every slice's heads, from the caller
+                const float2 v = reinterpret_cast<const float2*>(a.ssq_in)[t];
+                tq = v.x; tk = v.y;
+            } else {
+                const float4* r4 = reinterpret_cast<const float4*>(red + parity * 32);
+                float4 acc = r4[0];
+                for (int w = 1; w < (nwarps + 1) >> 1; ++w) {
+                    const float4 v = r4[w];
+                    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+                }
+                tq = acc.x + acc.z; tk = acc.y + acc.w;
+            }
+            rq = rsqrtf(tq * inv_nq + a.eps);
+            rk = rsqrtf(tk * inv_nk + a.eps);
+        }
+        if (FP8) {  // E4M3(value * scale): the scale rides on r
+            rq *= a.q_scale;
+            rk *= a.q_scale;
+        }
+        float cs[8], sn[8];
+        {
+            const float4* cp = reinterpret_cast<const float4*>(cst + (parity * L + l) * kCsPitch);
+            const float4 c0 = cp[0], c1 = cp[1], s0 = cp[2], s1 = cp[3];
+            cs[0] = c0.x; cs[1] = c0.y; cs[2] = c0.z; cs[3] = c0.w;
+            cs[4] = c1.x; cs[5] = c1.y; cs[6] = c1.z; cs[7] = c1.w;
+            sn[0] = s0.x; sn[1] = s0.y; sn[2] = s0.z; sn[3] = s0.w;
+            sn[4] = s1.x; sn[5] = s1.y; sn[6] = s1.z; sn[7] = s1.w;
+        }
+        uint8_t* const qrow = a.q_out + t * q_tok;
+        uint8_t* const krow = a.k_out + t * k_tok;
+        // Q slots with r_q on cos/sin, then K slots with r_k: the rotation is
+        // linear, so the norm factor (and the E4M3 scale) rides on it.
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+            const float r = pass == 0 ? rq : rk;
+            const float2 r2 = make_float2(r, r), nr2 = make_float2(-r, -r);
+            float2 C[4], Sv[4], NSv[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float2 c = make_float2(cs[2 * m], cs[2 * m + 1]);
+                const float2 s = make_float2(sn[2 * m], sn[2 * m + 1]);
+                C[m] = mul2(c, r2);
+                Sv[m] = mul2(s, r2);
+                NSv[m] = mul2(s, nr2);
+            }
+#pragma unroll
+            for (int k = 0; k < NS; ++k) {
+                if (roff[k] < 0 || isq[k] != (pass == 0)) continue;
+                const float2* xs = x[k];
+                float2 ya[4], yb[4];
+                if (norm) {
+                    const float4* w = wsm + woff[k];
+                    const float4 a0 = w[va], a1 = w[VPH + va], b0 = w[va + dv],
+                                 b1 = w[VPH + va + dv];
+                    ya[0] = mul2(xs[0], make_float2(a0.x, a0.y));
+                    ya[1] = mul2(xs[1], make_float2(a0.z, a0.w));
+                    ya[2] = mul2(xs[2], make_float2(a1.x, a1.y));
+                    ya[3] = mul2(xs[3], make_float2(a1.z, a1.w));
+                    yb[0] = mul2(xs[4], make_float2(b0.x, b0.y));
+                    yb[1] = mul2(xs[5], make_float2(b0.z, b0.w));
+                    yb[2] = mul2(xs[6], make_float2(b1.x, b1.y));
+                    yb[3] = mul2(xs[7], make_float2(b1.z, b1.w));
+                } else {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        ya[m] = xs[m];
+                        yb[m] = xs[4 + m];
+                    }
+                }
+                float2 oa[4], ob[4];
+                if constexpr (NEOX) {
+                    // channel e of vector a pairs with channel e of vector b
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        oa[m] = fma2(ya[m], C[m], mul2(yb[m], NSv[m]));
+                        ob[m] = fma2(yb[m], C[m], mul2(ya[m], Sv[m]));
+                    }
+                } else {
+                    // channels (2m, 2m+1) of a vector pair up: pair slot m of
+                    // vector a, 4 + m of vector b
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float ca = (m & 1) ? C[m >> 1].y : C[m >> 1].x;
+                        const float sa = (m & 1) ? Sv[m >> 1].y : Sv[m >> 1].x;
+                        const float cb = (m & 1) ? C[2 + (m >> 1)].y : C[2 + (m >> 1)].x;
+                        const float sb = (m & 1) ? Sv[2 + (m >> 1)].y : Sv[2 + (m >> 1)].x;
+                        oa[m].x = ya[m].x * ca - ya[m].y * sa;
+                        oa[m].y = ya[m].y * ca + ya[m].x * sa;
+                        ob[m].x = yb[m].x * cb - yb[m].y * sb;
+                        ob[m].y = yb[m].y * cb + yb[m].x * sb;
+                    }
+                }
+                uint8_t* o = (pass == 0 ? qrow : krow) + ooff[k];
+                if constexpr (FP8) {
+                    const float fa[8] = {oa[0].x, oa[0].y, oa[1].x, oa[1].y,
+                                         oa[2].x, oa[2].y, oa[3].x, oa[3].y};
+                    const float fb[8] = {ob[0].x, ob[0].y, ob[1].x, ob[1].y,
+                                         ob[2].x, ob[2].y, ob[3].x, ob[3].y};
+                    st_v2(o, pack8_e4m3_unscaled(fa));
+                    st_v2(o + 8 * dv, pack8_e4m3_unscaled(fb));
+                } else {
+                    st_v4(o, make_uint4(f2_to_bf16x2(oa[0]), f2_to_bf16x2(oa[1]),
+                                        f2_to_bf16x2(oa[2]), f2_to_bf16x2(oa[3])));
+                    st_v4(o + 16 * dv, make_uint4(f2_to_bf16x2(ob[0]), f2_to_bf16x2(ob[1]),
+                                                 f2_to_bf16x2(ob[2]), f2_to_bf16x2(ob[3])));
+                }
+            }
+        }
+    }
+    if (ctid == 0) {
+        if (aborted || *abort_flag) {
+            atomicOr(&g_rope3d_status, 1u);
+            // Loads of tokens i .. i+stages-1 may still be in flight (each
+            // buffer is refilled at its own token's barrier): drain them,
+            // bounded.
+            for (int64_t j = i; j < n_local && j < i + stages; ++j)
+                mbar_wait_bounded(&full[j % stages], (uint32_t)((j / stages) & 1),
+                                  a.wait_limit_ns);
+        }
+        if (v_bulk) bulk_wait_all();
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Fallback kernel: 128-bit loads into registers, no ring.
 // ---------------------------------------------------------------------------
 template <int D, bool NEOX, bool FP8, int S>
@@ -792,6 +1215,18 @@ int device_sms() {
     return cached_sm_count(&sms) == cudaSuccess ? sms : 0;
 }
 
+// Whether a CTA builds the shared cos/sin table: it must fit, and its
+// entries (one sincos each, per CTA) must not outnumber the angles the CTA
+// would otherwise evaluate per token (half a head's channels for each of its
+// tokens). Short calls (a few thousand tokens over all SMs) evaluate them
+// per token instead.
+bool table_pays(const Rope3DArgs& a, int half) {
+    if ((int64_t)a.table_entries * 8 > kMaxTableBytes) return false;
+    const int sms = std::max(1, device_sms());
+    const int64_t tokens_per_cta = (a.num_tokens + sms - 1) / sms;
+    return (int64_t)a.table_entries <= tokens_per_cta * half;
+}
+
 template <typename K>
 cudaError_t launch_grid(K kern, int block, int smem, int64_t tokens, const Rope3DArgs& args,
                         cudaStream_t stream, int* grid_out) {
@@ -822,7 +1257,7 @@ cudaError_t run(const Rope3DArgs& a, int block_mg, int block_reg, cudaStream_t s
     Rope3DArgs args = a;
     const bool partial = a.mode == kModePartialSsq;
     const int table_bytes = a.table_entries * 8;
-    args.use_table = (!partial && table_bytes <= kMaxTableBytes) ? 1 : 0;
+    args.use_table = (!partial && table_pays(a, HALF)) ? 1 : 0;
     const int used_table = args.use_table ? table_bytes : 0;
     const int row_bytes = partial ? (a.hq + a.hk) * D * 2 : (a.hq + a.hk + a.hv) * D * 2;
     const int weight_floats = (a.is_qk_norm && !partial) ? (a.hq + a.hk) * D : 0;
@@ -890,9 +1325,80 @@ cudaError_t run(const Rope3DArgs& a, int block_mg, int block_reg, cudaStream_t s
     return e;
 }
 
+// The register-resident kernel for a whole-transform call, when its shape
+// fits: NS slots per thread, at most rr_max_threads<NS>() threads per CTA, a
+// two-buffer ring per pipeline in shared memory. Returns cudaErrorNotSupported
+// (nothing launched) otherwise.
+template <int D, bool NEOX, bool FP8, int NS>
+cudaError_t run_rr(const Rope3DArgs& a, cudaStream_t stream, LaunchInfo* info) {
+    constexpr int L = D / 16;
+    if (a.mode == kModePartialSsq) return cudaErrorNotSupported;
+    const bool mixed = a.hq != a.hk;
+    const int nq = a.hq * L, nk = a.hk * L;
+    const int need = mixed ? (nq + nk + NS - 1) / NS : (std::max(nq, nk) + NS / 2 - 1) / (NS / 2);
+    int bg = std::max(32, (need + 31) / 32 * 32);
+    const int max_threads = rr_max_threads<NS>();
+    if (bg > max_threads) return cudaErrorNotSupported;
+    Rope3DArgs args = a;
+    const int table_bytes = a.table_entries * 8;
+    args.use_table = table_pays(a, D / 2) ? 1 : 0;
+    const int used_table = args.use_table ? table_bytes : 0;
+    const int row_bytes = (a.hq + a.hk + a.hv) * D * 2;
+    const int weight_floats = a.is_qk_norm ? (a.hq + a.hk) * D : 0;
+    if (args.norm_q_elems == 0) args.norm_q_elems = a.hq * D;
+    if (args.norm_k_elems == 0) args.norm_k_elems = a.hk * D;
+    int groups = std::min(kMaxGroups, max_threads / bg);
+    const int sms = device_sms();
+    if (sms <= 0) return cudaErrorNoDevice;
+    while (groups > 1 && (int64_t)sms * (groups - 1) >= a.num_tokens) --groups;
+    for (; groups >= 1; --groups)
+        if (mg_layout(D, groups, 2, row_bytes, weight_floats, used_table).total <= kSmemPerSm - 1024)
+            break;
+    if (groups < 1) return cudaErrorNotSupported;
+    int stages = 2;
+    if (mg_layout(D, groups, 3, row_bytes, weight_floats, used_table).total <= kSmemPerSm - 1024)
+        stages = 3;
+    args.stages = stages;
+    args.groups = groups;
+    args.v_bulk = FP8 ? 0 : 1;
+    if (args.wait_limit_ns == 0) args.wait_limit_ns = 2000000000ull;  // 2 s
+    const int smem = mg_layout(D, groups, stages, row_bytes, weight_floats, used_table).total;
+    const int block = bg * groups;
+    void (*kern)(const Rope3DArgs) = mixed ? rope3d_rr_kernel<D, NEOX, FP8, NS, true>
+                                           : rope3d_rr_kernel<D, NEOX, FP8, NS, false>;
+    int per_sm = 0;
+    cudaError_t e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), block, smem,
+                                              &per_sm);
+    if (e == cudaSuccess && per_sm < 1) e = cudaErrorInvalidConfiguration;
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<int64_t>(sms, (a.num_tokens + groups - 1) / groups);
+    e = launch_overlapped(kern, grid, block, smem, stream, args);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        forget_kernel(reinterpret_cast<const void*>(kern));
+        e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), block, smem, &per_sm);
+        if (e == cudaSuccess) e = launch_overlapped(kern, grid, block, smem, stream, args);
+    }
+    if (info) {
+        info->grid = grid;
+        info->block = block;
+        info->smem = smem;
+        info->kernel_id = 3200 + D / 64 * 10 + (NEOX ? 4 : 0) + (FP8 ? 2 : 0) + (mixed ? 1 : 0);
+    }
+    return e;
+}
+
 template <int D, bool NEOX, bool FP8>
 cudaError_t run_s(const Rope3DArgs& a, cudaStream_t stream, LaunchInfo* info) {
     constexpr int L = D / 16;
+    // The register-resident kernel where it measured faster (NeoX pairs or
+    // grouped-query heads with the norm), and for the per-axis NeoX layout,
+    // which only it builds; the pipelined kernel for the rest.
+    if (a.mode != kModePartialSsq &&
+        (a.neox_per_axis || (a.is_qk_norm && (NEOX || a.hq != a.hk)))) {
+        const cudaError_t e = run_rr<D, NEOX, FP8, 4>(a, stream, info);
+        if (e != cudaErrorNotSupported || a.neox_per_axis) return e;
+    }
     const int slots = std::max(std::max(a.hq, a.hk), 1) * L;
     int S = (slots + kMaxBlock - 1) / kMaxBlock;
     if (S > 4) return cudaErrorInvalidValue;  // rejected earlier by the host checks

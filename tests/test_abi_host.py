@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_strings(L):
-    assert L.qknr_abi_version() == Q.ABI_VERSION == 3
+    assert L.qknr_abi_version() == Q.ABI_VERSION == 4
     for s in range(8):
         assert L.qknr_status_string(s)
     assert L.qknr_status_string(0) == b"ok"
@@ -91,6 +91,8 @@ def _call3d(L, p):
     (dict(eps=-1.0), Q.QKNR_ERR_SHAPE, "eps"),
     (dict(qkv_ptr=0), Q.QKNR_ERR_NULL, "qkv"),
     (dict(qkv_ptr=A + 8), Q.QKNR_ERR_ALIGN, "16-byte"),
+    # NeoX pairs per axis group are built for groups that are multiples of 16
+    (dict(interleave=False, neox_per_axis=True), Q.QKNR_ERR_UNSUPPORTED, "multiples of 16"),
 ])
 def test_3d_validation(L, over, code, needle):
     p = _p3(**over)

@@ -62,3 +62,12 @@ def test_one_core_figure_restores_threads():
             w = dataclasses.replace(w, tokens=64)
         assert bench.one_core(w, inp, 0.05, chunk) > 0
         assert O.threads() == before
+
+
+def test_host_cost_program_builds():
+    """The C host-cost program (tests/host_cost.c) compiles and links against
+    libqknr.so; running it needs a GPU."""
+    import bench
+
+    exe = bench.host_cost_exe()
+    assert os.path.exists(exe) and os.access(exe, os.X_OK)

@@ -199,6 +199,47 @@ def test_3d_variants(case):
     check_3d_case(qkv, qw if norm else None, kw if norm else None, **p)
 
 
+CASES_PER_AXIS = [
+    # (T, Hq, Hk, Hv, D, grid, channels, fp8, norm, pos_offset)
+    (3001, 24, 24, 24, 128, (31, 24, 40), (32, 48, 48), True, True, 12345),   # FP8 NeoX geometry
+    (3001, 24, 24, 24, 128, (31, 24, 40), (32, 48, 48), True, False, 12345),  # without the norm
+    (3001, 24, 24, 24, 128, (31, 24, 40), (32, 48, 48), False, True, 5),      # bf16 out
+    (500, 5, 3, 2, 64, (2, 5, 50), (16, 16, 32), False, True, 7),             # grouped-query
+    (300, 2, 2, 1, 256, (3, 4, 25), (64, 96, 96), False, True, 0),            # head_dim 256
+    (300, 2, 2, 1, 256, (3, 4, 25), (64, 96, 96), True, True, 0),
+    (400, 4, 4, 4, 128, (1, 20, 20), (0, 64, 64), False, True, 0),            # empty frame group
+]
+
+
+@pytest.mark.parametrize("case", CASES_PER_AXIS, ids=[str(i) for i in range(len(CASES_PER_AXIS))])
+def test_3d_neox_per_axis(case):
+    """NeoX halves inside each axis group (neox_per_axis), the other reading
+    of the page's "NeoX-style", against the oracle's per-axis pair map."""
+    T, Hq, Hk, Hv, D, grid, ch, fp8, norm, off = case
+    qkv, qw, kw = _rand3d(T, Hq, Hk, Hv, D, std=2.0, seed=T + D + 1)
+    p = dict(ppf=grid[0], pph=grid[1], ppw=grid[2], num_frame_channels=ch[0],
+             num_height_channels=ch[1], num_width_channels=ch[2], num_heads_q=Hq, num_heads_k=Hk,
+             num_heads_v=Hv, head_dim=D, eps=1e-5, base=10000.0, interleave=False,
+             is_qk_norm=norm, output_fp8=fp8, output_quant_scale=0.75, v_quant_scale=1.5,
+             pos_offset=off, neox_per_axis=True)
+    outs = check_3d_case(qkv, qw if norm else None, kw if norm else None, **p)
+    whole = run_3d(qkv, qw if norm else None, kw if norm else None, **dict(p, neox_per_axis=False))
+    assert not torch.equal(outs[0].view(torch.uint8), whole[0].view(torch.uint8))
+
+
+def test_3d_neox_per_axis_ignored_when_interleaved():
+    """With adjacent pairs the two readings coincide: the flag changes nothing."""
+    qkv, qw, kw = _rand3d(200, 4, 4, 4, 128, seed=8)
+    p = dict(ppf=2, pph=10, ppw=10, num_frame_channels=32, num_height_channels=48,
+             num_width_channels=48, num_heads_q=4, num_heads_k=4, num_heads_v=4, head_dim=128,
+             interleave=True)
+    a = run_3d(qkv, qw, kw, **p)
+    b = run_3d(qkv, qw, kw, neox_per_axis=True, **p)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
 def test_3d_rope_only_origin_is_bit_copy():
     qkv, _, _ = _rand3d(16, 4, 4, 4, 64, std=3.0)
     p = dict(ppf=1, pph=4, ppw=4, num_frame_channels=16, num_height_channels=24,

@@ -23,13 +23,15 @@ def _slice_cols(qkv, heads, D, sl):
     return qkv[:, (heads + sl[0]) * D:(heads + sl[1]) * D]
 
 
-def _run_simulated(w, T, R, pos_offset=None):
+def _run_simulated(w, T, R, pos_offset=None, per_axis=False):
     inp = W.make_inputs(w, device="cpu", tokens=T)
     qkv, qw, kw = inp["qkv"], inp["q_weight"], inp["k_weight"]
     D = w.head_dim
     p = dict(w.params())
     if pos_offset is not None:
         p["pos_offset"] = pos_offset
+    if per_axis:
+        p["neox_per_axis"] = True
     slices = [(tp.head_slice(w.hq, R, r), tp.head_slice(w.hk, R, r), tp.head_slice(w.hv, R, r))
               for r in range(R)]
     locals_ = []
@@ -72,6 +74,12 @@ def test_tp_simulated_matches_oracle(name, R):
     want_k = x[:, w.hq * w.head_dim:(w.hq + w.hk) * w.head_dim].pow(2).sum(1)
     np.testing.assert_allclose(total[:, 0].cpu().numpy(), want_q.numpy(), rtol=1e-5)
     np.testing.assert_allclose(total[:, 1].cpu().numpy(), want_k.numpy(), rtol=1e-5)
+
+
+@pytest.mark.parametrize("R", [1, 3])
+def test_tp_simulated_neox_per_axis(R):
+    """The per-axis NeoX layout through the two tensor-parallel passes."""
+    _run_simulated(W.WORKLOADS["fp8neox"], 1201, R, pos_offset=333, per_axis=True)
 
 
 def test_tp_one_rank_nccl_group():

@@ -34,6 +34,9 @@ MUTATIONS = {
     "axis_order_swapped": ("int64_t pos[3] = {f, h, w};", "int64_t pos[3] = {w, h, f};"),
     "position_height_index": ("*h = (s / ppw) % pph;", "*h = (s / pph) % ppw;"),
     "pos_offset_ignored": ("int64_t s = (t + pos_offset) % P;", "int64_t s = t % P;"),
+    "per_axis_partner_mirrored": ("pb[off / 2 + i] = off + i + C[a] / 2;",
+                                  "pb[off / 2 + i] = off + C[a] - 1 - i;"),
+    "per_axis_flag_ignored": ("} else if (!neox_per_axis) {", "} else if (1) {"),
     "half_split_mirrored": ("pb[j] = interleaved ? 2 * j + 1 : j + rotary_dim / 2;",
                             "pb[j] = interleaved ? 2 * j + 1 : rotary_dim - 1 - j;"),
     "table_sin_column": ("s[j] = row[R / 2 + j];\n            } else {",

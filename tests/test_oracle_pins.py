@@ -496,6 +496,34 @@ def pin_width_axis_textbook_rope():
         assert np.allclose(q[t, 0, :8], y[t, :8], atol=1e-14)
 
 
+def pin_neox_per_axis_textbook_rope():
+    """The other reading of [F] interleave=False ("NeoX-style"), NeoX halves
+    inside each axis group, on a grid where only the height and width positions
+    vary: each group is a textbook 1D half-split RoPE of its own channels,
+    pairs (o + i, o + i + C/2) multiplied by exp(i * pos * base^(-2i/C)) as
+    numpy complex numbers; the frame group (position 0) is not turned. The
+    whole-head NeoX reading differs on the same input."""
+    D = 32
+    ch = (8, 8, 16)
+    qkv, qw, kw, p = _tiny3d(T=12, grid=(1, 3, 4), ch=ch, weights=False, H=(1, 1, 1), D=D)
+    p = dict(p, interleave=False)
+    q, _, _ = O.rope_3d(qkv, qw, kw, eps=0.0, exact=True, neox_per_axis=True, **p)
+    q_whole, _, _ = O.rope_3d(qkv, qw, kw, eps=0.0, exact=True, **p)
+    x = O.bf16_to_f64(qkv)[:, :D]
+    y = x / np.sqrt(np.mean(x ** 2, axis=1, keepdims=True))
+    for t in range(12):
+        pos = {0: 0, 1: t // 4, 2: t % 4}
+        o = 0
+        for a, C in enumerate(ch):
+            h = C // 2
+            freqs = 10000.0 ** (-np.arange(h) * 2.0 / C)
+            z = (y[t, o:o + h] + 1j * y[t, o + h:o + C]) * np.exp(1j * pos[a] * freqs)
+            assert np.allclose(q[t, 0, o:o + h], z.real, atol=1e-13)
+            assert np.allclose(q[t, 0, o + h:o + C], z.imag, atol=1e-13)
+            o += C
+    assert not np.allclose(q, q_whole)
+
+
 def pin_offset_and_batch_repeat():
     """A token range computed with pos_offset equals the same rows of the whole
     call, and a second batch (tokens P..2P-1) repeats the first's angles."""
