@@ -40,15 +40,15 @@ FALLBACK_HBM_GBS = 6650.0
 # rope_table.md, ucpe_cam_prep.md), valid only for the kernel sources whose
 # hash is stored beside it (the bench reports null otherwise).
 TRAFFIC = {
-    "video3d": (377564416 + 325334784, "f0170ddbe869b9f9"),
-    "fp8neox": (1097153280 + 517297920, "f0170ddbe869b9f9"),
-    "fp8neox_nonorm": (1097140224 + 517154816, "f0170ddbe869b9f9"),
-    "gqa3d": (189662976 + 139130624, "f0170ddbe869b9f9"),
-    "table_hs": (43562240 + 2029568, "9230c313092c6dc7"),
-    "table_il": (25730816 + 15616, "9230c313092c6dc7"),
-    "table_hs_f16": (42770176 + 2013952, "9230c313092c6dc7"),
-    "table_d72": (24805120 + 3584, "9230c313092c6dc7"),
-    "ucpe": (259064832 + 202290688, "a8106b18f58c9fbf"),
+    "video3d": (377566208 + 325051392, "5b35f23a7b87b432"),
+    "fp8neox": (1097155840 + 506035456, "5b35f23a7b87b432"),
+    "fp8neox_nonorm": (1097141504 + 516299008, "5b35f23a7b87b432"),
+    "gqa3d": (188821760 + 132320768, "5b35f23a7b87b432"),
+    "table_hs": (43556096 + 2080000, "e2facc58fbd531cb"),
+    "table_il": (25730304 + 0, "e2facc58fbd531cb"),
+    "table_hs_f16": (42769920 + 1963008, "e2facc58fbd531cb"),
+    "table_d72": (24805632 + 4608, "e2facc58fbd531cb"),
+    "ucpe": (263128576 + 204118016, "b20337bb3277e59c"),
 }
 KERNEL_FILES = {"3d": ("rope3d.cu",), "table": ("rope_table.cu",),
                 "ucpe": ("ucpe_launch.h", "ucpe.cu")}

@@ -253,10 +253,13 @@ int qknr_rope_3d_with_ssq(const qknr_rope_3d_params* params, const float* ssq,
  * k_scale          any finite float (the page's value is
  *                  head_dim^-0.5 * spatial_tokens^-0.5).
  * Alignment: every pointer 16-byte aligned (QKNR_ERR_ALIGN otherwise).
- * Any num_tokens is allowed. head_dim <= 128 with an even num_tokens and at
- * least two heads runs the pipelined kernel; other shapes run a general one,
- * which writes two bytes at a time when num_tokens is not a multiple of 8.
- * Range: both kernels apply k_scale to K's rotated result (the projection
+ * Any num_tokens is allowed. Kernels: with at least two heads, head_dim
+ * 72..120, device-memory q/k/v and batch*num_tokens >= 64, a warp-specialised
+ * pipelined kernel (any num_tokens); else, with at least two heads,
+ * head_dim <= 128 and an even num_tokens, a barrier-synchronised pipelined
+ * kernel; else a general one, which writes two bytes at a time when
+ * num_tokens is not a multiple of 8.
+ * Range: every kernel applies k_scale to K's rotated result (the projection
  * and the rotation are linear) and take the two fp32 sums of squares over the
  * unscaled ReLU key, so the scale itself never underflows or overflows them.
  * A key whose squares all underflow fp32 (every channel below about 1e-19 in
@@ -264,9 +267,11 @@ int qknr_rope_3d_with_ssq(const qknr_rope_3d_params* params, const float* ssq,
  * squares overflows fp32 (channels above about 1e18 at head_dim 256, 1.8e19
  * for one channel) gives inflation_sq NaN, where the fp64 definition stays
  * finite.
- * The kernels wait only on their own cp.async groups and bulk stores, which
- * always complete, so they have no timeout path and do not set the device
- * status word.
+ * The warp-specialised kernel's waits (its compute warps on the copy warp's
+ * ring stages, the copy warp on the compute warps) are bounded at 2 s; on
+ * expiry the launch abandons its remaining steps and raises bit 0 of the
+ * device status word (qknr_device_status). The other two kernels wait only on
+ * their own cp.async groups and CTA barriers, which always complete.
  */
 int qknr_ucpe_cam_prep(const void* q_normed, const void* k_normed, const void* v_raw,
                        const float* proj_q, const float* proj_kv, const float* rope_cos,
@@ -278,7 +283,8 @@ int qknr_ucpe_cam_prep(const void* q_normed, const void* k_normed, const void* v
 /*
  * Device-side status of this library's kernels on the current device, for
  * failures that can only be seen on the GPU. Bit 0: a kernel's wait on one of
- * its own bulk copies ran past its time limit (2 s), so that launch abandoned
+ * its own bulk copies (or, in the camera prep, on another warp of its CTA) ran
+ * past its time limit (2 s), so that launch abandoned
  * its remaining tokens and its outputs are incomplete; the kernel still ended
  * normally and the CUDA context stays usable. The word accumulates over
  * launches until cleared. Unlike every other entry point this one
@@ -290,7 +296,8 @@ int qknr_device_status(void* cuda_stream, uint32_t* status_out, int32_t clear);
 /*
  * Test hook for the timeout path above (not for production use). While
  * extra_bytes is non-zero, every later launch of a bulk-copy kernel (3D and
- * table forms) on any thread makes each ring buffer wait for extra_bytes more
+ * table forms, the camera prep's warp-specialised kernel) on any thread makes each
+ * ring buffer wait for extra_bytes more
  * than its copy delivers, so its waits
  * run out after limit_ns and the launch takes the abandon path; the copies
  * themselves complete, so nothing is left in flight. extra_bytes == 0 turns

@@ -150,10 +150,12 @@ int qknr_device_status(void* cuda_stream, uint32_t* status_out, int32_t clear) {
     if (!status_out) return fail(QKNR_ERR_NULL, "status_out is NULL");
     uint32_t v = 0, w = 0;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    uint32_t u = 0;
     cudaError_t e = qknr::read_device_status(&v, clear, st);
     if (e == cudaSuccess) e = qknr::read_table_status(&w, clear, st);
+    if (e == cudaSuccess) e = qknr::read_ucpe_status(&u, clear, st);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
-    *status_out = v | w;
+    *status_out = v | w | u;
     return ok();
 }
 
@@ -551,8 +553,23 @@ int qknr_ucpe_cam_prep(const void* q_normed, const void* k_normed, const void* v
     a.head_dim = head_dim;
     a.act_f16 = act_dtype == QKNR_DT_F16;
     a.k_scale = k_scale;
+    qknr::UcpeControl ctl{};
+    ctl.stall_tx_bytes = g_fault_extra_bytes.load(std::memory_order_relaxed);
+    ctl.wait_limit_ns = ctl.stall_tx_bytes ? g_fault_limit_ns.load() : 2000000000ull;  // 2 s
+    // The warp-specialised kernel reads q, k and v through tensor maps: only
+    // for device memory (page-locked host or managed buffers take another).
+    ctl.device_inputs = 1;
+    for (int i = 0; i < 3; ++i) {
+        cudaPointerAttributes attr;
+        if (cudaPointerGetAttributes(&attr, all[i]) != cudaSuccess) {
+            cudaGetLastError();
+            ctl.device_inputs = 0;
+        } else if (attr.type != cudaMemoryTypeDevice) {
+            ctl.device_inputs = 0;
+        }
+    }
     qknr::LaunchInfo info{};
-    e = qknr::launch_ucpe(a, static_cast<cudaStream_t>(cuda_stream), &info);
+    e = qknr::launch_ucpe(a, ctl, static_cast<cudaStream_t>(cuda_stream), &info);
     if (e != cudaSuccess) return cuda_fail(e, "camera prep kernel launch");
     return ok();
 }

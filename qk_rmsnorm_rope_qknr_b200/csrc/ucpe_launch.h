@@ -24,8 +24,22 @@ struct UcpeArgs {
     float k_scale;
 };
 
+// What only the warp-specialised kernel needs (kept out of UcpeArgs, whose
+// layout the other two kernels' register allocation is sensitive to).
+struct UcpeControl {
+    int32_t device_inputs;    // q, k, v are device memory (the kernel reads them by tensor maps)
+    uint32_t stall_tx_bytes;  // test hook: extra bytes a ring stage waits for (0 in use)
+    uint64_t wait_limit_ns;   // a wait on a copy or on another warp gives up after this long
+};
+
 // UCPE camera prep (head_dim a multiple of 8 up to 256; pointers 16-byte
 // aligned; sizes already checked).
-cudaError_t launch_ucpe(const UcpeArgs& a, cudaStream_t stream, LaunchInfo* info);
+cudaError_t launch_ucpe(const UcpeArgs& a, const UcpeControl& ctl, cudaStream_t stream,
+                        LaunchInfo* info);
+
+// Status word of the camera-prep kernels (bit 0: a wait ran past its limit and
+// the launch abandoned its remaining steps), read on `stream`; optionally
+// cleared.
+cudaError_t read_ucpe_status(uint32_t* out, int clear, cudaStream_t stream);
 
 }  // namespace qknr

@@ -1,6 +1,8 @@
 """Failure detection on the GPU without faulting it.
 
-The pipelined 3D kernel bounds every wait on its own bulk copies. The test
+The pipelined 3D and table kernels bound every wait on their own bulk copies,
+and the camera prep's warp-specialised kernel every wait on its copy warp and
+on its compute warps. The test
 hook makes each ring buffer expect 16 bytes more than its copy delivers (a
 count that nothing completes), with a 20 ms limit: the waits run out, the
 launch abandons its tokens, raises bit 0 of the device status word, drains its
@@ -88,6 +90,41 @@ def test_table_wait_timeout_raises_status_and_context_survives(shape):
     assert Q.qknr_device_status(clear=True) & 1
     again = [torch.empty_like(inp["q"]), torch.empty_like(inp["k"])]
     call(*again)
+    torch.cuda.synchronize()
+    for a, b in zip(good, again):
+        assert torch.equal(a, b)
+    assert Q.qknr_device_status() == 0
+
+
+def test_ucpe_wait_timeout_raises_status_and_context_survives():
+    """The camera prep's warp-specialised kernel: its compute warps wait on the copy
+    warp's ring stages and the copy warp on them, every wait bounded. With the
+    hook, the stages never fill: the waits run out, the launch abandons its
+    steps, raises bit 0, waits (bounded) for the copies it issued and ends."""
+    B, N, H, D = 1, 128, 3, 112
+    w = W.FormUcpe("case", batch=B, seq=N, heads=H, head_dim=D, spatial=N // 4, seed=6)
+    inp = W.make_inputs(w, device="cuda")
+    args = [inp[k] for k in ("q_normed", "k_normed", "v_raw", "proj_q", "proj_kv", "rope_cos",
+                             "rope_sin")]
+
+    def call():
+        outs = [torch.empty(B, H, D, N, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+        infl = torch.empty(B, H, N, device="cuda")
+        Q.qknr_ucpe_cam_prep(*args, *outs, infl, k_scale=w.k_scale)
+        return outs + [infl]
+
+    good = call()
+    torch.cuda.synchronize()
+    Q.qknr_device_status(clear=True)
+    L = Q.lib()
+    assert L.qknr_test_set_wait_fault(16, 20_000_000) == 0
+    try:
+        call()
+        torch.cuda.synchronize()
+    finally:
+        assert L.qknr_test_set_wait_fault(0, 0) == 0
+    assert Q.qknr_device_status(clear=True) & 1
+    again = call()
     torch.cuda.synchronize()
     for a, b in zip(good, again):
         assert torch.equal(a, b)

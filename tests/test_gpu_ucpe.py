@@ -57,10 +57,11 @@ def _compare(outs, ref, ref_exact, act, where=""):
 
 
 CASES = [
-    # B, N, H, D, act. The pipelined kernel takes head_dim <= 128, an even N
-    # and at least two heads: ring depths 3 (two heads, or head_dim 128) and 4,
-    # ragged last tiles (also of 2 mod 8 tokens), a single 8-token tile,
-    # several tiles per CTA.
+    # B, N, H, D, act. Pipelined kernels (at least two heads): the
+    # warp-specialised one for head_dim 72..120 (any N, at least 64 rows), the
+    # barrier-synchronised one for the other head_dims up to 128 with an even
+    # N; ring depths 3 (two heads, or head_dim 128) and 4, ragged last tiles
+    # (also of 2 mod 8 tokens), a single 8-token tile, several tiles per CTA.
     (1, 64, 3, 8, "bf16"),
     (2, 128, 4, 16, "bf16"),
     (1, 200, 5, 56, "bf16"),
@@ -74,7 +75,8 @@ CASES = [
     (2, 130, 2, 24, "bf16"),
     (1, 150, 3, 112, "f16"),
     (2, 64, 2, 40, "f16"),
-    # The general kernel: one head, odd N (two-byte stores), head_dim above
+    # Odd N: the warp-specialised kernel (head_dim 72..120, 16-bit stores),
+    # else the general kernel, which also takes one head and head_dim above
     # 128; tiles of 64 tokens with ragged tails, every chunk count parity
     (1, 64, 1, 8, "bf16"),
     (1, 201, 3, 16, "bf16"),
@@ -159,12 +161,12 @@ def test_ucpe_zero_k_scale(N):
 
 
 @pytest.mark.parametrize("k_scale", [1e-20, 1e20])
-@pytest.mark.parametrize("N", [61, 64])  # general kernel, pipelined kernel
-def test_ucpe_extreme_k_scale(N, k_scale):
+@pytest.mark.parametrize("N,D", [(61, 48), (64, 48), (97, 112)])  # general, synchronised,
+def test_ucpe_extreme_k_scale(N, D, k_scale):                      # warp-specialised kernel
     """A tiny or huge K scale: both kernels take the sums of squares over the
     unscaled key (the scale cancels in the gain), so inflation_sq neither
     underflows to 1 nor overflows to NaN, and k_trans carries the scale."""
-    B, H, D = 1, 3, 48
+    B, H = 1, 3
     w, inp = _case(B, N, H, D, seed=13)
     outs = Q.cam_prep_func(inp["q_normed"], inp["k_normed"], inp["v_raw"], proj_q=inp["proj_q"],
                            proj_kv=inp["proj_kv"], rope_cos=inp["rope_cos"],
