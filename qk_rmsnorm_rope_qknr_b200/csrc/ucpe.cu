@@ -11,10 +11,12 @@
 //   V: times proj_kv blockwise;
 // and the three results are stored transposed, [B, H, D, N].
 //
-// The work is a stream over HBM (about 1.5 flops per byte). Two kernels do it:
-// ucpe_fast_kernel (further down) for head_dim <= 128, an even token count and
-// at least two heads, and ucpe_prep_kernel for every other shape. Both are
-// built for coalescing on both sides of the transpose. The general kernel:
+// The work is a stream over HBM (about 1.5 flops per byte). Three kernels do
+// it, all built for coalescing on both sides of the transpose:
+// ucpe_fast_kernel (warp-specialised, further down) for head_dim 72..120 with
+// at least two heads; ucpe_sync_kernel (barrier-synchronised) for the other
+// head_dims up to 128 with an even token count and at least two heads; and
+// ucpe_prep_kernel for every other shape. The general kernel:
 //   - work unit: a tile of 64 consecutive tokens of one (batch, head), tiles
 //     numbered with the head fastest, so that the tiles in flight at once
 //     share their tokens' cos/sin rows and matrices in L2;
