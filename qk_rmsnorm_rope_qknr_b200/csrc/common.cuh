@@ -290,6 +290,17 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
 
 __device__ __forceinline__ uint32_t f2_to_bf16x2(float2 v) { return pack_bf16x2(v.x, v.y); }
 
+// acc + (lo^2, hi^2) for the bf16 pair in w: two mixed-precision FMAs (bf16
+// inputs, fp32 accumulation, one rounding each), the same results as widening
+// first and one fp32x2 FMA.
+__device__ __forceinline__ float2 ssq_bf16x2(uint32_t w, float2 acc) {
+    asm("{\n.reg .b16 lo, hi;\nmov.b32 {lo, hi}, %2;\n"
+        "fma.rn.f32.bf16 %0, lo, lo, %0;\nfma.rn.f32.bf16 %1, hi, hi, %1;\n}"
+        : "+f"(acc.x), "+f"(acc.y)
+        : "r"(w));
+    return acc;
+}
+
 // 16-bit activation pairs: bf16 (H16 = false) or IEEE binary16 (H16 = true).
 template <bool H16>
 __device__ __forceinline__ float2 act2_to_f2(uint32_t w) {

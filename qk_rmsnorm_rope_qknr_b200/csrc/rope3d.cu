@@ -266,14 +266,12 @@ __device__ __forceinline__ void apply_slot_wf(const uint4& va, const uint4& vb,
     }
 }
 
-// Sum of squares of the 16 channels of a vector pair, packed.
+// Sum of squares of the 16 channels of a vector pair (even channels in .x,
+// odd ones in .y), straight from the bf16 pairs.
 __device__ __forceinline__ float2 ssq_pair(const uint4& va, const uint4& vb, float2 acc) {
     const uint32_t w[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const float2 x = bf16x2_to_f2(w[m]);
-        acc = fma2(x, x, acc);
-    }
+    for (int m = 0; m < 8; ++m) acc = ssq_bf16x2(w[m], acc);
     return acc;
 }
 
@@ -673,11 +671,12 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
 // ---------------------------------------------------------------------------
 // Register-resident pipelined kernel: as rope3d_mg_kernel (G token pipelines
 // per CTA, bulk-copy rings, shared angle table and fp32 weights), but each
-// thread keeps its NS slots in registers, widened to fp32, from the sums of
-// squares to the stores. A token therefore needs NS/2 times fewer threads,
-// every slot is read from shared memory and widened once, and the token's
-// own ring buffer is free at the token's barrier: it is refilled there, one
-// and a half tokens of copy time ahead of its next use. The per-token work
+// thread keeps its NS slots in registers, as loaded (bf16 pairs), from the
+// sums of squares (mixed-precision FMAs on the pairs) to the stores. A token
+// therefore needs NS/2 times fewer threads, every slot is read from shared
+// memory once and widened once, and the token's own ring buffer is free at
+// the token's barrier: it is refilled there, one and a half tokens of copy
+// time ahead of its next use. The per-token work
 // that every warp repeats (the wait, the reductions, the barrier, r, the
 // cos/sin reads, the loop) is spread over NS slots per thread instead of two.
 //
@@ -843,22 +842,21 @@ __global__ void __launch_bounds__(rr_max_threads<NS>(), 1) rope3d_rr_kernel(cons
             bulk_store(a.v_out + t * vbytes, row + v_off, (uint32_t)vbytes);
             bulk_commit();
         }
-        float2 x[NS][8];
+        uint4 px[NS][2];  // the slots' channels as loaded (bf16 pairs)
         float2 sq2 = make_float2(0.0f, 0.0f), sk2 = make_float2(0.0f, 0.0f);
         if (ok) {
 #pragma unroll
             for (int k = 0; k < NS; ++k) {
                 if (roff[k] < 0) continue;
                 const uint4* v4 = reinterpret_cast<const uint4*>(row) + roff[k];
-                const uint4 ra = v4[0], rb = v4[dv];
-                x[k][0] = bf16x2_to_f2(ra.x); x[k][1] = bf16x2_to_f2(ra.y);
-                x[k][2] = bf16x2_to_f2(ra.z); x[k][3] = bf16x2_to_f2(ra.w);
-                x[k][4] = bf16x2_to_f2(rb.x); x[k][5] = bf16x2_to_f2(rb.y);
-                x[k][6] = bf16x2_to_f2(rb.z); x[k][7] = bf16x2_to_f2(rb.w);
+                px[k][0] = v4[0];
+                px[k][1] = v4[dv];
                 if (norm && !supplied) {
                     float2 acc = isq[k] ? sq2 : sk2;
+                    const uint32_t w[8] = {px[k][0].x, px[k][0].y, px[k][0].z, px[k][0].w,
+                                           px[k][1].x, px[k][1].y, px[k][1].z, px[k][1].w};
 #pragma unroll
-                    for (int m = 0; m < 8; ++m) acc = fma2(x[k][m], x[k][m], acc);
+                    for (int m = 0; m < 8; ++m) acc = ssq_bf16x2(w[m], acc);
                     if (isq[k]) sq2 = acc; else sk2 = acc;
                 }
             }
@@ -998,7 +996,10 @@ __global__ void __launch_bounds__(rr_max_threads<NS>(), 1) rope3d_rr_kernel(cons
 #pragma unroll
             for (int k = 0; k < NS; ++k) {
                 if (roff[k] < 0 || isq[k] != (pass == 0)) continue;
-                const float2* xs = x[k];
+                const float2 xs[8] = {
+                    bf16x2_to_f2(px[k][0].x), bf16x2_to_f2(px[k][0].y), bf16x2_to_f2(px[k][0].z),
+                    bf16x2_to_f2(px[k][0].w), bf16x2_to_f2(px[k][1].x), bf16x2_to_f2(px[k][1].y),
+                    bf16x2_to_f2(px[k][1].z), bf16x2_to_f2(px[k][1].w)};
                 float2 ya[4], yb[4];
                 if (norm) {
                     const float4* w = wsm + woff[k];
