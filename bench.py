@@ -44,11 +44,11 @@ TRAFFIC = {
     "fp8neox": (1097223424 + 511681024, "c498c206163b8263"),
     "fp8neox_nonorm": (1097139456 + 516128512, "c498c206163b8263"),
     "gqa3d": (188852992 + 131656960, "c498c206163b8263"),
-    "table_hs": (43556096 + 2080000, "e2facc58fbd531cb"),
-    "table_il": (25730304 + 0, "e2facc58fbd531cb"),
-    "table_hs_f16": (42769920 + 1963008, "e2facc58fbd531cb"),
-    "table_d72": (24805632 + 4608, "e2facc58fbd531cb"),
-    "ucpe": (263128576 + 204118016, "b20337bb3277e59c"),
+    "table_hs": (43556096 + 2207488, "d163d414d08677d2"),
+    "table_il": (25730048 + 0, "d163d414d08677d2"),
+    "table_hs_f16": (42769152 + 1724416, "d163d414d08677d2"),
+    "table_d72": (24805632 + 1024, "d163d414d08677d2"),
+    "ucpe": (263094016 + 204621056, "af3adacd4b1bec78"),
 }
 KERNEL_FILES = {"3d": ("rope3d.cu",), "table": ("rope_table.cu",),
                 "ucpe": ("ucpe_launch.h", "ucpe.cu")}
@@ -86,7 +86,8 @@ class ClockSampler:
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "clocks.mem")
 
     def __init__(self, gpu_index: int):
         # nvidia-smi numbers GPUs physically; under CUDA_VISIBLE_DEVICES the
@@ -134,7 +135,7 @@ class ClockSampler:
         """Median SM clock and the throttle reasons seen while the GPU was
         under load: from the start of the spin-up to the end of the timed
         region (samples of the idle start-up are left out)."""
-        sm, smax, reasons = [], None, set()
+        sm, smax, mem, reasons = [], None, [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for t, ln in self.lines:
             if self.load_from is not None and t < self.load_from:
@@ -152,10 +153,15 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
+            try:
+                mem.append(float(parts[9]))
+            except (IndexError, ValueError):
+                pass
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
                     "gpu": self.gpu}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
+                "mem_mhz": statistics.median(mem) if mem else None,
                 "reasons": sorted(reasons), "samples": len(sm), "gpu": self.gpu}
 
 
@@ -378,14 +384,17 @@ def time_steps(step, args, stream, local, dev, pg):
     stream. The kernels are programmatic dependent launches, so no event may
     sit between them: the average launch duration is the region's time over K.
 
-    The optional spin-up (--spin-ms, off by default) runs untimed steps for
-    that long with the clock sampler already running, so that the region
-    starts at the clock the GPU holds under sustained load. On a 1 kW B200
-    that is the power-capped clock: after 500 ms of this load the SM clock
-    sits near 1750-1850 MHz with sw_power_cap active, where a short region
-    that starts from a cool GPU runs at 1965 MHz. Both are real operating
-    points; the bench line carries the sampled clock and the time normalised
-    to the top clock, so either can be compared.
+    The spin-up (--spin-ms, 1000 ms by default; 0 turns it off) runs untimed
+    steps for that long with the clock sampler already running, so that the
+    K timed steps measure the state the GPU holds under sustained load, which
+    is how the op runs inside a model. On B200 that state differs from a cool
+    start in two ways: the 1 kW power cap lowers the SM clock (to about
+    1640-1700 MHz for these kernels, sw_power_cap active), and the kernels
+    nevertheless run faster than in the first few milliseconds after idle
+    (the FP8 3D workload: 260.6 us after 1 s of load at 1642 MHz against
+    288 us in 20 cold launches at 1965 MHz on the same box, memory clock at
+    its maximum in both). The bench line carries the sampled SM and memory
+    clocks and the time normalised to the top SM clock.
     Returns (ms per step, max over ranks; the clock sampler)."""
     import torch
 
@@ -1107,7 +1116,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="qknr", choices=["qknr", "reference"])
     ap.add_argument("--workload", default="fp8neox")
-    ap.add_argument("--spin-ms", type=float, default=0.0,
+    ap.add_argument("--spin-ms", type=float, default=1000.0,
                     help="untimed steps for this long before the warm-up, with the clock "
                          "sampler running")
     ap.add_argument("--e2e-steps", type=int, default=20)
