@@ -40,15 +40,15 @@ FALLBACK_HBM_GBS = 6650.0
 # rope_table.md, ucpe_cam_prep.md), valid only for the kernel sources whose
 # hash is stored beside it (the bench reports null otherwise).
 TRAFFIC = {
-    "video3d": (377564416 + 324862208, "c498c206163b8263"),
-    "fp8neox": (1097223424 + 511681024, "c498c206163b8263"),
-    "fp8neox_nonorm": (1097139456 + 516128512, "c498c206163b8263"),
-    "gqa3d": (188852992 + 131656960, "c498c206163b8263"),
-    "table_hs": (43556096 + 2207488, "d163d414d08677d2"),
-    "table_il": (25730048 + 0, "d163d414d08677d2"),
-    "table_hs_f16": (42769152 + 1724416, "d163d414d08677d2"),
-    "table_d72": (24805632 + 1024, "d163d414d08677d2"),
-    "ucpe": (263094016 + 204621056, "af3adacd4b1bec78"),
+    "video3d": (377567232 + 326036992, "789f04d7c18eb74c"),
+    "fp8neox": (1097157376 + 513794304, "789f04d7c18eb74c"),
+    "fp8neox_nonorm": (1097140480 + 516132352, "789f04d7c18eb74c"),
+    "gqa3d": (188861952 + 130926080, "789f04d7c18eb74c"),
+    "table_hs": (43556096 + 1905920, "e27ddf1ef866f0f6"),
+    "table_il": (25730304 + 0, "e27ddf1ef866f0f6"),
+    "table_hs_f16": (42768896 + 1988608, "e27ddf1ef866f0f6"),
+    "table_d72": (24805632 + 768, "e27ddf1ef866f0f6"),
+    "ucpe": (263099136 + 204933632, "f5ad21e8f37930cf"),
 }
 KERNEL_FILES = {"3d": ("rope3d.cu",), "table": ("rope_table.cu",),
                 "ucpe": ("ucpe_launch.h", "ucpe.cu")}

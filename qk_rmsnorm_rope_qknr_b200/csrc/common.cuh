@@ -290,6 +290,18 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
 
 __device__ __forceinline__ uint32_t f2_to_bf16x2(float2 v) { return pack_bf16x2(v.x, v.y); }
 
+// The products (x_lo * w_lo, x_hi * w_hi) of two bf16 pairs, exact in fp32
+// (mixed-precision FMAs with a -0 addend, which keeps the sign of a zero
+// product as a plain multiply does).
+__device__ __forceinline__ float2 mul_bf16x2(uint32_t x, uint32_t w) {
+    float2 r;
+    asm("{\n.reg .b16 xl, xh, wl, wh;\nmov.b32 {xl, xh}, %2;\nmov.b32 {wl, wh}, %3;\n"
+        "fma.rn.f32.bf16 %0, xl, wl, 0f80000000;\nfma.rn.f32.bf16 %1, xh, wh, 0f80000000;\n}"
+        : "=f"(r.x), "=f"(r.y)
+        : "r"(x), "r"(w));
+    return r;
+}
+
 // acc + (lo^2, hi^2) for the bf16 pair in w: two mixed-precision FMAs (bf16
 // inputs, fp32 accumulation, one rounding each), the same results as widening
 // first and one fp32x2 FMA.

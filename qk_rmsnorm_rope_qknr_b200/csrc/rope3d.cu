@@ -697,6 +697,11 @@ __global__ void __launch_bounds__(rr_max_threads<NS>(), 1) rope3d_rr_kernel(cons
     constexpr int HALF = D / 2;
     constexpr int OUTB = FP8 ? 1 : 2;
     constexpr int S = NS / 2;
+    // Weights in shared memory as stored (bf16, [head][D], multiplied with
+    // mixed-precision FMAs) for equal Q and K head counts; as fp32 pairs
+    // ([head][2][VPH] float4) for grouped-query heads, where the bf16 form
+    // measured slower.
+    constexpr bool BW = !MIXED;
 
     const int G = a.groups;
     const int Bg = blockDim.x / G;
@@ -704,11 +709,13 @@ __global__ void __launch_bounds__(rr_max_threads<NS>(), 1) rope3d_rr_kernel(cons
     const int stages = a.stages;
     const bool norm = a.is_qk_norm != 0;
     const bool supplied = a.mode == kModeSuppliedSsq;  // sums come from ssq_in
-    const MgLayout lay = mg_layout(D, G, stages, row_bytes, norm ? (a.hq + a.hk) * D : 0,
+    const MgLayout lay = mg_layout(D, G, stages, row_bytes,
+                                   norm ? (a.hq + a.hk) * D / (BW ? 2 : 1) : 0,
                                    a.use_table ? a.table_entries * 8 : 0);
     extern __shared__ __align__(128) unsigned char smem[];
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + lay.abort);
     float4* wsm = reinterpret_cast<float4*>(smem + lay.wts);
+    uint4* wsb = reinterpret_cast<uint4*>(smem + lay.wts);
     uint64_t* gq = reinterpret_cast<uint64_t*>(smem + lay.gq);
     float2* tab = reinterpret_cast<float2*>(smem + lay.tab);
 
@@ -749,7 +756,12 @@ __global__ void __launch_bounds__(rr_max_threads<NS>(), 1) rope3d_rr_kernel(cons
     setup_angles<D>(a, gq, tab);
     griddep_wait();
     griddep_launch_dependents();
-    if (norm) {
+    if (norm && BW) {  // Q heads, then K heads
+        const int nq16 = a.hq * VPH, n16 = (a.hq + a.hk) * VPH;
+        for (int q = tid; q < n16; q += blockDim.x)
+            wsb[q] = q < nq16 ? reinterpret_cast<const uint4*>(a.q_weight)[q]
+                              : reinterpret_cast<const uint4*>(a.k_weight)[q - nq16];
+    } else if (norm) {
         const int nq4 = a.hq * VPH * 2, n4 = (a.hq + a.hk) * VPH * 2;
         for (int q = tid; q < n4; q += blockDim.x) {
             const bool isk = q >= nq4;
@@ -771,7 +783,8 @@ __global__ void __launch_bounds__(rr_max_threads<NS>(), 1) rope3d_rr_kernel(cons
     const int nq = a.hq * L, nk = a.hk * L, nv = a.hv * VPH;
 
     // The thread's slots: the row vector of their first half (uint4 index in a
-    // row, -1 for none), their head's weights (float4 index in wsm), their
+    // row, -1 for none), their head's weights (uint4 index in wsb or float4
+    // index in wsm), their
     // byte offset in the output token row, and whether they are Q slots.
     int roff[NS], woff[NS], ooff[NS];
     bool isq[NS];
@@ -793,7 +806,7 @@ __global__ void __launch_bounds__(rr_max_threads<NS>(), 1) rope3d_rr_kernel(cons
         const int hg = q ? hh : a.hq + hh;
         isq[k] = q;
         roff[k] = valid ? hg * VPH + va : -1;
-        woff[k] = hg * 2 * VPH;
+        woff[k] = BW ? hg * VPH : hg * 2 * VPH;
         ooff[k] = hh * D * OUTB + (FP8 ? 8 : 16) * va;
     }
 
@@ -996,28 +1009,42 @@ __global__ void __launch_bounds__(rr_max_threads<NS>(), 1) rope3d_rr_kernel(cons
 #pragma unroll
             for (int k = 0; k < NS; ++k) {
                 if (roff[k] < 0 || isq[k] != (pass == 0)) continue;
-                const float2 xs[8] = {
-                    bf16x2_to_f2(px[k][0].x), bf16x2_to_f2(px[k][0].y), bf16x2_to_f2(px[k][0].z),
-                    bf16x2_to_f2(px[k][0].w), bf16x2_to_f2(px[k][1].x), bf16x2_to_f2(px[k][1].y),
-                    bf16x2_to_f2(px[k][1].z), bf16x2_to_f2(px[k][1].w)};
                 float2 ya[4], yb[4];
-                if (norm) {
-                    const float4* w = wsm + woff[k];
-                    const float4 a0 = w[va], a1 = w[VPH + va], b0 = w[va + dv],
-                                 b1 = w[VPH + va + dv];
-                    ya[0] = mul2(xs[0], make_float2(a0.x, a0.y));
-                    ya[1] = mul2(xs[1], make_float2(a0.z, a0.w));
-                    ya[2] = mul2(xs[2], make_float2(a1.x, a1.y));
-                    ya[3] = mul2(xs[3], make_float2(a1.z, a1.w));
-                    yb[0] = mul2(xs[4], make_float2(b0.x, b0.y));
-                    yb[1] = mul2(xs[5], make_float2(b0.z, b0.w));
-                    yb[2] = mul2(xs[6], make_float2(b1.x, b1.y));
-                    yb[3] = mul2(xs[7], make_float2(b1.z, b1.w));
-                } else {
+                if (norm && BW) {  // x * w, exact in fp32, from the bf16 pairs as loaded
+                    const uint32_t xa[4] = {px[k][0].x, px[k][0].y, px[k][0].z, px[k][0].w};
+                    const uint32_t xb[4] = {px[k][1].x, px[k][1].y, px[k][1].z, px[k][1].w};
+                    const uint4 wa = wsb[woff[k] + va], wb = wsb[woff[k] + va + dv];
+                    const uint32_t wa4[4] = {wa.x, wa.y, wa.z, wa.w};
+                    const uint32_t wb4[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
-                        ya[m] = xs[m];
-                        yb[m] = xs[4 + m];
+                        ya[m] = mul_bf16x2(xa[m], wa4[m]);
+                        yb[m] = mul_bf16x2(xb[m], wb4[m]);
+                    }
+                } else {
+                    const float2 xs[8] = {
+                        bf16x2_to_f2(px[k][0].x), bf16x2_to_f2(px[k][0].y),
+                        bf16x2_to_f2(px[k][0].z), bf16x2_to_f2(px[k][0].w),
+                        bf16x2_to_f2(px[k][1].x), bf16x2_to_f2(px[k][1].y),
+                        bf16x2_to_f2(px[k][1].z), bf16x2_to_f2(px[k][1].w)};
+                    if (norm) {
+                        const float4* w = wsm + woff[k];
+                        const float4 a0 = w[va], a1 = w[VPH + va], b0 = w[va + dv],
+                                     b1 = w[VPH + va + dv];
+                        ya[0] = mul2(xs[0], make_float2(a0.x, a0.y));
+                        ya[1] = mul2(xs[1], make_float2(a0.z, a0.w));
+                        ya[2] = mul2(xs[2], make_float2(a1.x, a1.y));
+                        ya[3] = mul2(xs[3], make_float2(a1.z, a1.w));
+                        yb[0] = mul2(xs[4], make_float2(b0.x, b0.y));
+                        yb[1] = mul2(xs[5], make_float2(b0.z, b0.w));
+                        yb[2] = mul2(xs[6], make_float2(b1.x, b1.y));
+                        yb[3] = mul2(xs[7], make_float2(b1.z, b1.w));
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            ya[m] = xs[m];
+                            yb[m] = xs[4 + m];
+                        }
                     }
                 }
                 float2 oa[4], ob[4];
@@ -1345,7 +1372,8 @@ cudaError_t run_rr(const Rope3DArgs& a, cudaStream_t stream, LaunchInfo* info) {
     args.use_table = table_pays(a, D / 2) ? 1 : 0;
     const int used_table = args.use_table ? table_bytes : 0;
     const int row_bytes = (a.hq + a.hk + a.hv) * D * 2;
-    const int weight_floats = a.is_qk_norm ? (a.hq + a.hk) * D : 0;
+    const bool bw = !mixed;  // the kernel's BW: bf16 weights in shared memory
+    const int weight_floats = a.is_qk_norm ? (a.hq + a.hk) * D / (bw ? 2 : 1) : 0;
     if (args.norm_q_elems == 0) args.norm_q_elems = a.hq * D;
     if (args.norm_k_elems == 0) args.norm_k_elems = a.hk * D;
     int groups = std::min(kMaxGroups, max_threads / bg);
