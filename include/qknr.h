@@ -258,7 +258,8 @@ int qknr_rope_3d_with_ssq(const qknr_rope_3d_params* params, const float* ssq,
  * pipelined kernel (any num_tokens); else, with at least two heads,
  * head_dim <= 128 and an even num_tokens, a barrier-synchronised pipelined
  * kernel; else a general one, which writes two bytes at a time when
- * num_tokens is not a multiple of 8.
+ * num_tokens is not a multiple of 8 and, when there are enough 64-token tiles
+ * to fill the GPU, takes whole tiles with all their heads per CTA.
  * Range: every kernel applies k_scale to K's rotated result (the projection
  * and the rotation are linear) and take the two fp32 sums of squares over the
  * unscaled ReLU key, so the scale itself never underflows or overflows them.

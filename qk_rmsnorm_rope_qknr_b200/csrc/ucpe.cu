@@ -17,9 +17,12 @@
 // at least two heads; ucpe_sync_kernel (barrier-synchronised) for the other
 // head_dims up to 128 with an even token count and at least two heads; and
 // ucpe_prep_kernel for every other shape. The general kernel:
-//   - work unit: a tile of 64 consecutive tokens of one (batch, head), tiles
-//     numbered with the head fastest, so that the tiles in flight at once
-//     share their tokens' cos/sin rows and matrices in L2;
+//   - work unit: a tile of 64 consecutive tokens of one (batch, head), units
+//     numbered with the head fastest, so that the units in flight at once
+//     share their tokens' cos/sin rows and matrices in L2; or, when there are
+//     enough tiles to give every CTA whole tiles (TILE_MAJOR), a tile with
+//     all its heads in turn, its matrices and cos/sin rows staged once
+//     (56.6 against 48.5% of HBM at head_dim 256, 8 heads);
 //   - a thread takes four tokens of one 8-channel chunk (two projection
 //     blocks, four rotation pairs). Consecutive threads read consecutive
 //     16-byte chunks of a token's row, so each warp load covers whole rows;
@@ -268,12 +271,15 @@ struct TileCursor {
     }
 };
 
-template <bool H16>
+template <bool H16, bool TILE_MAJOR>
 __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
     const int D = a.head_dim, C = D / 8, H = a.heads;
     const int64_t N = a.num_tokens;
     const int64_t tiles_n = (N + kTile - 1) / kTile;
-    const int64_t ntiles = a.batch * tiles_n * H;
+    // TILE_MAJOR: a CTA takes whole tiles and their heads in turn, staging the
+    // tile's matrices and cos/sin rows once; otherwise single (tile, head)
+    // units, the head fastest.
+    const int64_t nunits = a.batch * tiles_n * (TILE_MAJOR ? 1 : H);
     const int tid = threadIdx.x, nthr = blockDim.x;
     const bool vec_out = (N & 7) == 0;
 
@@ -288,13 +294,20 @@ __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
     const int p = tid / C, c = tid - (tid / C) * C;
     const bool has_item = tid < (kTile / 4) * C;
 
-    int64_t tile = blockIdx.x;
-    if (tile >= ntiles) return;
-    const int64_t step_bt = (int64_t)gridDim.x / H;
-    const int step_h = (int)((int64_t)gridDim.x - step_bt * H);
+    int64_t unit = blockIdx.x;
+    if (unit >= nunits) return;
     TileCursor cur;
-    cur.h = (int)(tile % H);
-    cur.tn = tile / H;
+    int64_t step_bt = 0;
+    int step_h = 0;
+    if constexpr (TILE_MAJOR) {
+        cur.h = 0;
+        cur.tn = unit;
+    } else {
+        step_bt = (int64_t)gridDim.x / H;
+        step_h = (int)((int64_t)gridDim.x - step_bt * H);
+        cur.h = (int)(unit % H);
+        cur.tn = unit / H;
+    }
     cur.b = cur.tn / tiles_n;
     cur.tn -= cur.b * tiles_n;
 
@@ -329,14 +342,31 @@ __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
         }
         __syncthreads();
 
-        // The next tile's inputs go out before this tile's stores.
-        tile += gridDim.x;
-        const bool more = tile < ntiles;
+        // The next unit's inputs go out before this one's stores; the tile's
+        // matrices and cos/sin rows only when the tile changes.
+        bool more, new_tile = true;
+        if constexpr (TILE_MAJOR) {
+            if (cur.h + 1 < H) {
+                ++cur.h;
+                more = true;
+                new_tile = false;
+            } else {
+                unit += gridDim.x;
+                more = unit < nunits;
+                if (more) {
+                    cur.h = 0;
+                    cur.advance(gridDim.x, 0, 1, tiles_n);
+                }
+            }
+        } else {
+            unit += gridDim.x;
+            more = unit < nunits;
+            if (more) cur.advance(step_bt, step_h, H, tiles_n);
+        }
         if (more) {
-            cur.advance(step_bt, step_h, H, tiles_n);
             const int64_t nn0 = cur.tn * kTile;
             const int ntv = (int)min((int64_t)kTile, N - nn0);
-            stage_token_inputs(a, cur.b, nn0, ntv, tid, nthr, proj, cosr, sinr);
+            if (new_tile) stage_token_inputs(a, cur.b, nn0, ntv, tid, nthr, proj, cosr, sinr);
             if (has_item) load_item(a, cur.b, nn0, cur.h, ntv, p, c, raw);
         }
 
@@ -387,34 +417,34 @@ __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
 // Work unit: a step is one head of a tile of 64 tokens of one batch element;
 // a CTA takes its tiles in turn and each tile's heads in order. The CTA is D/8
 // compute warps and one copy warp:
-//   - the copy warp brings each step's Q, K and V rows (64 tokens x D, three
-//     tensors) into a stage of a shared-memory ring with 16-byte cp.async
-//     copies, each lane arriving on the stage's "full" mbarrier once its
-//     copies have landed, STAGES - 1 steps ahead. (A bulk copy per 2D-byte
-//     row measured 2.6x slower: the copy engine took about 27 such small
+//   - the copy warp's lane 0 brings each step's Q, K and V rows (64 tokens,
+//     fast_row_elems(D) channels from the head's first) into a stage of a
+//     shared-memory ring with one 2D tensor copy per tensor, counted in bytes
+//     on the stage's "full" mbarrier, STAGES - 1 steps ahead. (One bulk copy
+//     per row measured 2.6x slower: the copy engine took about 27 such small
 //     copies per microsecond per SM, below what 192 rows per step need.)
-//     Before refilling a stage it
-//     waits on the stage's "empty" mbarrier, which every compute thread
-//     arrives on once it has read the stage. At a tile's first step it also
-//     writes the tile's two 4x4 matrices into shared memory, interleaved by
-//     token pair (double-buffered per tile, with their own full/empty
-//     mbarriers), and it adds up the key sums of finished steps and writes
-//     inflation_sq;
-//   - lane i of compute warp w owns the token pair (2i, 2i+1) and the
-//     8-channel chunk w. Per step it widens, projects, rotates and rounds its
-//     two tokens x eight channels of each tensor with packed fp32x2
+//     Before refilling a stage it waits on the stage's "empty" mbarrier, which
+//     every compute thread arrives on once it has read the stage. At a tile's
+//     first step it also writes the tile's two 4x4 matrices into shared
+//     memory, interleaved by the token pairs the compute lanes own
+//     (double-buffered per tile, with their own full/empty mbarriers), and it
+//     adds up the key sums of finished steps and writes inflation_sq;
+//   - lane i of compute warp w owns the tokens i and i + 32 of the tile and
+//     the 8-channel chunk w. Per step it widens, projects, rotates and rounds
+//     its two tokens x eight channels of each tensor with packed fp32x2
 //     instructions (the tile's cos/sin values sit in registers for all its
-//     heads) and stores one 32-bit word (both tokens) per channel straight to
-//     [B, H, D, N]: the 32 lanes of a warp write one whole 128-byte row. Its
-//     key sums go to a double-buffered shared array for the copy warp.
+//     heads) and stores 16-bit values straight to [B, H, D, N]: the 32 lanes
+//     of a warp write the two 64-byte halves of a 128-byte output row, so any
+//     token count works. Its key sums go to a double-buffered shared array for
+//     the copy warp.
 // No CTA-wide barrier: compute warps wait only for their data, so a slow warp
 // delays the others only when the ring runs dry. Every wait is bounded in
 // time; on expiry the waiter raises the CTA's abort flag and bit 0 of the
 // device status word, every other wait gives up at the flag, and the copy
 // warp waits for its own copies (which always land) before the CTA ends.
-// Padding: a token pair's two rows take 2D*2 + 16 bytes of a stage, so that
-// the 16-byte chunks that eight consecutive lanes read fall in distinct banks;
-// a pair's interleaved matrices take 144 bytes for the same reason.
+// Padding: a stage row is an odd number of 16-byte chunks (fast_row_elems),
+// so that the chunk c of eight consecutive rows falls in distinct bank groups;
+// a token pair's interleaved matrices take 144 bytes for the same reason.
 constexpr int kFastMaxD = 128;  // the barrier-synchronised kernel's limit
 constexpr int kWsMaxD = 120;    // the warp-specialised kernel's (16 warps of 32 threads)
 constexpr int kMatStride = 36;  // floats per token pair per matrix (32 used)
@@ -1297,14 +1327,29 @@ cudaError_t launch_ucpe(const UcpeArgs& a, const UcpeControl& ctl, cudaStream_t 
         }
     }
     const int block = ucpe_block(D), smem = ucpe_smem(D);
-    void (*kern)(const UcpeArgs) = a.act_f16 ? ucpe_prep_kernel<true> : ucpe_prep_kernel<false>;
+    void (*kern)(const UcpeArgs) =
+        a.act_f16 ? ucpe_prep_kernel<true, false> : ucpe_prep_kernel<false, false>;
     int sms = 0, per_sm = 0;
     cudaError_t e = cached_sm_count(&sms);
     if (e != cudaSuccess) return e;
     e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), block, smem, &per_sm);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const int64_t tiles = a.batch * ((a.num_tokens + kTile - 1) / kTile) * a.heads;
+    // Whole tiles per CTA (the tile's matrices and cos/sin rows staged once
+    // for all its heads) unless that leaves the last round of tiles so uneven
+    // that it takes over a quarter more (tile, head) rounds than single units.
+    const int64_t slots = (int64_t)sms * per_sm;
+    const int64_t tiles_bt = a.batch * ((a.num_tokens + kTile - 1) / kTile);
+    const int64_t rounds_tile = (tiles_bt + slots - 1) / slots * a.heads;
+    const int64_t rounds_unit = (tiles_bt * a.heads + slots - 1) / slots;
+    const bool tile_major = a.heads > 1 && 4 * rounds_tile <= 5 * rounds_unit;
+    if (tile_major) {
+        kern = a.act_f16 ? ucpe_prep_kernel<true, true> : ucpe_prep_kernel<false, true>;
+        e = cached_smem_and_occupancy(reinterpret_cast<const void*>(kern), block, smem, &per_sm);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    }
+    const int64_t tiles = tiles_bt * (tile_major ? 1 : a.heads);
     const int grid = (int)std::min<int64_t>((int64_t)sms * per_sm, tiles);
     e = launch_pdl(kern, grid, block, smem, stream, a);
     if (e != cudaSuccess) {
@@ -1317,7 +1362,7 @@ cudaError_t launch_ucpe(const UcpeArgs& a, const UcpeControl& ctl, cudaStream_t 
         info->grid = grid;
         info->block = block;
         info->smem = smem;
-        info->kernel_id = 5000 + (a.act_f16 ? 1 : 0);
+        info->kernel_id = 5000 + (a.act_f16 ? 1 : 0) + (tile_major ? 2 : 0);
     }
     return e;
 }

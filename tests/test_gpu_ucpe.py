@@ -89,6 +89,11 @@ CASES = [
     (1, 129, 2, 256, "bf16"),
     (1, 151, 3, 112, "f16"),
     (2, 65, 2, 40, "f16"),
+    # The general kernel with whole tiles per CTA (enough tiles to fill every
+    # SM): a tile's heads in turn over one staging of its matrices and cos/sin
+    (1, 18480, 2, 136, "bf16"),
+    (2, 9300, 2, 256, "f16"),
+    (1, 18481, 3, 192, "bf16"),
 ]
 
 
