@@ -217,6 +217,32 @@ def run_host_sweep(args):
         rows[form] = [host_cost(form, t) for t in (64, 128, 256, 512, 1024, 2048, 4096, 8192)]
     cross = {f: next((r["tokens"] for r in v if r["device_us_per_call"] >= r["host_us_per_call"]),
                      None) for f, v in rows.items()}
+    # The same 3D calls through the Python binding: the wrapper and a prepared call.
+    import torch
+
+    import qk_rmsnorm_rope_qknr_b200 as Q
+    import workloads as W
+
+    w = W.WORKLOADS["fp8neox"]
+    prm = dict(w.params(), pos_offset=0)
+    prepared = Q.Rope3DCall(**prm)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    row = (w.hq + w.hk + w.hv) * w.head_dim
+    for r in rows["3d"]:
+        T = r["tokens"]
+        qkv = torch.zeros(T, row, dtype=torch.bfloat16, device="cuda")
+        qw = torch.ones(w.hq * w.head_dim, dtype=torch.bfloat16, device="cuda")
+        kw = torch.ones(w.hk * w.head_dim, dtype=torch.bfloat16, device="cuda")
+        outs = [torch.empty(T, h, w.head_dim, dtype=torch.float8_e4m3fn, device="cuda")
+                for h in (w.hq, w.hk, w.hv)]
+        r["python_wrapper_us_per_call"] = python_call_us(
+            lambda: Q.qknr_rope_3d(qkv, qw, kw, *outs, stream=stream, **prm))
+        r["python_prepared_us_per_call"] = python_call_us(
+            lambda: prepared(qkv, qw, kw, *outs, stream=sh))
+    for key in ("python_wrapper_us_per_call", "python_prepared_us_per_call"):
+        cross["3d_" + key.replace("_us_per_call", "")] = next(
+            (r["tokens"] for r in rows["3d"] if r["device_us_per_call"] >= r[key]), None)
     print(json.dumps({"host_sweep": rows, "crossover_tokens": cross,
                       "shapes": {"3d": "24+24+24 heads of 128, E4M3 out (fp8neox per token)",
                                  "table": "32+8 heads of 128, rotary_dim 96, fp32 table "
@@ -477,7 +503,11 @@ def run_gpu(args, w):
     if rank == 0 and world == 1 and not args.no_e2e:
         # host cost of one call: through the Python binding (argument checks
         # and ctypes) and from C through the ABI, with the launch
-        host_us = {"python_binding": python_call_us(lambda: step(0))}
+        prepared = Q.Rope3DCall(**p)
+        sh = stream.cuda_stream
+        host_us = {"python_binding": python_call_us(lambda: step(0)),
+                   "python_prepared": python_call_us(
+                       lambda: prepared(qkv, qw, kw, *outs, stream=sh))}
         if not getattr(args, "tokens", None) and w.name == "fp8neox":
             hc = host_cost("3d", T)
             host_us.update({"c_abi": hc["host_us_per_call"],

@@ -9,6 +9,7 @@ Low-level names mirror the C entry points:
   qknr_rope_table(...)     table-driven per-head form
   qknr_rope_3d(...)        packed-QKV across-heads 3D form
   qknr_ucpe_cam_prep(...)  UCPE camera prep (ReLU, K scale, ray projection, RoPE)
+  Rope3DCall(**params)     qknr_rope_3d prepared once, for repeated small calls
 Page-shaped wrappers allocate missing outputs and return them:
   fused_qk_norm_rope(q, k, q_weight, k_weight, rope_table, eps, *, head_dim=None,
                      rotary_dim=None, interleaved=False) -> (q, k)
@@ -259,6 +260,58 @@ def qknr_rope_3d(qkv, q_weight, k_weight, q_out, k_out, v_out, *, stream=None, *
     _check(lib().qknr_rope_3d(C.byref(p), st))
 
 
+class Rope3DCall:
+    """A 3D-form call prepared once for repeated use: the page's keyword
+    arguments (as for qknr_rope_3d) are fixed here and the C parameter block is
+    built once. Each call checks only what changes between calls (the tensors'
+    dtype, density and element counts, which the kernel trusts), fills in the
+    six pointers and the token count, and launches: about a third of
+    qknr_rope_3d's Python cost. Pass the stream (a torch stream or its handle)
+    to skip the current-stream lookup. One instance is not for concurrent use
+    from several threads (the parameter block is reused)."""
+
+    def __init__(self, **params):
+        self._p = make_3d_params(None, None, None, None, None, None, num_tokens=0, **params)
+        p = self._p
+        self._row = (p.num_heads_q + p.num_heads_k + p.num_heads_v) * p.head_dim
+        self._sizes = (p.num_heads_q * p.head_dim, p.num_heads_k * p.head_dim,
+                       p.num_heads_v * p.head_dim)
+        self._odt = torch.float8_e4m3fn if p.output_fp8 else torch.bfloat16
+        self._norm = bool(p.is_qk_norm)
+        self._fn = lib().qknr_rope_3d
+        self._byref = C.byref(p)
+
+    def __call__(self, qkv, q_weight, k_weight, q_out, k_out, v_out, stream=None) -> None:
+        p = self._p
+        n = qkv.numel()
+        if qkv.dtype is not torch.bfloat16 or n % self._row or not qkv.is_contiguous():
+            raise QknrValueError(QKNR_ERR_SHAPE,
+                                 f"qkv must be a contiguous bf16 tensor [..., {self._row}]")
+        T = n // self._row
+        odt = self._odt
+        for o, sz in ((q_out, self._sizes[0]), (k_out, self._sizes[1]), (v_out, self._sizes[2])):
+            if sz and (o is None or o.numel() != T * sz or
+                       (o.dtype is not odt and o.dtype is not torch.uint8) or
+                       not o.is_contiguous()):
+                raise QknrValueError(QKNR_ERR_SHAPE,
+                                     f"outputs must be dense {odt} tensors of {T} tokens")
+        if self._norm:
+            for w, sz in ((q_weight, self._sizes[0]), (k_weight, self._sizes[1])):
+                if sz and (w is None or w.numel() != sz or w.dtype is not torch.bfloat16):
+                    raise QknrValueError(QKNR_ERR_SHAPE, f"weights must be bf16 [{sz}]")
+        p.qkv = qkv.data_ptr()
+        p.q_weight, p.k_weight = _ptr(q_weight), _ptr(k_weight)
+        p.q_out, p.k_out, p.v_out = _ptr(q_out), _ptr(k_out), _ptr(v_out)
+        p.num_tokens = T
+        if stream is None:
+            st = torch.cuda.current_stream(qkv.device).cuda_stream
+        else:
+            st = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        status = self._fn(self._byref, st)
+        if status:
+            _check(status)
+
+
 def qknr_rope_3d_partial_ssq(qkv, ssq_out, *, stream=None, **params) -> None:
     """Tensor-parallel pass 1 through the C ABI: per-token sums of x^2 over this
     call's Q and K heads into ssq_out (fp32 [tokens, 2])."""
@@ -407,4 +460,5 @@ __all__ = ["qknr_rope_table", "qknr_rope_3d", "qknr_rope_3d_partial_ssq", "qknr_
            "qknr_ucpe_cam_prep", "cam_prep_func",
            "qknr_device_status", "fused_qk_norm_rope", "fused_qk_rmsnorm_rope",
            "QknrError", "QknrValueError", "lib", "build", "make_3d_params", "Rope3DParams",
+           "Rope3DCall",
            "EXPORTS", "LIB_PATH"]

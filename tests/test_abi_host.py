@@ -202,6 +202,39 @@ def test_python_wrapper_raises_valueerror(L):
         Q.fused_qk_norm_rope(x.half(), x.half(), w.half(), w.half(), tbl.bfloat16(), 1e-6)
 
 
+
+def test_prepared_3d_call_checks_tensors_before_the_library(L):
+    """Rope3DCall checks what changes per call (dtype, density, element counts)
+    in Python and raises ValueError before any pointer reaches the library."""
+    import torch
+
+    p = dict(ppf=1, pph=2, ppw=3, num_frame_channels=16, num_height_channels=24,
+             num_width_channels=24, num_heads_q=2, num_heads_k=1, num_heads_v=1, head_dim=64,
+             interleave=False, output_fp8=True, pos_offset=0)
+    call = Q.Rope3DCall(**p)
+    T, row = 6, 4 * 64
+    qkv = torch.zeros(T, row, dtype=torch.bfloat16)
+    qw = torch.zeros(2 * 64, dtype=torch.bfloat16)
+    kw = torch.zeros(64, dtype=torch.bfloat16)
+    f8 = torch.float8_e4m3fn
+    outs = [torch.zeros(T, h, 64, dtype=f8) for h in (2, 1, 1)]
+    bad_cases = [
+        (qkv.float(), qw, kw, *outs),                                        # qkv dtype
+        (qkv[:, :-8].contiguous(), qw, kw, *outs),                           # not whole rows
+        (qkv.t().contiguous().t(), qw, kw, *outs),                           # not dense
+        (qkv, qw, kw, torch.zeros(T, 2, 64, dtype=torch.bfloat16), *outs[1:]),  # bf16 out, FP8 call
+        (qkv, qw, kw, outs[0][:-1], *outs[1:]),                              # too few tokens
+        (qkv, qw, kw, outs[0], outs[1], None),                               # missing output
+        (qkv, qw.float(), kw, *outs),                                        # weight dtype
+        (qkv, qw, kw[:-1], *outs),                                           # weight size
+        (qkv, None, kw, *outs),                                              # missing weight
+    ]
+    for args in bad_cases:
+        with pytest.raises(ValueError):
+            call(*args, stream=0)
+    with pytest.raises(ValueError):                       # a bad static parameter
+        Q.Rope3DCall(**dict(p, num_heads_q=-1))(qkv, qw, kw, *outs, stream=0)
+
 def test_wait_fault_hook_argument_checks(L):
     assert L.qknr_test_set_wait_fault(8, 1000) == Q.QKNR_ERR_SHAPE
     assert L.qknr_test_set_wait_fault(16, 0) == Q.QKNR_ERR_SHAPE

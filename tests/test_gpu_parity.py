@@ -344,6 +344,32 @@ def test_3d_deterministic_and_streams():
         assert torch.equal(x, y)
 
 
+
+@pytest.mark.parametrize("case", [CASES_3D[1], CASES_3D[6], CASES_3D[13]], ids=["neox_e4m3", "slots2", "gqa"])
+def test_3d_prepared_call_matches_wrapper(case):
+    """Rope3DCall (parameters fixed once) gives the wrapper's bytes, for a whole
+    call and for shards of other token counts through the same instance."""
+    T, Hq, Hk, Hv, D, grid, ch, il, fp8, norm, off = case
+    qkv, qw, kw = _rand3d(T, Hq, Hk, Hv, D, std=2.0, seed=T + D + 1)
+    p = dict(ppf=grid[0], pph=grid[1], ppw=grid[2], num_frame_channels=ch[0],
+             num_height_channels=ch[1], num_width_channels=ch[2], num_heads_q=Hq, num_heads_k=Hk,
+             num_heads_v=Hv, head_dim=D, eps=1e-5, base=10000.0, interleave=il, is_qk_norm=norm,
+             output_fp8=fp8, output_quant_scale=0.75, v_quant_scale=1.5, pos_offset=off)
+    call = Q.Rope3DCall(**p)
+    odt = torch.float8_e4m3fn if fp8 else torch.bfloat16
+    s = torch.cuda.Stream()
+    for t in (T, max(1, T // 3), 1):
+        ref = run_3d(qkv[:t], qw, kw, **p)
+        got = [torch.empty((t, h, D), dtype=odt, device=DEV) for h in (Hq, Hk, Hv)]
+        for g in got:
+            g.view(torch.uint8).fill_(7)
+        call(qkv[:t], qw, kw, *got, stream=s)
+        s.synchronize()
+        for x, y in zip(ref, got):
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8)), t
+    with pytest.raises(Q.QknrValueError):
+        call(qkv[:, :-1].contiguous(), qw, kw, *got, stream=s)
+
 def test_3d_batch_shape():
     w = W.WORKLOADS["tiny3d"]
     qkv, qw, kw = _rand3d(64, 4, 4, 4, 64)
