@@ -670,9 +670,11 @@ __global__ void __launch_bounds__(768, 1) rope3d_mg_kernel(const Rope3DArgs a) {
 
 // ---------------------------------------------------------------------------
 // Register-resident pipelined kernel: as rope3d_mg_kernel (G token pipelines
-// per CTA, bulk-copy rings, shared angle table and fp32 weights), but each
-// thread keeps its NS slots in registers, as loaded (bf16 pairs), from the
-// sums of squares (mixed-precision FMAs on the pairs) to the stores. A token
+// per CTA, bulk-copy rings, shared angle table), but each thread keeps its NS
+// slots in registers, as loaded (bf16 pairs), from the sums of squares
+// (mixed-precision FMAs on the pairs) to the stores. With equal Q and K head
+// counts the weights stay bf16 in shared memory and x * w is a mixed-precision
+// product too; with grouped-query heads they are widened to fp32 once. A token
 // therefore needs NS/2 times fewer threads, every slot is read from shared
 // memory once and widened once, and the token's own ring buffer is free at
 // the token's barrier: it is refilled there, one and a half tokens of copy
