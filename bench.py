@@ -240,9 +240,23 @@ def run_host_sweep(args):
             lambda: Q.qknr_rope_3d(qkv, qw, kw, *outs, stream=stream, **prm))
         r["python_prepared_us_per_call"] = python_call_us(
             lambda: prepared(qkv, qw, kw, *outs, stream=sh))
-    for key in ("python_wrapper_us_per_call", "python_prepared_us_per_call"):
-        cross["3d_" + key.replace("_us_per_call", "")] = next(
-            (r["tokens"] for r in rows["3d"] if r["device_us_per_call"] >= r[key]), None)
+    tcall = Q.RopeTableCall(heads_q=32, heads_k=8, head_dim=128, eps=1e-6, rotary_dim=96)
+    for r in rows["table"]:
+        T = r["tokens"]
+        q = torch.zeros(T, 32, 128, dtype=torch.bfloat16, device="cuda")
+        k = torch.zeros(T, 8, 128, dtype=torch.bfloat16, device="cuda")
+        qo, ko = torch.empty_like(q), torch.empty_like(k)
+        wt = torch.ones(128, dtype=torch.bfloat16, device="cuda")
+        tbl = torch.zeros(T, 96, dtype=torch.float32, device="cuda")
+        r["python_wrapper_us_per_call"] = python_call_us(
+            lambda: Q.qknr_rope_table(q, k, qo, ko, wt, wt, tbl, eps=1e-6, rotary_dim=96,
+                                      stream=stream))
+        r["python_prepared_us_per_call"] = python_call_us(
+            lambda: tcall(q, k, qo, ko, wt, wt, tbl, stream=sh))
+    for form in ("3d", "table"):
+        for key in ("python_wrapper_us_per_call", "python_prepared_us_per_call"):
+            cross[form + "_" + key.replace("_us_per_call", "")] = next(
+                (r["tokens"] for r in rows[form] if r["device_us_per_call"] >= r[key]), None)
     print(json.dumps({"host_sweep": rows, "crossover_tokens": cross,
                       "shapes": {"3d": "24+24+24 heads of 128, E4M3 out (fp8neox per token)",
                                  "table": "32+8 heads of 128, rotary_dim 96, fp32 table "

@@ -10,6 +10,7 @@ Low-level names mirror the C entry points:
   qknr_rope_3d(...)        packed-QKV across-heads 3D form
   qknr_ucpe_cam_prep(...)  UCPE camera prep (ReLU, K scale, ray projection, RoPE)
   Rope3DCall(**params)     qknr_rope_3d prepared once, for repeated small calls
+  RopeTableCall(...)       qknr_rope_table prepared once, likewise
 Page-shaped wrappers allocate missing outputs and return them:
   fused_qk_norm_rope(q, k, q_weight, k_weight, rope_table, eps, *, head_dim=None,
                      rotary_dim=None, interleaved=False) -> (q, k)
@@ -199,6 +200,64 @@ def qknr_rope_table(q, k, q_out, k_out, q_weight, k_weight, rope_table, *, eps: 
                                  _table_dtype(rope_table, q.dtype), act, T, Hq,
                                  Hk, D, R, qs, ks, qos, kos, float(eps), int(bool(interleaved)),
                                  st))
+
+
+class RopeTableCall:
+    """The table form prepared once for repeated use: head counts, head_dim,
+    rotary_dim, eps, the pair layout and the dtypes are fixed here. Each call
+    checks the tensors' shapes, dtypes and head density, takes their token
+    strides and launches (about two thirds of qknr_rope_table's Python cost). Pass
+    the stream (a torch stream or its handle) to skip the current-stream
+    lookup."""
+
+    def __init__(self, *, heads_q: int, heads_k: int, head_dim: int, eps: float,
+                 rotary_dim: int = 0, interleaved: bool = False,
+                 act_dtype: torch.dtype = torch.bfloat16,
+                 table_dtype: torch.dtype = torch.float32):
+        if act_dtype not in _ACT_DTYPES:
+            raise QknrValueError(QKNR_ERR_SHAPE, f"act_dtype {act_dtype} is not bfloat16/float16")
+        self._tcode = _table_dtype(torch.empty(0, dtype=table_dtype), act_dtype)
+        self._acode = _ACT_DTYPES[act_dtype]
+        self._act, self._tdt = act_dtype, table_dtype
+        self._hq, self._hk, self._d = int(heads_q), int(heads_k), int(head_dim)
+        self._r = int(rotary_dim) or self._d
+        self._eps, self._il = float(eps), int(bool(interleaved))
+        self._fn = lib().qknr_rope_table
+
+    def _stride(self, t, heads, T):
+        sh = t.shape
+        if len(sh) != 3 or sh[0] != T or sh[1] != heads or sh[2] != self._d or \
+                t.dtype is not self._act:
+            raise QknrValueError(QKNR_ERR_SHAPE,
+                                 f"expected {self._act} [{T}, {heads}, {self._d}] tensors")
+        st = t.stride()
+        if T > 0 and heads > 0 and (st[2] != 1 or (heads > 1 and st[1] != self._d)):
+            raise QknrValueError(QKNR_ERR_SHAPE, "heads must be dense inside a token")
+        return st[0]
+
+    def __call__(self, q, k, q_out, k_out, q_weight, k_weight, rope_table, stream=None) -> None:
+        T = q.shape[0] if q.dim() == 3 else -1
+        qs = self._stride(q, self._hq, T)
+        ks = self._stride(k, self._hk, T)
+        qos = self._stride(q_out, self._hq, T)
+        kos = self._stride(k_out, self._hk, T)
+        if rope_table.dtype is not self._tdt or tuple(rope_table.shape) != (T, self._r) or \
+                not rope_table.is_contiguous():
+            raise QknrValueError(QKNR_ERR_SHAPE,
+                                 f"rope_table must be a dense {self._tdt} [{T}, {self._r}]")
+        for w in (q_weight, k_weight):
+            if w.dtype is not self._act or w.numel() != self._d or not w.is_contiguous():
+                raise QknrValueError(QKNR_ERR_SHAPE, f"weights must be dense {self._act} [{self._d}]")
+        if stream is None:
+            st = torch.cuda.current_stream(q.device).cuda_stream
+        else:
+            st = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        status = self._fn(q.data_ptr(), k.data_ptr(), q_out.data_ptr(), k_out.data_ptr(),
+                          q_weight.data_ptr(), k_weight.data_ptr(), rope_table.data_ptr(),
+                          self._tcode, self._acode, T, self._hq, self._hk, self._d, self._r, qs,
+                          ks, qos, kos, self._eps, self._il, st)
+        if status:
+            _check(status)
 
 
 def make_3d_params(qkv, q_weight, k_weight, q_out, k_out, v_out, *, ppf, pph, ppw,
@@ -460,5 +519,5 @@ __all__ = ["qknr_rope_table", "qknr_rope_3d", "qknr_rope_3d_partial_ssq", "qknr_
            "qknr_ucpe_cam_prep", "cam_prep_func",
            "qknr_device_status", "fused_qk_norm_rope", "fused_qk_rmsnorm_rope",
            "QknrError", "QknrValueError", "lib", "build", "make_3d_params", "Rope3DParams",
-           "Rope3DCall",
+           "Rope3DCall", "RopeTableCall",
            "EXPORTS", "LIB_PATH"]

@@ -235,6 +235,34 @@ def test_prepared_3d_call_checks_tensors_before_the_library(L):
     with pytest.raises(ValueError):                       # a bad static parameter
         Q.Rope3DCall(**dict(p, num_heads_q=-1))(qkv, qw, kw, *outs, stream=0)
 
+
+def test_prepared_table_call_checks_tensors_before_the_library(L):
+    """RopeTableCall raises ValueError on a wrong shape, dtype, head layout,
+    table or weight before any pointer reaches the library."""
+    import torch
+
+    call = Q.RopeTableCall(heads_q=3, heads_k=2, head_dim=64, eps=1e-6, rotary_dim=48)
+    T = 5
+    q = torch.zeros(T, 3, 64, dtype=torch.bfloat16)
+    k = torch.zeros(T, 2, 64, dtype=torch.bfloat16)
+    w = torch.zeros(64, dtype=torch.bfloat16)
+    tbl = torch.zeros(T, 48)
+    bad_cases = [
+        (q.half(), k, q, k, w, w, tbl),                          # activation dtype
+        (q, k[:-1], q, k, w, w, tbl),                            # token counts differ
+        (q, k, q[:, :2], k, w, w, tbl),                          # head count
+        (q.transpose(1, 2).contiguous().transpose(1, 2), k, q, k, w, w, tbl),  # heads not dense
+        (q, k, q, k, w, w, tbl[:, :46]),                         # table width
+        (q, k, q, k, w, w, tbl.bfloat16()),                      # table dtype
+        (q, k, q, k, w[:-1], w, tbl),                            # weight size
+        (q, k, q, k, w, w.float(), tbl),                         # weight dtype
+    ]
+    for args in bad_cases:
+        with pytest.raises(ValueError):
+            call(*args, stream=0)
+    with pytest.raises(ValueError):                       # table dtype not f32 / activation
+        Q.RopeTableCall(heads_q=3, heads_k=2, head_dim=64, eps=1e-6, table_dtype=torch.float16)
+
 def test_wait_fault_hook_argument_checks(L):
     assert L.qknr_test_set_wait_fault(8, 1000) == Q.QKNR_ERR_SHAPE
     assert L.qknr_test_set_wait_fault(16, 0) == Q.QKNR_ERR_SHAPE

@@ -422,6 +422,27 @@ def test_table_variants(case):
     check_table_against_oracle(inp, qo.cpu(), ko.cpu(), 1e-5, R, il, str(case))
 
 
+@pytest.mark.parametrize("case", [CASES_TABLE[0], CASES_TABLE[1], CASES_TABLE[6], CASES_TABLE[11]],
+                         ids=["fast_hs", "fast_il", "general", "smem_no_q"])
+def test_table_prepared_call_matches_wrapper(case):
+    """RopeTableCall gives the wrapper's bytes, on dense tensors and on Q/K
+    views of one fused [T, Hq + Hk, D] tensor (token stride above the row)."""
+    T, Hq, Hk, D, R, f32, il = case
+    inp = _rand_table_inputs(T, Hq, Hk, D, R, f32, seed=D + R + 2, std=2.0)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    call = Q.RopeTableCall(heads_q=Hq, heads_k=Hk, head_dim=D, eps=1e-5, rotary_dim=R,
+                           interleaved=il, table_dtype=g["rope_table"].dtype)
+    fused = torch.cat([g["q"], g["k"]], dim=1)
+    fused_out = torch.empty_like(fused)
+    for q, k, qo, ko in ((g["q"], g["k"], torch.empty_like(g["q"]), torch.empty_like(g["k"])),
+                         (fused[:, :Hq], fused[:, Hq:], fused_out[:, :Hq], fused_out[:, Hq:])):
+        rq, rk = Q.fused_qk_norm_rope(q, k, g["q_weight"], g["k_weight"], g["rope_table"], 1e-5,
+                                      rotary_dim=R, interleaved=il)
+        call(q, k, qo, ko, g["q_weight"], g["k_weight"], g["rope_table"])
+        torch.cuda.synchronize()
+        assert torch.equal(rq.view(torch.int16), qo.contiguous().view(torch.int16))
+        assert torch.equal(rk.view(torch.int16), ko.contiguous().view(torch.int16))
+
 @pytest.mark.parametrize("case", CASES_TABLE, ids=[str(i) for i in range(len(CASES_TABLE))])
 def test_table_variants_f16(case):
     """The same shapes with IEEE binary16 activations and weights (the table
