@@ -427,15 +427,17 @@ def time_steps(step, args, stream, local, dev, pg):
     The spin-up (--spin-ms, 1000 ms by default; 0 turns it off) runs untimed
     steps for that long with the clock sampler already running, so that the
     K timed steps measure the state the GPU holds under sustained load, which
-    is how the op runs inside a model. On B200 that state differs from a cool
-    start in two ways: the 1 kW power cap lowers the SM clock (to about
-    1640-1700 MHz for these kernels, sw_power_cap active), and the kernels
-    nevertheless run faster than in the first few milliseconds after idle
+    is how the op runs inside a model. On most B200 boxes that state differs
+    from a cool start in two ways: the 1 kW power cap lowers the SM clock (to
+    about 1560-1870 MHz for these kernels, sw_power_cap active), and the
+    kernels nevertheless run faster than in the first milliseconds after idle
     (the FP8 3D workload: 260.6 us after 1 s of load at 1642 MHz against
-    288 us in 20 cold launches at 1965 MHz on the same box, memory clock at
-    its maximum in both). The bench line carries the sampled SM and memory
-    clocks and the time normalised to the top SM clock.
-    Returns (ms per step, max over ranks; the clock sampler)."""
+    288 us in 20 cold launches at 1965 MHz on one box, memory clock at its
+    maximum in both); on others the clock stays at 1965 MHz and the time with
+    it. The bench line carries the sampled SM and memory clocks, the time
+    normalised to the top SM clock, and the spread of single launches timed
+    one by one after the region.
+    Returns (ms per step, max over ranks; the clock sampler; the spread)."""
     import torch
 
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -459,6 +461,19 @@ def time_steps(step, args, stream, local, dev, pg):
         t_end.record(stream)
         torch.cuda.synchronize()
         clocks.load_to = time.perf_counter()
+        # The spread: the same steps again, each between its own events (an
+        # event between two launches ends their overlap, so these are single
+        # launches, reported beside the headline, not in it).
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for i, (a, b) in enumerate(ev):
+            a.record(stream)
+            step(i)
+            b.record(stream)
+        torch.cuda.synchronize()
+    one = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)
+    spread = {"min_us": one[0], "median_us": one[len(one) // 2], "max_us": one[-1],
+              "launches": len(one)} if one else None
     if pg:
         pg.barrier()
     total_ms = t_start.elapsed_time(t_end)
@@ -466,7 +481,7 @@ def time_steps(step, args, stream, local, dev, pg):
         t = torch.tensor([total_ms], device=dev)
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
         total_ms = t.item()
-    return total_ms / args.steps, clocks
+    return total_ms / args.steps, clocks, spread
 
 
 def clock_normalised(us_per_launch, clk):
@@ -503,7 +518,7 @@ def run_gpu(args, w):
     def step(i):
         Q.qknr_rope_3d(qkv, qw, kw, *outs, stream=stream, **p)
 
-    ms_per_step, clocks = time_steps(step, args, stream, local, dev, pg)
+    ms_per_step, clocks, spread = time_steps(step, args, stream, local, dev, pg)
     avg_launch_ms = ms_per_step
     tokens_per_s = world * T / (ms_per_step / 1e3)
 
@@ -566,6 +581,7 @@ def run_gpu(args, w):
                          "algorithmic_bytes_per_launch": alg_bytes},
             "cpu_baseline": cpu, "clocks": clk, "e2e": e2e, "gpu_launches": args.steps,
             "clock_normalised": clock_normalised(avg_launch_ms * 1e3, clk),
+            "launch_spread": spread,
             "host_us_per_call": host_us,
         }
         print(json.dumps(line), flush=True)
@@ -633,7 +649,7 @@ def run_gpu_table(args, w):
             rest.replay()
 
     graph_args = argparse.Namespace(steps=1, warmup=0, spin_ms=args.spin_ms)
-    ms_region, clocks = time_steps(region, graph_args, stream, local, dev, pg)
+    ms_region, clocks, _ = time_steps(region, graph_args, stream, local, dev, pg)
     ms_per_step = ms_region / args.steps
     tokens_per_s = world * T / (ms_per_step / 1e3)
     peak, peak_kind = measured_peaks()
@@ -974,7 +990,7 @@ def run_gpu_ucpe(args, w):
         if rc:
             Q._check(rc)
 
-    ms_per_step, clocks = time_steps(step, args, stream, local, dev, pg)
+    ms_per_step, clocks, spread = time_steps(step, args, stream, local, dev, pg)
     tokens_per_s = world * B * N / (ms_per_step / 1e3)
     alg_bytes = W.algorithmic_bytes(w)
     peak, peak_kind = measured_peaks()
@@ -1016,6 +1032,7 @@ def run_gpu_ucpe(args, w):
                          "algorithmic_bytes_per_launch": alg_bytes},
             "cpu_baseline": cpu, "clocks": clk, "e2e": e2e,
             "gpu_launches": args.steps, "clock_normalised": clock_normalised(ms_per_step * 1e3, clk),
+            "launch_spread": spread,
         }
         print(json.dumps(line), flush=True)
     if pg:
