@@ -48,7 +48,7 @@ TRAFFIC = {
     "table_il": (25730304 + 0, "e27ddf1ef866f0f6"),
     "table_hs_f16": (42768896 + 1988608, "e27ddf1ef866f0f6"),
     "table_d72": (24805632 + 768, "e27ddf1ef866f0f6"),
-    "ucpe": (263094272 + 204836864, "9bc6a6bf0edbf6fe"),
+    "ucpe": (263120896 + 205809920, "3edf98a9ef178c04"),
 }
 KERNEL_FILES = {"3d": ("rope3d.cu",), "table": ("rope_table.cu",),
                 "ucpe": ("ucpe_launch.h", "ucpe.cu")}

@@ -254,8 +254,8 @@ int qknr_rope_3d_with_ssq(const qknr_rope_3d_params* params, const float* ssq,
  *                  head_dim^-0.5 * spatial_tokens^-0.5).
  * Alignment: every pointer 16-byte aligned (QKNR_ERR_ALIGN otherwise).
  * Any num_tokens is allowed; a multiple of 16 is fastest (every output row
- * then starts on a 32-byte sector: 15% slower at a multiple of 8, about 38%
- * otherwise, at head_dim 112). Kernels: with at least two heads, head_dim
+ * then starts on a 32-byte sector: about 7% slower at 8 mod 16, 38% at counts
+ * that are not multiples of 8, at head_dim 112). Kernels: with at least two heads, head_dim
  * 72..120, device-memory q/k/v and batch*num_tokens >= 64, a warp-specialised
  * pipelined kernel (any num_tokens); else, with at least two heads,
  * head_dim <= 128 and an even num_tokens, a barrier-synchronised pipelined

@@ -435,8 +435,10 @@ __global__ void __launch_bounds__(512) ucpe_prep_kernel(const UcpeArgs a) {
 //     instructions (the tile's cos/sin values sit in registers for all its
 //     heads) and stores 16-bit values straight to [B, H, D, N]: the 32 lanes
 //     of a warp write the two 64-byte halves of a 128-byte output row, so any
-//     token count works. Its key sums go to a double-buffered shared array for
-//     the copy warp.
+//     token count works. When num_tokens is 8 mod 16 (rows 16 bytes off a
+//     32-byte sector) the warp instead writes its 8 x 64 results into its own
+//     1 KB shared buffer and sends whole rows as 16-byte stores. Its key sums
+//     go to a double-buffered shared array for the copy warp.
 // No CTA-wide barrier: compute warps wait only for their data, so a slow warp
 // delays the others only when the ring runs dry. Every wait is bounded in
 // time; on expiry the waiter raises the CTA's abort flag and bit 0 of the
@@ -465,18 +467,20 @@ __host__ __device__ inline int fast_row_pitch(int D) { return 2 * fast_row_elems
 __host__ __device__ inline int fast_stage_bytes(int D) { return 3 * kTile * fast_row_pitch(D); }
 
 struct FastLayout {
-    int ring, mats, part, bars, abort, total, stages;
+    int ring, out, mats, part, bars, abort, total, stages;
 };
 
-// The ring, two matrix buffers, two key-sum buffers, the mbarriers
+// The ring, the compute warps' 1 KB output buffers (staged), two matrix
+// buffers, two key-sum buffers, the mbarriers
 // (full[STAGES], empty[STAGES], mats_full[2], mats_empty[2], sums_full[2],
 // sums_empty[2]) and the abort flag.
-__host__ __device__ inline FastLayout fast_layout(int D, int stages) {
+__host__ __device__ inline FastLayout fast_layout(int D, int stages, bool staged) {
     FastLayout L;
     const int C = D / 8;
     L.stages = stages;
     L.ring = 0;
-    L.mats = stages * fast_stage_bytes(D);              // [2][2][32][kMatStride] f32
+    L.out = stages * fast_stage_bytes(D);               // [C][8][kTile] 16-bit
+    L.mats = L.out + (staged ? C * 8 * kTile * 2 : 0);  // [2][2][32][kMatStride] f32
     L.part = L.mats + 2 * 2 * kPairs * kMatStride * 4;  // [2][C][64] float2
     L.bars = L.part + 2 * C * kTile * 8;
     L.abort = L.bars + (2 * stages + 8) * 8;
@@ -578,13 +582,15 @@ __device__ __forceinline__ bool fast_reduce_sums(const UcpeArgs& a, const FastSt
 // K), project, rotate (Q, K), scale (K), round; each channel's two results are
 // stored straight to the output as 16-bit values (the 32 lanes of a warp write
 // the 64-byte halves of one 128-byte output row), each only if its token is in
-// the tile (va, vb). For K, the two tokens' sums of squares go to si/so.
-template <bool H16, int X>
+// the tile (va, vb). STAGED: the warp's 8 x 64 results go through its 1 KB
+// buffer obuf instead and leave as 16-byte stores of whole rows (tokens past
+// tv left out). For K, the two tokens' sums of squares go to si/so.
+template <bool H16, int X, bool STAGED>
 __device__ __forceinline__ void fast_tensor(const unsigned char* in, const float* mats,
                                             const float2 (&cj)[4], const float2 (&sj)[4],
                                             int pitch, int i, int c, float k_scale,
                                             uint8_t* out_row0, int64_t row_bytes, bool va, bool vb,
-                                            float2& si, float2& so) {
+                                            float2& si, float2& so, unsigned char* obuf, int tv) {
     const unsigned char* r0 = in + (X * kTile + i) * pitch + 16 * c;
     const uint4 ra = *reinterpret_cast<const uint4*>(r0);
     const uint4 rb = *reinterpret_cast<const uint4*>(r0 + kPairs * pitch);
@@ -637,18 +643,52 @@ __device__ __forceinline__ void fast_tensor(const unsigned char* in, const float
 #pragma unroll
         for (int e = 0; e < 8; ++e) y[e] = mul2(y[e], ks);
     }
-    uint8_t* o = out_row0 + 2 * i;
+    if constexpr (STAGED) {
+        const uint32_t sb = smem_u32(obuf);
+        __syncwarp();  // the warp has read back the previous tensor's tile
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const uint32_t w = f2_to_act2<H16>(y[e]);
-        if (va) st_u16(o + (int64_t)e * row_bytes, (uint16_t)w);
-        if (vb) st_u16(o + (int64_t)e * row_bytes + 2 * kPairs, (uint16_t)(w >> 16));
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t w = f2_to_act2<H16>(y[e]);
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(sb + e * 2 * kTile + 2 * i),
+                         "h"((uint16_t)w)
+                         : "memory");
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(sb + e * 2 * kTile + 2 * kPairs + 2 * i),
+                         "h"((uint16_t)(w >> 16))
+                         : "memory");
+        }
+        __syncwarp();
+        const int q = i & 7;  // 16-byte chunk q (tokens 8q..8q+7) of rows i/8 and i/8 + 4
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int r = (i >> 3) + 4 * hf;
+            uint4 v;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(sb + r * 2 * kTile + 16 * q)
+                         : "memory");
+            uint8_t* dst = out_row0 + (int64_t)r * row_bytes + 16 * q;
+            if (8 * q + 8 <= tv) {
+                st_v4(dst, v);
+            } else {
+                const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+                for (int t = 0; t < 8 && 8 * q + t < tv; ++t)
+                    st_u16(dst + 2 * t, (uint16_t)(ww[t >> 1] >> ((t & 1) * 16)));
+            }
+        }
+    } else {
+        uint8_t* o = out_row0 + 2 * i;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t w = f2_to_act2<H16>(y[e]);
+            if (va) st_u16(o + (int64_t)e * row_bytes, (uint16_t)w);
+            if (vb) st_u16(o + (int64_t)e * row_bytes + 2 * kPairs, (uint16_t)(w >> 16));
+        }
     }
 }
 
 // At most 15 compute warps (head_dim <= 120) and the copy warp: four warps per
 // scheduler, which leaves 128 registers a thread.
-template <bool H16, int STAGES>
+template <bool H16, int STAGES, bool STAGED>
 __global__ void __launch_bounds__(512, 1)
     ucpe_fast_kernel(const UcpeArgs a, const __grid_constant__ UcpeMaps maps,
                      const UcpeControl ctl) {
@@ -657,7 +697,7 @@ __global__ void __launch_bounds__(512, 1)
     const int64_t tiles_n = (N + kTile - 1) / kTile;
     const int64_t ntiles = a.batch * tiles_n;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const FastLayout L = fast_layout(D, STAGES);
+    const FastLayout L = fast_layout(D, STAGES, STAGED);
 
     extern __shared__ __align__(128) unsigned char smem[];
     float2* part = reinterpret_cast<float2*>(smem + L.part);  // [2][C][64]
@@ -775,10 +815,12 @@ __global__ void __launch_bounds__(512, 1)
                 sj[2] = make_float2(s0.z, s1.z); sj[3] = make_float2(s0.w, s1.w);
                 ok = mbar_wait_abortable(&mats_full[m], (uint32_t)((st.ti / 2) & 1),
                                          ctl.wait_limit_ns, abort_flag);
+                if (STAGED) ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
             }
             ok = mbar_wait_abortable(&full[slot], (uint32_t)((s / STAGES) & 1), ctl.wait_limit_ns,
                                      abort_flag);
+            if (STAGED) ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             const unsigned char* in = smem + L.ring + slot * fast_stage_bytes(D);
             const float* mats = mats_base + m * 2 * kPairs * kMatStride;
@@ -786,22 +828,24 @@ __global__ void __launch_bounds__(512, 1)
             const int64_t col = st.n0 * 2;
             float2 si = make_float2(0.f, 0.f), so = si;
             const bool va = i < st.tv, vb = i + kPairs < st.tv;
-            if (va) {
-                fast_tensor<H16, 0>(in, mats, cj, sj, pitch, i, c, a.k_scale,
-                                    a.q_out + head_row0 * row_bytes + col, row_bytes, va, vb, si,
-                                    so);
-                fast_tensor<H16, 1>(in, mats, cj, sj, pitch, i, c, a.k_scale,
-                                    a.k_out + head_row0 * row_bytes + col, row_bytes, va, vb, si,
-                                    so);
-                fast_tensor<H16, 2>(in, mats, cj, sj, pitch, i, c, a.k_scale,
-                                    a.v_out + head_row0 * row_bytes + col, row_bytes, va, vb, si,
-                                    so);
+            unsigned char* ob = smem + L.out + c * 8 * kTile * 2;
+            if (va || STAGED) {  // staged: the whole warp (rows past the tile end are zeros)
+                fast_tensor<H16, 0, STAGED>(in, mats, cj, sj, pitch, i, c, a.k_scale,
+                                            a.q_out + head_row0 * row_bytes + col, row_bytes, va,
+                                            vb, si, so, ob, st.tv);
+                fast_tensor<H16, 1, STAGED>(in, mats, cj, sj, pitch, i, c, a.k_scale,
+                                            a.k_out + head_row0 * row_bytes + col, row_bytes, va,
+                                            vb, si, so, ob, st.tv);
+                fast_tensor<H16, 2, STAGED>(in, mats, cj, sj, pitch, i, c, a.k_scale,
+                                            a.v_out + head_row0 * row_bytes + col, row_bytes, va,
+                                            vb, si, so, ob, st.tv);
             }
             mbar_arrive(&empty[slot]);  // the stage is read
             if (st.h == H - 1) mbar_arrive(&mats_empty[m]);
             if (s >= 2) {  // the copy warp has read step s - 2's key sums
                 ok = mbar_wait_abortable(&sums_empty[s & 1], (uint32_t)((s / 2 - 1) & 1),
                                          ctl.wait_limit_ns, abort_flag);
+                if (STAGED) ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
             }
             float2* pc = part + (s & 1) * C * kTile + c * kTile;
@@ -1198,27 +1242,42 @@ cudaError_t launch_fast(const UcpeArgs& a, const UcpeControl& ctl, cudaStream_t 
     // fit, take the one that keeps the most head stages in flight per SM
     // (CTAs per SM x (depth - 1)), the deeper ring on a tie.
     int stages = 0, per_sm = 0, best = 0;
+    bool staged = false;
     void (*kern)(const UcpeArgs, const UcpeMaps, const UcpeControl) = nullptr;
     for (int s = std::min(4, a.heads + 1); s >= 3; --s) {
-        if (fast_layout(D, s).total > optin) continue;
-        void (*k)(const UcpeArgs, const UcpeMaps, const UcpeControl) =
-            s == 4 ? (a.act_f16 ? ucpe_fast_kernel<true, 4> : ucpe_fast_kernel<false, 4>)
-                   : (a.act_f16 ? ucpe_fast_kernel<true, 3> : ucpe_fast_kernel<false, 3>);
-        int n = 0;
-        if (cached_smem_and_occupancy(reinterpret_cast<const void*>(k), block,
-                                      fast_layout(D, s).total, &n) != cudaSuccess) {
-            cudaGetLastError();
-            continue;
-        }
-        if (n * (s - 1) > best) {
-            best = n * (s - 1);
-            stages = s;
-            per_sm = n;
-            kern = k;
+        // Rows staged through shared memory and written with 16-byte stores
+        // when num_tokens is 8 mod 16: its rows then start 16 bytes past a
+        // 32-byte sector, where the direct 16-bit stores touch three sectors
+        // per 64-byte half row (117 -> 106.5 us at head_dim 112, 20 heads);
+        // elsewhere the extra instructions cost more than they save.
+        for (int sg = (a.num_tokens % 16 == 8) ? 1 : 0; sg >= 0; --sg) {
+            if (fast_layout(D, s, sg).total > optin) continue;
+            void (*k)(const UcpeArgs, const UcpeMaps, const UcpeControl) =
+                sg ? (s == 4 ? (a.act_f16 ? ucpe_fast_kernel<true, 4, true>
+                                          : ucpe_fast_kernel<false, 4, true>)
+                             : (a.act_f16 ? ucpe_fast_kernel<true, 3, true>
+                                          : ucpe_fast_kernel<false, 3, true>))
+                   : (s == 4 ? (a.act_f16 ? ucpe_fast_kernel<true, 4, false>
+                                          : ucpe_fast_kernel<false, 4, false>)
+                             : (a.act_f16 ? ucpe_fast_kernel<true, 3, false>
+                                          : ucpe_fast_kernel<false, 3, false>));
+            int n = 0;
+            if (cached_smem_and_occupancy(reinterpret_cast<const void*>(k), block,
+                                          fast_layout(D, s, sg).total, &n) != cudaSuccess) {
+                cudaGetLastError();
+                continue;
+            }
+            if (n * (s - 1) > best) {
+                best = n * (s - 1);
+                stages = s;
+                staged = sg;
+                per_sm = n;
+                kern = k;
+            }
         }
     }
     if (!kern) return cudaSuccess;  // does not fit: the general kernel runs instead
-    const FastLayout L = fast_layout(D, stages);
+    const FastLayout L = fast_layout(D, stages, staged);
     const int64_t tiles = a.batch * ((a.num_tokens + kTile - 1) / kTile);
     const int grid = (int)std::min<int64_t>((int64_t)sms * per_sm, tiles);
     e = launch_pdl(kern, grid, block, L.total, stream, a, maps, ctl);
@@ -1233,7 +1292,7 @@ cudaError_t launch_fast(const UcpeArgs& a, const UcpeControl& ctl, cudaStream_t 
         info->grid = grid;
         info->block = block;
         info->smem = L.total;
-        info->kernel_id = 5100 + 10 * stages + (a.act_f16 ? 1 : 0);
+        info->kernel_id = 5100 + 10 * stages + (a.act_f16 ? 1 : 0) + (staged ? 200 : 0);
     }
     return e;
 }

@@ -96,12 +96,14 @@ def test_table_wait_timeout_raises_status_and_context_survives(shape):
     assert Q.qknr_device_status() == 0
 
 
-def test_ucpe_wait_timeout_raises_status_and_context_survives():
+@pytest.mark.parametrize("N", [128, 136], ids=["direct_stores", "staged_stores"])
+def test_ucpe_wait_timeout_raises_status_and_context_survives(N):
     """The camera prep's warp-specialised kernel: its compute warps wait on the copy
     warp's ring stages and the copy warp on them, every wait bounded. With the
     hook, the stages never fill: the waits run out, the launch abandons its
-    steps, raises bit 0, waits (bounded) for the copies it issued and ends."""
-    B, N, H, D = 1, 128, 3, 112
+    steps, raises bit 0, waits (bounded) for the copies it issued and ends.
+    N = 136 (8 mod 16) takes the staged-store form, whose warps leave together."""
+    B, H, D = 1, 3, 112
     w = W.FormUcpe("case", batch=B, seq=N, heads=H, head_dim=D, spatial=N // 4, seed=6)
     inp = W.make_inputs(w, device="cuda")
     args = [inp[k] for k in ("q_normed", "k_normed", "v_raw", "proj_q", "proj_kv", "rope_cos",

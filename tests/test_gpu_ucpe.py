@@ -89,6 +89,11 @@ CASES = [
     (1, 129, 2, 256, "bf16"),
     (1, 151, 3, 112, "f16"),
     (2, 65, 2, 40, "f16"),
+    # N = 8 mod 16: the warp-specialised kernel stages each warp's rows in
+    # shared memory and writes 16-byte stores (last tiles of 8 and 40 tokens)
+    (1, 1000, 3, 112, "bf16"),
+    (2, 136, 4, 96, "f16"),
+    (1, 72, 2, 80, "bf16"),
     # The general kernel with whole tiles per CTA (enough tiles to fill every
     # SM): a tile's heads in turn over one staging of its matrices and cos/sin
     (1, 18480, 2, 136, "bf16"),
